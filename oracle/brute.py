@@ -1,0 +1,95 @@
+"""Pure-Python loop version of the HSTU layer (tiny inputs only).
+
+TEST INFRASTRUCTURE ONLY: used to pin the vectorised oracle in `oracle.hstu`.
+It is written independently of that module (scalar loops and the `math`
+module, no numpy arithmetic) so that an indexing, ordering or sign mistake in
+either one shows up as a disagreement.
+
+Follows the review of "Actions Speak Louder than Words" (xllm-io paper-review
+of arXiv 2402.17152), section 三 核心公式 Eq. 1-3, with the same readings as
+`oracle.hstu` (SiLU/ReLU/identity phi2, 1/n_u, LayerNorm over H*dv,
+ln(dt+1)/0.301 time buckets, min(i-j, P-1) position buckets, residual).
+"""
+from __future__ import annotations
+
+import math
+
+
+def _act(x, kind):
+    if kind == "relu":
+        return x if x > 0.0 else 0.0
+    if kind == "silu":
+        # x * sigmoid(x), written in the numerically safe form for both signs
+        if x >= 0:
+            return x / (1.0 + math.exp(-x))
+        ex = math.exp(x)
+        return x * ex / (1.0 + ex)
+    if kind == "identity":
+        return x
+    raise ValueError(kind)
+
+
+def _tbucket(dt, Tb):
+    if dt < 0:
+        return 0
+    b = int(math.floor(math.log(float(dt) + 1.0) / 0.301))
+    return max(0, min(Tb - 1, b))
+
+
+def layer(x, offsets, ts, w1, b1, w2, b2, rab_pos, rab_time, H, dqk, dv,
+          phi1="relu", phi2="silu", eps=1e-5, gamma=None, beta=None):
+    """One layer with explicit loops.  All arguments are nested lists / scalars."""
+    T = len(x)
+    d = len(x[0]) if T else 0
+    n1 = len(w1)
+    P, Tb = len(rab_pos[0]), len(rab_time[0])
+    hv = H * dv
+    y = [[0.0] * d for _ in range(T)]
+    for uu in range(len(offsets) - 1):
+        s, e = offsets[uu], offsets[uu + 1]
+        n = e - s
+        # Eq. 1, row by row
+        z = []
+        for i in range(s, e):
+            row = []
+            for c in range(n1):
+                acc = b1[c]
+                for t in range(d):
+                    acc += w1[c][t] * x[i][t]
+                row.append(_act(acc, phi1))
+            z.append(row)
+        U = [r[0:hv] for r in z]
+        V = [r[hv:2 * hv] for r in z]
+        Q = [r[2 * hv:2 * hv + H * dqk] for r in z]
+        K = [r[2 * hv + H * dqk:2 * hv + 2 * H * dqk] for r in z]
+        for i in range(n):
+            # Eq. 2 for row i, every head
+            o = [0.0] * hv
+            for h in range(H):
+                for j in range(i + 1):
+                    dot = 0.0
+                    for t in range(dqk):
+                        dot += Q[i][h * dqk + t] * K[j][h * dqk + t]
+                    bp = min(i - j, P - 1)
+                    bt = _tbucket(ts[s + i] - ts[s + j], Tb)
+                    a = _act(dot + rab_pos[h][bp] + rab_time[h][bt], phi2) / n
+                    for t in range(dv):
+                        o[h * dv + t] += a * V[j][h * dv + t]
+            # Eq. 3: LayerNorm over all heads, gate with U, project, residual
+            mean = sum(o) / hv
+            var = sum((val - mean) * (val - mean) for val in o) / hv
+            inv = 1.0 / math.sqrt(var + eps)
+            g = []
+            for c in range(hv):
+                nv = (o[c] - mean) * inv
+                if gamma is not None:
+                    nv *= gamma[c]
+                if beta is not None:
+                    nv += beta[c]
+                g.append(nv * U[i][c])
+            for c in range(d):
+                acc = b2[c]
+                for t in range(hv):
+                    acc += w2[c][t] * g[t]
+                y[s + i][c] = x[s + i][c] + acc
+    return y
