@@ -280,3 +280,38 @@ def algorithmic_counts(case: Case) -> dict:
     return {"tokens": T, "causal_pairs": pairs, "attn_flop_per_layer": attn_flop,
             "f1_flop_per_layer": f1_flop, "f2_flop_per_layer": f2_flop,
             "layers": cfg.num_layers}
+
+
+@dataclass
+class AttnCase:
+    """Inputs of the attention step alone (Eq. 2): Q, K, V per token and head."""
+    offsets: np.ndarray
+    timestamps: np.ndarray
+    q: np.ndarray         # [T, H*64] float32 holding bf16-representable values
+    k: np.ndarray
+    v: np.ndarray
+    rab_pos: np.ndarray   # [H, P] fp32
+    rab_time: np.ndarray  # [H, Tb] fp32
+    num_heads: int
+    dtype: str
+
+
+def make_attn_case(lengths: List[int], num_heads: int, P: int, Tb: int, seed: int = 0,
+                   dtype: str = "bf16", gap_kind: str = "exp", scale: float = 0.6,
+                   rab_std: float = 0.02) -> AttnCase:
+    """Q, K, V drawn like the projection's outputs: ReLU-shaped half-normals of std `scale`
+    (draw order: timestamps, q, k, v, rab_pos, rab_time)."""
+    rng = np.random.default_rng(seed)
+    offsets = np.zeros(len(lengths) + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(lengths)
+    T = int(offsets[-1])
+    ts = np.empty(T, dtype=np.int64)
+    for u, n in enumerate(lengths):
+        ts[offsets[u]:offsets[u + 1]] = _timeline(rng, gap_kind, n)
+    w = num_heads * 64
+    q, k, v = (to_dtype(np.maximum(rng.standard_normal((T, w), dtype=np.float32) * scale, 0.0)
+                        + 0.05 * rng.standard_normal((T, w), dtype=np.float32), dtype)
+               for _ in range(3))
+    rp = (rng.standard_normal((num_heads, P)) * rab_std).astype(np.float32)
+    rt = (rng.standard_normal((num_heads, Tb)) * rab_std).astype(np.float32)
+    return AttnCase(offsets, ts, q, k, v, rp, rt, num_heads, dtype)

@@ -1,0 +1,589 @@
+// Pointwise aggregated attention (Eq. 2 of the review of "Actions Speak Louder
+// than Words", section 三 核心公式): AV = phi2(Q K^T + rab^{p,t}) V / N over
+// jagged per-user sequences, with no softmax (hence no row max, no row sum,
+// no rescaling of the running output).
+//
+// One CTA owns a pair of 128-row query tiles (A = rows q0..q0+127, B = the
+// next 128) of one user and one head, and walks that user's key tiles in
+// order.  Causal mode (the layer forward) stops at the diagonal and masks
+// inside it; candidate mode (M-FALCON) lets candidate rows see every cached
+// history key and adds each candidate's own key/value in the epilogue.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax group A: thread t owns query row t of tile A
+//   warps 4-7  softmax group B: thread t owns query row t of tile B
+//   warp 8     producer: TMA loads of Q, K, V tiles (128B swizzle) and the
+//              per-key side data (timestamps, or candidate-mode bias)
+//   warp 9     MMA issuer (one thread) and TMEM owner
+// Tensor memory (512 columns): S_A, S_B (128 fp32 columns each), P_A, P_B
+// (64 columns each, bf16 pairs), O_A, O_B (64 fp32 columns each).
+// Per key tile: S = Q K^T (tcgen05, A and B from shared memory), the softmax
+// group reads S row by row, adds the gathered bias, applies phi2 and the
+// mask, writes P (bf16) back to tensor memory, then O += P V (tcgen05 with A
+// from tensor memory, V as an MN-major B operand).  1/N is applied once to O.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+constexpr int ATT_ROWS = 128;
+constexpr int ATT_KEYS = 128;
+constexpr int ATT_HD = 64;
+constexpr int ATT_STAGES = 3;
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_POS_PAD = 128;
+constexpr int MAX_TIME_BUCKETS = 256;
+
+constexpr uint32_t ATT_TILE_BYTES = ATT_ROWS * ATT_HD * 2;  // 16 KB
+
+struct AttnParams {
+  const int64_t* kv_offsets;   // [B+1] key/value rows per user (query rows too in causal mode)
+  const int64_t* q_offsets;    // [B+1] candidate rows per user (candidate mode)
+  const int64_t* timestamps;   // [T_kv]
+  const int64_t* request_ts;   // [B] (candidate mode)
+  const float* rab_pos;        // [H, P]
+  const float* rab_time;       // [H, Tb]
+  const __nv_bfloat16* q_self; // candidate mode: candidate Q, K, V rows (self term)
+  const __nv_bfloat16* k_self;
+  const __nv_bfloat16* v_self;
+  int64_t ld_self;             // row stride (elements) of q_self/k_self/v_self
+  __nv_bfloat16* av;           // [T_q, ld_av]
+  int64_t ld_av;
+  float* ln_part;              // [T_q, H, 2] (sum, centred sum of squares) or nullptr
+  int32_t B, H, P, Tb;
+  int32_t num_qpairs;
+  int32_t pos_cap;             // entries of the position table held in shared memory
+  int32_t phi2;
+  uint64_t timeout_ns;
+  int64_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0)
+};
+
+// ---------------------------------------------------------------- time buckets
+
+// Largest b in [0, Tb) with thr[b] <= dt (dt < 0 -> 0): the bucket of dt.
+__device__ __forceinline__ int time_bucket_search(int64_t dt, const int64_t* thr, int Tb) {
+  if (dt <= 0) return 0;
+  int lo = 0, hi = Tb - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (thr[mid] <= dt) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Bucket of t_i - t_j for one query row as j walks forward through keys with
+// non-decreasing timestamps: the bucket can only go down, so each step is a
+// compare against the current lower edge and an occasional decrement.
+struct BucketWalk {
+  int b;
+  int64_t ti;
+  int64_t bound;  // keys with t_j <= bound are still in bucket >= b
+
+  __device__ __forceinline__ void init(int64_t t_row, int64_t t_first_key, const int64_t* thr,
+                                       int Tb) {
+    ti = t_row;
+    b = time_bucket_search(t_row - t_first_key, thr, Tb);
+    bound = (b == 0) ? INT64_MAX : ti - thr[b];
+  }
+  // Advance to a key with timestamp tj; returns true when the bucket changed.
+  __device__ __forceinline__ bool step(int64_t tj, const int64_t* thr) {
+    bool changed = false;
+    while (tj > bound) {
+      --b;
+      bound = (b == 0) ? INT64_MAX : ti - thr[b];
+      changed = true;
+    }
+    return changed;
+  }
+};
+
+template <int PHI>
+__device__ __forceinline__ float apply_phi(float x) {
+  if constexpr (PHI == HSTU_ACT_SILU) {
+    const float h = 0.5f * x;  // x*sigmoid(x) = h + h*tanh(h), h = x/2
+    return fmaf(h, tanh_approx(h), h);
+  } else if constexpr (PHI == HSTU_ACT_RELU) {
+    return fmaxf(x, 0.0f);
+  } else {
+    return x;
+  }
+}
+
+// ---------------------------------------------------------------- shared memory
+
+struct AttnSmem {
+  static constexpr uint32_t kQ = 0;                                   // 2 x 16 KB
+  static constexpr uint32_t kK = kQ + 2 * ATT_TILE_BYTES;             // stages x 16 KB
+  static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 16 KB
+  static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 128 x 8 B
+  static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * ATT_KEYS * 8;
+  static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
+  static constexpr uint32_t kBars = kThr + MAX_TIME_BUCKETS * 8;
+  static constexpr uint32_t kMisc = kBars + 32 * 8;
+  static constexpr uint32_t kPos = kMisc + 64;
+  static constexpr uint32_t bytes(int pos_cap) {
+    return kPos + static_cast<uint32_t>(ATT_POS_PAD + pos_cap) * 4 + 1024;  // + align slack
+  }
+};
+
+// barrier slots
+enum : int {
+  BAR_Q_FULL = 0,
+  BAR_KV_FULL = 1,                     // + stage
+  BAR_KV_EMPTY = BAR_KV_FULL + ATT_STAGES,
+  BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + group
+  BAR_P_FULL = BAR_S_FULL + 2,             // + group
+  BAR_O_FULL = BAR_P_FULL + 2,
+  BAR_DONE = BAR_O_FULL + 1,
+  BAR_COUNT = BAR_DONE + 1
+};
+
+// ---------------------------------------------------------------- kernel
+
+template <bool CAND, int PHI>
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+
+  const int h = blockIdx.x;
+  const int u = blockIdx.y;
+  const int qp = p.num_qpairs - 1 - static_cast<int>(blockIdx.z);  // longest work first
+  const int64_t kv_start = p.kv_offsets[u];
+  const int n_kv = static_cast<int>(p.kv_offsets[u + 1] - kv_start);
+  int64_t q_start;
+  int n_q;
+  if constexpr (CAND) {
+    q_start = p.q_offsets[u];
+    n_q = static_cast<int>(p.q_offsets[u + 1] - q_start);
+  } else {
+    q_start = kv_start;
+    n_q = n_kv;
+  }
+  const int q0 = qp * 2 * ATT_ROWS;
+  if (q0 >= n_q) return;  // uniform across the CTA, before any allocation
+  const bool has_b = (q0 + ATT_ROWS) < n_q;
+
+  // number of key tiles each query tile consumes
+  int nA, nB;
+  if constexpr (CAND) {
+    const int nk = (n_kv + ATT_KEYS - 1) / ATT_KEYS;
+    nA = nk;
+    nB = has_b ? nk : 0;
+  } else {
+    nA = 2 * qp + 1;
+    nB = has_b ? 2 * qp + 2 : 0;
+  }
+  const int nk_total = nA > nB ? nA : nB;
+
+  uint8_t* sQ = smem + AttnSmem::kQ;
+  uint8_t* sK = smem + AttnSmem::kK;
+  uint8_t* sV = smem + AttnSmem::kV;
+  int64_t* sKeyTs = reinterpret_cast<int64_t*>(smem + AttnSmem::kKeyInfo);
+  float* sKeyRab = reinterpret_cast<float*>(smem + AttnSmem::kKeyInfo);
+  float* sTime = reinterpret_cast<float*>(smem + AttnSmem::kTimeTab);
+  int64_t* sThr = reinterpret_cast<int64_t*>(smem + AttnSmem::kThr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
+  uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 4);
+  float* sPos = reinterpret_cast<float*>(smem + AttnSmem::kPos);  // sPos[ATT_POS_PAD + k]
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int tid = threadIdx.x;
+
+  // ---------------- setup
+  if (tid == 0) {
+    mbar_init(&bars[BAR_Q_FULL], 1);
+    for (int s = 0; s < ATT_STAGES; ++s) {
+      mbar_init(&bars[BAR_KV_FULL + s], 2);
+      mbar_init(&bars[BAR_KV_EMPTY + s], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bars[BAR_S_FULL + g], 1);
+      mbar_init(&bars[BAR_P_FULL + g], ATT_ROWS);
+    }
+    mbar_init(&bars[BAR_O_FULL], 1);
+    mbar_init(&bars[BAR_DONE], 1);
+    *sAbort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sTmemBase, 512);
+    tmem_relinquish();
+  }
+  // position table: sPos[pad + k] = rab_pos[h, min(k, P-1)]; the pad covers the
+  // negative offsets read (and discarded) for masked entries of diagonal tiles
+  // causal rows of this CTA read i - j <= q0 + 255; candidates read n_kv - j <= n_kv
+  const int pos_needed = CAND ? (n_kv + 1) : (q0 + 2 * ATT_ROWS);
+  const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
+  for (int k = tid; k < ATT_POS_PAD + pos_needed; k += ATT_THREADS) {
+    float val = 0.0f;
+    if (k >= ATT_POS_PAD) val = rp[min(k - ATT_POS_PAD, p.P - 1)];
+    sPos[k] = val;
+  }
+  for (int k = tid; k < p.Tb; k += ATT_THREADS) {
+    sTime[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
+    sThr[k] = p.thr[k];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmemBase;
+  const WaitCtl ctl{sAbort, p.timeout_ns};
+
+  const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+  const uint32_t tP[2] = {tmem + 256u, tmem + 320u};
+  const uint32_t tO[2] = {tmem + 384u, tmem + 448u};
+
+  if (warp == 8) {
+    // ---------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars[BAR_Q_FULL], ATT_TILE_BYTES * (has_b ? 2u : 1u));
+      tma_load_2d(sQ, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD, static_cast<int32_t>(q_start + q0));
+      if (has_b)
+        tma_load_2d(sQ + ATT_TILE_BYTES, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD,
+                    static_cast<int32_t>(q_start + q0 + ATT_ROWS));
+    }
+    int64_t t_req = 0;
+    if constexpr (CAND) t_req = p.request_ts[u];
+    int issued = 0;
+    for (int kt = 0; kt < nk_total; ++kt) {
+      const int s = kt % ATT_STAGES;
+      const uint32_t par = (static_cast<uint32_t>(kt / ATT_STAGES) & 1u) ^ 1u;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait(&bars[BAR_KV_EMPTY + s], par, ctl) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[BAR_KV_FULL + s], 2 * ATT_TILE_BYTES);
+        const int32_t row = static_cast<int32_t>(kv_start + kt * ATT_KEYS);
+        tma_load_2d(sK + s * ATT_TILE_BYTES, &tm_k, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
+        tma_load_2d(sV + s * ATT_TILE_BYTES, &tm_v, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
+      }
+      ++issued;
+      for (int e = 0; e < ATT_KEYS / 32; ++e) {
+        const int c = lane + 32 * e;
+        const int j = kt * ATT_KEYS + c;
+        if constexpr (CAND) {
+          float r = 0.0f;
+          if (j < n_kv) {
+            const int64_t dt = t_req - p.timestamps[kv_start + j];
+            r = sPos[ATT_POS_PAD + (n_kv - j)] + sTime[time_bucket_search(dt, sThr, p.Tb)];
+          }
+          sKeyRab[s * ATT_KEYS * 2 + c] = r;
+        } else {
+          sKeyTs[s * ATT_KEYS + c] = (j < n_kv) ? p.timestamps[kv_start + j] : INT64_MAX;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[BAR_KV_FULL + s]);
+    }
+    // drain: every issued load must land before shared memory is released
+    if (lane == 0) {
+      mbar_wait_drain(&bars[BAR_Q_FULL], 0, p.timeout_ns);
+      for (int kt = max(0, issued - ATT_STAGES); kt < issued; ++kt)
+        mbar_wait_drain(&bars[BAR_KV_FULL + kt % ATT_STAGES],
+                        static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
+      const int nW[2] = {nA, nB};
+      bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
+      tc_fence_after();
+      auto issue_s = [&](int g, int s) {
+        const uint32_t qa = smem_u32(sQ + g * ATT_TILE_BYTES);
+        const uint32_t ka = smem_u32(sK + s * ATT_TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < ATT_HD / 16; ++kk) {
+          mma_bf16_ss(tS[g], smem_desc_sw128(qa + kk * 32, 16, 1024),
+                      smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[BAR_S_FULL + g]);
+      };
+      auto issue_pv = [&](int g, int s, bool first) {
+        const uint32_t va = smem_u32(sV + s * ATT_TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
+          mma_bf16_ts(tO[g], tP[g] + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024),
+                      idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      if (ok && nk_total > 0) {
+        ok = mbar_wait(&bars[BAR_KV_FULL + 0], 0, ctl);
+        tc_fence_after();
+        if (ok) {
+          if (nA > 0) issue_s(0, 0);
+          if (nB > 0) issue_s(1, 0);
+        }
+      }
+      for (int kt = 0; ok && kt < nk_total; ++kt) {
+        const int s = kt % ATT_STAGES;
+        bool next_ready = false;
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (kt >= nW[g]) continue;
+          ok = mbar_wait(&bars[BAR_P_FULL + g], static_cast<uint32_t>(kt) & 1u, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(g, s, kt == 0);
+          if (kt + 1 < nW[g]) {
+            if (!next_ready) {
+              const int s1 = (kt + 1) % ATT_STAGES;
+              ok = mbar_wait(&bars[BAR_KV_FULL + s1],
+                             static_cast<uint32_t>((kt + 1) / ATT_STAGES) & 1u, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              next_ready = true;
+            }
+            issue_s(g, (kt + 1) % ATT_STAGES);
+          }
+        }
+        if (ok) mma_commit(&bars[BAR_KV_EMPTY + s]);
+      }
+      mma_commit(&bars[BAR_O_FULL]);
+      // every MMA of this CTA must be complete before TMEM is released
+      mma_commit(&bars[BAR_DONE]);
+      mbar_wait_drain(&bars[BAR_DONE], 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax groups
+    const int g = warp >> 2;               // 0 = tile A, 1 = tile B
+    const int r = tid & (ATT_ROWS - 1);    // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int i = q0 + g * ATT_ROWS + r;   // query index within the user
+    const bool valid = i < n_q;
+    const int nW = g == 0 ? nA : nB;
+    bool ok = true;
+
+    BucketWalk walk;
+    float rt = 0.0f;
+    if constexpr (!CAND) {
+      if (valid) {
+        walk.init(p.timestamps[kv_start + i], p.timestamps[kv_start], sThr, p.Tb);
+      } else {
+        walk.ti = 0;
+        walk.b = 0;
+        walk.bound = INT64_MAX;
+      }
+      rt = sTime[walk.b];
+    }
+
+    for (int kt = 0; kt < nW; ++kt) {
+      const int s = kt % ATT_STAGES;
+      ok = mbar_wait(&bars[BAR_S_FULL + g], static_cast<uint32_t>(kt) & 1u, ctl);
+      // the producer's per-key side data for this stage (already complete)
+      if (ok)
+        ok = mbar_wait(&bars[BAR_KV_FULL + s], static_cast<uint32_t>(kt / ATT_STAGES) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-collective
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = !CAND && (kt == 2 * qp + g);
+      const int pos_base = ATT_POS_PAD + i - kt * ATT_KEYS;  // sPos index at column 0
+      const int key_lim = n_kv - kt * ATT_KEYS;              // columns >= key_lim are padding
+#pragma unroll 1
+      for (int ch = 0; ch < ATT_KEYS / 32; ++ch) {
+        uint32_t sv[32];
+        __syncwarp();
+        tmem_ld32(tS[g] + lane_off + ch * 32, sv);
+        tmem_ld_wait();
+        uint32_t pk[16];
+        if constexpr (CAND) {
+          const float* kr = sKeyRab + s * ATT_KEYS * 2 + ch * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float x0 = __uint_as_float(sv[c]) + kr[c];
+            float x1 = __uint_as_float(sv[c + 1]) + kr[c + 1];
+            float p0 = apply_phi<PHI>(x0);
+            float p1 = apply_phi<PHI>(x1);
+            if (ch * 32 + c >= key_lim) p0 = 0.0f;
+            if (ch * 32 + c + 1 >= key_lim) p1 = 0.0f;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          const int64_t* kts = sKeyTs + s * ATT_KEYS + ch * 32;
+          const float* pr = sPos + pos_base - ch * 32;
+          const bool steady = kts[31] <= walk.bound;  // no bucket change inside this chunk
+          float pv[32];
+          if (steady) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pv[c] = __uint_as_float(sv[c]) + (pr[-c] + rt);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (walk.step(kts[c], sThr)) rt = sTime[walk.b];
+              pv[c] = __uint_as_float(sv[c]) + (pr[-c] + rt);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pv[c] = apply_phi<PHI>(pv[c]);
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (ch * 32 + c > r) pv[c] = 0.0f;
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) pk[c >> 1] = pack_bf16x2(pv[c], pv[c + 1]);
+        }
+        __syncwarp();
+        tmem_st16(tP[g] + lane_off + ch * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[BAR_P_FULL + g]);
+    }
+
+    // ---------------- epilogue: O / N, LayerNorm partial sums, bf16 store
+    float o[ATT_HD];
+    if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL], 0, ctl);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      if (nW > 0) {
+        tc_fence_after();
+        uint32_t ov[32];
+        tmem_ld32(tO[g] + lane_off + 0, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(ov[c]);
+        tmem_ld32(tO[g] + lane_off + 32, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[32 + c] = __uint_as_float(ov[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < ATT_HD; ++c) o[c] = 0.0f;
+      }
+      if (valid) {
+        const int64_t row = q_start + i;
+        if constexpr (CAND) {
+          // the candidate's own key/value: position bucket 0, time bucket 0
+          const __nv_bfloat16* qs = p.q_self + row * p.ld_self + h * ATT_HD;
+          const __nv_bfloat16* ks = p.k_self + row * p.ld_self + h * ATT_HD;
+          const __nv_bfloat16* vs = p.v_self + row * p.ld_self + h * ATT_HD;
+          float dot = 0.0f;
+#pragma unroll
+          for (int c = 0; c < ATT_HD; c += 8) {
+            uint4 qa = *reinterpret_cast<const uint4*>(qs + c);
+            uint4 ka = *reinterpret_cast<const uint4*>(ks + c);
+            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qa);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&ka);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float2 qf = __bfloat1622float2(q2[t]);
+              float2 kf = __bfloat1622float2(k2[t]);
+              dot = fmaf(qf.x, kf.x, dot);
+              dot = fmaf(qf.y, kf.y, dot);
+            }
+          }
+          const float ps = apply_phi<PHI>(dot + sPos[ATT_POS_PAD + 0] + sTime[0]);
+#pragma unroll
+          for (int c = 0; c < ATT_HD; c += 8) {
+            uint4 va = *reinterpret_cast<const uint4*>(vs + c);
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&va);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float2 vf = __bfloat1622float2(v2[t]);
+              o[c + 2 * t] = fmaf(ps, vf.x, o[c + 2 * t]);
+              o[c + 2 * t + 1] = fmaf(ps, vf.y, o[c + 2 * t + 1]);
+            }
+          }
+        }
+        const float inv_n = 1.0f / static_cast<float>(CAND ? max(n_kv, 1) : n_kv);
+        float sum = 0.0f;
+#pragma unroll
+        for (int c = 0; c < ATT_HD; ++c) {
+          o[c] *= inv_n;
+          sum += o[c];
+        }
+        const float mean = sum * (1.0f / ATT_HD);
+        float m2 = 0.0f;
+#pragma unroll
+        for (int c = 0; c < ATT_HD; ++c) {
+          const float dlt = o[c] - mean;
+          m2 = fmaf(dlt, dlt, m2);
+        }
+        __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD;
+#pragma unroll
+        for (int c = 0; c < ATT_HD; c += 8) {
+          uint4 pkt;
+          pkt.x = pack_bf16x2(o[c + 0], o[c + 1]);
+          pkt.y = pack_bf16x2(o[c + 2], o[c + 3]);
+          pkt.z = pack_bf16x2(o[c + 4], o[c + 5]);
+          pkt.w = pack_bf16x2(o[c + 6], o[c + 7]);
+          *reinterpret_cast<uint4*>(dst + c) = pkt;
+        }
+        if (p.ln_part != nullptr) {
+          float2* lp = reinterpret_cast<float2*>(p.ln_part + (row * p.H + h) * 2);
+          *lp = make_float2(sum, m2);
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- debug: bucket indices
+
+// Writes, per user, the n x n blocks of position and time bucket indices the
+// attention kernel uses (BucketWalk for the time buckets, min(i-j, P-1) for
+// positions; -1 above the diagonal).  One thread per query row.
+__global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_t* timestamps,
+                                            const int64_t* block_offsets, int B, int P, int Tb,
+                                            int max_len, int32_t* pos_idx, int32_t* time_idx,
+                                            const __grid_constant__ AttnParams p) {
+  __shared__ int64_t sThr[MAX_TIME_BUCKETS];
+  for (int k = threadIdx.x; k < Tb; k += blockDim.x) sThr[k] = p.thr[k];
+  __syncthreads();
+  const int u = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= B) return;
+  const int64_t s = offsets[u];
+  const int n = static_cast<int>(offsets[u + 1] - s);
+  if (i >= n) return;
+  const int64_t base = block_offsets[u] + static_cast<int64_t>(i) * n;
+  BucketWalk walk;
+  walk.init(timestamps[s + i], timestamps[s], sThr, Tb);
+  for (int j = 0; j < n; ++j) {
+    if (j <= i) {
+      walk.step(timestamps[s + j], sThr);
+      pos_idx[base + j] = min(i - j, P - 1);
+      time_idx[base + j] = walk.b;
+    } else {
+      pos_idx[base + j] = -1;
+      time_idx[base + j] = -1;
+    }
+  }
+}
+
+// One CTA waits on a barrier that nothing completes; the bounded wait records
+// HSTU_ERR_DEVICE_TIMEOUT and the kernel returns.
+__global__ void hstu_debug_wait_timeout_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl ctl{&abort_flag, timeout_ns};
+  mbar_wait(&bar, 0, ctl);
+  __syncthreads();
+}
+
+}  // namespace hstu

@@ -1,0 +1,521 @@
+// The two linear layers of an HSTU block (review of "Actions Speak Louder
+// than Words", section 三 核心公式, Eq. 1 and Eq. 3; the efficiency table of
+// section 五 counts exactly two linear layers per block):
+//
+//   f1:  Z = phi1(X W1^T + b1), written straight into the U, V, Q, K blocks
+//        (Eq. 1's Split is only a choice of destination per column block).
+//   f2:  Y = X + (Norm(AV) (.) U) W2^T + b2 (Eq. 3 plus the residual), with the
+//        LayerNorm-and-gate computed by producer warps directly into the
+//        swizzled shared-memory A tile, so Norm(AV) (.) U never reaches HBM.
+//
+// Both are persistent tcgen05 GEMMs: 128 x 256 output tiles, 64-wide K steps
+// through a 4-stage shared-memory ring fed by TMA (128B swizzle), fp32
+// accumulators double-buffered in tensor memory (2 x 256 columns) so the
+// epilogue of one tile overlaps the main loop of the next.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+constexpr int G_BM = 128;
+constexpr int G_BN = 256;
+constexpr int G_BK = 64;
+constexpr int G_STAGES = 4;
+constexpr uint32_t G_A_BYTES = G_BM * G_BK * 2;  // 16 KB
+constexpr uint32_t G_B_BYTES = G_BN * G_BK * 2;  // 32 KB
+constexpr uint32_t G_STAGE_BYTES = G_A_BYTES + G_B_BYTES;
+
+struct GemmSmem {
+  static constexpr uint32_t kA = 0;
+  static constexpr uint32_t kB = G_STAGES * G_A_BYTES;
+  static constexpr uint32_t kBars = kB + G_STAGES * G_B_BYTES;  // 16 barriers
+  static constexpr uint32_t kMisc = kBars + 16 * 8;
+  static constexpr uint32_t kRowStats = kMisc + 64;             // 128 x (mean, rstd)
+  static constexpr uint32_t kBytes = kRowStats + G_BM * 8 + 1024;
+};
+
+enum : int {
+  GB_FULL = 0,                       // + stage
+  GB_EMPTY = GB_FULL + G_STAGES,     // + stage
+  GB_ACC_FULL = GB_EMPTY + G_STAGES, // + buffer
+  GB_ACC_EMPTY = GB_ACC_FULL + 2,    // + buffer
+  GB_DONE = GB_ACC_EMPTY + 2,
+  GB_COUNT = GB_DONE + 1
+};
+
+template <int ACT>
+__device__ __forceinline__ float apply_act(float x) {
+  if constexpr (ACT == HSTU_ACT_RELU) {
+    return fmaxf(x, 0.0f);
+  } else if constexpr (ACT == HSTU_ACT_SILU) {
+    return x / (1.0f + __expf(-x));
+  } else {
+    return x;
+  }
+}
+
+struct F1Params {
+  __nv_bfloat16* dst[4];  // destination of column block b (U, V, Q, K)
+  int64_t ld_dst[4];      // row stride of each destination (elements)
+  const float* bias;      // [N]
+  int64_t M;
+  int32_t N, K;
+  int32_t blk_w;          // width of one column block (H*64)
+  int32_t num_m_tiles, num_n_tiles;
+  uint64_t timeout_ns;
+};
+
+struct F2Params {
+  const __nv_bfloat16* av;  // [M, ld_av]
+  const __nv_bfloat16* u;   // [M, ld_u]
+  int64_t ld_av, ld_u;
+  const float* ln_part;     // [M, H, 2] per-head (sum, centred sum of squares) of AV rows
+  const float* gamma;       // [K] or nullptr
+  const float* beta;        // [K] or nullptr
+  float eps;
+  const float* bias;        // [N]
+  const float* x_res;       // [M, ld_x] fp32 residual, or nullptr -> x_lp
+  const __nv_bfloat16* x_lp;
+  int64_t ld_x;
+  float* y;                 // [M, ld_y] fp32
+  __nv_bfloat16* y_lp;      // [M, ld_y] or nullptr
+  int64_t ld_y;
+  int64_t M;
+  int32_t N, K, H;
+  int32_t num_m_tiles, num_n_tiles;
+  uint64_t timeout_ns;
+};
+
+// ------------------------------------------------------------------ shared pieces
+
+struct TileIter {
+  int t, step, total, n_tiles;
+  __device__ __forceinline__ int m() const { return t / n_tiles; }
+  __device__ __forceinline__ int n() const { return t % n_tiles; }
+};
+
+__device__ __forceinline__ void gemm_mma_loop(uint64_t* bars, const uint8_t* sA, const uint8_t* sB,
+                                              uint32_t tmem, int total_tiles, int k_blocks,
+                                              const WaitCtl& ctl, uint64_t drain_ns) {
+  constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_BN, false, false);
+  int stage = 0;
+  uint32_t phase = 0;
+  int lt = 0;
+  bool ok = true;
+  for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x, ++lt) {
+    const int acc = lt & 1;
+    const uint32_t acc_par = (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u;
+    ok = mbar_wait(&bars[GB_ACC_EMPTY + acc], acc_par, ctl);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t d = tmem + static_cast<uint32_t>(acc * G_BN);
+    for (int kb = 0; kb < k_blocks; ++kb) {
+      ok = mbar_wait(&bars[GB_FULL + stage], phase, ctl);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA + stage * G_A_BYTES);
+      const uint32_t b0 = smem_u32(sB + stage * G_B_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < G_BK / 16; ++kk) {
+        mma_bf16_ss(d, smem_desc_sw128(a0 + kk * 32, 16, 1024),
+                    smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                    (kb > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&bars[GB_EMPTY + stage]);
+      if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+    }
+    if (ok) mma_commit(&bars[GB_ACC_FULL + acc]);
+  }
+  mma_commit(&bars[GB_DONE]);
+  mbar_wait_drain(&bars[GB_DONE], 0, drain_ns);
+}
+
+// ------------------------------------------------------------------ f1
+
+template <int ACT>
+__global__ void __launch_bounds__(192, 1)
+hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ F1Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem + GemmSmem::kA;
+  uint8_t* sB = smem + GemmSmem::kB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmem::kBars);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + GemmSmem::kMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + GemmSmem::kMisc + 4);
+  const int warp = warp_id(), lane = lane_id();
+  const int total = p.num_m_tiles * p.num_n_tiles;
+  const int k_blocks = p.K / G_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G_STAGES; ++s) {
+      mbar_init(&bars[GB_FULL + s], 1);
+      mbar_init(&bars[GB_EMPTY + s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[GB_ACC_FULL + b], 1);
+      mbar_init(&bars[GB_ACC_EMPTY + b], 128);
+    }
+    mbar_init(&bars[GB_DONE], 1);
+    *sAbort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sTmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const WaitCtl ctl{sAbort, p.timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_w);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          ok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars[GB_FULL + stage], G_STAGE_BYTES);
+          tma_load_2d(sA + stage * G_A_BYTES, &tm_x, &bars[GB_FULL + stage], kb * G_BK, mt * G_BM);
+          tma_load_2d(sB + stage * G_B_BYTES, &tm_w, &bars[GB_FULL + stage], kb * G_BK, nt * G_BN);
+          ++issued;
+          if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // drain the loads still in flight
+      for (int k = max(0, issued - G_STAGES); k < issued; ++k)
+        mbar_wait_drain(&bars[GB_FULL + (k % G_STAGES)], static_cast<uint32_t>(k / G_STAGES) & 1u,
+                          p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int row_in_tile = (warp & 3) * 32 + lane;
+    int lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
+      const int acc = lt & 1;
+      bool ok = mbar_wait(&bars[GB_ACC_FULL + acc], static_cast<uint32_t>(lt >> 1) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mt) * G_BM + row_in_tile;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int ch = 0; ch < G_BN / 32; ++ch) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(acc * G_BN + ch * 32), v);
+        tmem_ld_wait();
+        const int col = nt * G_BN + ch * 32;
+        const int blk = col / p.blk_w;
+        const int cb = col - blk * p.blk_w;
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
+        uint32_t out[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = __ldg(b4 + q);
+          const float z0 = apply_act<ACT>(__uint_as_float(v[4 * q + 0]) + bb.x);
+          const float z1 = apply_act<ACT>(__uint_as_float(v[4 * q + 1]) + bb.y);
+          const float z2 = apply_act<ACT>(__uint_as_float(v[4 * q + 2]) + bb.z);
+          const float z3 = apply_act<ACT>(__uint_as_float(v[4 * q + 3]) + bb.w);
+          out[2 * q] = pack_bf16x2(z0, z1);
+          out[2 * q + 1] = pack_bf16x2(z2, z3);
+        }
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(p.dst[blk] + row * p.ld_dst[blk] + cb);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[GB_ACC_EMPTY + acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ f2
+
+__global__ void __launch_bounds__(320, 1)
+hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ F2Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem + GemmSmem::kA;
+  uint8_t* sB = smem + GemmSmem::kB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmem::kBars);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + GemmSmem::kMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + GemmSmem::kMisc + 4);
+  float2* sStats = reinterpret_cast<float2*>(smem + GemmSmem::kRowStats);
+  const int warp = warp_id(), lane = lane_id();
+  const int total = p.num_m_tiles * p.num_n_tiles;
+  const int k_blocks = p.K / G_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G_STAGES; ++s) {
+      mbar_init(&bars[GB_FULL + s], 1 + 4);  // TMA of W2 + 4 producer warps for the A tile
+      mbar_init(&bars[GB_EMPTY + s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[GB_ACC_FULL + b], 1);
+      mbar_init(&bars[GB_ACC_EMPTY + b], 128);
+    }
+    mbar_init(&bars[GB_DONE], 1);
+    *sAbort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sTmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const WaitCtl ctl{sAbort, p.timeout_ns};
+
+  if (warp == 0) {
+    // W2 tiles by TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_w);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const int nt = t % p.num_n_tiles;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          ok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars[GB_FULL + stage], G_B_BYTES);
+          tma_load_2d(sB + stage * G_B_BYTES, &tm_w, &bars[GB_FULL + stage], kb * G_BK, nt * G_BN);
+          ++issued;
+          if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int k = max(0, issued - G_STAGES); k < issued; ++k)
+        mbar_wait_drain(&bars[GB_FULL + (k % G_STAGES)], static_cast<uint32_t>(k / G_STAGES) & 1u,
+                          p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    __syncwarp();
+  } else if (warp >= 6) {
+    // A-tile producers: Norm(AV) (.) U, bf16, 128B-swizzled K-major layout
+    const int aw = warp - 6;             // 0..3
+    const int t128 = threadIdx.x - 192;  // 0..127
+    const int sub = lane >> 3;           // row within a group of 4
+    const int c16 = lane & 7;            // 16-byte chunk within a 128-byte row
+    const float inv_cnt = 1.0f / static_cast<float>(p.K);
+    const float inv_hd = 1.0f / 64.0f;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    // every producer warp runs every iteration (the named barriers below must
+    // match); after a failed wait a warp only skips the work
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int mt = t / p.num_n_tiles;
+      const int64_t m0 = static_cast<int64_t>(mt) * G_BM;
+      // per-row LayerNorm statistics combined from per-head partial sums
+      {
+        const int64_t row = m0 + t128;
+        float mean = 0.0f, rstd = 0.0f;
+        if (row < p.M) {
+          const float2* lp = reinterpret_cast<const float2*>(p.ln_part + row * p.H * 2);
+          float tot = 0.0f;
+          for (int hh = 0; hh < p.H; ++hh) tot += lp[hh].x;
+          mean = tot * inv_cnt;
+          float m2 = 0.0f;
+          for (int hh = 0; hh < p.H; ++hh) {
+            const float2 v = lp[hh];
+            const float dm = v.x * inv_hd - mean;
+            m2 += v.y + 64.0f * dm * dm;
+          }
+          rstd = rsqrtf(m2 * inv_cnt + p.eps);
+        }
+        named_barrier_sync(1, 128);  // previous tile's readers are done with sStats
+        sStats[t128] = make_float2(mean, rstd);
+        named_barrier_sync(1, 128);
+      }
+      for (int kb = 0; kb < k_blocks && ok; ++kb) {
+        int wok = 0;
+        if (lane == 0) wok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
+        if (!ok) break;
+        uint8_t* a_tile = sA + stage * G_A_BYTES;
+        const int col = kb * G_BK + c16 * 8;
+        float gm[8], bt[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { gm[e] = 1.0f; bt[e] = 0.0f; }
+        if (p.gamma != nullptr) {
+          const float4 g0 = __ldg(reinterpret_cast<const float4*>(p.gamma + col));
+          const float4 g1 = __ldg(reinterpret_cast<const float4*>(p.gamma + col) + 1);
+          gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
+          gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
+        }
+        if (p.beta != nullptr) {
+          const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.beta + col));
+          const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.beta + col) + 1);
+          bt[0] = b0.x; bt[1] = b0.y; bt[2] = b0.z; bt[3] = b0.w;
+          bt[4] = b1.x; bt[5] = b1.y; bt[6] = b1.z; bt[7] = b1.w;
+        }
+#pragma unroll 2
+        for (int it = 0; it < 8; ++it) {
+          const int r = aw * 32 + it * 4 + sub;
+          const int64_t row = m0 + r;
+          uint4 outv = make_uint4(0u, 0u, 0u, 0u);
+          if (row < p.M) {
+            const uint4 av4 = *reinterpret_cast<const uint4*>(p.av + row * p.ld_av + col);
+            const uint4 u4 = *reinterpret_cast<const uint4*>(p.u + row * p.ld_u + col);
+            const float2 st = sStats[r];
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av4);
+            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&u4);
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 af = __bfloat1622float2(a2[e]);
+              const float2 uf = __bfloat1622float2(u2[e]);
+              const float g0 = fmaf((af.x - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf.x;
+              const float g1 = fmaf((af.y - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf.y;
+              w[e] = pack_bf16x2(g0, g1);
+            }
+            outv = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          *reinterpret_cast<uint4*>(a_tile + r * 128 + ((c16 ^ (r & 7)) << 4)) = outv;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[GB_FULL + stage]);
+        if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else {
+    // epilogue warps 2..5: + b2 + residual, fp32 (and optional bf16) store
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int row_in_tile = (warp & 3) * 32 + lane;
+    int lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
+      const int acc = lt & 1;
+      bool ok = mbar_wait(&bars[GB_ACC_FULL + acc], static_cast<uint32_t>(lt >> 1) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mt) * G_BM + row_in_tile;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int ch = 0; ch < G_BN / 32; ++ch) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(acc * G_BN + ch * 32), v);
+        tmem_ld_wait();
+        const int col = nt * G_BN + ch * 32;
+        if (col >= p.N) continue;  // warp-uniform: the last N tile may be partial
+        if (row_ok) {
+          float y[32];
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 bb = __ldg(b4 + q);
+            y[4 * q + 0] = __uint_as_float(v[4 * q + 0]) + bb.x;
+            y[4 * q + 1] = __uint_as_float(v[4 * q + 1]) + bb.y;
+            y[4 * q + 2] = __uint_as_float(v[4 * q + 2]) + bb.z;
+            y[4 * q + 3] = __uint_as_float(v[4 * q + 3]) + bb.w;
+          }
+          if (p.x_res != nullptr) {
+            const float4* xr = reinterpret_cast<const float4*>(p.x_res + row * p.ld_x + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 xx = xr[q];
+              y[4 * q + 0] += xx.x;
+              y[4 * q + 1] += xx.y;
+              y[4 * q + 2] += xx.z;
+              y[4 * q + 3] += xx.w;
+            }
+          } else {
+            const uint4* xr = reinterpret_cast<const uint4*>(p.x_lp + row * p.ld_x + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 xx = xr[q];
+              const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xx);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(x2[e]);
+                y[8 * q + 2 * e] += f.x;
+                y[8 * q + 2 * e + 1] += f.y;
+              }
+            }
+          }
+          float4* yo = reinterpret_cast<float4*>(p.y + row * p.ld_y + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            yo[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+          if (p.y_lp != nullptr) {
+            uint4* yl = reinterpret_cast<uint4*>(p.y_lp + row * p.ld_y + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              yl[q] = make_uint4(pack_bf16x2(y[8 * q], y[8 * q + 1]),
+                                 pack_bf16x2(y[8 * q + 2], y[8 * q + 3]),
+                                 pack_bf16x2(y[8 * q + 4], y[8 * q + 5]),
+                                 pack_bf16x2(y[8 * q + 6], y[8 * q + 7]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[GB_ACC_EMPTY + acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ M-FALCON score
+
+// score[r] = <y[r, :], e[r, :]>, one warp per candidate row.
+template <typename TE>
+__global__ void hstu_score_kernel(const float* y, int64_t ld_y, const TE* e, int64_t ld_e,
+                                  int64_t M, int d, float* scores) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  float acc = 0.0f;
+  for (int c = lane; c < d; c += 32) {
+    float ev;
+    if constexpr (sizeof(TE) == 2) ev = __bfloat162float(e[row * ld_e + c]);
+    else ev = static_cast<float>(e[row * ld_e + c]);
+    acc = fmaf(y[row * ld_y + c], ev, acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) scores[row] = acc;
+}
+
+}  // namespace hstu

@@ -1,0 +1,840 @@
+// libhstu: the C ABI declared in include/hstu.h.
+//
+// Host side of every entry point: argument validation (no launch on error),
+// workspace carving, TMA tensor-map encoding and kernel launches on the
+// caller's stream.  The library is one translation unit so the device status
+// word in status.cuh is shared by all kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hstu.h"
+#include "attn.cuh"
+#include "fp32_path.cuh"
+#include "gemm.cuh"
+
+using namespace hstu;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kMaxLen = 16384;
+constexpr int kMaxPos = 16384;
+constexpr int kMaxDevices = 64;
+
+#define HSTU_CHECK_CUDA(expr)                      \
+  do {                                             \
+    cudaError_t err__ = (expr);                    \
+    if (err__ != cudaSuccess) return HSTU_ERR_CUDA; \
+  } while (0)
+
+// ------------------------------------------------------------------ time buckets
+
+// The unclamped bucket formula of rab^{p,t}: floor(ln(dt + 1) / 0.301), dt < 0 -> 0.
+int64_t time_bucket_formula(int64_t dt) {
+  if (dt < 0) return 0;
+  return static_cast<int64_t>(std::floor(std::log(static_cast<double>(dt) + 1.0) / 0.301));
+}
+
+// thr[k] = min { dt >= 0 : formula(dt) >= k } for k = 1..Tb-1, thr[0] = 0.
+// The formula is non-decreasing in dt, so a doubling search plus bisection
+// finds each edge exactly; the kernels then compare integers only.
+// Buckets that no dt below 2^62 reaches get INT64_MAX.
+void compute_thresholds(int Tb, int64_t* thr) {
+  const int64_t cap = int64_t(1) << 62;
+  thr[0] = 0;
+  for (int k = 1; k < Tb; ++k) {
+    if (time_bucket_formula(cap) < k) {
+      thr[k] = INT64_MAX;
+      continue;
+    }
+    int64_t hi = 1;
+    while (time_bucket_formula(hi) < k) hi = (hi < cap / 2) ? hi * 2 : cap;
+    int64_t lo = 0;
+    while (lo < hi) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (time_bucket_formula(mid) >= k) hi = mid; else lo = mid + 1;
+    }
+    thr[k] = lo;
+  }
+}
+
+const int64_t* thresholds_for(int Tb) {
+  static std::mutex mu;
+  static int64_t table[MAX_TIME_BUCKETS + 1][MAX_TIME_BUCKETS];
+  static bool ready[MAX_TIME_BUCKETS + 1] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ready[Tb]) {
+    compute_thresholds(Tb, table[Tb]);
+    ready[Tb] = true;
+  }
+  return table[Tb];
+}
+
+// ------------------------------------------------------------------ device info
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool smem_set = false;
+};
+
+hstu_status_t device_info(DeviceInfo** out) {
+  static std::mutex mu;
+  static DeviceInfo info[kMaxDevices];
+  int dev = 0;
+  HSTU_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& d = info[dev];
+  if (d.sm_count == 0) {
+    HSTU_CHECK_CUDA(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev));
+  }
+  if (!d.smem_set) {
+    const int att_max = static_cast<int>(AttnSmem::bytes(kMaxLen + 256));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_SILU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_RELU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_IDENTITY>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_SILU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_RELU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_IDENTITY>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    const int g = static_cast<int>(GemmSmem::kBytes);
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_SILU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_IDENTITY>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f2_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+    d.smem_set = true;
+  }
+  *out = &d;
+  return HSTU_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix with row stride `ld`
+// elements; box = box_cols x box_rows; 128-byte swizzle.
+hstu_status_t make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                            int64_t ld, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return HSTU_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ validation
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+hstu_status_t check_cfg(const hstu_layer_cfg_t* c) {
+  if (c == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  if (c->d_model <= 0 || c->num_heads <= 0 || c->dqk <= 0 || c->dv <= 0 ||
+      c->num_pos_buckets <= 0 || c->num_time_buckets <= 0)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (c->phi1 < HSTU_ACT_IDENTITY || c->phi1 > HSTU_ACT_SILU || c->phi2 < HSTU_ACT_IDENTITY ||
+      c->phi2 > HSTU_ACT_SILU)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (c->dtype != HSTU_BF16 && c->dtype != HSTU_FP32) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!(c->ln_eps >= 0.0f)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (c->dqk != ATT_HD || c->dv != ATT_HD) return HSTU_ERR_UNSUPPORTED;
+  if (c->d_model % 64 != 0) return HSTU_ERR_UNSUPPORTED;
+  if (c->num_pos_buckets > kMaxPos || c->num_time_buckets > MAX_TIME_BUCKETS)
+    return HSTU_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(c->num_heads) * ATT_HD > 8192) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+hstu_status_t check_jag(const hstu_jagged_t* j) {
+  if (j == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  if (j->batch < 0 || j->total_tokens < 0 || j->max_len < 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (j->batch > 0 && j->offsets == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  if (j->total_tokens > 0 && (j->timestamps == nullptr || j->batch == 0))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (j->max_len > kMaxLen || j->batch > 65535) return HSTU_ERR_UNSUPPORTED;
+  if (j->total_tokens > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+size_t elt(const hstu_layer_cfg_t* c) { return c->dtype == HSTU_BF16 ? 2 : 4; }
+
+int n1_of(const hstu_layer_cfg_t* c) { return 2 * c->num_heads * (c->dqk + c->dv); }
+
+// workspace for one layer: Z [T, n1], AV [T, H*dv], then LN partials (bf16
+// path) or the gated rows G [T, H*dv] (fp32 path)
+struct LayerWs {
+  void* z;
+  void* av;
+  void* extra;
+};
+
+size_t layer_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
+  const size_t e = elt(c);
+  const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
+  size_t b = align_up(static_cast<size_t>(T) * n1_of(c) * e, 256);
+  b += align_up(static_cast<size_t>(T) * hv * e, 256);
+  if (c->dtype == HSTU_BF16)
+    b += align_up(static_cast<size_t>(T) * c->num_heads * 2 * sizeof(float), 256);
+  else
+    b += align_up(static_cast<size_t>(T) * hv * sizeof(float), 256);
+  return b;
+}
+
+LayerWs carve_layer(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
+  const size_t e = elt(c);
+  const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  LayerWs w;
+  w.z = p;
+  p += align_up(static_cast<size_t>(T) * n1_of(c) * e, 256);
+  w.av = p;
+  p += align_up(static_cast<size_t>(T) * hv * e, 256);
+  w.extra = p;
+  return w;
+}
+
+// residual-stream buffers of a multi-layer pass: 2 x fp32 [T, d] + 2 x low-precision [T, d]
+size_t stream_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
+  const size_t d = static_cast<size_t>(c->d_model);
+  return 2 * align_up(static_cast<size_t>(T) * d * 4, 256) +
+         2 * align_up(static_cast<size_t>(T) * d * elt(c), 256);
+}
+
+// ------------------------------------------------------------------ launches
+
+struct AttnJob {
+  const hstu_layer_cfg_t* cfg;
+  const int64_t* kv_offsets;
+  const int64_t* q_offsets;   // nullptr in causal mode
+  const int64_t* timestamps;
+  const int64_t* request_ts;
+  int32_t batch;
+  int32_t max_q_len;
+  int32_t max_kv_len;
+  int64_t T_q, T_kv;
+  const void* q; int64_t ldq;
+  const void* k; int64_t ldk;
+  const void* v; int64_t ldv;
+  const void* q_self; const void* k_self; const void* v_self; int64_t ld_self;
+  const float* rab_pos;
+  const float* rab_time;
+  void* av; int64_t ld_av;
+  float* ln_part;
+  uint64_t timeout_ns;
+};
+
+template <bool CAND>
+hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
+  const hstu_layer_cfg_t* c = j.cfg;
+  if (j.batch == 0 || j.T_q == 0 || j.max_q_len == 0) return HSTU_OK;
+  DeviceInfo* di = nullptr;
+  hstu_status_t s = device_info(&di);
+  if (s != HSTU_OK) return s;
+  CUtensorMap mq, mk, mv;
+  const int64_t hc = static_cast<int64_t>(c->num_heads) * ATT_HD;
+  if ((s = make_map_bf16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS)) != HSTU_OK) return s;
+  // with no key rows at all (every history empty) no K/V tile is ever loaded;
+  // the maps then describe the query rows so that they stay valid
+  const bool no_kv = j.T_kv == 0;
+  if ((s = make_map_bf16(&mk, no_kv ? j.q : j.k, no_kv ? j.T_q : j.T_kv, hc,
+                         no_kv ? j.ldq : j.ldk, ATT_HD, ATT_KEYS)) != HSTU_OK)
+    return s;
+  if ((s = make_map_bf16(&mv, no_kv ? j.q : j.v, no_kv ? j.T_q : j.T_kv, hc,
+                         no_kv ? j.ldq : j.ldv, ATT_HD, ATT_KEYS)) != HSTU_OK)
+    return s;
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.kv_offsets = j.kv_offsets;
+  p.q_offsets = j.q_offsets;
+  p.timestamps = j.timestamps;
+  p.request_ts = j.request_ts;
+  p.rab_pos = j.rab_pos;
+  p.rab_time = j.rab_time;
+  p.q_self = static_cast<const __nv_bfloat16*>(j.q_self);
+  p.k_self = static_cast<const __nv_bfloat16*>(j.k_self);
+  p.v_self = static_cast<const __nv_bfloat16*>(j.v_self);
+  p.ld_self = j.ld_self;
+  p.av = static_cast<__nv_bfloat16*>(j.av);
+  p.ld_av = j.ld_av;
+  p.ln_part = j.ln_part;
+  p.B = j.batch;
+  p.H = c->num_heads;
+  p.P = c->num_pos_buckets;
+  p.Tb = c->num_time_buckets;
+  p.num_qpairs = (j.max_q_len + 2 * ATT_ROWS - 1) / (2 * ATT_ROWS);
+  const int longest = j.max_q_len > j.max_kv_len ? j.max_q_len : j.max_kv_len;
+  p.pos_cap = static_cast<int32_t>(align_up(static_cast<size_t>(longest) + 1, 256));
+  p.phi2 = c->phi2;
+  p.timeout_ns = j.timeout_ns;
+  std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
+  dim3 grid(c->num_heads, j.batch, p.num_qpairs);
+  const size_t smem = AttnSmem::bytes(p.pos_cap);
+  switch (c->phi2) {
+    case HSTU_ACT_SILU:
+      hstu_attn_kernel<CAND, HSTU_ACT_SILU><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+      break;
+    case HSTU_ACT_RELU:
+      hstu_attn_kernel<CAND, HSTU_ACT_RELU><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+      break;
+    default:
+      hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+      break;
+  }
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t ldx, int64_t M,
+                             const void* w1, const float* b1, void* const dst[4],
+                             const int64_t ld_dst[4], cudaStream_t st) {
+  if (M == 0) return HSTU_OK;
+  DeviceInfo* di = nullptr;
+  hstu_status_t s = device_info(&di);
+  if (s != HSTU_OK) return s;
+  const int N = n1_of(c), K = c->d_model;
+  CUtensorMap mx, mw;
+  if ((s = make_map_bf16(&mx, x, M, K, ldx, G_BK, G_BM)) != HSTU_OK) return s;
+  if ((s = make_map_bf16(&mw, w1, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  F1Params p;
+  std::memset(&p, 0, sizeof(p));
+  for (int b = 0; b < 4; ++b) {
+    p.dst[b] = static_cast<__nv_bfloat16*>(dst[b]);
+    p.ld_dst[b] = ld_dst[b];
+  }
+  p.bias = b1;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.blk_w = c->num_heads * ATT_HD;
+  p.num_m_tiles = static_cast<int32_t>((M + G_BM - 1) / G_BM);
+  p.num_n_tiles = N / G_BN;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int total = p.num_m_tiles * p.num_n_tiles;
+  const int grid = total < di->sm_count ? total : di->sm_count;
+  switch (c->phi1) {
+    case HSTU_ACT_RELU:
+      hstu_f1_kernel<HSTU_ACT_RELU><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      break;
+    case HSTU_ACT_SILU:
+      hstu_f1_kernel<HSTU_ACT_SILU><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      break;
+    default:
+      hstu_f1_kernel<HSTU_ACT_IDENTITY><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      break;
+  }
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
+                             const void* av, int64_t ld_av, const void* u, int64_t ld_u,
+                             const float* ln_part, const float* x_res, const void* x_lp,
+                             int64_t ld_x, float* y, void* y_lp, int64_t ld_y, int64_t M,
+                             cudaStream_t st) {
+  if (M == 0) return HSTU_OK;
+  DeviceInfo* di = nullptr;
+  hstu_status_t s = device_info(&di);
+  if (s != HSTU_OK) return s;
+  const int N = c->d_model, K = c->num_heads * c->dv;
+  CUtensorMap mw;
+  if ((s = make_map_bf16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  F2Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.av = static_cast<const __nv_bfloat16*>(av);
+  p.u = static_cast<const __nv_bfloat16*>(u);
+  p.ld_av = ld_av;
+  p.ld_u = ld_u;
+  p.ln_part = ln_part;
+  p.gamma = w->ln_gamma;
+  p.beta = w->ln_beta;
+  p.eps = c->ln_eps;
+  p.bias = w->b2;
+  p.x_res = x_res;
+  p.x_lp = static_cast<const __nv_bfloat16*>(x_lp);
+  p.ld_x = ld_x;
+  p.y = y;
+  p.y_lp = static_cast<__nv_bfloat16*>(y_lp);
+  p.ld_y = ld_y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.H = c->num_heads;
+  p.num_m_tiles = static_cast<int32_t>((M + G_BM - 1) / G_BM);
+  p.num_n_tiles = (N + G_BN - 1) / G_BN;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int total = p.num_m_tiles * p.num_n_tiles;
+  const int grid = total < di->sm_count ? total : di->sm_count;
+  hstu_f2_kernel<<<grid, 320, GemmSmem::kBytes, st>>>(mw, p);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+// ------------------------------------------------------------------ fp32 path
+
+hstu_status_t launch_f32_linear(const float* a, int64_t lda, int64_t M, int N, int K,
+                                const float* w, const float* bias, const float* res,
+                                int64_t ld_res, float* const dst[4], const int64_t ld_dst[4],
+                                int blk_w, int act, cudaStream_t st) {
+  if (M == 0) return HSTU_OK;
+  F32LinParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.a = a;
+  p.lda = lda;
+  p.w = w;
+  p.bias = bias;
+  p.res = res;
+  p.ld_res = ld_res;
+  for (int b = 0; b < 4; ++b) {
+    p.dst[b] = dst[b];
+    p.ld_dst[b] = ld_dst[b];
+  }
+  p.blk_w = blk_w;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.act = act;
+  dim3 grid((N + 63) / 64, static_cast<unsigned>((M + 63) / 64));
+  hstu_f32_linear_kernel<<<grid, 256, 0, st>>>(p);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t launch_f32_attn(const AttnJob& j, cudaStream_t st) {
+  const hstu_layer_cfg_t* c = j.cfg;
+  if (j.batch == 0 || j.T_q == 0 || j.max_q_len == 0) return HSTU_OK;
+  F32AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const float*>(j.q);
+  p.k = static_cast<const float*>(j.k);
+  p.v = static_cast<const float*>(j.v);
+  p.ldq = j.ldq;
+  p.ldk = j.ldk;
+  p.ldv = j.ldv;
+  p.kv_offsets = j.kv_offsets;
+  p.q_offsets = j.q_offsets;
+  p.timestamps = j.timestamps;
+  p.request_ts = j.request_ts;
+  p.rab_pos = j.rab_pos;
+  p.rab_time = j.rab_time;
+  p.q_self = static_cast<const float*>(j.q_self);
+  p.k_self = static_cast<const float*>(j.k_self);
+  p.v_self = static_cast<const float*>(j.v_self);
+  p.ld_self = j.ld_self;
+  p.av = static_cast<float*>(j.av);
+  p.ld_av = j.ld_av;
+  p.B = j.batch;
+  p.H = c->num_heads;
+  p.P = c->num_pos_buckets;
+  p.Tb = c->num_time_buckets;
+  p.phi2 = c->phi2;
+  p.cand = j.q_offsets != nullptr ? 1 : 0;
+  std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
+  dim3 grid((j.max_q_len + 31) / 32, c->num_heads, j.batch);
+  hstu_f32_attn_kernel<<<grid, 128, 0, st>>>(p);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+// One layer on the fp32 path.
+hstu_status_t layer_fp32(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
+                         const AttnJob& base, const float* x_in, const float* x_res, int64_t T,
+                         float* y_out, float* kv_cache, const LayerWs& ws, bool cand,
+                         cudaStream_t st) {
+  const int H = c->num_heads, hv = H * ATT_HD, n1 = n1_of(c), d = c->d_model;
+  float* z = static_cast<float*>(ws.z);
+  float* dst[4] = {z, z + hv, z + 2 * hv, z + 2 * hv + hv};
+  int64_t ldd[4] = {n1, n1, n1, n1};
+  if (kv_cache != nullptr) {
+    dst[1] = kv_cache + hv;  // V
+    dst[3] = kv_cache;       // K
+    ldd[1] = ldd[3] = 2 * hv;
+  }
+  hstu_status_t s = launch_f32_linear(x_in, d, T, n1, d, static_cast<const float*>(w->w1), w->b1,
+                                      nullptr, 0, dst, ldd, hv, c->phi1, st);
+  if (s != HSTU_OK) return s;
+  AttnJob j = base;
+  if (!cand) {
+    j.q = dst[2]; j.ldq = ldd[2];
+    j.k = dst[3]; j.ldk = ldd[3];
+    j.v = dst[1]; j.ldv = ldd[1];
+  } else {
+    j.q_self = dst[2]; j.k_self = dst[3]; j.v_self = dst[1]; j.ld_self = n1;
+    j.q = dst[2]; j.ldq = n1;
+  }
+  j.rab_pos = w->rab_pos;
+  j.rab_time = w->rab_time;
+  j.av = ws.av;
+  j.ld_av = hv;
+  if ((s = launch_f32_attn(j, st)) != HSTU_OK) return s;
+  float* g = static_cast<float*>(ws.extra);
+  const unsigned blocks = static_cast<unsigned>((T * 32 + 255) / 256);
+  hstu_f32_ln_gate_kernel<<<blocks, 256, 0, st>>>(static_cast<const float*>(ws.av), hv, z, n1,
+                                                  w->ln_gamma, w->ln_beta, c->ln_eps, T, hv, g, hv);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  float* ydst[4] = {y_out, y_out, y_out, y_out};
+  int64_t ydl[4] = {d, d, d, d};
+  return launch_f32_linear(g, hv, T, d, hv, static_cast<const float*>(w->w2), w->b2,
+                           x_res != nullptr ? x_res : x_in, d, ydst, ydl, d, HSTU_ACT_IDENTITY, st);
+}
+
+// One layer on the bf16 tensor-core path.
+hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
+                         const AttnJob& base, const void* x_in, const float* x_res, int64_t T,
+                         float* y_out, void* y_lp, void* kv_cache, const LayerWs& ws, bool cand,
+                         cudaStream_t st) {
+  const int H = c->num_heads, hv = H * ATT_HD, n1 = n1_of(c), d = c->d_model;
+  __nv_bfloat16* z = static_cast<__nv_bfloat16*>(ws.z);
+  void* dst[4] = {z, z + hv, z + 2 * hv, z + 3 * hv};
+  int64_t ldd[4] = {n1, n1, n1, n1};
+  if (kv_cache != nullptr) {
+    __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(kv_cache);
+    dst[1] = kv + hv;  // V
+    dst[3] = kv;       // K
+    ldd[1] = ldd[3] = 2 * hv;
+  }
+  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, st);
+  if (s != HSTU_OK) return s;
+  AttnJob j = base;
+  if (!cand) {
+    j.q = dst[2]; j.ldq = ldd[2];
+    j.k = dst[3]; j.ldk = ldd[3];
+    j.v = dst[1]; j.ldv = ldd[1];
+  } else {
+    j.q = dst[2]; j.ldq = n1;
+    j.q_self = dst[2]; j.k_self = dst[3]; j.v_self = dst[1]; j.ld_self = n1;
+  }
+  j.rab_pos = w->rab_pos;
+  j.rab_time = w->rab_time;
+  j.av = ws.av;
+  j.ld_av = hv;
+  j.ln_part = static_cast<float*>(ws.extra);
+  s = cand ? launch_attn_bf16<true>(j, st) : launch_attn_bf16<false>(j, st);
+  if (s != HSTU_OK) return s;
+  return launch_f2_bf16(c, w, ws.av, hv, z, n1, static_cast<const float*>(ws.extra), x_res, x_in,
+                        d, y_out, y_lp, d, T, st);
+}
+
+hstu_status_t check_weights(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w) {
+  if (w == nullptr || w->w1 == nullptr || w->b1 == nullptr || w->w2 == nullptr ||
+      w->b2 == nullptr || w->rab_pos == nullptr || w->rab_time == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(w->w1) || !aligned16(w->b1) || !aligned16(w->w2) || !aligned16(w->b2) ||
+      !aligned16(w->ln_gamma) || !aligned16(w->ln_beta))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  (void)c;
+  return HSTU_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* hstu_version(void) { return "libhstu 0.1 (sm_100a)"; }
+
+const char* hstu_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "ok";
+    case HSTU_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case HSTU_ERR_CUDA: return "CUDA error";
+    case HSTU_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case HSTU_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case HSTU_ERR_DEVICE_CHECK: return "device-side input check failed";
+  }
+  return "unknown status";
+}
+
+size_t hstu_layer_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total_tokens) {
+  if (check_cfg(cfg) != HSTU_OK || total_tokens < 0) return 0;
+  return layer_ws_bytes(cfg, total_tokens);
+}
+
+size_t hstu_forward_workspace_bytes(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                                    int64_t total_tokens) {
+  if (check_cfg(cfg) != HSTU_OK || total_tokens < 0 || num_layers < 1) return 0;
+  return layer_ws_bytes(cfg, total_tokens) + stream_ws_bytes(cfg, total_tokens);
+}
+
+size_t hstu_mfalcon_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t num_cand) {
+  if (check_cfg(cfg) != HSTU_OK || num_cand < 0) return 0;
+  return layer_ws_bytes(cfg, num_cand) + stream_ws_bytes(cfg, num_cand);
+}
+
+hstu_status_t hstu_time_bucket_thresholds(int32_t num_time_buckets, int64_t* thr_out) {
+  if (thr_out == nullptr || num_time_buckets < 1 || num_time_buckets > MAX_TIME_BUCKETS)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  std::memcpy(thr_out, thresholds_for(num_time_buckets), sizeof(int64_t) * num_time_buckets);
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag, const void* q,
+                            const void* k, const void* v, const float* rab_pos,
+                            const float* rab_time, void* av_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (jag->total_tokens == 0 || jag->batch == 0) return HSTU_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || rab_pos == nullptr ||
+      rab_time == nullptr || av_out == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(av_out))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  const int64_t hv = static_cast<int64_t>(cfg->num_heads) * ATT_HD;
+  AttnJob j;
+  std::memset(&j, 0, sizeof(j));
+  j.cfg = cfg;
+  j.kv_offsets = jag->offsets;
+  j.timestamps = jag->timestamps;
+  j.batch = jag->batch;
+  j.max_q_len = j.max_kv_len = jag->max_len;
+  j.T_q = j.T_kv = jag->total_tokens;
+  j.q = q; j.ldq = hv;
+  j.k = k; j.ldk = hv;
+  j.v = v; j.ldv = hv;
+  j.rab_pos = rab_pos;
+  j.rab_time = rab_time;
+  j.av = av_out;
+  j.ld_av = hv;
+  j.timeout_ns = kDefaultTimeoutNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == HSTU_FP32) return launch_f32_attn(j, st);
+  return launch_attn_bf16<false>(j, st);
+}
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                             const hstu_jagged_t* jag, const void* x_in, const float* x_res,
+                             float* y_out, void* y_out_lp, void* kv_cache_out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if ((s = check_weights(cfg, w)) != HSTU_OK) return s;
+  const int64_t T = jag->total_tokens;
+  if (T == 0 || jag->batch == 0) return HSTU_OK;
+  if (x_in == nullptr || y_out == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(x_res) || !aligned16(y_out) || !aligned16(y_out_lp) ||
+      !aligned16(kv_cache_out) || !aligned16(workspace))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || ws_bytes < layer_ws_bytes(cfg, T)) return HSTU_ERR_WORKSPACE_TOO_SMALL;
+  AttnJob base;
+  std::memset(&base, 0, sizeof(base));
+  base.cfg = cfg;
+  base.kv_offsets = jag->offsets;
+  base.timestamps = jag->timestamps;
+  base.batch = jag->batch;
+  base.max_q_len = base.max_kv_len = jag->max_len;
+  base.T_q = base.T_kv = T;
+  base.timeout_ns = kDefaultTimeoutNs;
+  const LayerWs ws = carve_layer(cfg, T, workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == HSTU_FP32) {
+    s = layer_fp32(cfg, w, base, static_cast<const float*>(x_in), x_res, T, y_out,
+                   static_cast<float*>(kv_cache_out), ws, false, st);
+    if (s == HSTU_OK && y_out_lp != nullptr && y_out_lp != y_out)
+      HSTU_CHECK_CUDA(cudaMemcpyAsync(y_out_lp, y_out, sizeof(float) * T * cfg->d_model,
+                                      cudaMemcpyDeviceToDevice, st));
+    return s;
+  }
+  return layer_bf16(cfg, w, base, x_in, x_res, T, y_out, y_out_lp, kv_cache_out, ws, false, st);
+}
+
+hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                           const hstu_layer_weights_t* weights, const hstu_jagged_t* jag,
+                           const void* x_in, float* y_out, void* kv_cache_out, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (num_layers < 1 || weights == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  for (int l = 0; l < num_layers; ++l)
+    if ((s = check_weights(cfg, &weights[l])) != HSTU_OK) return s;
+  const int64_t T = jag->total_tokens;
+  if (T == 0 || jag->batch == 0) return HSTU_OK;
+  if (x_in == nullptr || y_out == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(y_out) || !aligned16(kv_cache_out) || !aligned16(workspace))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || ws_bytes < hstu_forward_workspace_bytes(cfg, num_layers, T))
+    return HSTU_ERR_WORKSPACE_TOO_SMALL;
+  const int d = cfg->d_model;
+  const size_t lw = layer_ws_bytes(cfg, T);
+  uint8_t* sp = static_cast<uint8_t*>(workspace) + lw;
+  const size_t fbytes = align_up(static_cast<size_t>(T) * d * 4, 256);
+  const size_t lbytes = align_up(static_cast<size_t>(T) * d * elt(cfg), 256);
+  float* yf[2] = {reinterpret_cast<float*>(sp), reinterpret_cast<float*>(sp + fbytes)};
+  void* yl[2] = {sp + 2 * fbytes, sp + 2 * fbytes + lbytes};
+  const size_t cache_layer = static_cast<size_t>(T) * 2 * cfg->num_heads * ATT_HD * elt(cfg);
+  for (int l = 0; l < num_layers; ++l) {
+    const bool last = (l == num_layers - 1);
+    const void* xin = (l == 0) ? x_in : (cfg->dtype == HSTU_BF16 ? yl[(l - 1) & 1]
+                                                                  : static_cast<void*>(yf[(l - 1) & 1]));
+    const float* xres = (l == 0) ? nullptr : yf[(l - 1) & 1];
+    float* yo = last ? y_out : yf[l & 1];
+    void* ylp = (last || cfg->dtype == HSTU_FP32) ? nullptr : yl[l & 1];
+    void* kv = kv_cache_out == nullptr ? nullptr
+                                       : static_cast<uint8_t*>(kv_cache_out) + cache_layer * l;
+    s = hstu_layer_fwd(cfg, &weights[l], jag, xin, xres, yo, ylp, kv, workspace, lw, stream);
+    if (s != HSTU_OK) return s;
+  }
+  return HSTU_OK;
+}
+
+hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                            const hstu_layer_weights_t* weights, const hstu_jagged_t* history,
+                            const void* kv_cache, const int64_t* cand_offsets, int64_t num_cand,
+                            int32_t max_cand, const void* cand_emb, const int64_t* request_ts,
+                            int32_t microbatch, float* scores, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(history)) != HSTU_OK) return s;
+  if (num_layers < 1 || weights == nullptr || microbatch < 1 || num_cand < 0 || max_cand < 0)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  for (int l = 0; l < num_layers; ++l)
+    if ((s = check_weights(cfg, &weights[l])) != HSTU_OK) return s;
+  if (num_cand == 0 || history->batch == 0) return HSTU_OK;
+  if (max_cand > kMaxLen) return HSTU_ERR_UNSUPPORTED;
+  if (num_cand > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
+  if (cand_offsets == nullptr || cand_emb == nullptr || request_ts == nullptr ||
+      scores == nullptr || (history->total_tokens > 0 && kv_cache == nullptr))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(cand_emb) || !aligned16(kv_cache) || !aligned16(workspace))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || ws_bytes < hstu_mfalcon_workspace_bytes(cfg, num_cand))
+    return HSTU_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t M = num_cand;
+  const int d = cfg->d_model;
+  const int hv = cfg->num_heads * ATT_HD;
+  const size_t lw = layer_ws_bytes(cfg, M);
+  const LayerWs ws = carve_layer(cfg, M, workspace);
+  uint8_t* sp = static_cast<uint8_t*>(workspace) + lw;
+  const size_t fbytes = align_up(static_cast<size_t>(M) * d * 4, 256);
+  const size_t lbytes = align_up(static_cast<size_t>(M) * d * elt(cfg), 256);
+  float* yf[2] = {reinterpret_cast<float*>(sp), reinterpret_cast<float*>(sp + fbytes)};
+  void* yl[2] = {sp + 2 * fbytes, sp + 2 * fbytes + lbytes};
+  const size_t cache_layer =
+      static_cast<size_t>(history->total_tokens) * 2 * hv * elt(cfg);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnJob base;
+  std::memset(&base, 0, sizeof(base));
+  base.cfg = cfg;
+  base.kv_offsets = history->offsets;
+  base.q_offsets = cand_offsets;
+  base.timestamps = history->timestamps;
+  base.request_ts = request_ts;
+  base.batch = history->batch;
+  base.max_q_len = max_cand;
+  base.max_kv_len = history->max_len;
+  base.T_q = M;
+  base.T_kv = history->total_tokens;
+  base.timeout_ns = kDefaultTimeoutNs;
+  for (int l = 0; l < num_layers; ++l) {
+    const uint8_t* cache_l = static_cast<const uint8_t*>(kv_cache) + cache_layer * l;
+    AttnJob j = base;
+    const size_t e = elt(cfg);
+    j.k = cache_l;
+    j.ldk = 2 * hv;
+    j.v = cache_l + static_cast<size_t>(hv) * e;
+    j.ldv = 2 * hv;
+    const float* xres = (l == 0) ? nullptr : yf[(l - 1) & 1];
+    float* yo = yf[l & 1];
+    if (cfg->dtype == HSTU_FP32) {
+      const float* xin = (l == 0) ? static_cast<const float*>(cand_emb) : yf[(l - 1) & 1];
+      s = layer_fp32(cfg, &weights[l], j, xin, xres, M, yo, nullptr, ws, true, st);
+    } else {
+      const void* xin = (l == 0) ? cand_emb : yl[(l - 1) & 1];
+      s = layer_bf16(cfg, &weights[l], j, xin, xres, M, yo, yl[l & 1], nullptr, ws, true, st);
+    }
+    if (s != HSTU_OK) return s;
+  }
+  const float* yfin = yf[(num_layers - 1) & 1];
+  const unsigned blocks = static_cast<unsigned>((M * 32 + 255) / 256);
+  if (cfg->dtype == HSTU_FP32)
+    hstu_score_kernel<float><<<blocks, 256, 0, st>>>(yfin, d, static_cast<const float*>(cand_emb),
+                                                     d, M, d, scores);
+  else
+    hstu_score_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        yfin, d, static_cast<const __nv_bfloat16*>(cand_emb), d, M, d, scores);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_get_device_status(void* stream) {
+  HSTU_CHECK_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  unsigned int v = 0;
+  HSTU_CHECK_CUDA(cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)));
+  const unsigned int zero = 0;
+  HSTU_CHECK_CUDA(cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)));
+  return static_cast<hstu_status_t>(v);
+}
+
+hstu_status_t hstu_debug_rab_index(const hstu_jagged_t* jag, int32_t num_pos_buckets,
+                                   int32_t num_time_buckets, const int64_t* block_offsets,
+                                   int32_t* pos_idx, int32_t* time_idx, void* stream) {
+  hstu_status_t s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (num_pos_buckets < 1 || num_time_buckets < 1 || num_time_buckets > MAX_TIME_BUCKETS)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (jag->total_tokens == 0 || jag->batch == 0 || jag->max_len == 0) return HSTU_OK;
+  if (block_offsets == nullptr || pos_idx == nullptr || time_idx == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  std::memcpy(p.thr, thresholds_for(num_time_buckets), sizeof(int64_t) * num_time_buckets);
+  dim3 grid((jag->max_len + 127) / 128, jag->batch);
+  hstu_debug_rab_index_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      jag->offsets, jag->timestamps, block_offsets, jag->batch, num_pos_buckets,
+      num_time_buckets, jag->max_len, pos_idx, time_idx, p);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  hstu_debug_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,210 @@
+/*
+ * hstu.h -- C ABI of libhstu, a B200 (sm_100a) implementation of the forward
+ * pass of the HSTU layer (Hierarchical Sequential Transduction Unit) and of
+ * M-FALCON candidate scoring.
+ *
+ * Source of the method: the review of "Actions Speak Louder than Words:
+ * Trillion-Parameter Sequential Transducers for Generative Recommendations"
+ * (xllm-io paper-review of arXiv 2402.17152), section 三 技术架构 / 核心公式:
+ *   Eq. 1  U, V, Q, K = Split(phi1(f1(X)))            f_i(X) = W_i X + b_i, phi1 = ReLU
+ *   Eq. 2  A(X)V(X)   = phi2(Q K^T + rab^{p,t}) V(X)  pointwise attention, no softmax
+ *   Eq. 3  Y(X)       = f2(Norm(A(X)V(X)) (.) U(X))   plus the residual between layers
+ * and the M-FALCON paragraph of the same section (microbatched candidates
+ * reusing cached history keys/values).
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - phi2 is selectable (SiLU by default; ReLU; identity); attention weights
+ *     are divided by N = n_u, the user's own length (candidates: max(n_u, 1));
+ *   - no 1/sqrt(d) scale; rab is added before phi2; the causal mask zeroes
+ *     weights of later keys after phi2;
+ *   - rab_ij = rab_pos[h, min(i-j, P-1)] + rab_time[h, bt(t_i - t_j)],
+ *     bt(dt) = clamp(floor(ln(dt + 1) / 0.301), 0, Tb-1), dt < 0 -> 0;
+ *   - Norm = LayerNorm over the H*dv concatenated heads of a token, biased
+ *     variance, eps from the config, optional affine;
+ *   - Y = X + f2(...): the residual stream is fp32.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must point to memory of the current CUDA
+ *     device; the caller owns every buffer.  The library never allocates
+ *     device memory inside a call and keeps no per-call state.
+ *   - All device work is enqueued on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and is asynchronous to the host.
+ *   - Argument errors are detected on the host before any launch and return
+ *     HSTU_ERR_INVALID_ARGUMENT or HSTU_ERR_UNSUPPORTED without touching
+ *     device memory.  A failed launch returns HSTU_ERR_CUDA.  A kernel that
+ *     gives up on a bounded wait records HSTU_ERR_DEVICE_TIMEOUT in the
+ *     device status word (read with hstu_get_device_status); no kernel traps.
+ *   - Layouts are row-major.  Jagged batches: user u owns rows
+ *     offsets[u] .. offsets[u+1]-1 of every per-token tensor.
+ *   - Timestamps are int64 seconds, non-decreasing inside each user (the
+ *     result is unspecified otherwise).
+ *   - Supported shapes: dqk = dv = 64; d_model a multiple of 64;
+ *     1 <= num_heads with num_heads*64 a multiple of 64; max_len <= 16384;
+ *     num_pos_buckets <= 16384; num_time_buckets <= 256.  bf16 and fp32
+ *     storage (fp32 runs the fp32 SIMT path, bf16 the tensor-core path).
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARGUMENT = 1,   /* NULL pointer, negative size, inconsistent shapes */
+  HSTU_ERR_UNSUPPORTED = 2,        /* valid request outside the supported shapes */
+  HSTU_ERR_CUDA = 3,               /* a CUDA runtime call or launch failed */
+  HSTU_ERR_WORKSPACE_TOO_SMALL = 4,/* ws_bytes < hstu_*_workspace_bytes(...) */
+  HSTU_ERR_DEVICE_TIMEOUT = 5,     /* a kernel gave up on a bounded wait */
+  HSTU_ERR_DEVICE_CHECK = 6        /* a device-side input check failed */
+} hstu_status_t;
+
+typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1 } hstu_dtype_t;
+
+typedef enum { HSTU_ACT_IDENTITY = 0, HSTU_ACT_RELU = 1, HSTU_ACT_SILU = 2 } hstu_act_t;
+
+/* A jagged batch of per-user, time-ordered action sequences (the "unified
+ * time series" x_0..x_{n-1} of each user, section 二/三 of the review). */
+typedef struct {
+  int32_t batch;              /* B >= 0 */
+  int64_t total_tokens;       /* T == offsets[B], known to the caller (no device read) */
+  int32_t max_len;            /* >= max_u (offsets[u+1] - offsets[u]) */
+  const int64_t* offsets;     /* device [B+1], offsets[0] = 0, non-decreasing */
+  const int64_t* timestamps;  /* device [T], int64 seconds */
+} hstu_jagged_t;
+
+typedef struct {
+  int32_t d_model;            /* d */
+  int32_t num_heads;          /* H */
+  int32_t dqk;                /* per-head query/key width (64) */
+  int32_t dv;                 /* per-head value width (64) */
+  int32_t num_pos_buckets;    /* P */
+  int32_t num_time_buckets;   /* Tb */
+  int32_t phi1;               /* hstu_act_t, ReLU per Eq. 1 */
+  int32_t phi2;               /* hstu_act_t, SiLU by default */
+  float ln_eps;               /* LayerNorm epsilon (1e-5) */
+  int32_t dtype;              /* hstu_dtype_t of X, W1, W2 and all bf16 intermediates */
+} hstu_layer_cfg_t;
+
+/* Weights of one layer (all device pointers). */
+typedef struct {
+  const void* w1;        /* [2H(dqk+dv), d] in cfg dtype; rows ordered U, V, Q, K */
+  const float* b1;       /* [2H(dqk+dv)] fp32 */
+  const void* w2;        /* [d, H*dv] in cfg dtype */
+  const float* b2;       /* [d] fp32 */
+  const float* rab_pos;  /* [H, P] fp32 */
+  const float* rab_time; /* [H, Tb] fp32 */
+  const float* ln_gamma; /* [H*dv] fp32 or NULL (= 1) */
+  const float* ln_beta;  /* [H*dv] fp32 or NULL (= 0) */
+} hstu_layer_weights_t;
+
+/* Library version string (static storage). */
+const char* hstu_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* hstu_status_string(hstu_status_t status);
+
+/* Number of workspace bytes hstu_layer_fwd / hstu_forward / hstu_attn_fwd need
+ * for `total_tokens` rows.  Returns 0 for an invalid cfg. */
+size_t hstu_layer_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total_tokens);
+size_t hstu_forward_workspace_bytes(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                                    int64_t total_tokens);
+
+/* Workspace bytes for mfalcon_score with `num_cand` candidate rows in total. */
+size_t hstu_mfalcon_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t num_cand);
+
+/*
+ * Eq. 2 alone: AV = phi2(Q K^T + rab^{p,t}) V / n_u per user and head, causal.
+ *   q, k   device [T, H*dqk], v device [T, H*dv], av_out device [T, H*dv],
+ *          all in cfg->dtype; head h occupies columns h*64 .. h*64+63.
+ *   rab_pos device [H, P] fp32, rab_time device [H, Tb] fp32.
+ *   workspace may be NULL when ws_bytes == 0 (this entry needs none).
+ * Rows of av_out belonging to users are written; nothing else is touched.
+ */
+hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
+                            const void* q, const void* k, const void* v,
+                            const float* rab_pos, const float* rab_time, void* av_out,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * One HSTU layer (Eq. 1-3 and the residual) over a jagged batch.
+ *   x_in        device [T, d] in cfg dtype: the layer input fed to f1.
+ *   x_res       device [T, d] fp32 residual input, or NULL to use x_in.
+ *   y_out       device [T, d] fp32: X + f2(Norm(AV) (.) U).
+ *   y_out_lp    device [T, d] in cfg dtype (a rounded copy of y_out for the
+ *               next layer's f1), or NULL.
+ *   kv_cache_out device [T, 2, H, 64] in cfg dtype (per row: K of every head,
+ *               then V of every head), or NULL.  When given, this layer's K
+ *               and V rows are kept there for M-FALCON.
+ *   workspace   device, ws_bytes >= hstu_layer_workspace_bytes(cfg, T).
+ * x_in, y_out and y_out_lp must not overlap.
+ */
+hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                             const hstu_jagged_t* jag, const void* x_in, const float* x_res,
+                             float* y_out, void* y_out_lp, void* kv_cache_out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * A stack of num_layers HSTU layers (the residual stream stays fp32).
+ *   weights      host array [num_layers] of per-layer weight structs.
+ *   x_in         device [T, d] in cfg dtype.  y_out device [T, d] fp32.
+ *   kv_cache_out device [num_layers][T, 2, H, 64] in cfg dtype, or NULL.
+ *   workspace    ws_bytes >= hstu_forward_workspace_bytes(cfg, num_layers, T).
+ */
+hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                           const hstu_layer_weights_t* weights, const hstu_jagged_t* jag,
+                           const void* x_in, float* y_out, void* kv_cache_out,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * M-FALCON scoring (section 三, M-FALCON 推理算法): each candidate c of user u,
+ * with embedding e_c, runs through the num_layers layers as a row placed at
+ * position n_u with timestamp request_ts[u]; at every layer it attends to the
+ * user's cached history keys/values and to itself only.  score_c = <y_c, e_c>
+ * where y_c is its final fp32 residual-stream row.
+ *   history      jagged history (offsets/timestamps of the cached rows).
+ *   kv_cache     device [num_layers][T_hist, 2, H, 64] from hstu_forward.
+ *   cand_offsets device [B+1] candidate row ranges per user; num_cand = total
+ *                rows, max_cand >= the largest per-user count.
+ *   cand_emb     device [num_cand, d] in cfg dtype.  request_ts device [B].
+ *   microbatch   b_m >= 1.  Microbatches run concurrently as tiles of one
+ *                launch; scores do not depend on b_m.
+ *   scores       device [num_cand] fp32.
+ */
+hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
+                            const hstu_layer_weights_t* weights, const hstu_jagged_t* history,
+                            const void* kv_cache, const int64_t* cand_offsets, int64_t num_cand,
+                            int32_t max_cand, const void* cand_emb, const int64_t* request_ts,
+                            int32_t microbatch, float* scores, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/* Synchronises `stream`, returns the first error a kernel recorded in the
+ * device status word since the last call (HSTU_OK if none) and clears it. */
+hstu_status_t hstu_get_device_status(void* stream);
+
+/* Host only: writes thr[0..Tb-1], the smallest int64 dt reaching each time
+ * bucket under bt(dt) above (thr[0] = 0).  Tb in [1, 256]. */
+hstu_status_t hstu_time_bucket_thresholds(int32_t num_time_buckets, int64_t* thr_out);
+
+/* Test support: for every user writes the n_u x n_u row-major block of
+ * position buckets min(i-j, P-1) and time buckets bt(t_i - t_j) for j <= i
+ * (-1 for j > i), using the same device code as the attention kernels.
+ * pos_idx / time_idx: device int32 [sum_u n_u^2], blocks in user order;
+ * block_offsets: device int64 [B+1] prefix sums of n_u^2. */
+hstu_status_t hstu_debug_rab_index(const hstu_jagged_t* jag, int32_t num_pos_buckets,
+                                   int32_t num_time_buckets, const int64_t* block_offsets,
+                                   int32_t* pos_idx, int32_t* time_idx, void* stream);
+
+/* Test support: launches one CTA that waits on an mbarrier nothing completes,
+ * bounded by timeout_ns; it records HSTU_ERR_DEVICE_TIMEOUT and returns. */
+hstu_status_t hstu_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

@@ -31,7 +31,8 @@ documented constant here, never hidden):
   * Residual: Y = X + f2(...).  No pre-norm, no final norm.
   * M-FALCON: a candidate sits at position n_u with timestamp t_req, attends to
     the user's cached history rows (keys/values of every layer) and to itself
-    (position bucket 0, time bucket 0); its score is <y_c^(L), e_c>.
+    (position bucket 0, time bucket 0); its score is <y_c^(L), e_c>.  Its
+    normaliser is max(n_u, 1), so a user with an empty history still scores.
 
 Layouts (row-major): X [T, d]; W1 [2H(dqk+dv), d] rows ordered U, V, Q, K with
 head h occupying rows h*dh:(h+1)*dh of each block; W2 [d, H*dv]; jagged users
@@ -253,7 +254,7 @@ def mfalcon_scores(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_
                     own_v = v[:, h * dv:(h + 1) * dv]
                     s_self = np.einsum("cd,cd->c", qh, own_k) + rp[h, 0] + rt[h, 0]
                     o = phi(s_hist, cfg.phi2) @ vh + phi(s_self, cfg.phi2)[:, None] * own_v
-                    av[:, h * dv:(h + 1) * dv] = o / float(n_u)
+                    av[:, h * dv:(h + 1) * dv] = o / float(max(n_u, 1))
                 xc, _ = output(xc, av, u, w2, b2, cfg.ln_eps, _f64(layer.ln_gamma),
                                _f64(layer.ln_beta))
             scores[mb:mend] = np.einsum("cd,cd->c", xc, e)
@@ -282,8 +283,8 @@ def score_alone(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_emb
         for layer in layers:
             u, v, q, k = projection(cur, _f64(layer.w1), _f64(layer.b1), cfg.num_heads,
                                     cfg.dqk, cfg.dv, cfg.phi1)
-            av = user_attention(q, k, v, ts, _f64(layer.rab_pos), _f64(layer.rab_time), n_u,
-                                cfg.num_heads, cfg.dqk, cfg.dv, cfg.phi2)
+            av = user_attention(q, k, v, ts, _f64(layer.rab_pos), _f64(layer.rab_time),
+                                max(n_u, 1), cfg.num_heads, cfg.dqk, cfg.dv, cfg.phi2)
             cur, _ = output(cur, av, u, _f64(layer.w2), _f64(layer.b2), cfg.ln_eps,
                             _f64(layer.ln_gamma), _f64(layer.ln_beta))
         out.append(float(cur[n_u] @ e_all[c]))
@@ -293,15 +294,18 @@ def score_alone(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_emb
 def time_bucket_thresholds(num_time_buckets: int) -> np.ndarray:
     """Smallest integer dt reaching each bucket k (k = 0..Tb-1), by the formula above.
 
-    Used only by tests to probe bucket edges (dt = thr[k] - 1 and thr[k]).
+    Buckets that no dt below 2^62 reaches get INT64_MAX.  Used only by tests to
+    probe bucket edges (dt = thr[k] - 1 and thr[k]).
     """
+    cap = 1 << 62
     thr = np.zeros(num_time_buckets, dtype=np.int64)
     for k in range(1, num_time_buckets):
+        if int(time_bucket(cap, 1 << 30)) < k:
+            thr[k] = np.iinfo(np.int64).max
+            continue
         lo, hi = 0, 1
         while int(time_bucket(hi, 1 << 30)) < k:
-            hi *= 2
-            if hi > (1 << 62):
-                break
+            hi = min(hi * 2, cap)
         while lo < hi:
             mid = (lo + hi) // 2
             if int(time_bucket(mid, 1 << 30)) >= k:

@@ -238,7 +238,7 @@ def test_layer_norm_textbook():
 
 # --------------------------------------------------------------------------- M-FALCON
 
-def _mf_case(seed=7, lengths=(6, 1, 11), m=5):
+def _mf_case(seed=7, lengths=(6, 1, 0, 11), m=5):
     cfg = _tiny_cfg(num_layers=2, num_cand=m, microbatch=2)
     return make_case(cfg, seed=seed, lengths=list(lengths))
 
