@@ -48,7 +48,8 @@ struct AttnParams {
   const __nv_bfloat16* k_self;
   const __nv_bfloat16* v_self;
   int64_t ld_self;             // row stride (elements) of q_self/k_self/v_self
-  __nv_bfloat16* av;           // [T_q, ld_av]
+  __nv_bfloat16* av;           // [T_q, ld_av] bf16 output, or
+  float* av_f32;               // [T_q, ld_av] fp32 output (the layer path feeds LayerNorm)
   int64_t ld_av;
   float* ln_part;              // [T_q, H, 2] (sum, centred sum of squares) or nullptr
   int32_t B, H, P, Tb;
@@ -510,15 +511,22 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const float dlt = o[c] - mean;
           m2 = fmaf(dlt, dlt, m2);
         }
-        __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD;
+        if (p.av_f32 != nullptr) {
+          float4* dst = reinterpret_cast<float4*>(p.av_f32 + row * p.ld_av + h * ATT_HD);
 #pragma unroll
-        for (int c = 0; c < ATT_HD; c += 8) {
-          uint4 pkt;
-          pkt.x = pack_bf16x2(o[c + 0], o[c + 1]);
-          pkt.y = pack_bf16x2(o[c + 2], o[c + 3]);
-          pkt.z = pack_bf16x2(o[c + 4], o[c + 5]);
-          pkt.w = pack_bf16x2(o[c + 6], o[c + 7]);
-          *reinterpret_cast<uint4*>(dst + c) = pkt;
+          for (int c = 0; c < ATT_HD; c += 4)
+            dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        } else {
+          __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD;
+#pragma unroll
+          for (int c = 0; c < ATT_HD; c += 8) {
+            uint4 pkt;
+            pkt.x = pack_bf16x2(o[c + 0], o[c + 1]);
+            pkt.y = pack_bf16x2(o[c + 2], o[c + 3]);
+            pkt.z = pack_bf16x2(o[c + 4], o[c + 5]);
+            pkt.w = pack_bf16x2(o[c + 6], o[c + 7]);
+            *reinterpret_cast<uint4*>(dst + c) = pkt;
+          }
         }
         if (p.ln_part != nullptr) {
           float2* lp = reinterpret_cast<float2*>(p.ln_part + (row * p.H + h) * 2);

@@ -56,8 +56,9 @@ __device__ __forceinline__ float apply_act(float x) {
 }
 
 struct F1Params {
-  __nv_bfloat16* dst[4];  // destination of column block b (U, V, Q, K)
+  void* dst[4];           // destination of column block b (U, V, Q, K)
   int64_t ld_dst[4];      // row stride of each destination (elements)
+  uint32_t f32_mask;      // bit b set: block b is stored as fp32, else bf16
   const float* bias;      // [N]
   int64_t M;
   int32_t N, K;
@@ -67,8 +68,8 @@ struct F1Params {
 };
 
 struct F2Params {
-  const __nv_bfloat16* av;  // [M, ld_av]
-  const __nv_bfloat16* u;   // [M, ld_u]
+  const float* av;          // [M, ld_av] fp32 attention output
+  const float* u;           // [M, ld_u] fp32 gate
   int64_t ld_av, ld_u;
   const float* ln_part;     // [M, H, 2] per-head (sum, centred sum of squares) of AV rows
   const float* gamma;       // [K] or nullptr
@@ -225,22 +226,32 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int blk = col / p.blk_w;
         const int cb = col - blk * p.blk_w;
         const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
-        uint32_t out[16];
+        float z[32];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 bb = __ldg(b4 + q);
-          const float z0 = apply_act<ACT>(__uint_as_float(v[4 * q + 0]) + bb.x);
-          const float z1 = apply_act<ACT>(__uint_as_float(v[4 * q + 1]) + bb.y);
-          const float z2 = apply_act<ACT>(__uint_as_float(v[4 * q + 2]) + bb.z);
-          const float z3 = apply_act<ACT>(__uint_as_float(v[4 * q + 3]) + bb.w);
-          out[2 * q] = pack_bf16x2(z0, z1);
-          out[2 * q + 1] = pack_bf16x2(z2, z3);
+          z[4 * q + 0] = apply_act<ACT>(__uint_as_float(v[4 * q + 0]) + bb.x);
+          z[4 * q + 1] = apply_act<ACT>(__uint_as_float(v[4 * q + 1]) + bb.y);
+          z[4 * q + 2] = apply_act<ACT>(__uint_as_float(v[4 * q + 2]) + bb.z);
+          z[4 * q + 3] = apply_act<ACT>(__uint_as_float(v[4 * q + 3]) + bb.w);
         }
         if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dst[blk] + row * p.ld_dst[blk] + cb);
+          if ((p.f32_mask >> blk) & 1u) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dst[blk]) +
+                                                    row * p.ld_dst[blk] + cb);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dst[blk]) +
+                                                  row * p.ld_dst[blk] + cb);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(z[8 * q], z[8 * q + 1]),
+                                  pack_bf16x2(z[8 * q + 2], z[8 * q + 3]),
+                                  pack_bf16x2(z[8 * q + 4], z[8 * q + 5]),
+                                  pack_bf16x2(z[8 * q + 6], z[8 * q + 7]));
+          }
         }
       }
       tc_fence_before();
@@ -388,18 +399,18 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           const int64_t row = m0 + r;
           uint4 outv = make_uint4(0u, 0u, 0u, 0u);
           if (row < p.M) {
-            const uint4 av4 = *reinterpret_cast<const uint4*>(p.av + row * p.ld_av + col);
-            const uint4 u4 = *reinterpret_cast<const uint4*>(p.u + row * p.ld_u + col);
+            const float4* ap = reinterpret_cast<const float4*>(p.av + row * p.ld_av + col);
+            const float4* up = reinterpret_cast<const float4*>(p.u + row * p.ld_u + col);
+            const float4 a0 = ap[0], a1 = ap[1], u0 = up[0], u1 = up[1];
+            const float af[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float uf[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             const float2 st = sStats[r];
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av4);
-            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&u4);
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 af = __bfloat1622float2(a2[e]);
-              const float2 uf = __bfloat1622float2(u2[e]);
-              const float g0 = fmaf((af.x - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf.x;
-              const float g1 = fmaf((af.y - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf.y;
+              const float g0 = fmaf((af[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf[2 * e];
+              const float g1 =
+                  fmaf((af[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
               w[e] = pack_bf16x2(g0, g1);
             }
             outv = make_uint4(w[0], w[1], w[2], w[3]);

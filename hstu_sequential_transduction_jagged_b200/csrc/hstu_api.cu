@@ -198,35 +198,44 @@ size_t elt(const hstu_layer_cfg_t* c) { return c->dtype == HSTU_BF16 ? 2 : 4; }
 
 int n1_of(const hstu_layer_cfg_t* c) { return 2 * c->num_heads * (c->dqk + c->dv); }
 
-// workspace for one layer: Z [T, n1], AV [T, H*dv], then LN partials (bf16
-// path) or the gated rows G [T, H*dv] (fp32 path)
+// Workspace of one layer.
+//   bf16 path: VQK [T, 3*H*dv] bf16 (V, Q, K blocks; K/V may go to a cache
+//              instead), U [T, H*dv] fp32, AV [T, H*dv] fp32, LN partials
+//              [T, H, 2] fp32.  AV and U stay fp32 because LayerNorm removes the
+//              large common mean of AV and would magnify bf16 rounding there.
+//   fp32 path: Z [T, n1] fp32, AV [T, H*dv] fp32, G [T, H*dv] fp32.
 struct LayerWs {
-  void* z;
+  void* z;      // bf16: VQK; fp32: Z
+  float* u;     // bf16 path: U fp32
   void* av;
-  void* extra;
+  void* extra;  // bf16: LN partials; fp32: G
 };
 
 size_t layer_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
-  const size_t e = elt(c);
+  const size_t t = static_cast<size_t>(T);
   const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
-  size_t b = align_up(static_cast<size_t>(T) * n1_of(c) * e, 256);
-  b += align_up(static_cast<size_t>(T) * hv * e, 256);
   if (c->dtype == HSTU_BF16)
-    b += align_up(static_cast<size_t>(T) * c->num_heads * 2 * sizeof(float), 256);
-  else
-    b += align_up(static_cast<size_t>(T) * hv * sizeof(float), 256);
-  return b;
+    return align_up(t * 3 * hv * 2, 256) + 2 * align_up(t * hv * 4, 256) +
+           align_up(t * c->num_heads * 2 * sizeof(float), 256);
+  return align_up(t * n1_of(c) * 4, 256) + 2 * align_up(t * hv * 4, 256);
 }
 
 LayerWs carve_layer(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
-  const size_t e = elt(c);
+  const size_t t = static_cast<size_t>(T);
   const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
   uint8_t* p = static_cast<uint8_t*>(ws);
   LayerWs w;
   w.z = p;
-  p += align_up(static_cast<size_t>(T) * n1_of(c) * e, 256);
+  if (c->dtype == HSTU_BF16) {
+    p += align_up(t * 3 * hv * 2, 256);
+    w.u = reinterpret_cast<float*>(p);
+    p += align_up(t * hv * 4, 256);
+  } else {
+    p += align_up(t * n1_of(c) * 4, 256);
+    w.u = nullptr;
+  }
   w.av = p;
-  p += align_up(static_cast<size_t>(T) * hv * e, 256);
+  p += align_up(t * hv * 4, 256);
   w.extra = p;
   return w;
 }
@@ -256,7 +265,8 @@ struct AttnJob {
   const void* q_self; const void* k_self; const void* v_self; int64_t ld_self;
   const float* rab_pos;
   const float* rab_time;
-  void* av; int64_t ld_av;
+  void* av; int64_t ld_av;      // bf16 [.., ld_av] output (attention alone)
+  float* av_f32;                // fp32 output (layer path)
   float* ln_part;
   uint64_t timeout_ns;
 };
@@ -293,6 +303,7 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.v_self = static_cast<const __nv_bfloat16*>(j.v_self);
   p.ld_self = j.ld_self;
   p.av = static_cast<__nv_bfloat16*>(j.av);
+  p.av_f32 = j.av_f32;
   p.ld_av = j.ld_av;
   p.ln_part = j.ln_part;
   p.B = j.batch;
@@ -324,7 +335,7 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
 
 hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t ldx, int64_t M,
                              const void* w1, const float* b1, void* const dst[4],
-                             const int64_t ld_dst[4], cudaStream_t st) {
+                             const int64_t ld_dst[4], uint32_t f32_mask, cudaStream_t st) {
   if (M == 0) return HSTU_OK;
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
@@ -336,9 +347,10 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   F1Params p;
   std::memset(&p, 0, sizeof(p));
   for (int b = 0; b < 4; ++b) {
-    p.dst[b] = static_cast<__nv_bfloat16*>(dst[b]);
+    p.dst[b] = dst[b];
     p.ld_dst[b] = ld_dst[b];
   }
+  p.f32_mask = f32_mask;
   p.bias = b1;
   p.M = M;
   p.N = N;
@@ -365,7 +377,7 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
 }
 
 hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
-                             const void* av, int64_t ld_av, const void* u, int64_t ld_u,
+                             const float* av, int64_t ld_av, const float* u, int64_t ld_u,
                              const float* ln_part, const float* x_res, const void* x_lp,
                              int64_t ld_x, float* y, void* y_lp, int64_t ld_y, int64_t M,
                              cudaStream_t st) {
@@ -378,8 +390,8 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   if ((s = make_map_bf16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
   F2Params p;
   std::memset(&p, 0, sizeof(p));
-  p.av = static_cast<const __nv_bfloat16*>(av);
-  p.u = static_cast<const __nv_bfloat16*>(u);
+  p.av = av;
+  p.u = u;
   p.ld_av = ld_av;
   p.ld_u = ld_u;
   p.ln_part = ln_part;
@@ -520,36 +532,39 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
                          const AttnJob& base, const void* x_in, const float* x_res, int64_t T,
                          float* y_out, void* y_lp, void* kv_cache, const LayerWs& ws, bool cand,
                          cudaStream_t st) {
-  const int H = c->num_heads, hv = H * ATT_HD, n1 = n1_of(c), d = c->d_model;
-  __nv_bfloat16* z = static_cast<__nv_bfloat16*>(ws.z);
-  void* dst[4] = {z, z + hv, z + 2 * hv, z + 3 * hv};
-  int64_t ldd[4] = {n1, n1, n1, n1};
+  const int hv = c->num_heads * ATT_HD, d = c->d_model;
+  __nv_bfloat16* vqk = static_cast<__nv_bfloat16*>(ws.z);
+  // f1 column blocks U, V, Q, K -> U (fp32), V, Q, K (bf16; K/V into the cache if given)
+  void* dst[4] = {ws.u, vqk, vqk + hv, vqk + 2 * hv};
+  int64_t ldd[4] = {hv, 3 * hv, 3 * hv, 3 * hv};
   if (kv_cache != nullptr) {
     __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(kv_cache);
     dst[1] = kv + hv;  // V
     dst[3] = kv;       // K
     ldd[1] = ldd[3] = 2 * hv;
   }
-  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, st);
+  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, 1u, st);
   if (s != HSTU_OK) return s;
   AttnJob j = base;
+  j.q = dst[2];
+  j.ldq = ldd[2];
   if (!cand) {
-    j.q = dst[2]; j.ldq = ldd[2];
     j.k = dst[3]; j.ldk = ldd[3];
     j.v = dst[1]; j.ldv = ldd[1];
   } else {
-    j.q = dst[2]; j.ldq = n1;
-    j.q_self = dst[2]; j.k_self = dst[3]; j.v_self = dst[1]; j.ld_self = n1;
+    j.q_self = dst[2]; j.k_self = dst[3]; j.v_self = dst[1]; j.ld_self = 3 * hv;
   }
   j.rab_pos = w->rab_pos;
   j.rab_time = w->rab_time;
-  j.av = ws.av;
+  j.av = nullptr;
+  j.av_f32 = static_cast<float*>(ws.av);
   j.ld_av = hv;
   j.ln_part = static_cast<float*>(ws.extra);
   s = cand ? launch_attn_bf16<true>(j, st) : launch_attn_bf16<false>(j, st);
   if (s != HSTU_OK) return s;
-  return launch_f2_bf16(c, w, ws.av, hv, z, n1, static_cast<const float*>(ws.extra), x_res, x_in,
-                        d, y_out, y_lp, d, T, st);
+  return launch_f2_bf16(c, w, static_cast<const float*>(ws.av), hv, ws.u, hv,
+                        static_cast<const float*>(ws.extra), x_res, x_in, d, y_out, y_lp, d, T,
+                        st);
 }
 
 hstu_status_t check_weights(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w) {

@@ -20,9 +20,18 @@ def errors(got, want):
     return max_abs, rel
 
 
-def assert_close(got, want, what="", max_abs=MAX_ABS, rel_l2=REL_L2):
+def assert_close(got, want, what="", max_abs=MAX_ABS, rel_l2=REL_L2, scaled=False):
+    """max |got - want| <= max_abs and ||got - want|| / ||want|| <= rel_l2.
+
+    scaled=True is for bf16-stored intermediates (AV, cached K/V): one bf16 ulp
+    is 2^-7 relative, so the max-abs bound is applied to |got - want| / max(1, |want|).
+    """
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     ma, rl = errors(got, want)
-    assert np.all(np.isfinite(np.asarray(got))), f"{what}: non-finite values"
+    if scaled:
+        ma = float(np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want)))) if got.size else 0.0
     assert ma <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
     return ma, rl
 
