@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/hstu.h"
 #include "attn.cuh"
@@ -74,6 +75,63 @@ const int64_t* thresholds_for(int Tb) {
   }
   return table[Tb];
 }
+
+// ------------------------------------------------------------------ profiler
+
+enum KernelKind : int {
+  K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_COUNT
+};
+const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
+                                           "mfalcon_attention", "score",    "fp32_linear",
+                                           "fp32_attention",    "fp32_ln_gate"};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec { int kind; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+
+// Brackets one kernel launch with events while the profiler is on.
+class ProfScope {
+ public:
+  ProfScope(int kind, cudaStream_t st) : kind_(kind), st_(st) {
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (!p.on) return;
+    a_ = p.get();
+    b_ = p.get();
+    if (a_ != nullptr) cudaEventRecord(a_, st_);
+  }
+  ~ProfScope() {
+    if (a_ == nullptr || b_ == nullptr) return;
+    cudaEventRecord(b_, st_);
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> lock(p.mu);
+    p.recs.push_back({kind_, a_, b_});
+  }
+
+ private:
+  int kind_;
+  cudaStream_t st_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
 
 // ------------------------------------------------------------------ device info
 
@@ -318,6 +376,7 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
   dim3 grid(c->num_heads, j.batch, p.num_qpairs);
   const size_t smem = AttnSmem::bytes(p.pos_cap);
+  ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
   switch (c->phi2) {
     case HSTU_ACT_SILU:
       hstu_attn_kernel<CAND, HSTU_ACT_SILU><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
@@ -361,6 +420,7 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   p.timeout_ns = kDefaultTimeoutNs;
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
+  ProfScope prof(K_F1, st);
   switch (c->phi1) {
     case HSTU_ACT_RELU:
       hstu_f1_kernel<HSTU_ACT_RELU><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
@@ -414,6 +474,7 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   p.timeout_ns = kDefaultTimeoutNs;
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
+  ProfScope prof(K_F2, st);
   hstu_f2_kernel<<<grid, 320, GemmSmem::kBytes, st>>>(mw, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
@@ -444,6 +505,7 @@ hstu_status_t launch_f32_linear(const float* a, int64_t lda, int64_t M, int N, i
   p.K = K;
   p.act = act;
   dim3 grid((N + 63) / 64, static_cast<unsigned>((M + 63) / 64));
+  ProfScope prof(K_F32_LINEAR, st);
   hstu_f32_linear_kernel<<<grid, 256, 0, st>>>(p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
@@ -480,6 +542,7 @@ hstu_status_t launch_f32_attn(const AttnJob& j, cudaStream_t st) {
   p.cand = j.q_offsets != nullptr ? 1 : 0;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
   dim3 grid((j.max_q_len + 31) / 32, c->num_heads, j.batch);
+  ProfScope prof(K_F32_ATTN, st);
   hstu_f32_attn_kernel<<<grid, 128, 0, st>>>(p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
@@ -518,6 +581,7 @@ hstu_status_t layer_fp32(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
   if ((s = launch_f32_attn(j, st)) != HSTU_OK) return s;
   float* g = static_cast<float*>(ws.extra);
   const unsigned blocks = static_cast<unsigned>((T * 32 + 255) / 256);
+  ProfScope prof(K_F32_LN, st);
   hstu_f32_ln_gate_kernel<<<blocks, 256, 0, st>>>(static_cast<const float*>(ws.av), hv, z, n1,
                                                   w->ln_gamma, w->ln_beta, c->ln_eps, T, hv, g, hv);
   HSTU_CHECK_CUDA(cudaGetLastError());
@@ -806,6 +870,7 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
   }
   const float* yfin = yf[(num_layers - 1) & 1];
   const unsigned blocks = static_cast<unsigned>((M * 32 + 255) / 256);
+  ProfScope prof(K_SCORE, st);
   if (cfg->dtype == HSTU_FP32)
     hstu_score_kernel<float><<<blocks, 256, 0, st>>>(yfin, d, static_cast<const float*>(cand_emb),
                                                      d, M, d, scores);
@@ -814,6 +879,47 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
         yfin, d, static_cast<const __nv_bfloat16*>(cand_emb), d, M, d, scores);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
+}
+
+hstu_status_t hstu_profiler_start(void) {
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  for (auto& r : p.recs) {
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.recs.clear();
+  p.on = true;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_profiler_stop(hstu_kernel_time_t* out, int32_t capacity, int32_t* count) {
+  if (count == nullptr || capacity < 0 || (capacity > 0 && out == nullptr))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  p.on = false;
+  double total[K_COUNT] = {};
+  int32_t n[K_COUNT] = {};
+  hstu_status_t st = HSTU_OK;
+  for (auto& r : p.recs) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      st = HSTU_ERR_CUDA;
+    total[r.kind] += ms;
+    n[r.kind] += 1;
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.recs.clear();
+  int32_t k = 0;
+  for (int i = 0; i < K_COUNT; ++i) {
+    if (n[i] == 0) continue;
+    if (k < capacity) out[k] = hstu_kernel_time_t{kKernelNames[i], n[i], total[i]};
+    ++k;
+  }
+  *count = k;
+  return st;
 }
 
 hstu_status_t hstu_get_device_status(void* stream) {

@@ -45,6 +45,11 @@ class LayerCfgT(ctypes.Structure):
                 ("dtype", ctypes.c_int32)]
 
 
+class KernelTimeT(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int32),
+                ("total_ms", ctypes.c_double)]
+
+
 class LayerWeightsT(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w1", "b1", "w2", "b2", "rab_pos", "rab_time", "ln_gamma", "ln_beta")]
@@ -67,6 +72,8 @@ EXPORTS = {
                                      ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hstu_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "hstu_profiler_start": (ctypes.c_int, []),
+    "hstu_profiler_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]),
     "hstu_time_bucket_thresholds": (ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p]),
     "hstu_debug_rab_index": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -288,3 +295,16 @@ def debug_rab_index(jag: Jagged, num_pos_buckets: int, num_time_buckets: int, st
 
 def debug_wait_timeout(timeout_ns: int, stream=None):
     _check(lib().hstu_debug_wait_timeout(timeout_ns, _stream(stream)), "hstu_debug_wait_timeout")
+
+
+def profiler_start():
+    """Start bracketing every library kernel launch with CUDA events."""
+    _check(lib().hstu_profiler_start(), "hstu_profiler_start")
+
+
+def profiler_stop() -> dict:
+    """Stop the profiler; returns {kernel name: (launches, total milliseconds)}."""
+    arr = (KernelTimeT * 16)()
+    n = ctypes.c_int32(0)
+    _check(lib().hstu_profiler_stop(arr, 16, ctypes.byref(n)), "hstu_profiler_stop")
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}

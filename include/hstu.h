@@ -182,6 +182,22 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                             int32_t microbatch, float* scores, void* workspace, size_t ws_bytes,
                             void* stream);
 
+/* Per-kernel timing.  Between hstu_profiler_start() and hstu_profiler_stop()
+ * every kernel the library launches is bracketed by CUDA events recorded on
+ * its own stream (device time, no host synchronisation while running).
+ * stop() waits for the recorded events, writes up to `capacity` entries (one
+ * per kernel kind that ran: name, launch count, summed milliseconds) and sets
+ * *count.  The profiler is process-wide; calls from several threads are
+ * serialised. */
+typedef struct {
+  const char* name;      /* static string, e.g. "attention", "f1_gemm", "f2_gemm" */
+  int32_t launches;
+  double total_ms;
+} hstu_kernel_time_t;
+
+hstu_status_t hstu_profiler_start(void);
+hstu_status_t hstu_profiler_stop(hstu_kernel_time_t* out, int32_t capacity, int32_t* count);
+
 /* Synchronises `stream`, returns the first error a kernel recorded in the
  * device status word since the last call (HSTU_OK if none) and clears it. */
 hstu_status_t hstu_get_device_status(void* stream);
