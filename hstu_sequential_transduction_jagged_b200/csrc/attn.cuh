@@ -21,6 +21,17 @@
 // group reads S row by row, adds the gathered bias, applies phi2 and the
 // mask, writes P (bf16) back to tensor memory, then O += P V (tcgen05 with A
 // from tensor memory, V as an MN-major B operand).  1/N is applied once to O.
+//
+// Elementwise work per (query, key, head), SiLU case: x = s + rab, and
+// x*sigmoid(x) = h + h*tanh(h) with h = x/2.  The 1/2 is folded into the bias
+// tables when they are staged, so h = fma(s, 1/2, rab/2) and only one
+// transcendental (tanh) is needed.  The position bias is staged reversed in
+// two copies offset by one entry, so every thread reads the biases of two
+// adjacent keys with one aligned 8-byte shared load; pairs of keys then go
+// through packed fp32x2 adds and FMAs.  The time bucket only decreases along
+// a row (keys are time-ordered), so a 32-key chunk whose last key still lies
+// in the current bucket needs no per-key work; otherwise a short integer
+// walk over the bucket edges runs per key.
 #pragma once
 
 #include "ptx.cuh"
@@ -32,7 +43,6 @@ constexpr int ATT_KEYS = 128;
 constexpr int ATT_HD = 64;
 constexpr int ATT_STAGES = 3;
 constexpr int ATT_THREADS = 320;
-constexpr int ATT_POS_PAD = 128;
 constexpr int MAX_TIME_BUCKETS = 256;
 
 constexpr uint32_t ATT_TILE_BYTES = ATT_ROWS * ATT_HD * 2;  // 16 KB
@@ -54,7 +64,7 @@ struct AttnParams {
   float* ln_part;              // [T_q, H, 2] (sum, centred sum of squares) or nullptr
   int32_t B, H, P, Tb;
   int32_t num_qpairs;
-  int32_t pos_cap;             // entries of the position table held in shared memory
+  int32_t pos_len;             // floats per staged copy of the position table
   int32_t phi2;
   uint64_t timeout_ns;
   int64_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0)
@@ -76,33 +86,60 @@ __device__ __forceinline__ int time_bucket_search(int64_t dt, const int64_t* thr
 // Bucket of t_i - t_j for one query row as j walks forward through keys with
 // non-decreasing timestamps: the bucket can only go down, so each step is a
 // compare against the current lower edge and an occasional decrement.
+// T is int64_t (absolute seconds) or int32_t (seconds since the user's first
+// event, used when the user's whole span fits).
+template <typename T>
 struct BucketWalk {
   int b;
-  int64_t ti;
-  int64_t bound;  // keys with t_j <= bound are still in bucket >= b
+  T ti;
+  T bound;  // keys with t_j <= bound are still in bucket >= b
 
-  __device__ __forceinline__ void init(int64_t t_row, int64_t t_first_key, const int64_t* thr,
-                                       int Tb) {
+  __device__ __forceinline__ void init(T t_row, T t_first_key, const int64_t* thr, int Tb) {
     ti = t_row;
-    b = time_bucket_search(t_row - t_first_key, thr, Tb);
-    bound = (b == 0) ? INT64_MAX : ti - thr[b];
+    b = time_bucket_search(static_cast<int64_t>(t_row) - static_cast<int64_t>(t_first_key), thr, Tb);
+    set_bound(thr);
+  }
+  __device__ __forceinline__ void set_bound(const int64_t* thr) {
+    if constexpr (sizeof(T) == 8) {
+      bound = (b == 0) ? INT64_MAX : ti - thr[b];
+    } else {
+      bound = (b == 0) ? INT32_MAX : static_cast<T>(static_cast<int64_t>(ti) - thr[b]);
+    }
   }
   // Advance to a key with timestamp tj; returns true when the bucket changed.
-  __device__ __forceinline__ bool step(int64_t tj, const int64_t* thr) {
+  __device__ __forceinline__ bool step(T tj, const int64_t* thr) {
     bool changed = false;
     while (tj > bound) {
       --b;
-      bound = (b == 0) ? INT64_MAX : ti - thr[b];
+      set_bound(thr);
       changed = true;
     }
     return changed;
   }
 };
 
+// phi2 applied to a pair given h = (scaled) pre-activation; returns bf16x2.
+// SiLU: tables carry x/2, so p = h + h*tanh(h); ReLU / identity: h = x.
+template <int PHI>
+__device__ __forceinline__ uint32_t phi_pair(uint64_t h2) {
+  if constexpr (PHI == HSTU_ACT_SILU) {
+    float h0, h1;
+    f2_unpack(h2, h0, h1);
+    const uint64_t t2 = f2_pack(tanh_approx(h0), tanh_approx(h1));
+    return f2_to_bf16x2(f2_fma(h2, t2, h2));
+  } else if constexpr (PHI == HSTU_ACT_RELU) {
+    float h0, h1;
+    f2_unpack(h2, h0, h1);
+    return pack_bf16x2(fmaxf(h0, 0.0f), fmaxf(h1, 0.0f));
+  } else {
+    return f2_to_bf16x2(h2);
+  }
+}
+
 template <int PHI>
 __device__ __forceinline__ float apply_phi(float x) {
   if constexpr (PHI == HSTU_ACT_SILU) {
-    const float h = 0.5f * x;  // x*sigmoid(x) = h + h*tanh(h), h = x/2
+    const float h = 0.5f * x;
     return fmaf(h, tanh_approx(h), h);
   } else if constexpr (PHI == HSTU_ACT_RELU) {
     return fmaxf(x, 0.0f);
@@ -111,20 +148,31 @@ __device__ __forceinline__ float apply_phi(float x) {
   }
 }
 
+template <int PHI>
+__host__ __device__ constexpr float phi_scale() { return PHI == HSTU_ACT_SILU ? 0.5f : 1.0f; }
+
+// Zero the keys of a bf16 pair at columns c, c+1 that are above `last`.
+__device__ __forceinline__ uint32_t mask_pair(uint32_t w, int c, int last) {
+  const uint32_t lo = (c <= last) ? 0x0000FFFFu : 0u;
+  const uint32_t hi = (c + 1 <= last) ? 0xFFFF0000u : 0u;
+  return w & (lo | hi);
+}
+
 // ---------------------------------------------------------------- shared memory
 
 struct AttnSmem {
   static constexpr uint32_t kQ = 0;                                   // 2 x 16 KB
   static constexpr uint32_t kK = kQ + 2 * ATT_TILE_BYTES;             // stages x 16 KB
   static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 16 KB
-  static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 128 x 8 B
-  static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * ATT_KEYS * 8;
+  static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 1 KB
+  static constexpr uint32_t kKeyStride = ATT_KEYS * 8;                // bytes per stage
+  static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * kKeyStride;
   static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
   static constexpr uint32_t kBars = kThr + MAX_TIME_BUCKETS * 8;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kPos = kMisc + 64;
-  static constexpr uint32_t bytes(int pos_cap) {
-    return kPos + static_cast<uint32_t>(ATT_POS_PAD + pos_cap) * 4 + 1024;  // + align slack
+  static constexpr uint32_t bytes(int pos_len, bool pairs) {
+    return kPos + static_cast<uint32_t>(pos_len) * 4u * (pairs ? 2u : 1u) + 1024u;  // + align slack
   }
 };
 
@@ -142,7 +190,7 @@ enum : int {
 
 // ---------------------------------------------------------------- kernel
 
-template <bool CAND, int PHI>
+template <bool CAND, int PHI, bool PAIRS>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -180,21 +228,32 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   const int nk_total = nA > nB ? nA : nB;
 
+  // causal rows read position offsets i - j in [-127, q0 + 255]; candidates
+  // read n_kv - j in [1, n_kv].  The staged table holds scale * rab_pos at
+  // index x = D - (i - j).
+  const int D = CAND ? n_kv : q0 + 2 * ATT_ROWS;
+  constexpr float kScale = phi_scale<PHI>();
+
   uint8_t* sQ = smem + AttnSmem::kQ;
   uint8_t* sK = smem + AttnSmem::kK;
   uint8_t* sV = smem + AttnSmem::kV;
-  int64_t* sKeyTs = reinterpret_cast<int64_t*>(smem + AttnSmem::kKeyInfo);
-  float* sKeyRab = reinterpret_cast<float*>(smem + AttnSmem::kKeyInfo);
+  uint8_t* sKey = smem + AttnSmem::kKeyInfo;
   float* sTime = reinterpret_cast<float*>(smem + AttnSmem::kTimeTab);
   int64_t* sThr = reinterpret_cast<int64_t*>(smem + AttnSmem::kThr);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 4);
-  float* sPos = reinterpret_cast<float*>(smem + AttnSmem::kPos);  // sPos[ATT_POS_PAD + k]
+  float* sRv = reinterpret_cast<float*>(smem + AttnSmem::kPos);
 
   const int warp = warp_id();
   const int lane = lane_id();
   const int tid = threadIdx.x;
+
+  // timestamps relative to the user's first event fit in int32 unless the
+  // user spans more than ~68 years; then the int64 walk is used
+  const int64_t t_first = n_kv > 0 ? p.timestamps[kv_start] : 0;
+  const bool ts32 = CAND || (n_kv == 0) ||
+                    (p.timestamps[kv_start + n_kv - 1] - t_first < static_cast<int64_t>(INT32_MAX) - 1);
 
   // ---------------- setup
   if (tid == 0) {
@@ -216,18 +275,20 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tmem_alloc(sTmemBase, 512);
     tmem_relinquish();
   }
-  // position table: sPos[pad + k] = rab_pos[h, min(k, P-1)]; the pad covers the
-  // negative offsets read (and discarded) for masked entries of diagonal tiles
-  // causal rows of this CTA read i - j <= q0 + 255; candidates read n_kv - j <= n_kv
-  const int pos_needed = CAND ? (n_kv + 1) : (q0 + 2 * ATT_ROWS);
-  const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
-  for (int k = tid; k < ATT_POS_PAD + pos_needed; k += ATT_THREADS) {
-    float val = 0.0f;
-    if (k >= ATT_POS_PAD) val = rp[min(k - ATT_POS_PAD, p.P - 1)];
-    sPos[k] = val;
+  {
+    const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
+    const int xend = min(p.pos_len, D + ATT_KEYS + 2);
+    for (int x = tid; x < xend; x += ATT_THREADS) {
+      const int d0 = D - x;  // copy 0 holds offset D - x
+      sRv[x] = (d0 >= 0) ? kScale * rp[min(d0, p.P - 1)] : 0.0f;
+      if constexpr (PAIRS) {
+        const int d1 = D + 1 - x;  // copy 1 holds offset D + 1 - x
+        sRv[p.pos_len + x] = (d1 >= 0) ? kScale * rp[min(d1, p.P - 1)] : 0.0f;
+      }
+    }
   }
   for (int k = tid; k < p.Tb; k += ATT_THREADS) {
-    sTime[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
+    sTime[k] = kScale * p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     sThr[k] = p.thr[k];
   }
   tc_fence_before();
@@ -235,10 +296,6 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *sTmemBase;
   const WaitCtl ctl{sAbort, p.timeout_ns};
-
-  const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-  const uint32_t tP[2] = {tmem + 256u, tmem + 320u};
-  const uint32_t tO[2] = {tmem + 384u, tmem + 448u};
 
   if (warp == 8) {
     // ---------------- producer
@@ -268,18 +325,23 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tma_load_2d(sV + s * ATT_TILE_BYTES, &tm_v, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
       }
       ++issued;
+      uint8_t* key = sKey + s * AttnSmem::kKeyStride;
       for (int e = 0; e < ATT_KEYS / 32; ++e) {
         const int c = lane + 32 * e;
         const int j = kt * ATT_KEYS + c;
         if constexpr (CAND) {
+          // the whole per-key bias: candidates share position n_kv and time t_req
           float r = 0.0f;
           if (j < n_kv) {
             const int64_t dt = t_req - p.timestamps[kv_start + j];
-            r = sPos[ATT_POS_PAD + (n_kv - j)] + sTime[time_bucket_search(dt, sThr, p.Tb)];
+            r = sRv[j] + sTime[time_bucket_search(dt, sThr, p.Tb)];
           }
-          sKeyRab[s * ATT_KEYS * 2 + c] = r;
+          reinterpret_cast<float*>(key)[c] = r;
+        } else if (ts32) {
+          reinterpret_cast<int32_t*>(key)[c] =
+              (j < n_kv) ? static_cast<int32_t>(p.timestamps[kv_start + j] - t_first) : INT32_MAX;
         } else {
-          sKeyTs[s * ATT_KEYS + c] = (j < n_kv) ? p.timestamps[kv_start + j] : INT64_MAX;
+          reinterpret_cast<int64_t*>(key)[c] = (j < n_kv) ? p.timestamps[kv_start + j] : INT64_MAX;
         }
       }
       __syncwarp();
@@ -297,25 +359,27 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
-      const int nW[2] = {nA, nB};
       bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
       tc_fence_after();
       auto issue_s = [&](int g, int s) {
         const uint32_t qa = smem_u32(sQ + g * ATT_TILE_BYTES);
         const uint32_t ka = smem_u32(sK + s * ATT_TILE_BYTES);
+        const uint32_t d = tmem + static_cast<uint32_t>(g * 128);
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk) {
-          mma_bf16_ss(tS[g], smem_desc_sw128(qa + kk * 32, 16, 1024),
+          mma_bf16_ss(d, smem_desc_sw128(qa + kk * 32, 16, 1024),
                       smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[BAR_S_FULL + g]);
       };
       auto issue_pv = [&](int g, int s, bool first) {
         const uint32_t va = smem_u32(sV + s * ATT_TILE_BYTES);
+        const uint32_t d = tmem + 384u + static_cast<uint32_t>(g * 64);
+        const uint32_t a = tmem + 256u + static_cast<uint32_t>(g * 64);
 #pragma unroll
         for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
-          mma_bf16_ts(tO[g], tP[g] + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024),
-                      idesc_pv, (first && kk == 0) ? 0u : 1u);
+          mma_bf16_ts(d, a + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
+                      (first && kk == 0) ? 0u : 1u);
         }
       };
       if (ok && nk_total > 0) {
@@ -330,12 +394,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int s = kt % ATT_STAGES;
         bool next_ready = false;
         for (int g = 0; g < 2 && ok; ++g) {
-          if (kt >= nW[g]) continue;
+          const int nW = g == 0 ? nA : nB;
+          if (kt >= nW) continue;
           ok = mbar_wait(&bars[BAR_P_FULL + g], static_cast<uint32_t>(kt) & 1u, ctl);
           if (!ok) break;
           tc_fence_after();
           issue_pv(g, s, kt == 0);
-          if (kt + 1 < nW[g]) {
+          if (kt + 1 < nW) {
             if (!next_ready) {
               const int s1 = (kt + 1) % ATT_STAGES;
               ok = mbar_wait(&bars[BAR_KV_FULL + s1],
@@ -360,23 +425,117 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int g = warp >> 2;               // 0 = tile A, 1 = tile B
     const int r = tid & (ATT_ROWS - 1);    // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(g * 128);
+    const uint32_t tP = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64);
+    const uint32_t tO = tmem + lane_off + 384u + static_cast<uint32_t>(g * 64);
     const int i = q0 + g * ATT_ROWS + r;   // query index within the user
     const bool valid = i < n_q;
     const int nW = g == 0 ? nA : nB;
     bool ok = true;
+    const uint64_t scale2 = f2_pack(kScale, kScale);
 
-    BucketWalk walk;
+    // causal: per-row time-bucket walk and staged position-table copy
+    BucketWalk<int32_t> w32;
+    BucketWalk<int64_t> w64;
     float rt = 0.0f;
+    int copy = 0;
+    const float* rv = sRv;
     if constexpr (!CAND) {
-      if (valid) {
-        walk.init(p.timestamps[kv_start + i], p.timestamps[kv_start], sThr, p.Tb);
+      const int64_t ti = valid ? p.timestamps[kv_start + i] : t_first;
+      if (ts32) {
+        w32.init(static_cast<int32_t>(ti - t_first), 0, sThr, p.Tb);
+        rt = sTime[w32.b];
       } else {
-        walk.ti = 0;
-        walk.b = 0;
-        walk.bound = INT64_MAX;
+        w64.init(ti, t_first, sThr, p.Tb);
+        rt = sTime[w64.b];
       }
-      rt = sTime[walk.b];
+      if constexpr (PAIRS) copy = (D - i) & 1;
+      rv = sRv + copy * p.pos_len;
     }
+
+    // one 32-key chunk: S values in `sv`, packed bf16 P pairs to `pk`
+    auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int ch, int s,
+                     bool diag) {
+      const uint8_t* key = sKey + s * AttnSmem::kKeyStride;
+      if constexpr (CAND) {
+        const float* kr = reinterpret_cast<const float*>(key) + ch * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                     scale2, lds_b64(kr + c));
+          pk[c >> 1] = phi_pair<PHI>(h2);
+        }
+        const int last = n_kv - 1 - (kt * ATT_KEYS + ch * 32);  // last live column
+        if (last < 31) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
+        }
+      } else {
+        const int xc = D - i + kt * ATT_KEYS + ch * 32 + copy;  // table index at column 0
+        float rtv[32];
+        bool steady;
+        if (ts32) {
+          const int32_t* kts = reinterpret_cast<const int32_t*>(key) + ch * 32;
+          // warp-uniform fast path: no row of this warp changes bucket in the chunk
+          steady = __all_sync(0xffffffffu, kts[31] <= w32.bound);
+          if (!steady) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) rtv[c] = rt;
+            // each bucket change point applies the new time bias to the rest of
+            // the chunk; the first key past the current edge is found by binary
+            // search over the chunk's sorted key times
+            while (kts[31] > w32.bound) {
+              int lo = 0, hi = 31;
+              while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (kts[mid] > w32.bound) hi = mid; else lo = mid + 1;
+              }
+              w32.step(kts[lo], sThr);
+              rt = sTime[w32.b];
+#pragma unroll
+              for (int c = 0; c < 32; ++c) rtv[c] = (c >= lo) ? rt : rtv[c];
+            }
+          }
+        } else {
+          const int64_t* kts = reinterpret_cast<const int64_t*>(key) + ch * 32;
+          steady = kts[31] <= w64.bound;
+          if (!steady) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (w64.step(kts[c], sThr)) rt = sTime[w64.b];
+              rtv[c] = rt;
+            }
+          }
+        }
+        if (steady) {
+          const uint64_t rt2 = f2_pack(rt, rt);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            uint64_t pp;
+            if constexpr (PAIRS) pp = lds_b64(rv + xc + c);
+            else pp = f2_pack(rv[xc + c], rv[xc + c + 1]);
+            const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                       scale2, f2_add(pp, rt2));
+            pk[c >> 1] = phi_pair<PHI>(h2);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            uint64_t pp;
+            if constexpr (PAIRS) pp = lds_b64(rv + xc + c);
+            else pp = f2_pack(rv[xc + c], rv[xc + c + 1]);
+            const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                       scale2, f2_add(pp, f2_pack(rtv[c], rtv[c + 1])));
+            pk[c >> 1] = phi_pair<PHI>(h2);
+          }
+        }
+        if (diag) {
+          const int last = r - ch * 32;  // keys at columns <= r are visible
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
+        }
+      }
+    };
 
     for (int kt = 0; kt < nW; ++kt) {
       const int s = kt % ATT_STAGES;
@@ -388,61 +547,34 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) break;
       tc_fence_after();
       const bool diag = !CAND && (kt == 2 * qp + g);
-      const int pos_base = ATT_POS_PAD + i - kt * ATT_KEYS;  // sPos index at column 0
-      const int key_lim = n_kv - kt * ATT_KEYS;              // columns >= key_lim are padding
-#pragma unroll 1
-      for (int ch = 0; ch < ATT_KEYS / 32; ++ch) {
-        uint32_t sv[32];
-        __syncwarp();
-        tmem_ld32(tS[g] + lane_off + ch * 32, sv);
-        tmem_ld_wait();
-        uint32_t pk[16];
-        if constexpr (CAND) {
-          const float* kr = sKeyRab + s * ATT_KEYS * 2 + ch * 32;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float x0 = __uint_as_float(sv[c]) + kr[c];
-            float x1 = __uint_as_float(sv[c + 1]) + kr[c + 1];
-            float p0 = apply_phi<PHI>(x0);
-            float p1 = apply_phi<PHI>(x1);
-            if (ch * 32 + c >= key_lim) p0 = 0.0f;
-            if (ch * 32 + c + 1 >= key_lim) p1 = 0.0f;
-            pk[c >> 1] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          const int64_t* kts = sKeyTs + s * ATT_KEYS + ch * 32;
-          const float* pr = sPos + pos_base - ch * 32;
-          const bool steady = kts[31] <= walk.bound;  // no bucket change inside this chunk
-          float pv[32];
-          if (steady) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pv[c] = __uint_as_float(sv[c]) + (pr[-c] + rt);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (walk.step(kts[c], sThr)) rt = sTime[walk.b];
-              pv[c] = __uint_as_float(sv[c]) + (pr[-c] + rt);
-            }
-          }
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pv[c] = apply_phi<PHI>(pv[c]);
-          if (diag) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (ch * 32 + c > r) pv[c] = 0.0f;
-          }
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) pk[c >> 1] = pack_bf16x2(pv[c], pv[c + 1]);
-        }
-        __syncwarp();
-        tmem_st16(tP[g] + lane_off + ch * 16, pk);
-      }
+      // chunks of 32 keys; the TMEM load of chunk ch+1 overlaps the math of ch
+      uint32_t sa[32], sb[32], pk[16];
+      tmem_ld32(tS + 0, sa);
+      tmem_ld_wait(sa);
+      tmem_ld32(tS + 32, sb);
+      chunk(sa, pk, kt, 0, s, diag);
+      __syncwarp();
+      tmem_st16(tP + 0, pk);
+      tmem_ld_wait(sb);
+      tmem_ld32(tS + 64, sa);
+      chunk(sb, pk, kt, 1, s, diag);
+      __syncwarp();
+      tmem_st16(tP + 16, pk);
+      tmem_ld_wait(sa);
+      tmem_ld32(tS + 96, sb);
+      chunk(sa, pk, kt, 2, s, diag);
+      __syncwarp();
+      tmem_st16(tP + 32, pk);
+      tmem_ld_wait(sb);
+      chunk(sb, pk, kt, 3, s, diag);
+      __syncwarp();
+      tmem_st16(tP + 48, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P_FULL + g]);
     }
 
-    // ---------------- epilogue: O / N, LayerNorm partial sums, bf16 store
+    // ---------------- epilogue: O / N, LayerNorm partial sums, store
     float o[ATT_HD];
     if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL], 0, ctl);
     ok = __all_sync(0xffffffffu, ok);
@@ -450,12 +582,12 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (nW > 0) {
         tc_fence_after();
         uint32_t ov[32];
-        tmem_ld32(tO[g] + lane_off + 0, ov);
-        tmem_ld_wait();
+        tmem_ld32(tO + 0, ov);
+        tmem_ld_wait(ov);
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(ov[c]);
-        tmem_ld32(tO[g] + lane_off + 32, ov);
-        tmem_ld_wait();
+        tmem_ld32(tO + 32, ov);
+        tmem_ld_wait(ov);
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[32 + c] = __uint_as_float(ov[c]);
       } else {
@@ -484,7 +616,9 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               dot = fmaf(qf.y, kf.y, dot);
             }
           }
-          const float ps = apply_phi<PHI>(dot + sPos[ATT_POS_PAD + 0] + sTime[0]);
+          const float rab0 = (p.rab_pos[static_cast<int64_t>(h) * p.P] +
+                              p.rab_time[static_cast<int64_t>(h) * p.Tb]);
+          const float ps = apply_phi<PHI>(dot + rab0);
 #pragma unroll
           for (int c = 0; c < ATT_HD; c += 8) {
             uint4 va = *reinterpret_cast<const uint4*>(vs + c);
@@ -548,8 +682,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // ---------------------------------------------------------------- debug: bucket indices
 
 // Writes, per user, the n x n blocks of position and time bucket indices the
-// attention kernel uses (BucketWalk for the time buckets, min(i-j, P-1) for
-// positions; -1 above the diagonal).  One thread per query row.
+// attention kernel uses (the int32 and int64 BucketWalk for the time buckets,
+// min(i-j, P-1) for positions; -1 above the diagonal).  One thread per query row.
 __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_t* timestamps,
                                             const int64_t* block_offsets, int B, int P, int Tb,
                                             int max_len, int32_t* pos_idx, int32_t* time_idx,
@@ -564,13 +698,24 @@ __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_
   const int n = static_cast<int>(offsets[u + 1] - s);
   if (i >= n) return;
   const int64_t base = block_offsets[u] + static_cast<int64_t>(i) * n;
-  BucketWalk walk;
-  walk.init(timestamps[s + i], timestamps[s], sThr, Tb);
+  const int64_t t0 = timestamps[s];
+  const bool ts32 = timestamps[s + n - 1] - t0 < static_cast<int64_t>(INT32_MAX) - 1;
+  BucketWalk<int32_t> w32;
+  BucketWalk<int64_t> w64;
+  if (ts32) w32.init(static_cast<int32_t>(timestamps[s + i] - t0), 0, sThr, Tb);
+  else w64.init(timestamps[s + i], t0, sThr, Tb);
   for (int j = 0; j < n; ++j) {
     if (j <= i) {
-      walk.step(timestamps[s + j], sThr);
+      int b;
+      if (ts32) {
+        w32.step(static_cast<int32_t>(timestamps[s + j] - t0), sThr);
+        b = w32.b;
+      } else {
+        w64.step(timestamps[s + j], sThr);
+        b = w64.b;
+      }
       pos_idx[base + j] = min(i - j, P - 1);
-      time_idx[base + j] = walk.b;
+      time_idx[base + j] = b;
     } else {
       pos_idx[base + j] = -1;
       time_idx[base + j] = -1;

@@ -135,6 +135,23 @@ class ProfScope {
 
 // ------------------------------------------------------------------ device info
 
+using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                              const AttnParams);
+
+template <bool CAND, bool PAIRS>
+AttnKernelFn attn_kernel_for(int phi) {
+  switch (phi) {
+    case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS>;
+    case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS>;
+    default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS>;
+  }
+}
+
+AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs) {
+  if (cand) return pairs ? attn_kernel_for<true, true>(phi) : attn_kernel_for<true, false>(phi);
+  return pairs ? attn_kernel_for<false, true>(phi) : attn_kernel_for<false, false>(phi);
+}
+
 struct DeviceInfo {
   int sm_count = 0;
   bool smem_set = false;
@@ -152,19 +169,13 @@ hstu_status_t device_info(DeviceInfo** out) {
     HSTU_CHECK_CUDA(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev));
   }
   if (!d.smem_set) {
-    const int att_max = static_cast<int>(AttnSmem::bytes(kMaxLen + 256));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_SILU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_RELU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<false, HSTU_ACT_IDENTITY>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_SILU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_RELU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_attn_kernel<true, HSTU_ACT_IDENTITY>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    const int att_max = 227 * 1024;
+    for (int cand = 0; cand < 2; ++cand)
+      for (int phi = 0; phi < 3; ++phi)
+        for (int pairs = 0; pairs < 2; ++pairs)
+          HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(cand != 0, phi, pairs != 0),
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               att_max));
     const int g = static_cast<int>(GemmSmem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g));
@@ -369,25 +380,21 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.P = c->num_pos_buckets;
   p.Tb = c->num_time_buckets;
   p.num_qpairs = (j.max_q_len + 2 * ATT_ROWS - 1) / (2 * ATT_ROWS);
-  const int longest = j.max_q_len > j.max_kv_len ? j.max_q_len : j.max_kv_len;
-  p.pos_cap = static_cast<int32_t>(align_up(static_cast<size_t>(longest) + 1, 256));
+  // largest staged-table origin D over the CTAs, plus the diagonal overhang
+  const size_t dmax = CAND ? static_cast<size_t>(j.max_kv_len)
+                           : align_up(static_cast<size_t>(j.max_q_len), 2 * ATT_ROWS);
+  // per-copy length = 16 (mod 32) floats: the two copies' 8-byte pair reads
+  // by neighbouring lanes then fall in disjoint shared-memory banks
+  p.pos_len = static_cast<int32_t>(align_up(dmax + ATT_KEYS + 2, 32) + 16);
   p.phi2 = c->phi2;
   p.timeout_ns = j.timeout_ns;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
   dim3 grid(c->num_heads, j.batch, p.num_qpairs);
-  const size_t smem = AttnSmem::bytes(p.pos_cap);
+  const bool pairs = AttnSmem::bytes(p.pos_len, true) <= 227u * 1024u;
+  const size_t smem = AttnSmem::bytes(p.pos_len, pairs);
+  if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
-  switch (c->phi2) {
-    case HSTU_ACT_SILU:
-      hstu_attn_kernel<CAND, HSTU_ACT_SILU><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
-      break;
-    case HSTU_ACT_RELU:
-      hstu_attn_kernel<CAND, HSTU_ACT_RELU><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
-      break;
-    default:
-      hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY><<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
-      break;
-  }
+  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
