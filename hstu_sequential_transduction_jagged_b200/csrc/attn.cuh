@@ -15,12 +15,18 @@
 //   warp 8     producer: TMA loads of Q, K, V tiles (128B swizzle) and the
 //              per-key side data (timestamps, or candidate-mode bias)
 //   warp 9     MMA issuer (one thread) and TMEM owner
-// Tensor memory (512 columns): S_A, S_B (128 fp32 columns each), P_A, P_B
-// (64 columns each, bf16 pairs), O_A, O_B (64 fp32 columns each).
-// Per key tile: S = Q K^T (tcgen05, A and B from shared memory), the softmax
-// group reads S row by row, adds the gathered bias, applies phi2 and the
-// mask, writes P (bf16) back to tensor memory, then O += P V (tcgen05 with A
-// from tensor memory, V as an MN-major B operand).  1/N is applied once to O.
+// Tensor memory (448 of 512 columns): S_A, S_B (128 fp32 columns each; P,
+// bf16 pairs, overwrites the first 64 columns of its S once they are read),
+// O_A, O_B (64 fp32 columns each), Q_A, Q_B (32 columns each, bf16 pairs).
+// Q is written to tensor memory once per CTA by the softmax threads, so the
+// QK^T MMA reads only K from shared memory (an M=128, N=128 MMA with both
+// operands in shared memory would need the whole shared-memory bandwidth).
+// Per key tile: S = Q K^T (tcgen05, A from tensor memory), the softmax group
+// reads S row by row, adds the gathered bias, applies phi2 and the mask,
+// writes P (bf16) back over S, then O += P V (tcgen05 with A from tensor
+// memory, V as an MN-major B operand).  The MMAs of one CTA execute in issue
+// order, so S of the next tile is only written after P V has read P.
+// 1/N is applied once to O.
 //
 // Elementwise work per (query, key, head), SiLU case: x = s + rab, and
 // x*sigmoid(x) = h + h*tanh(h) with h = x/2.  The 1/2 is folded into the bias
@@ -54,6 +60,8 @@ struct AttnParams {
   const int64_t* request_ts;   // [B] (candidate mode)
   const float* rab_pos;        // [H, P]
   const float* rab_time;       // [H, Tb]
+  const __nv_bfloat16* q;      // [T_q, ld_q] query rows (head h at columns h*64..)
+  int64_t ld_q;
   const __nv_bfloat16* q_self; // candidate mode: candidate Q, K, V rows (self term)
   const __nv_bfloat16* k_self;
   const __nv_bfloat16* v_self;
@@ -68,6 +76,7 @@ struct AttnParams {
   int32_t phi2;
   uint64_t timeout_ns;
   int64_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0)
+  int4 oct[32];                   // per octave k of dt+1: {t1, t2, t3, bucket(2^k - 1)}
 };
 
 // ---------------------------------------------------------------- time buckets
@@ -118,6 +127,17 @@ struct BucketWalk {
   }
 };
 
+// Time bucket of 0 <= dt < 2^31 - 1 without a walk.  For dt + 1 in the octave
+// [2^k, 2^(k+1)) the bucket is oct[k].w plus the number of the next three
+// bucket edges oct[k].x/y/z it reaches (edges are ~1.35x apart, so at most
+// three fall inside one octave; INT32_MAX pads missing edges).
+__device__ __forceinline__ int time_bucket_octave(int32_t dt, const int4* oct) {
+  const int32_t d = dt > 0 ? dt : 0;
+  const int k = 31 - __clz(d + 1);
+  const int4 o = oct[k];
+  return o.w + (d >= o.x ? 1 : 0) + (d >= o.y ? 1 : 0) + (d >= o.z ? 1 : 0);
+}
+
 // phi2 applied to a pair given h = (scaled) pre-activation; returns bf16x2.
 // SiLU: tables carry x/2, so p = h + h*tanh(h); ReLU / identity: h = x.
 template <int PHI>
@@ -161,14 +181,14 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t w, int c, int last) {
 // ---------------------------------------------------------------- shared memory
 
 struct AttnSmem {
-  static constexpr uint32_t kQ = 0;                                   // 2 x 16 KB
-  static constexpr uint32_t kK = kQ + 2 * ATT_TILE_BYTES;             // stages x 16 KB
+  static constexpr uint32_t kK = 0;                                   // stages x 16 KB
   static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 16 KB
   static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 1 KB
   static constexpr uint32_t kKeyStride = ATT_KEYS * 8;                // bytes per stage
   static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * kKeyStride;
   static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
-  static constexpr uint32_t kBars = kThr + MAX_TIME_BUCKETS * 8;
+  static constexpr uint32_t kOct = kThr + MAX_TIME_BUCKETS * 8;      // 32 x int4
+  static constexpr uint32_t kBars = kOct + 32 * 16;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kPos = kMisc + 64;
   static constexpr uint32_t bytes(int pos_len, bool pairs) {
@@ -188,12 +208,101 @@ enum : int {
   BAR_COUNT = BAR_DONE + 1
 };
 
+// ---------------------------------------------------------------- causal chunk
+
+// One 32-key chunk of one causal row: S values in `sv` -> packed bf16 P in `pk`.
+// `rvx` points at the staged position table entry of column 0 (entries for
+// consecutive columns are consecutive), `kts` at the chunk's key times
+// (seconds since the user's first event, 16-byte aligned).  Columns above
+// `lim` are masked (P = 0) and never move the time-bucket walk; lim < 0 masks
+// the whole chunk.  The walk `w` enters at the bucket of the previous key and
+// leaves at the bucket of the last visible key.  Per warp the chunk falls in
+// one of three cases:
+//   every row keeps one bucket      -> one time bias per row;
+//   two buckets B, B+1 in the warp  -> per key: B+1 iff t_j <= t_i - thr[B+1];
+//   more (near the diagonal)        -> per key bucket from the octave table.
+template <int PHI, bool PAIRS>
+__device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16],
+                                             const float* rvx, const int32_t* kts, int lim,
+                                             BucketWalk<int32_t>& w, const float* sTime,
+                                             const int64_t* sThr, const int4* sOct,
+                                             uint64_t scale2) {
+  const unsigned full = 0xffffffffu;
+  const bool live = lim >= 0;
+  const int last = lim < 31 ? lim : 31;
+  int32_t kt[32];
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(kts + c);
+    kt[c] = v.x; kt[c + 1] = v.y; kt[c + 2] = v.z; kt[c + 3] = v.w;
+  }
+  int b_first = -1, b_last = 1 << 30;
+  bool lane_steady = true;
+  if (live) {
+    w.step(kt[0], sThr);
+    b_first = w.b;
+    const int32_t k_last = kts[last];
+    lane_steady = k_last <= w.bound;
+    if (!lane_steady) w.step(k_last, sThr);
+    b_last = w.b;
+  }
+  auto pos_pair = [&](int c) -> uint64_t {
+    if constexpr (PAIRS) return lds_b64(rvx + c);
+    else return f2_pack(rvx[c], rvx[c + 1]);
+  };
+  auto s_pair = [&](int c) -> uint64_t {
+    return f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+  };
+  if (__all_sync(full, lane_steady)) {
+    if (live) {
+      const float rt = sTime[b_first];
+      const uint64_t rt2 = f2_pack(rt, rt);
+#pragma unroll
+      for (int c = 0; c < 32; c += 2)
+        pk[c >> 1] = phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
+    }
+  } else {
+    const int B_hi = __reduce_max_sync(full, b_first);
+    const int B_lo = __reduce_min_sync(full, b_last);
+    if (B_hi - B_lo == 1) {
+      if (live) {
+        const float rt_hi = sTime[B_hi], rt_lo = sTime[B_lo];
+        const int64_t e = static_cast<int64_t>(w.ti) - sThr[B_hi];
+        const int32_t edge =
+            e < static_cast<int64_t>(INT32_MIN) ? INT32_MIN : static_cast<int32_t>(e);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float r0 = (kt[c] <= edge) ? rt_hi : rt_lo;
+          const float r1 = (kt[c + 1] <= edge) ? rt_hi : rt_lo;
+          pk[c >> 1] =
+              phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
+        }
+      }
+    } else if (live) {
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        const float r0 = sTime[time_bucket_octave(w.ti - kt[c], sOct)];
+        const float r1 = sTime[time_bucket_octave(w.ti - kt[c + 1], sOct)];
+        pk[c >> 1] =
+            phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
+      }
+    }
+  }
+  if (!live) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) pk[q] = 0u;
+  } else if (lim < 31) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, lim);
+  }
+}
+
 // ---------------------------------------------------------------- kernel
 
 template <bool CAND, int PHI, bool PAIRS>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
+hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -234,12 +343,12 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int D = CAND ? n_kv : q0 + 2 * ATT_ROWS;
   constexpr float kScale = phi_scale<PHI>();
 
-  uint8_t* sQ = smem + AttnSmem::kQ;
   uint8_t* sK = smem + AttnSmem::kK;
   uint8_t* sV = smem + AttnSmem::kV;
   uint8_t* sKey = smem + AttnSmem::kKeyInfo;
   float* sTime = reinterpret_cast<float*>(smem + AttnSmem::kTimeTab);
   int64_t* sThr = reinterpret_cast<int64_t*>(smem + AttnSmem::kThr);
+  int4* sOct = reinterpret_cast<int4*>(smem + AttnSmem::kOct);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 4);
@@ -249,15 +358,17 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int lane = lane_id();
   const int tid = threadIdx.x;
 
-  // timestamps relative to the user's first event fit in int32 unless the
-  // user spans more than ~68 years; then the int64 walk is used
+  // key times are kept as int32 seconds since the user's first event; a user
+  // spanning 2^31 - 1 seconds (68 years) or more is outside the contract and
+  // is reported through the device status word (times are then clamped)
   const int64_t t_first = n_kv > 0 ? p.timestamps[kv_start] : 0;
-  const bool ts32 = CAND || (n_kv == 0) ||
-                    (p.timestamps[kv_start + n_kv - 1] - t_first < static_cast<int64_t>(INT32_MAX) - 1);
+  if (!CAND && n_kv > 0 && tid == 0 &&
+      p.timestamps[kv_start + n_kv - 1] - t_first >= static_cast<int64_t>(INT32_MAX) - 1)
+    record_status(HSTU_ERR_DEVICE_CHECK);
 
   // ---------------- setup
   if (tid == 0) {
-    mbar_init(&bars[BAR_Q_FULL], 1);
+    mbar_init(&bars[BAR_Q_FULL], 2 * ATT_ROWS);  // every softmax thread stores its Q row
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&bars[BAR_KV_FULL + s], 2);
       mbar_init(&bars[BAR_KV_EMPTY + s], 1);
@@ -291,6 +402,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     sTime[k] = kScale * p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     sThr[k] = p.thr[k];
   }
+  if (tid < 32) sOct[tid] = p.oct[tid];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -300,14 +412,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp == 8) {
     // ---------------- producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars[BAR_Q_FULL], ATT_TILE_BYTES * (has_b ? 2u : 1u));
-      tma_load_2d(sQ, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD, static_cast<int32_t>(q_start + q0));
-      if (has_b)
-        tma_load_2d(sQ + ATT_TILE_BYTES, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD,
-                    static_cast<int32_t>(q_start + q0 + ATT_ROWS));
     }
     int64_t t_req = 0;
     if constexpr (CAND) t_req = p.request_ts[u];
@@ -337,11 +443,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             r = sRv[j] + sTime[time_bucket_search(dt, sThr, p.Tb)];
           }
           reinterpret_cast<float*>(key)[c] = r;
-        } else if (ts32) {
-          reinterpret_cast<int32_t*>(key)[c] =
-              (j < n_kv) ? static_cast<int32_t>(p.timestamps[kv_start + j] - t_first) : INT32_MAX;
         } else {
-          reinterpret_cast<int64_t*>(key)[c] = (j < n_kv) ? p.timestamps[kv_start + j] : INT64_MAX;
+          int32_t rel = INT32_MAX;
+          if (j < n_kv) {
+            const int64_t d = p.timestamps[kv_start + j] - t_first;
+            rel = d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d);
+          }
+          reinterpret_cast<int32_t*>(key)[c] = rel;
         }
       }
       __syncwarp();
@@ -349,7 +457,6 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     // drain: every issued load must land before shared memory is released
     if (lane == 0) {
-      mbar_wait_drain(&bars[BAR_Q_FULL], 0, p.timeout_ns);
       for (int kt = max(0, issued - ATT_STAGES); kt < issued; ++kt)
         mbar_wait_drain(&bars[BAR_KV_FULL + kt % ATT_STAGES],
                         static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
@@ -362,20 +469,20 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
       tc_fence_after();
       auto issue_s = [&](int g, int s) {
-        const uint32_t qa = smem_u32(sQ + g * ATT_TILE_BYTES);
+        const uint32_t qa = tmem + 384u + static_cast<uint32_t>(g * 32);
         const uint32_t ka = smem_u32(sK + s * ATT_TILE_BYTES);
         const uint32_t d = tmem + static_cast<uint32_t>(g * 128);
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk) {
-          mma_bf16_ss(d, smem_desc_sw128(qa + kk * 32, 16, 1024),
-                      smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(d, qa + kk * 8, smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk,
+                      kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[BAR_S_FULL + g]);
       };
       auto issue_pv = [&](int g, int s, bool first) {
         const uint32_t va = smem_u32(sV + s * ATT_TILE_BYTES);
-        const uint32_t d = tmem + 384u + static_cast<uint32_t>(g * 64);
-        const uint32_t a = tmem + 256u + static_cast<uint32_t>(g * 64);
+        const uint32_t d = tmem + 256u + static_cast<uint32_t>(g * 64);
+        const uint32_t a = tmem + static_cast<uint32_t>(g * 128);  // P over S
 #pragma unroll
         for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
           mma_bf16_ts(d, a + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
@@ -426,29 +533,42 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int r = tid & (ATT_ROWS - 1);    // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(g * 128);
-    const uint32_t tP = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64);
-    const uint32_t tO = tmem + lane_off + 384u + static_cast<uint32_t>(g * 64);
+    const uint32_t tP = tS;  // P overwrites the S columns it was computed from
+    const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64);
+    const uint32_t tQ = tmem + lane_off + 384u + static_cast<uint32_t>(g * 32);
     const int i = q0 + g * ATT_ROWS + r;   // query index within the user
     const bool valid = i < n_q;
     const int nW = g == 0 ? nA : nB;
     bool ok = true;
+    {
+      // this row's query (64 bf16 = 32 columns of packed pairs) into tensor memory
+      uint32_t qv[32];
+      if (valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + (q_start + i) * p.ld_q + h * ATT_HD);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v4 = src[c];
+          qv[4 * c] = v4.x; qv[4 * c + 1] = v4.y; qv[4 * c + 2] = v4.z; qv[4 * c + 3] = v4.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) qv[c] = 0u;
+      }
+      tmem_st32(tQ, qv);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[BAR_Q_FULL]);
+    }
     const uint64_t scale2 = f2_pack(kScale, kScale);
 
     // causal: per-row time-bucket walk and staged position-table copy
     BucketWalk<int32_t> w32;
-    BucketWalk<int64_t> w64;
-    float rt = 0.0f;
     int copy = 0;
     const float* rv = sRv;
     if constexpr (!CAND) {
-      const int64_t ti = valid ? p.timestamps[kv_start + i] : t_first;
-      if (ts32) {
-        w32.init(static_cast<int32_t>(ti - t_first), 0, sThr, p.Tb);
-        rt = sTime[w32.b];
-      } else {
-        w64.init(ti, t_first, sThr, p.Tb);
-        rt = sTime[w64.b];
-      }
+      const int64_t d = (valid ? p.timestamps[kv_start + i] : t_first) - t_first;
+      w32.init(d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d), 0,
+               sThr, p.Tb);
       if constexpr (PAIRS) copy = (D - i) & 1;
       rv = sRv + copy * p.pos_len;
     }
@@ -472,68 +592,11 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       } else {
         const int xc = D - i + kt * ATT_KEYS + ch * 32 + copy;  // table index at column 0
-        float rtv[32];
-        bool steady;
-        if (ts32) {
-          const int32_t* kts = reinterpret_cast<const int32_t*>(key) + ch * 32;
-          // warp-uniform fast path: no row of this warp changes bucket in the chunk
-          steady = __all_sync(0xffffffffu, kts[31] <= w32.bound);
-          if (!steady) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) rtv[c] = rt;
-            // each bucket change point applies the new time bias to the rest of
-            // the chunk; the first key past the current edge is found by binary
-            // search over the chunk's sorted key times
-            while (kts[31] > w32.bound) {
-              int lo = 0, hi = 31;
-              while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (kts[mid] > w32.bound) hi = mid; else lo = mid + 1;
-              }
-              w32.step(kts[lo], sThr);
-              rt = sTime[w32.b];
-#pragma unroll
-              for (int c = 0; c < 32; ++c) rtv[c] = (c >= lo) ? rt : rtv[c];
-            }
-          }
-        } else {
-          const int64_t* kts = reinterpret_cast<const int64_t*>(key) + ch * 32;
-          steady = kts[31] <= w64.bound;
-          if (!steady) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (w64.step(kts[c], sThr)) rt = sTime[w64.b];
-              rtv[c] = rt;
-            }
-          }
-        }
-        if (steady) {
-          const uint64_t rt2 = f2_pack(rt, rt);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            uint64_t pp;
-            if constexpr (PAIRS) pp = lds_b64(rv + xc + c);
-            else pp = f2_pack(rv[xc + c], rv[xc + c + 1]);
-            const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                       scale2, f2_add(pp, rt2));
-            pk[c >> 1] = phi_pair<PHI>(h2);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            uint64_t pp;
-            if constexpr (PAIRS) pp = lds_b64(rv + xc + c);
-            else pp = f2_pack(rv[xc + c], rv[xc + c + 1]);
-            const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                       scale2, f2_add(pp, f2_pack(rtv[c], rtv[c + 1])));
-            pk[c >> 1] = phi_pair<PHI>(h2);
-          }
-        }
-        if (diag) {
-          const int last = r - ch * 32;  // keys at columns <= r are visible
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
-        }
+        // last visible column: the diagonal masks keys after the row; rows past
+        // the user's end are not stored and skip the work
+        const int lim = !valid ? -1 : (diag ? r - ch * 32 : 31);
+        causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + ch * 32,
+                                 lim, w32, sTime, sThr, sOct, scale2);
       }
     };
 
@@ -547,28 +610,16 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) break;
       tc_fence_after();
       const bool diag = !CAND && (kt == 2 * qp + g);
-      // chunks of 32 keys; the TMEM load of chunk ch+1 overlaps the math of ch
-      uint32_t sa[32], sb[32], pk[16];
-      tmem_ld32(tS + 0, sa);
-      tmem_ld_wait(sa);
-      tmem_ld32(tS + 32, sb);
-      chunk(sa, pk, kt, 0, s, diag);
-      __syncwarp();
-      tmem_st16(tP + 0, pk);
-      tmem_ld_wait(sb);
-      tmem_ld32(tS + 64, sa);
-      chunk(sb, pk, kt, 1, s, diag);
-      __syncwarp();
-      tmem_st16(tP + 16, pk);
-      tmem_ld_wait(sa);
-      tmem_ld32(tS + 96, sb);
-      chunk(sa, pk, kt, 2, s, diag);
-      __syncwarp();
-      tmem_st16(tP + 32, pk);
-      tmem_ld_wait(sb);
-      chunk(sb, pk, kt, 3, s, diag);
-      __syncwarp();
-      tmem_st16(tP + 48, pk);
+      // four chunks of 32 keys: TMEM -> registers -> bias, phi2, mask -> P back to TMEM
+      uint32_t sa[32], pk[16];
+#pragma unroll 1
+      for (int ch = 0; ch < ATT_KEYS / 32; ++ch) {
+        tmem_ld32(tS + ch * 32, sa);
+        tmem_ld_wait(sa);
+        chunk(sa, pk, kt, ch, s, diag);
+        __syncwarp();
+        tmem_st16(tP + ch * 16, pk);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P_FULL + g]);
@@ -689,7 +740,9 @@ __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_
                                             int max_len, int32_t* pos_idx, int32_t* time_idx,
                                             const __grid_constant__ AttnParams p) {
   __shared__ int64_t sThr[MAX_TIME_BUCKETS];
+  __shared__ int4 sOct[32];
   for (int k = threadIdx.x; k < Tb; k += blockDim.x) sThr[k] = p.thr[k];
+  if (threadIdx.x < 32) sOct[threadIdx.x] = p.oct[threadIdx.x];
   __syncthreads();
   const int u = blockIdx.y;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -714,6 +767,10 @@ __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_
         w64.step(timestamps[s + j], sThr);
         b = w64.b;
       }
+      // the attention kernels use both the walk and the octave table; a
+      // disagreement between them is reported as -2
+      if (ts32 && b != time_bucket_octave(static_cast<int32_t>(timestamps[s + i] - timestamps[s + j]), sOct))
+        b = -2;
       pos_idx[base + j] = min(i - j, P - 1);
       time_idx[base + j] = b;
     } else {

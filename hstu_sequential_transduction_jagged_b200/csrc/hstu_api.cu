@@ -64,6 +64,27 @@ void compute_thresholds(int Tb, int64_t* thr) {
   }
 }
 
+// Octave table for dt < 2^31 - 1: for dt + 1 in [2^k, 2^(k+1)), {t1, t2, t3}
+// are the next three bucket edges after bucket(2^k - 1) (INT32_MAX when the
+// bucket index would reach Tb or the edge does not fit), w = bucket(2^k - 1).
+// Returns false if some octave holds more than three edges.
+bool compute_octaves(int Tb, const int64_t* thr, int4* oct) {
+  for (int k = 0; k < 32; ++k) {
+    const int64_t lo = (int64_t(1) << k) - 1;
+    const int64_t hi = (int64_t(2) << k) - 2;  // largest dt with dt + 1 < 2^(k+1)
+    int b = 0;
+    while (b + 1 < Tb && thr[b + 1] <= lo) ++b;
+    int32_t t[4];
+    for (int e = 0; e < 4; ++e) {
+      const int idx = b + 1 + e;
+      t[e] = (idx < Tb && thr[idx] < INT32_MAX) ? static_cast<int32_t>(thr[idx]) : INT32_MAX;
+    }
+    if (static_cast<int64_t>(t[3]) <= hi && t[3] != INT32_MAX) return false;
+    oct[k] = make_int4(t[0], t[1], t[2], b);
+  }
+  return true;
+}
+
 const int64_t* thresholds_for(int Tb) {
   static std::mutex mu;
   static int64_t table[MAX_TIME_BUCKETS + 1][MAX_TIME_BUCKETS];
@@ -135,8 +156,7 @@ class ProfScope {
 
 // ------------------------------------------------------------------ device info
 
-using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                              const AttnParams);
+using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const AttnParams);
 
 template <bool CAND, bool PAIRS>
 AttnKernelFn attn_kernel_for(int phi) {
@@ -347,9 +367,8 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mk, mv;
   const int64_t hc = static_cast<int64_t>(c->num_heads) * ATT_HD;
-  if ((s = make_map_bf16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS)) != HSTU_OK) return s;
   // with no key rows at all (every history empty) no K/V tile is ever loaded;
   // the maps then describe the query rows so that they stay valid
   const bool no_kv = j.T_kv == 0;
@@ -367,6 +386,8 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.request_ts = j.request_ts;
   p.rab_pos = j.rab_pos;
   p.rab_time = j.rab_time;
+  p.q = static_cast<const __nv_bfloat16*>(j.q);
+  p.ld_q = j.ldq;
   p.q_self = static_cast<const __nv_bfloat16*>(j.q_self);
   p.k_self = static_cast<const __nv_bfloat16*>(j.k_self);
   p.v_self = static_cast<const __nv_bfloat16*>(j.v_self);
@@ -389,12 +410,13 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.phi2 = c->phi2;
   p.timeout_ns = j.timeout_ns;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
+  if (!compute_octaves(c->num_time_buckets, p.thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
   dim3 grid(c->num_heads, j.batch, p.num_qpairs);
   const bool pairs = AttnSmem::bytes(p.pos_len, true) <= 227u * 1024u;
   const size_t smem = AttnSmem::bytes(p.pos_len, pairs);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
-  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mk, mv, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
@@ -951,6 +973,7 @@ hstu_status_t hstu_debug_rab_index(const hstu_jagged_t* jag, int32_t num_pos_buc
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
   std::memcpy(p.thr, thresholds_for(num_time_buckets), sizeof(int64_t) * num_time_buckets);
+  if (!compute_octaves(num_time_buckets, p.thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
   dim3 grid((jag->max_len + 127) / 128, jag->batch);
   hstu_debug_rab_index_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
       jag->offsets, jag->timestamps, block_offsets, jag->batch, num_pos_buckets,
