@@ -671,6 +671,28 @@ hstu_status_t check_weights(const hstu_layer_cfg_t* c, const hstu_layer_weights_
   return HSTU_OK;
 }
 
+// Scratch for hstu_layer_fwd_static: a fixed block in the library's own device
+// memory, for callers that cannot allocate.  Host code may not use the symbol
+// as an address; static_scratch() looks the device address up once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[HSTU_STATIC_SCRATCH_BYTES];
+
+hstu_status_t static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  HSTU_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    HSTU_CHECK_CUDA(cudaGetSymbolAddress(&p, g_static_scratch));
+    if (p == nullptr) return HSTU_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return HSTU_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -787,6 +809,21 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
     return s;
   }
   return layer_bf16(cfg, w, base, x_in, x_res, T, y_out, y_out_lp, kv_cache_out, ws, false, st);
+}
+
+hstu_status_t hstu_layer_fwd_static(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                                    const hstu_jagged_t* jag, const void* x_in,
+                                    const float* x_res, float* y_out, void* y_out_lp,
+                                    void* kv_cache_out, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (layer_ws_bytes(cfg, jag->total_tokens) > HSTU_STATIC_SCRATCH_BYTES)
+    return HSTU_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != HSTU_OK) return s;
+  return hstu_layer_fwd(cfg, w, jag, x_in, x_res, y_out, y_out_lp, kv_cache_out, scratch,
+                        HSTU_STATIC_SCRATCH_BYTES, stream);
 }
 
 hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,

@@ -64,6 +64,7 @@ EXPORTS = {
     "hstu_mfalcon_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int64]),
     "hstu_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hstu_layer_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "hstu_layer_fwd_static": (ctypes.c_int, [ctypes.c_void_p] * 9),
     "hstu_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32] + [ctypes.c_void_p] * 6
                      + [ctypes.c_size_t, ctypes.c_void_p]),
     "mfalcon_score": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
@@ -226,6 +227,24 @@ def layer_fwd(cfg: LayerConfig, w: LayerWeights, jag: Jagged, x_in, x_res=None, 
     _check(lib().hstu_layer_fwd(ctypes.byref(c), ctypes.byref(wc), ctypes.byref(j), _p(x_in),
                                 _p(x_res), _p(y_out), _p(y_out_lp), _p(kv_cache_out), _p(ws),
                                 ws.numel(), _stream(stream)), "hstu_layer_fwd")
+    return y_out
+
+
+STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def layer_fwd_static(cfg: LayerConfig, w: LayerWeights, jag: Jagged, x_in, x_res=None,
+                     y_out=None, y_out_lp=None, kv_cache_out=None, stream=None) -> torch.Tensor:
+    """hstu_layer_fwd without a caller workspace: the library's fixed scratch array
+    (STATIC_SCRATCH_BYTES per GPU) is used, so the C call itself allocates nothing."""
+    if y_out is None:
+        y_out = torch.empty((jag.total_tokens, cfg.d_model), dtype=torch.float32,
+                            device=x_in.device)
+    c, j, wc = cfg.c(), jag.c(), w.c()
+    _check(lib().hstu_layer_fwd_static(ctypes.byref(c), ctypes.byref(wc), ctypes.byref(j),
+                                       _p(x_in), _p(x_res), _p(y_out), _p(y_out_lp),
+                                       _p(kv_cache_out), _stream(stream)),
+           "hstu_layer_fwd_static")
     return y_out
 
 

@@ -198,6 +198,36 @@ typedef struct {
 hstu_status_t hstu_profiler_start(void);
 hstu_status_t hstu_profiler_stop(hstu_kernel_time_t* out, int32_t capacity, int32_t* count);
 
+/*
+ * hstu_layer_fwd for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is an interface convenience.  Some callers
+ * are handed only their input and output buffers: a plugin inside a serving
+ * engine that owns every byte of device memory, or a process whose memory is
+ * pre-reserved by another allocator.  Others must not call cudaMalloc on a
+ * latency-critical path, because it can synchronise the device.  This entry
+ * takes the same arguments as hstu_layer_fwd minus the workspace.  Its
+ * scratch is one fixed array inside the library,
+ * HSTU_STATIC_SCRATCH_BYTES (64 MiB) per GPU, which every GPU that loads the
+ * library keeps until the process exits.
+ *   - Size limit: hstu_layer_workspace_bytes(cfg, T) must not exceed
+ *     HSTU_STATIC_SCRATCH_BYTES (about 9,000 tokens at d_model 512 and 8 heads,
+ *     about 18,000 at d_model 256 and 4 heads).  A larger request returns
+ *     HSTU_ERR_WORKSPACE_TOO_SMALL before any launch.
+ *   - No call allocates: no cudaMalloc, no cudaFree, no allocating library.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current).  Make that first call
+ *     before capturing any stream.
+ *   - Every call on a device shares the same array and leaves its contents
+ *     behind.  The layer writes every scratch byte it reads, so nothing needs
+ *     clearing, but two calls whose work overlaps on the GPU (different
+ *     streams, or different host threads) race on the array: order them.
+ */
+#define HSTU_STATIC_SCRATCH_BYTES (64ull << 20)
+hstu_status_t hstu_layer_fwd_static(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                                    const hstu_jagged_t* jag, const void* x_in,
+                                    const float* x_res, float* y_out, void* y_out_lp,
+                                    void* kv_cache_out, void* stream);
+
 /* Synchronises `stream`, returns the first error a kernel recorded in the
  * device status word since the last call (HSTU_OK if none) and clears it. */
 hstu_status_t hstu_get_device_status(void* stream);
