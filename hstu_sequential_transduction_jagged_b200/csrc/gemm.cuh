@@ -269,7 +269,10 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
 // ------------------------------------------------------------------ f2
 
-__global__ void __launch_bounds__(320, 1)
+constexpr int F2_PRODUCER_WARPS = 8;
+constexpr int F2_THREADS = (6 + F2_PRODUCER_WARPS) * 32;
+
+__global__ void __launch_bounds__(F2_THREADS, 1)
 hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ F2Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -286,7 +289,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G_STAGES; ++s) {
-      mbar_init(&bars[GB_FULL + s], 1 + 4);  // TMA of W2 + 4 producer warps for the A tile
+      mbar_init(&bars[GB_FULL + s], 1 + F2_PRODUCER_WARPS);  // TMA of W2 + A-tile producer warps
       mbar_init(&bars[GB_EMPTY + s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -335,11 +338,16 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     if (lane == 0) gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
     __syncwarp();
   } else if (warp >= 6) {
-    // A-tile producers: Norm(AV) (.) U, bf16, 128B-swizzled K-major layout
-    const int aw = warp - 6;             // 0..3
-    const int t128 = threadIdx.x - 192;  // 0..127
-    const int sub = lane >> 3;           // row within a group of 4
-    const int c16 = lane & 7;            // 16-byte chunk within a 128-byte row
+    // A-tile producers: Norm(AV) (.) U, bf16, 128B-swizzled K-major layout.
+    // Each warp owns 16 rows of the tile; all of a k-block's loads (4 rows x
+    // 8 fp32 of AV and of U per thread) are issued before the smem stage is
+    // awaited, so a whole k-block (64 KB per CTA) is in flight at once.
+    const int aw = warp - 6;                 // 0..F2_PRODUCER_WARPS-1
+    const int tp = threadIdx.x - 6 * 32;     // 0..255
+    const int sub = lane >> 3;               // row within a group of 4
+    const int c16 = lane & 7;                // 16-byte chunk within a 128-byte row
+    constexpr int kRowsPerWarp = G_BM / F2_PRODUCER_WARPS;  // 16
+    constexpr int kIters = kRowsPerWarp / 4;                // 4
     const float inv_cnt = 1.0f / static_cast<float>(p.K);
     const float inv_hd = 1.0f / 64.0f;
     int stage = 0;
@@ -352,32 +360,42 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       const int64_t m0 = static_cast<int64_t>(mt) * G_BM;
       // per-row LayerNorm statistics combined from per-head partial sums
       {
-        const int64_t row = m0 + t128;
-        float mean = 0.0f, rstd = 0.0f;
-        if (row < p.M) {
-          const float2* lp = reinterpret_cast<const float2*>(p.ln_part + row * p.H * 2);
-          float tot = 0.0f;
-          for (int hh = 0; hh < p.H; ++hh) tot += lp[hh].x;
-          mean = tot * inv_cnt;
-          float m2 = 0.0f;
-          for (int hh = 0; hh < p.H; ++hh) {
-            const float2 v = lp[hh];
-            const float dm = v.x * inv_hd - mean;
-            m2 += v.y + 64.0f * dm * dm;
+        named_barrier_sync(1, 32 * F2_PRODUCER_WARPS);  // previous tile's readers are done
+        if (tp < G_BM) {
+          const int64_t row = m0 + tp;
+          float mean = 0.0f, rstd = 0.0f;
+          if (row < p.M) {
+            const float2* lp = reinterpret_cast<const float2*>(p.ln_part + row * p.H * 2);
+            float tot = 0.0f;
+            for (int hh = 0; hh < p.H; ++hh) tot += lp[hh].x;
+            mean = tot * inv_cnt;
+            float m2 = 0.0f;
+            for (int hh = 0; hh < p.H; ++hh) {
+              const float2 v = lp[hh];
+              const float dm = v.x * inv_hd - mean;
+              m2 += v.y + 64.0f * dm * dm;
+            }
+            rstd = rsqrtf(m2 * inv_cnt + p.eps);
           }
-          rstd = rsqrtf(m2 * inv_cnt + p.eps);
+          sStats[tp] = make_float2(mean, rstd);
         }
-        named_barrier_sync(1, 128);  // previous tile's readers are done with sStats
-        sStats[t128] = make_float2(mean, rstd);
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, 32 * F2_PRODUCER_WARPS);
       }
       for (int kb = 0; kb < k_blocks && ok; ++kb) {
-        int wok = 0;
-        if (lane == 0) wok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
-        if (!ok) break;
-        uint8_t* a_tile = sA + stage * G_A_BYTES;
         const int col = kb * G_BK + c16 * 8;
+        float4 av[kIters][2], uv[kIters][2];
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+          const int64_t row = m0 + aw * kRowsPerWarp + it * 4 + sub;
+          if (row < p.M) {
+            const float4* ap = reinterpret_cast<const float4*>(p.av + row * p.ld_av + col);
+            const float4* up = reinterpret_cast<const float4*>(p.u + row * p.ld_u + col);
+            av[it][0] = ap[0]; av[it][1] = ap[1];
+            uv[it][0] = up[0]; uv[it][1] = up[1];
+          } else {
+            av[it][0] = av[it][1] = uv[it][0] = uv[it][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
         float gm[8], bt[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) { gm[e] = 1.0f; bt[e] = 0.0f; }
@@ -393,29 +411,30 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           bt[0] = b0.x; bt[1] = b0.y; bt[2] = b0.z; bt[3] = b0.w;
           bt[4] = b1.x; bt[5] = b1.y; bt[6] = b1.z; bt[7] = b1.w;
         }
-#pragma unroll 2
-        for (int it = 0; it < 8; ++it) {
-          const int r = aw * 32 + it * 4 + sub;
-          const int64_t row = m0 + r;
-          uint4 outv = make_uint4(0u, 0u, 0u, 0u);
-          if (row < p.M) {
-            const float4* ap = reinterpret_cast<const float4*>(p.av + row * p.ld_av + col);
-            const float4* up = reinterpret_cast<const float4*>(p.u + row * p.ld_u + col);
-            const float4 a0 = ap[0], a1 = ap[1], u0 = up[0], u1 = up[1];
-            const float af[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float uf[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            const float2 st = sStats[r];
-            uint32_t w[4];
+        int wok = 0;
+        if (lane == 0) wok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
+        if (!ok) break;
+        uint8_t* a_tile = sA + stage * G_A_BYTES;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float g0 = fmaf((af[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf[2 * e];
-              const float g1 =
-                  fmaf((af[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
-              w[e] = pack_bf16x2(g0, g1);
-            }
-            outv = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int it = 0; it < kIters; ++it) {
+          const int r = aw * kRowsPerWarp + it * 4 + sub;
+          const float2 st = sStats[r];
+          const float af[8] = {av[it][0].x, av[it][0].y, av[it][0].z, av[it][0].w,
+                               av[it][1].x, av[it][1].y, av[it][1].z, av[it][1].w};
+          const float uf[8] = {uv[it][0].x, uv[it][0].y, uv[it][0].z, uv[it][0].w,
+                               uv[it][1].x, uv[it][1].y, uv[it][1].z, uv[it][1].w};
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g0 = fmaf((af[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf[2 * e];
+            const float g1 =
+                fmaf((af[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
+            w4[e] = pack_bf16x2(g0, g1);
           }
-          *reinterpret_cast<uint4*>(a_tile + r * 128 + ((c16 ^ (r & 7)) << 4)) = outv;
+          // rows past the end carry zeros (their stats are zero and the data too)
+          *reinterpret_cast<uint4*>(a_tile + r * 128 + ((c16 ^ (r & 7)) << 4)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

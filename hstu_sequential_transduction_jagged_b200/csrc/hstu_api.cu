@@ -504,7 +504,7 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
   ProfScope prof(K_F2, st);
-  hstu_f2_kernel<<<grid, 320, GemmSmem::kBytes, st>>>(mw, p);
+  hstu_f2_kernel<<<grid, F2_THREADS, GemmSmem::kBytes, st>>>(mw, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
