@@ -36,7 +36,10 @@ WORKLOAD_TEXT = {
     "sl-bf16": "4 HSTU layers bf16, d_model 512, 8 heads x 64, 64 users, Stochastic Length "
                "(alpha 1.6) subsample of 4096",
     "tiny-fp32": "1 HSTU layer fp32, d_model 64, 1 head x 64, 4 users, lengths U{8..64}",
+    "mfalcon": "M-FALCON ranking: 4 HSTU layers bf16, d_model 512, 8 heads x 64, 16 users x 4096 "
+               "cached history, 2048 candidates per user in microbatches of 256",
 }
+MFALCON_METRIC = "M-FALCON candidate scores/sec at 1 B200 (cached history K/V)"
 
 
 def load_peaks():
@@ -183,6 +186,135 @@ def traffic_from_profiles(kernel: str):
         return None
 
 
+def run_mfalcon(args, rank, world, local):
+    """Time mfalcon_score over every candidate of the M-FALCON workload (the
+    history is encoded once beforehand, with its K/V kept per layer)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from gen import make_case
+    from gen.device import case_tensors
+    from hstu_sequential_transduction_jagged_b200 import build as hbuild
+    from hstu_sequential_transduction_jagged_b200 import hstu as H
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        hbuild.build()
+    if world > 1:
+        dist.barrier()
+    case = make_case("mfalcon", batch=args.batch)
+    c = case.cfg
+    t = case_tensors(case, dev)
+    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
+    weights = [H.LayerWeights(**lw) for lw in t["layers"]]
+    cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets)
+    L, T, hv = c.num_layers, case.total_tokens, c.num_heads * 64
+    M = t["cand_emb"].shape[0]
+    kv = torch.empty((L, T, 2 * hv), dtype=torch.bfloat16, device=dev)
+    ws_h = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=dev)
+    ws_c = torch.empty(H.mfalcon_workspace_bytes(cfg, M), dtype=torch.uint8, device=dev)
+    scores = torch.empty(M, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    # history encode (timed on its own)
+    for _ in range(2):
+        H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv, workspace=ws_h)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv, workspace=ws_h)
+    b.record(stream)
+    torch.cuda.synchronize()
+    hist_ms = a.elapsed_time(b)
+
+    def step(emb):
+        H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], emb, t["request_ts"],
+                        c.microbatch, c.num_cand, scores=scores, workspace=ws_c)
+
+    for _ in range(args.warmup):
+        step(t["cand_emb"])
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    H.profiler_start()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step(t["cand_emb"])
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    kernels = H.profiler_stop()
+    clocks = sampler.stop()
+    assert H.device_status() == 0
+    total_ms = sum(x.elapsed_time(y) for x, y in evs)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms = total_ms / args.steps
+    value = world * M / (ms / 1000.0)
+    # end to end: candidate embeddings in, scores out
+    emb_host = t["cand_emb"].cpu().pin_memory()
+    sc_host = torch.empty(M, dtype=torch.float32).pin_memory()
+    emb_dev = torch.empty_like(t["cand_emb"])
+
+    def e2e_step():
+        emb_dev.copy_(emb_host, non_blocking=True)
+        step(emb_dev)
+        sc_host.copy_(scores, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e_ms = a.elapsed_time(b) / n_e2e
+    peaks, peak_src = load_peaks()
+    peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    n_u = case.lengths.astype(np.float64)
+    cand_flop = float(((n_u + 1) * c.num_cand).sum()) * c.num_heads * 256  # per layer
+    ca_n, ca_ms = kernels.get("mfalcon_attention", (0, 0.0))
+    ca_tf = cand_flop / (ca_ms / ca_n / 1000.0) / 1e12 if ca_n else None
+    kern = {k: {"launches": n, "ms_per_launch": m / n} for k, (n, m) in kernels.items()}
+    line = {"metric": MFALCON_METRIC, "value": value, "unit": "candidates/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT["mfalcon"], "candidates_per_step": world * M,
+                       "history_tokens": T, "layers": L, "microbatch": c.microbatch,
+                       "l2": "flushed between timed steps (256 MiB write outside the events)",
+                       "parallelism": f"dp{world}: users sharded, no collective"},
+            "history_encode_ms": hist_ms,
+            "roofline": {"kernel": "hstu_attn_kernel (candidate)", "bound": "tensor",
+                         "achieved": ca_tf, "peak": peak_sus, "unit": "TFLOP/s",
+                         "frac": ca_tf / peak_sus if ca_tf else None, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 dense, sustained",
+                         "algorithmic_flop_per_launch": cand_flop},
+            "kernels": kern, "gpu_launches": sum(n for n, _ in kernels.values()),
+            "clocks": clocks,
+            "e2e": {"value": world * M / (e_ms / 1000.0), "unit": "candidates/s",
+                    "ms_per_step": e_ms, "h2d_bytes_per_step": int(emb_host.numel() * 2),
+                    "d2h_bytes_per_step": int(M * 4)}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -205,6 +337,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload == "mfalcon":
+        run_mfalcon(args, rank, world, local)
         return
 
     import numpy as np
