@@ -15,9 +15,12 @@
 //   warp 8     producer: TMA loads of Q, K, V tiles (128B swizzle) and the
 //              per-key side data (timestamps, or candidate-mode bias)
 //   warp 9     MMA issuer (one thread) and TMEM owner
-// Tensor memory (448 of 512 columns): S_A, S_B (128 fp32 columns each; P,
-// bf16 pairs, overwrites the first 64 columns of its S once they are read),
-// O_A, O_B (64 fp32 columns each), Q_A, Q_B (32 columns each, bf16 pairs).
+// Key tiles are 64 keys.  Tensor memory (448 of 512 columns): two S buffers
+// per group (64 fp32 columns each; P, bf16 pairs, overwrites the first 32
+// columns of its S once they are read), O_A, O_B (64 fp32 columns each),
+// Q_A, Q_B (32 columns each, bf16 pairs).  With two S buffers the MMA warp
+// computes S of tile k+1 while the group works on tile k, so a group never
+// waits for the MMA round trip.
 // Q is written to tensor memory once per CTA by the softmax threads, so the
 // QK^T MMA reads only K from shared memory (an M=128, N=128 MMA with both
 // operands in shared memory would need the whole shared-memory bandwidth).
@@ -45,13 +48,13 @@
 namespace hstu {
 
 constexpr int ATT_ROWS = 128;
-constexpr int ATT_KEYS = 128;
+constexpr int ATT_KEYS = 64;
 constexpr int ATT_HD = 64;
-constexpr int ATT_STAGES = 3;
+constexpr int ATT_STAGES = 6;
 constexpr int ATT_THREADS = 320;
 constexpr int MAX_TIME_BUCKETS = 256;
 
-constexpr uint32_t ATT_TILE_BYTES = ATT_ROWS * ATT_HD * 2;  // 16 KB
+constexpr uint32_t ATT_TILE_BYTES = ATT_KEYS * ATT_HD * 2;  // one K or V tile: 8 KB
 
 struct AttnParams {
   const int64_t* kv_offsets;   // [B+1] key/value rows per user (query rows too in causal mode)
@@ -181,10 +184,10 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t w, int c, int last) {
 // ---------------------------------------------------------------- shared memory
 
 struct AttnSmem {
-  static constexpr uint32_t kK = 0;                                   // stages x 16 KB
-  static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 16 KB
-  static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 1 KB
-  static constexpr uint32_t kKeyStride = ATT_KEYS * 8;                // bytes per stage
+  static constexpr uint32_t kK = 0;                                   // stages x 8 KB
+  static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 8 KB
+  static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 256 B
+  static constexpr uint32_t kKeyStride = ATT_KEYS * 4;                // bytes per stage
   static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * kKeyStride;
   static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
   static constexpr uint32_t kOct = kThr + MAX_TIME_BUCKETS * 8;      // 32 x int4
@@ -201,9 +204,9 @@ enum : int {
   BAR_Q_FULL = 0,
   BAR_KV_FULL = 1,                     // + stage
   BAR_KV_EMPTY = BAR_KV_FULL + ATT_STAGES,
-  BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + group
-  BAR_P_FULL = BAR_S_FULL + 2,             // + group
-  BAR_O_FULL = BAR_P_FULL + 2,
+  BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + 2 * group + buffer
+  BAR_P_FULL = BAR_S_FULL + 4,             // + 2 * group + buffer
+  BAR_O_FULL = BAR_P_FULL + 4,
   BAR_DONE = BAR_O_FULL + 1,
   BAR_COUNT = BAR_DONE + 1
 };
@@ -332,8 +335,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     nA = nk;
     nB = has_b ? nk : 0;
   } else {
-    nA = 2 * qp + 1;
-    nB = has_b ? 2 * qp + 2 : 0;
+    nA = (q0 + ATT_ROWS) / ATT_KEYS;      // keys 0 .. q0 + 127
+    nB = has_b ? (q0 + 2 * ATT_ROWS) / ATT_KEYS : 0;
   }
   const int nk_total = nA > nB ? nA : nB;
 
@@ -374,8 +377,12 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(&bars[BAR_KV_EMPTY + s], 1);
     }
     for (int g = 0; g < 2; ++g) {
-      mbar_init(&bars[BAR_S_FULL + g], 1);
-      mbar_init(&bars[BAR_P_FULL + g], ATT_ROWS);
+      // one S-ready and one P-ready barrier per S buffer: a group can run a
+      // tile ahead of the MMA warp, but never two phases ahead on one barrier
+      mbar_init(&bars[BAR_S_FULL + 2 * g], 1);
+      mbar_init(&bars[BAR_S_FULL + 2 * g + 1], 1);
+      mbar_init(&bars[BAR_P_FULL + 2 * g], ATT_ROWS);
+      mbar_init(&bars[BAR_P_FULL + 2 * g + 1], ATT_ROWS);
     }
     mbar_init(&bars[BAR_O_FULL], 1);
     mbar_init(&bars[BAR_DONE], 1);
@@ -388,7 +395,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   }
   {
     const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
-    const int xend = min(p.pos_len, D + ATT_KEYS + 2);
+    const int xend = min(p.pos_len, D + ATT_ROWS + 2);
     for (int x = tid; x < xend; x += ATT_THREADS) {
       const int d0 = D - x;  // copy 0 holds offset D - x
       sRv[x] = (d0 >= 0) ? kScale * rp[min(d0, p.P - 1)] : 0.0f;
@@ -468,58 +475,62 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
       bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
       tc_fence_after();
-      auto issue_s = [&](int g, int s) {
+      // S of tile kt for group g into buffer kt & 1
+      auto issue_s = [&](int g, int kt) {
         const uint32_t qa = tmem + 384u + static_cast<uint32_t>(g * 32);
-        const uint32_t ka = smem_u32(sK + s * ATT_TILE_BYTES);
-        const uint32_t d = tmem + static_cast<uint32_t>(g * 128);
+        const uint32_t ka = smem_u32(sK + (kt % ATT_STAGES) * ATT_TILE_BYTES);
+        const uint32_t d = tmem + static_cast<uint32_t>(g * 128 + (kt & 1) * 64);
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk) {
           mma_bf16_ts(d, qa + kk * 8, smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk,
                       kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[BAR_S_FULL + g]);
+        mma_commit(&bars[BAR_S_FULL + 2 * g + (kt & 1)]);
       };
-      auto issue_pv = [&](int g, int s, bool first) {
-        const uint32_t va = smem_u32(sV + s * ATT_TILE_BYTES);
+      // O_g += P(kt) V(kt); P sits over the S buffer of tile kt
+      auto issue_pv = [&](int g, int kt) {
+        const uint32_t va = smem_u32(sV + (kt % ATT_STAGES) * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256u + static_cast<uint32_t>(g * 64);
-        const uint32_t a = tmem + static_cast<uint32_t>(g * 128);  // P over S
+        const uint32_t a = tmem + static_cast<uint32_t>(g * 128 + (kt & 1) * 64);
 #pragma unroll
         for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
           mma_bf16_ts(d, a + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
-                      (first && kk == 0) ? 0u : 1u);
+                      (kt == 0 && kk == 0) ? 0u : 1u);
         }
       };
-      if (ok && nk_total > 0) {
-        ok = mbar_wait(&bars[BAR_KV_FULL + 0], 0, ctl);
-        tc_fence_after();
-        if (ok) {
-          if (nA > 0) issue_s(0, 0);
-          if (nB > 0) issue_s(1, 0);
+      const int nW[2] = {nA, nB};
+      int kv_ready = 0;  // key tiles whose K/V have been awaited
+      auto await_kv = [&](int kt) -> bool {
+        while (kv_ready <= kt) {
+          if (!mbar_wait(&bars[BAR_KV_FULL + kv_ready % ATT_STAGES],
+                         static_cast<uint32_t>(kv_ready / ATT_STAGES) & 1u, ctl))
+            return false;
+          tc_fence_after();
+          ++kv_ready;
         }
+        return true;
+      };
+      // two tiles ahead per group: S(0), S(1) before any P exists
+      for (int t = 0; ok && t < 2 && t < nk_total; ++t) {
+        ok = await_kv(t);
+        for (int g = 0; ok && g < 2; ++g)
+          if (t < nW[g]) issue_s(g, t);
       }
       for (int kt = 0; ok && kt < nk_total; ++kt) {
-        const int s = kt % ATT_STAGES;
-        bool next_ready = false;
         for (int g = 0; g < 2 && ok; ++g) {
-          const int nW = g == 0 ? nA : nB;
-          if (kt >= nW) continue;
-          ok = mbar_wait(&bars[BAR_P_FULL + g], static_cast<uint32_t>(kt) & 1u, ctl);
+          if (kt >= nW[g]) continue;
+          ok = mbar_wait(&bars[BAR_P_FULL + 2 * g + (kt & 1)], static_cast<uint32_t>(kt >> 1) & 1u,
+                         ctl);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(g, s, kt == 0);
-          if (kt + 1 < nW) {
-            if (!next_ready) {
-              const int s1 = (kt + 1) % ATT_STAGES;
-              ok = mbar_wait(&bars[BAR_KV_FULL + s1],
-                             static_cast<uint32_t>((kt + 1) / ATT_STAGES) & 1u, ctl);
-              if (!ok) break;
-              tc_fence_after();
-              next_ready = true;
-            }
-            issue_s(g, (kt + 1) % ATT_STAGES);
+          issue_pv(g, kt);
+          if (kt + 2 < nW[g]) {
+            ok = await_kv(kt + 2);
+            if (!ok) break;
+            issue_s(g, kt + 2);  // into the buffer PV(kt) has just been issued to read
           }
         }
-        if (ok) mma_commit(&bars[BAR_KV_EMPTY + s]);
+        if (ok) mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
       }
       mma_commit(&bars[BAR_O_FULL]);
       // every MMA of this CTA must be complete before TMEM is released
@@ -532,8 +543,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const int g = warp >> 2;               // 0 = tile A, 1 = tile B
     const int r = tid & (ATT_ROWS - 1);    // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(g * 128);
-    const uint32_t tP = tS;  // P overwrites the S columns it was computed from
+    const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(g * 128);  // buffer 0; +64: 1
     const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64);
     const uint32_t tQ = tmem + lane_off + 384u + static_cast<uint32_t>(g * 32);
     const int i = q0 + g * ATT_ROWS + r;   // query index within the user
@@ -574,8 +584,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
 
     // one 32-key chunk: S values in `sv`, packed bf16 P pairs to `pk`
-    auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int ch, int s,
-                     bool diag) {
+    auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int ch, int s) {
       const uint8_t* key = sKey + s * AttnSmem::kKeyStride;
       if constexpr (CAND) {
         const float* kr = reinterpret_cast<const float*>(key) + ch * 32;
@@ -592,9 +601,9 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       } else {
         const int xc = D - i + kt * ATT_KEYS + ch * 32 + copy;  // table index at column 0
-        // last visible column: the diagonal masks keys after the row; rows past
-        // the user's end are not stored and skip the work
-        const int lim = !valid ? -1 : (diag ? r - ch * 32 : 31);
+        // last visible column: keys after the row are masked; rows past the
+        // user's end are not stored and skip the work
+        const int lim = !valid ? -1 : i - (kt * ATT_KEYS + ch * 32);
         causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + ch * 32,
                                  lim, w32, sTime, sThr, sOct, scale2);
       }
@@ -602,27 +611,27 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     for (int kt = 0; kt < nW; ++kt) {
       const int s = kt % ATT_STAGES;
-      ok = mbar_wait(&bars[BAR_S_FULL + g], static_cast<uint32_t>(kt) & 1u, ctl);
+      ok = mbar_wait(&bars[BAR_S_FULL + 2 * g + (kt & 1)], static_cast<uint32_t>(kt >> 1) & 1u, ctl);
       // the producer's per-key side data for this stage (already complete)
       if (ok)
         ok = mbar_wait(&bars[BAR_KV_FULL + s], static_cast<uint32_t>(kt / ATT_STAGES) & 1u, ctl);
       ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-collective
       if (!ok) break;
       tc_fence_after();
-      const bool diag = !CAND && (kt == 2 * qp + g);
-      // four chunks of 32 keys: TMEM -> registers -> bias, phi2, mask -> P back to TMEM
+      const uint32_t tS = tS0 + static_cast<uint32_t>((kt & 1) * 64);
+      // two chunks of 32 keys: TMEM -> registers -> bias, phi2, mask -> P over S
       uint32_t sa[32], pk[16];
 #pragma unroll 1
       for (int ch = 0; ch < ATT_KEYS / 32; ++ch) {
         tmem_ld32(tS + ch * 32, sa);
         tmem_ld_wait(sa);
-        chunk(sa, pk, kt, ch, s, diag);
+        chunk(sa, pk, kt, ch, s);
         __syncwarp();
-        tmem_st16(tP + ch * 16, pk);
+        tmem_st16(tS + ch * 16, pk);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[BAR_P_FULL + g]);
+      mbar_arrive(&bars[BAR_P_FULL + 2 * g + (kt & 1)]);
     }
 
     // ---------------- epilogue: O / N, LayerNorm partial sums, store

@@ -406,7 +406,7 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
                            : align_up(static_cast<size_t>(j.max_q_len), 2 * ATT_ROWS);
   // per-copy length = 16 (mod 32) floats: the two copies' 8-byte pair reads
   // by neighbouring lanes then fall in disjoint shared-memory banks
-  p.pos_len = static_cast<int32_t>(align_up(dmax + ATT_KEYS + 2, 32) + 16);
+  p.pos_len = static_cast<int32_t>(align_up(dmax + ATT_ROWS + 2, 32) + 16);
   p.phi2 = c->phi2;
   p.timeout_ns = j.timeout_ns;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
