@@ -9,18 +9,23 @@
 // inside it; candidate mode (M-FALCON) lets candidate rows see every cached
 // history key and adds each candidate's own key/value in the epilogue.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax group A: thread t owns query row t of tile A
-//   warps 4-7  softmax group B: thread t owns query row t of tile B
-//   warp 8     producer: TMA loads of Q, K, V tiles (128B swizzle) and the
-//              per-key side data (timestamps, or candidate-mode bias)
-//   warp 9     MMA issuer (one thread) and TMEM owner
+// Warp roles (576 threads):
+//   warps 0-7   element group A (query tile A): warps 0-3 own key columns
+//               0-31 of every S tile, warps 4-7 columns 32-63; within each
+//               warpgroup thread t owns query row t
+//   warps 8-15  element group B, the same for tile B
+//   warp 16     producer: TMA loads of K, V tiles (128B swizzle) and the
+//               per-key side data (timestamps, or candidate-mode bias)
+//   warp 17     MMA issuer (one thread) and TMEM owner
+// Two warpgroups per query tile halve the elements each thread handles per
+// key tile and double the warps that hide tensor-memory, shared-memory and
+// MUFU latency; the work per element is one row-thread's arithmetic either way.
 // Key tiles are 64 keys.  Tensor memory (448 of 512 columns): two S buffers
-// per group (64 fp32 columns each; P, bf16 pairs, overwrites the first 32
-// columns of its S once they are read), O_A, O_B (64 fp32 columns each),
-// Q_A, Q_B (32 columns each, bf16 pairs).  With two S buffers the MMA warp
-// computes S of tile k+1 while the group works on tile k, so a group never
-// waits for the MMA round trip.
+// per group (64 fp32 columns each; each half writes its 32 keys of P, bf16
+// pairs, over the first 16 columns of its own 32-column half once they are
+// read), O_A, O_B (64 fp32 columns each), Q_A, Q_B (32 columns each, bf16
+// pairs).  With two S buffers the MMA warp computes S of tile k+1 while the
+// group works on tile k, so a group never waits for the MMA round trip.
 // Q is written to tensor memory once per CTA by the softmax threads, so the
 // QK^T MMA reads only K from shared memory (an M=128, N=128 MMA with both
 // operands in shared memory would need the whole shared-memory bandwidth).
@@ -51,7 +56,9 @@ constexpr int ATT_ROWS = 128;
 constexpr int ATT_KEYS = 64;
 constexpr int ATT_HD = 64;
 constexpr int ATT_STAGES = 6;
-constexpr int ATT_THREADS = 320;
+constexpr int ATT_THREADS = 576;
+constexpr int ATT_PRODUCER_WARP = 16;
+constexpr int ATT_MMA_WARP = 17;
 constexpr int MAX_TIME_BUCKETS = 256;
 
 constexpr uint32_t ATT_TILE_BYTES = ATT_KEYS * ATT_HD * 2;  // one K or V tile: 8 KB
@@ -193,7 +200,8 @@ struct AttnSmem {
   static constexpr uint32_t kOct = kThr + MAX_TIME_BUCKETS * 8;      // 32 x int4
   static constexpr uint32_t kBars = kOct + 32 * 16;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
-  static constexpr uint32_t kPos = kMisc + 64;
+  static constexpr uint32_t kLnX = kMisc + 64;                        // 2 x 128 float2
+  static constexpr uint32_t kPos = kLnX + 2 * ATT_ROWS * 8;
   static constexpr uint32_t bytes(int pos_len, bool pairs) {
     return kPos + static_cast<uint32_t>(pos_len) * 4u * (pairs ? 2u : 1u) + 1024u;  // + align slack
   }
@@ -233,16 +241,13 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
   const unsigned full = 0xffffffffu;
   const bool live = lim >= 0;
   const int last = lim < 31 ? lim : 31;
-  int32_t kt[32];
-#pragma unroll
-  for (int c = 0; c < 32; c += 4) {
-    const int4 v = *reinterpret_cast<const int4*>(kts + c);
-    kt[c] = v.x; kt[c + 1] = v.y; kt[c + 2] = v.z; kt[c + 3] = v.w;
-  }
+  // key times of a pair of columns (broadcast shared loads, only off the
+  // one-bucket path)
+  auto kt_pair = [&](int c) -> int2 { return *reinterpret_cast<const int2*>(kts + c); };
   int b_first = -1, b_last = 1 << 30;
   bool lane_steady = true;
   if (live) {
-    w.step(kt[0], sThr);
+    w.step(kts[0], sThr);
     b_first = w.b;
     const int32_t k_last = kts[last];
     lane_steady = k_last <= w.bound;
@@ -275,8 +280,9 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
             e < static_cast<int64_t>(INT32_MIN) ? INT32_MIN : static_cast<int32_t>(e);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float r0 = (kt[c] <= edge) ? rt_hi : rt_lo;
-          const float r1 = (kt[c + 1] <= edge) ? rt_hi : rt_lo;
+          const int2 k2 = kt_pair(c);
+          const float r0 = (k2.x <= edge) ? rt_hi : rt_lo;
+          const float r1 = (k2.y <= edge) ? rt_hi : rt_lo;
           pk[c >> 1] =
               phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
         }
@@ -284,8 +290,9 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
     } else if (live) {
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        const float r0 = sTime[time_bucket_octave(w.ti - kt[c], sOct)];
-        const float r1 = sTime[time_bucket_octave(w.ti - kt[c + 1], sOct)];
+        const int2 k2 = kt_pair(c);
+        const float r0 = sTime[time_bucket_octave(w.ti - k2.x, sOct)];
+        const float r1 = sTime[time_bucket_octave(w.ti - k2.y, sOct)];
         pk[c >> 1] =
             phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
       }
@@ -354,6 +361,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   int4* sOct = reinterpret_cast<int4*>(smem + AttnSmem::kOct);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
+  float2* sLnX = reinterpret_cast<float2*>(smem + AttnSmem::kLnX);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 4);
   float* sRv = reinterpret_cast<float*>(smem + AttnSmem::kPos);
 
@@ -381,15 +389,15 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // tile ahead of the MMA warp, but never two phases ahead on one barrier
       mbar_init(&bars[BAR_S_FULL + 2 * g], 1);
       mbar_init(&bars[BAR_S_FULL + 2 * g + 1], 1);
-      mbar_init(&bars[BAR_P_FULL + 2 * g], ATT_ROWS);
-      mbar_init(&bars[BAR_P_FULL + 2 * g + 1], ATT_ROWS);
+      mbar_init(&bars[BAR_P_FULL + 2 * g], 2 * ATT_ROWS);  // both column halves
+      mbar_init(&bars[BAR_P_FULL + 2 * g + 1], 2 * ATT_ROWS);
     }
     mbar_init(&bars[BAR_O_FULL], 1);
     mbar_init(&bars[BAR_DONE], 1);
     *sAbort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == ATT_MMA_WARP) {
     tmem_alloc(sTmemBase, 512);
     tmem_relinquish();
   }
@@ -416,7 +424,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const uint32_t tmem = *sTmemBase;
   const WaitCtl ctl{sAbort, p.timeout_ns};
 
-  if (warp == 8) {
+  if (warp == ATT_PRODUCER_WARP) {
     // ---------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
@@ -468,7 +476,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         mbar_wait_drain(&bars[BAR_KV_FULL + kt % ATT_STAGES],
                         static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == ATT_MMA_WARP) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
@@ -487,14 +495,16 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         mma_commit(&bars[BAR_S_FULL + 2 * g + (kt & 1)]);
       };
-      // O_g += P(kt) V(kt); P sits over the S buffer of tile kt
+      // O_g += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
+      // buffer of tile kt, P of keys 32-63 at columns 32-47
       auto issue_pv = [&](int g, int kt) {
         const uint32_t va = smem_u32(sV + (kt % ATT_STAGES) * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256u + static_cast<uint32_t>(g * 64);
         const uint32_t a = tmem + static_cast<uint32_t>(g * 128 + (kt & 1) * 64);
 #pragma unroll
         for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
-          mma_bf16_ts(d, a + kk * 8, smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
+          mma_bf16_ts(d, a + (kk >> 1) * 32 + (kk & 1) * 8,
+                      smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
                       (kt == 0 && kk == 0) ? 0u : 1u);
         }
       };
@@ -539,18 +549,20 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     __syncwarp();
   } else {
-    // ---------------- softmax groups
-    const int g = warp >> 2;               // 0 = tile A, 1 = tile B
+    // ---------------- element groups
+    const int g = warp >> 3;               // 0 = tile A, 1 = tile B
+    const int half = (warp >> 2) & 1;      // key columns 32*half .. 32*half + 31 of each tile
     const int r = tid & (ATT_ROWS - 1);    // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(g * 128);  // buffer 0; +64: 1
-    const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64);
+    // this half's 32 columns of S buffer 0 (+64: buffer 1)
+    const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(g * 128 + half * 32);
+    const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64 + half * 32);
     const uint32_t tQ = tmem + lane_off + 384u + static_cast<uint32_t>(g * 32);
     const int i = q0 + g * ATT_ROWS + r;   // query index within the user
     const bool valid = i < n_q;
     const int nW = g == 0 ? nA : nB;
     bool ok = true;
-    {
+    if (half == 0) {
       // this row's query (64 bf16 = 32 columns of packed pairs) into tensor memory
       uint32_t qv[32];
       if (valid) {
@@ -583,28 +595,29 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       rv = sRv + copy * p.pos_len;
     }
 
-    // one 32-key chunk: S values in `sv`, packed bf16 P pairs to `pk`
-    auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int ch, int s) {
+    // this half's 32 keys of tile kt: S values in `sv`, packed bf16 P pairs to `pk`
+    auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int s) {
       const uint8_t* key = sKey + s * AttnSmem::kKeyStride;
+      const int j0 = kt * ATT_KEYS + half * 32;  // key index of column 0
       if constexpr (CAND) {
-        const float* kr = reinterpret_cast<const float*>(key) + ch * 32;
+        const float* kr = reinterpret_cast<const float*>(key) + half * 32;
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
                                      scale2, lds_b64(kr + c));
           pk[c >> 1] = phi_pair<PHI>(h2);
         }
-        const int last = n_kv - 1 - (kt * ATT_KEYS + ch * 32);  // last live column
+        const int last = n_kv - 1 - j0;  // last live column
         if (last < 31) {
 #pragma unroll
           for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
         }
       } else {
-        const int xc = D - i + kt * ATT_KEYS + ch * 32 + copy;  // table index at column 0
+        const int xc = D - i + j0 + copy;  // table index at column 0
         // last visible column: keys after the row are masked; rows past the
         // user's end are not stored and skip the work
-        const int lim = !valid ? -1 : i - (kt * ATT_KEYS + ch * 32);
-        causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + ch * 32,
+        const int lim = !valid ? -1 : i - j0;
+        causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + half * 32,
                                  lim, w32, sTime, sThr, sOct, scale2);
       }
     };
@@ -619,48 +632,46 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (!ok) break;
       tc_fence_after();
       const uint32_t tS = tS0 + static_cast<uint32_t>((kt & 1) * 64);
-      // two chunks of 32 keys: TMEM -> registers -> bias, phi2, mask -> P over S
+      // 32 keys: TMEM -> registers -> bias, phi2, mask -> P over this half's S
       uint32_t sa[32], pk[16];
-#pragma unroll 1
-      for (int ch = 0; ch < ATT_KEYS / 32; ++ch) {
-        tmem_ld32(tS + ch * 32, sa);
-        tmem_ld_wait(sa);
-        chunk(sa, pk, kt, ch, s);
-        __syncwarp();
-        tmem_st16(tS + ch * 16, pk);
-      }
+      tmem_ld32(tS, sa);
+      tmem_ld_wait(sa);
+      chunk(sa, pk, kt, s);
+      __syncwarp();
+      tmem_st16(tS, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P_FULL + 2 * g + (kt & 1)]);
     }
 
     // ---------------- epilogue: O / N, LayerNorm partial sums, store
-    float o[ATT_HD];
+    // Each half finishes its 32 columns of O; the two halves' (sum, centred
+    // sum of squares) merge by the pairwise update for equal counts:
+    // M2 = M2_0 + M2_1 + (mean_0 - mean_1)^2 * 32 * 32 / 64.
+    constexpr int HC = ATT_HD / 2;
+    float o[HC];
     if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL], 0, ctl);
     ok = __all_sync(0xffffffffu, ok);
+    float hsum = 0.0f, hm2 = 0.0f;
+    const int64_t row = q_start + i;
     if (ok) {
       if (nW > 0) {
         tc_fence_after();
         uint32_t ov[32];
-        tmem_ld32(tO + 0, ov);
+        tmem_ld32(tO, ov);
         tmem_ld_wait(ov);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(ov[c]);
-        tmem_ld32(tO + 32, ov);
-        tmem_ld_wait(ov);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[32 + c] = __uint_as_float(ov[c]);
+        for (int c = 0; c < HC; ++c) o[c] = __uint_as_float(ov[c]);
       } else {
 #pragma unroll
-        for (int c = 0; c < ATT_HD; ++c) o[c] = 0.0f;
+        for (int c = 0; c < HC; ++c) o[c] = 0.0f;
       }
       if (valid) {
-        const int64_t row = q_start + i;
         if constexpr (CAND) {
           // the candidate's own key/value: position bucket 0, time bucket 0
           const __nv_bfloat16* qs = p.q_self + row * p.ld_self + h * ATT_HD;
           const __nv_bfloat16* ks = p.k_self + row * p.ld_self + h * ATT_HD;
-          const __nv_bfloat16* vs = p.v_self + row * p.ld_self + h * ATT_HD;
+          const __nv_bfloat16* vs = p.v_self + row * p.ld_self + h * ATT_HD + half * HC;
           float dot = 0.0f;
 #pragma unroll
           for (int c = 0; c < ATT_HD; c += 8) {
@@ -680,7 +691,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                               p.rab_time[static_cast<int64_t>(h) * p.Tb]);
           const float ps = apply_phi<PHI>(dot + rab0);
 #pragma unroll
-          for (int c = 0; c < ATT_HD; c += 8) {
+          for (int c = 0; c < HC; c += 8) {
             uint4 va = *reinterpret_cast<const uint4*>(vs + c);
             const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&va);
 #pragma unroll
@@ -692,28 +703,26 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           }
         }
         const float inv_n = 1.0f / static_cast<float>(CAND ? max(n_kv, 1) : n_kv);
-        float sum = 0.0f;
 #pragma unroll
-        for (int c = 0; c < ATT_HD; ++c) {
+        for (int c = 0; c < HC; ++c) {
           o[c] *= inv_n;
-          sum += o[c];
+          hsum += o[c];
         }
-        const float mean = sum * (1.0f / ATT_HD);
-        float m2 = 0.0f;
+        const float mean = hsum * (1.0f / HC);
 #pragma unroll
-        for (int c = 0; c < ATT_HD; ++c) {
+        for (int c = 0; c < HC; ++c) {
           const float dlt = o[c] - mean;
-          m2 = fmaf(dlt, dlt, m2);
+          hm2 = fmaf(dlt, dlt, hm2);
         }
         if (p.av_f32 != nullptr) {
-          float4* dst = reinterpret_cast<float4*>(p.av_f32 + row * p.ld_av + h * ATT_HD);
+          float4* dst = reinterpret_cast<float4*>(p.av_f32 + row * p.ld_av + h * ATT_HD + half * HC);
 #pragma unroll
-          for (int c = 0; c < ATT_HD; c += 4)
+          for (int c = 0; c < HC; c += 4)
             dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         } else {
-          __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD;
+          __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD + half * HC;
 #pragma unroll
-          for (int c = 0; c < ATT_HD; c += 8) {
+          for (int c = 0; c < HC; c += 8) {
             uint4 pkt;
             pkt.x = pack_bf16x2(o[c + 0], o[c + 1]);
             pkt.y = pack_bf16x2(o[c + 2], o[c + 3]);
@@ -722,18 +731,23 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             *reinterpret_cast<uint4*>(dst + c) = pkt;
           }
         }
-        if (p.ln_part != nullptr) {
-          float2* lp = reinterpret_cast<float2*>(p.ln_part + (row * p.H + h) * 2);
-          *lp = make_float2(sum, m2);
-        }
       }
+    }
+    // every thread of the group's 256 reaches this barrier (no early exit)
+    if (half == 1) sLnX[g * ATT_ROWS + r] = make_float2(hsum, hm2);
+    named_barrier_sync(1 + g, 2 * ATT_ROWS);
+    if (half == 0 && ok && valid && p.ln_part != nullptr) {
+      const float2 other = sLnX[g * ATT_ROWS + r];
+      const float dm = (hsum - other.x) * (1.0f / HC);
+      float2* lp = reinterpret_cast<float2*>(p.ln_part + (row * p.H + h) * 2);
+      *lp = make_float2(hsum + other.x, hm2 + other.y + dm * dm * (HC * HC / (2.0f * HC)));
     }
   }
 
   // ---------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == ATT_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
