@@ -16,7 +16,12 @@
 //   warps 8-15  element group B, the same for tile B
 //   warp 16     producer: TMA loads of K, V tiles (128B swizzle) and the
 //               per-key side data (timestamps, or candidate-mode bias)
-//   warp 17     MMA issuer (one thread) and TMEM owner
+//   warp 17     MMA issuer of tile A (one thread) and TMEM owner
+//   warp 18     MMA issuer of tile B (one thread)
+// One issuing thread per query tile: a single thread issuing both tiles'
+// MMAs, with an mbarrier wait in front of every batch, could not keep the
+// tensor pipe fed.  The two issuers touch disjoint tensor memory; a K/V stage
+// is released by one commit from each.
 // Two warpgroups per query tile halve the elements each thread handles per
 // key tile and double the warps that hide tensor-memory, shared-memory and
 // MUFU latency; the work per element is one row-thread's arithmetic either way.
@@ -56,9 +61,9 @@ constexpr int ATT_ROWS = 128;
 constexpr int ATT_KEYS = 64;
 constexpr int ATT_HD = 64;
 constexpr int ATT_STAGES = 6;
-constexpr int ATT_THREADS = 576;
+constexpr int ATT_THREADS = 608;
 constexpr int ATT_PRODUCER_WARP = 16;
-constexpr int ATT_MMA_WARP = 17;
+constexpr int ATT_MMA_WARP = 17;  // + query tile (A: 17, B: 18)
 constexpr int MAX_TIME_BUCKETS = 256;
 
 constexpr uint32_t ATT_TILE_BYTES = ATT_KEYS * ATT_HD * 2;  // one K or V tile: 8 KB
@@ -214,9 +219,9 @@ enum : int {
   BAR_KV_EMPTY = BAR_KV_FULL + ATT_STAGES,
   BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + 2 * group + buffer
   BAR_P_FULL = BAR_S_FULL + 4,             // + 2 * group + buffer
-  BAR_O_FULL = BAR_P_FULL + 4,
-  BAR_DONE = BAR_O_FULL + 1,
-  BAR_COUNT = BAR_DONE + 1
+  BAR_O_FULL = BAR_P_FULL + 4,             // + group
+  BAR_DONE = BAR_O_FULL + 2,               // + group
+  BAR_COUNT = BAR_DONE + 2
 };
 
 // ---------------------------------------------------------------- causal chunk
@@ -382,7 +387,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     mbar_init(&bars[BAR_Q_FULL], 2 * ATT_ROWS);  // every softmax thread stores its Q row
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&bars[BAR_KV_FULL + s], 2);
-      mbar_init(&bars[BAR_KV_EMPTY + s], 1);
+      mbar_init(&bars[BAR_KV_EMPTY + s], 2);  // one commit per issuer
     }
     for (int g = 0; g < 2; ++g) {
       // one S-ready and one P-ready barrier per S buffer: a group can run a
@@ -392,8 +397,10 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(&bars[BAR_P_FULL + 2 * g], 2 * ATT_ROWS);  // both column halves
       mbar_init(&bars[BAR_P_FULL + 2 * g + 1], 2 * ATT_ROWS);
     }
-    mbar_init(&bars[BAR_O_FULL], 1);
-    mbar_init(&bars[BAR_DONE], 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bars[BAR_O_FULL + g], 1);
+      mbar_init(&bars[BAR_DONE + g], 1);
+    }
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -476,40 +483,25 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         mbar_wait_drain(&bars[BAR_KV_FULL + kt % ATT_STAGES],
                         static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
     }
-  } else if (warp == ATT_MMA_WARP) {
-    // ---------------- MMA issuer
+  } else if (warp >= ATT_MMA_WARP) {
+    // ---------------- MMA issuers, one thread per query tile
+    const int g = warp - ATT_MMA_WARP;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
+      const int nWg = g == 0 ? nA : nB;
+      // tensor memory: S buffers (P over them), O, Q of this tile
+      const uint32_t tS = tmem + static_cast<uint32_t>(g * 128);
+      const uint32_t tOg = tmem + 256u + static_cast<uint32_t>(g * 64);
+      const uint32_t tQg = tmem + 384u + static_cast<uint32_t>(g * 32);
+      // descriptors of stage 0; stage s adds s * 8 KB (s * 512 in 16-byte
+      // units) to the start-address field
+      const uint64_t dK0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_u32(sV), 8192, 1024);
+      constexpr uint64_t kStageDesc = ATT_TILE_BYTES >> 4;
       bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
       tc_fence_after();
-      // S of tile kt for group g into buffer kt & 1
-      auto issue_s = [&](int g, int kt) {
-        const uint32_t qa = tmem + 384u + static_cast<uint32_t>(g * 32);
-        const uint32_t ka = smem_u32(sK + (kt % ATT_STAGES) * ATT_TILE_BYTES);
-        const uint32_t d = tmem + static_cast<uint32_t>(g * 128 + (kt & 1) * 64);
-#pragma unroll
-        for (int kk = 0; kk < ATT_HD / 16; ++kk) {
-          mma_bf16_ts(d, qa + kk * 8, smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[BAR_S_FULL + 2 * g + (kt & 1)]);
-      };
-      // O_g += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
-      // buffer of tile kt, P of keys 32-63 at columns 32-47
-      auto issue_pv = [&](int g, int kt) {
-        const uint32_t va = smem_u32(sV + (kt % ATT_STAGES) * ATT_TILE_BYTES);
-        const uint32_t d = tmem + 256u + static_cast<uint32_t>(g * 64);
-        const uint32_t a = tmem + static_cast<uint32_t>(g * 128 + (kt & 1) * 64);
-#pragma unroll
-        for (int kk = 0; kk < ATT_KEYS / 16; ++kk) {
-          mma_bf16_ts(d, a + (kk >> 1) * 32 + (kk & 1) * 8,
-                      smem_desc_sw128(va + kk * 2048, 8192, 1024), idesc_pv,
-                      (kt == 0 && kk == 0) ? 0u : 1u);
-        }
-      };
-      const int nW[2] = {nA, nB};
-      int kv_ready = 0;  // key tiles whose K/V have been awaited
+      int kv_ready = 0;  // key tiles whose K/V this thread has seen land
       auto await_kv = [&](int kt) -> bool {
         while (kv_ready <= kt) {
           if (!mbar_wait(&bars[BAR_KV_FULL + kv_ready % ATT_STAGES],
@@ -520,32 +512,55 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         return true;
       };
-      // two tiles ahead per group: S(0), S(1) before any P exists
-      for (int t = 0; ok && t < 2 && t < nk_total; ++t) {
+      // S of tile kt into buffer kt & 1
+      auto issue_s = [&](int kt) {
+        const uint64_t dk = dK0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
+        const uint32_t d = tS + static_cast<uint32_t>((kt & 1) * 64);
+#pragma unroll
+        for (int kk = 0; kk < ATT_HD / 16; ++kk)
+          mma_bf16_ts(d, tQg + kk * 8, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[BAR_S_FULL + 2 * g + (kt & 1)]);
+      };
+      // O += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
+      // buffer of tile kt, P of keys 32-63 at columns 32-47
+      auto issue_pv = [&](int kt) {
+        const uint64_t dv = dV0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
+        const uint32_t a = tS + static_cast<uint32_t>((kt & 1) * 64);
+        const uint32_t acc0 = kt > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < ATT_KEYS / 16; ++kk)
+          mma_bf16_ts(tOg, a + (kk >> 1) * 32 + (kk & 1) * 8, dv + 128 * kk, idesc_pv,
+                      kk > 0 ? 1u : acc0);
+      };
+      // two tiles ahead: S(0), S(1) before any P exists
+      for (int t = 0; ok && t < 2 && t < nWg; ++t) {
         ok = await_kv(t);
-        for (int g = 0; ok && g < 2; ++g)
-          if (t < nW[g]) issue_s(g, t);
+        if (ok) issue_s(t);
       }
       for (int kt = 0; ok && kt < nk_total; ++kt) {
-        for (int g = 0; g < 2 && ok; ++g) {
-          if (kt >= nW[g]) continue;
+        if (kt < nWg) {
           ok = mbar_wait(&bars[BAR_P_FULL + 2 * g + (kt & 1)], static_cast<uint32_t>(kt >> 1) & 1u,
                          ctl);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(g, kt);
-          if (kt + 2 < nW[g]) {
+          issue_pv(kt);
+          if (kt + 2 < nWg) {
             ok = await_kv(kt + 2);
             if (!ok) break;
-            issue_s(g, kt + 2);  // into the buffer PV(kt) has just been issued to read
+            issue_s(kt + 2);  // into the buffer P V(kt) has just been issued to read
           }
+        } else {
+          // past this tile's last key tile: the release below must still
+          // follow the stage's load, so it counts toward this tile's phase
+          ok = await_kv(kt);
+          if (!ok) break;
         }
-        if (ok) mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
+        mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
       }
-      mma_commit(&bars[BAR_O_FULL]);
-      // every MMA of this CTA must be complete before TMEM is released
-      mma_commit(&bars[BAR_DONE]);
-      mbar_wait_drain(&bars[BAR_DONE], 0, p.timeout_ns);
+      mma_commit(&bars[BAR_O_FULL + g]);
+      // every MMA of this thread must be complete before TMEM is released
+      mma_commit(&bars[BAR_DONE + g]);
+      mbar_wait_drain(&bars[BAR_DONE + g], 0, p.timeout_ns);
     }
     __syncwarp();
   } else {
@@ -650,7 +665,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // M2 = M2_0 + M2_1 + (mean_0 - mean_1)^2 * 32 * 32 / 64.
     constexpr int HC = ATT_HD / 2;
     float o[HC];
-    if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL], 0, ctl);
+    if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL + g], 0, ctl);
     ok = __all_sync(0xffffffffu, ok);
     float hsum = 0.0f, hm2 = 0.0f;
     const int64_t row = q_start + i;
