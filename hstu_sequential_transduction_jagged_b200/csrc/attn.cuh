@@ -25,15 +25,14 @@
 // Two warpgroups per query tile halve the elements each thread handles per
 // key tile and double the warps that hide tensor-memory, shared-memory and
 // MUFU latency; the work per element is one row-thread's arithmetic either way.
-// Key tiles are 64 keys.  Tensor memory (448 of 512 columns): two S buffers
+// Key tiles are 64 keys.  Tensor memory (all 512 columns): three S buffers
 // per group (64 fp32 columns each; each half writes its 32 keys of P, bf16
 // pairs, over the first 16 columns of its own 32-column half once they are
-// read), O_A, O_B (64 fp32 columns each), Q_A, Q_B (32 columns each, bf16
-// pairs).  With two S buffers the MMA warp computes S of tile k+1 while the
-// group works on tile k, so a group never waits for the MMA round trip.
-// Q is written to tensor memory once per CTA by the softmax threads, so the
-// QK^T MMA reads only K from shared memory (an M=128, N=128 MMA with both
-// operands in shared memory would need the whole shared-memory bandwidth).
+// read) and O_A, O_B (64 fp32 columns each).  S of tile k+3 reuses the buffer
+// of tile k, so it can be issued as soon as P V of tile k is: the MMAs for a
+// tile are issued two tiles before the group needs them, which covers the
+// issue-to-completion latency of the tensor pipe.  Q_A, Q_B live in shared
+// memory (TMA, 128B swizzle) and S = Q K^T reads both operands from there.
 // Per key tile: S = Q K^T (tcgen05, A from tensor memory), the softmax group
 // reads S row by row, adds the gathered bias, applies phi2 and the mask,
 // writes P (bf16) back over S, then O += P V (tcgen05 with A from tensor
@@ -67,6 +66,8 @@ constexpr int ATT_MMA_WARP = 17;  // + query tile (A: 17, B: 18)
 constexpr int MAX_TIME_BUCKETS = 256;
 
 constexpr uint32_t ATT_TILE_BYTES = ATT_KEYS * ATT_HD * 2;  // one K or V tile: 8 KB
+constexpr uint32_t ATT_Q_BYTES = ATT_ROWS * ATT_HD * 2;     // one Q tile: 16 KB
+constexpr int ATT_SBUF = 3;                                 // S buffers per query tile
 
 struct AttnParams {
   const int64_t* kv_offsets;   // [B+1] key/value rows per user (query rows too in causal mode)
@@ -75,8 +76,6 @@ struct AttnParams {
   const int64_t* request_ts;   // [B] (candidate mode)
   const float* rab_pos;        // [H, P]
   const float* rab_time;       // [H, Tb]
-  const __nv_bfloat16* q;      // [T_q, ld_q] query rows (head h at columns h*64..)
-  int64_t ld_q;
   const __nv_bfloat16* q_self; // candidate mode: candidate Q, K, V rows (self term)
   const __nv_bfloat16* k_self;
   const __nv_bfloat16* v_self;
@@ -196,7 +195,8 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t w, int c, int last) {
 // ---------------------------------------------------------------- shared memory
 
 struct AttnSmem {
-  static constexpr uint32_t kK = 0;                                   // stages x 8 KB
+  static constexpr uint32_t kQ = 0;                                   // 2 x 16 KB
+  static constexpr uint32_t kK = kQ + 2 * ATT_Q_BYTES;                // stages x 8 KB
   static constexpr uint32_t kV = kK + ATT_STAGES * ATT_TILE_BYTES;    // stages x 8 KB
   static constexpr uint32_t kKeyInfo = kV + ATT_STAGES * ATT_TILE_BYTES;  // stages x 256 B
   static constexpr uint32_t kKeyStride = ATT_KEYS * 4;                // bytes per stage
@@ -217,9 +217,9 @@ enum : int {
   BAR_Q_FULL = 0,
   BAR_KV_FULL = 1,                     // + stage
   BAR_KV_EMPTY = BAR_KV_FULL + ATT_STAGES,
-  BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + 2 * group + buffer
-  BAR_P_FULL = BAR_S_FULL + 4,             // + 2 * group + buffer
-  BAR_O_FULL = BAR_P_FULL + 4,             // + group
+  BAR_S_FULL = BAR_KV_EMPTY + ATT_STAGES,  // + ATT_SBUF * group + buffer
+  BAR_P_FULL = BAR_S_FULL + 2 * ATT_SBUF,  // + ATT_SBUF * group + buffer
+  BAR_O_FULL = BAR_P_FULL + 2 * ATT_SBUF,  // + group
   BAR_DONE = BAR_O_FULL + 2,               // + group
   BAR_COUNT = BAR_DONE + 2
 };
@@ -316,7 +316,8 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
 
 template <bool CAND, int PHI, bool PAIRS>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -358,6 +359,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const int D = CAND ? n_kv : q0 + 2 * ATT_ROWS;
   constexpr float kScale = phi_scale<PHI>();
 
+  uint8_t* sQ = smem + AttnSmem::kQ;
   uint8_t* sK = smem + AttnSmem::kK;
   uint8_t* sV = smem + AttnSmem::kV;
   uint8_t* sKey = smem + AttnSmem::kKeyInfo;
@@ -384,18 +386,19 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
   // ---------------- setup
   if (tid == 0) {
-    mbar_init(&bars[BAR_Q_FULL], 2 * ATT_ROWS);  // every softmax thread stores its Q row
+    mbar_init(&bars[BAR_Q_FULL], 1);  // the producer's expect-tx arrival + the Q bytes
     for (int s = 0; s < ATT_STAGES; ++s) {
       mbar_init(&bars[BAR_KV_FULL + s], 2);
       mbar_init(&bars[BAR_KV_EMPTY + s], 2);  // one commit per issuer
     }
     for (int g = 0; g < 2; ++g) {
-      // one S-ready and one P-ready barrier per S buffer: a group can run a
-      // tile ahead of the MMA warp, but never two phases ahead on one barrier
-      mbar_init(&bars[BAR_S_FULL + 2 * g], 1);
-      mbar_init(&bars[BAR_S_FULL + 2 * g + 1], 1);
-      mbar_init(&bars[BAR_P_FULL + 2 * g], 2 * ATT_ROWS);  // both column halves
-      mbar_init(&bars[BAR_P_FULL + 2 * g + 1], 2 * ATT_ROWS);
+      // one S-ready and one P-ready barrier per S buffer: S of tile k+3 is
+      // only issued once P of tile k has been seen, so no barrier can run a
+      // phase ahead of its waiters
+      for (int b = 0; b < ATT_SBUF; ++b) {
+        mbar_init(&bars[BAR_S_FULL + ATT_SBUF * g + b], 1);
+        mbar_init(&bars[BAR_P_FULL + ATT_SBUF * g + b], 2 * ATT_ROWS);  // both column halves
+      }
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bars[BAR_O_FULL + g], 1);
@@ -436,6 +439,14 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      // both query tiles (rows past the tensor's end read as zeros; rows of
+      // the next user are loaded but their results are never stored)
+      mbar_arrive_expect_tx(&bars[BAR_Q_FULL], 2 * ATT_Q_BYTES);
+      const int64_t qrow = q_start + q0;  // < 2^31 (row counts are checked on the host)
+      const int64_t qrow_b = min(qrow + ATT_ROWS, static_cast<int64_t>(INT32_MAX));
+      tma_load_2d(sQ, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD, static_cast<int32_t>(qrow));
+      tma_load_2d(sQ + ATT_Q_BYTES, &tm_q, &bars[BAR_Q_FULL], h * ATT_HD,
+                  static_cast<int32_t>(qrow_b));
     }
     int64_t t_req = 0;
     if constexpr (CAND) t_req = p.request_ts[u];
@@ -479,6 +490,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     // drain: every issued load must land before shared memory is released
     if (lane == 0) {
+      mbar_wait_drain(&bars[BAR_Q_FULL], 0, p.timeout_ns);
       for (int kt = max(0, issued - ATT_STAGES); kt < issued; ++kt)
         mbar_wait_drain(&bars[BAR_KV_FULL + kt % ATT_STAGES],
                         static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
@@ -490,12 +502,12 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
       const int nWg = g == 0 ? nA : nB;
-      // tensor memory: S buffers (P over them), O, Q of this tile
-      const uint32_t tS = tmem + static_cast<uint32_t>(g * 128);
-      const uint32_t tOg = tmem + 256u + static_cast<uint32_t>(g * 64);
-      const uint32_t tQg = tmem + 384u + static_cast<uint32_t>(g * 32);
-      // descriptors of stage 0; stage s adds s * 8 KB (s * 512 in 16-byte
-      // units) to the start-address field
+      // tensor memory: S buffers (P over them) and O of this tile
+      const uint32_t tS = tmem + static_cast<uint32_t>(g * ATT_SBUF * 64);
+      const uint32_t tOg = tmem + static_cast<uint32_t>(2 * ATT_SBUF * 64 + g * 64);
+      // this tile's Q, and the K/V descriptors of stage 0; stage s adds
+      // s * 8 KB (s * 512 in 16-byte units) to the start-address field
+      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ + g * ATT_Q_BYTES), 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_u32(sV), 8192, 1024);
       constexpr uint64_t kStageDesc = ATT_TILE_BYTES >> 4;
@@ -512,42 +524,47 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         return true;
       };
-      // S of tile kt into buffer kt & 1
-      auto issue_s = [&](int kt) {
+      // S of tile kt into buffer b = kt mod 3
+      auto issue_s = [&](int kt, int b) {
         const uint64_t dk = dK0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
-        const uint32_t d = tS + static_cast<uint32_t>((kt & 1) * 64);
+        const uint32_t d = tS + static_cast<uint32_t>(b * 64);
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk)
-          mma_bf16_ts(d, tQg + kk * 8, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(&bars[BAR_S_FULL + 2 * g + (kt & 1)]);
+          mma_bf16_ss(d, dQ + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[BAR_S_FULL + ATT_SBUF * g + b]);
       };
       // O += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
       // buffer of tile kt, P of keys 32-63 at columns 32-47
-      auto issue_pv = [&](int kt) {
+      auto issue_pv = [&](int kt, int b) {
         const uint64_t dv = dV0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
-        const uint32_t a = tS + static_cast<uint32_t>((kt & 1) * 64);
+        const uint32_t a = tS + static_cast<uint32_t>(b * 64);
         const uint32_t acc0 = kt > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < ATT_KEYS / 16; ++kk)
           mma_bf16_ts(tOg, a + (kk >> 1) * 32 + (kk & 1) * 8, dv + 128 * kk, idesc_pv,
                       kk > 0 ? 1u : acc0);
       };
-      // two tiles ahead: S(0), S(1) before any P exists
-      for (int t = 0; ok && t < 2 && t < nWg; ++t) {
+      // three tiles ahead: S(0), S(1), S(2) before any P exists
+      for (int t = 0; ok && t < ATT_SBUF && t < nWg; ++t) {
         ok = await_kv(t);
-        if (ok) issue_s(t);
+        if (ok) issue_s(t, t);
       }
+      int b = 0;         // buffer of tile kt
+      uint32_t ph = 0;   // phase parity of that buffer's barriers at tile kt
       for (int kt = 0; ok && kt < nk_total; ++kt) {
         if (kt < nWg) {
-          ok = mbar_wait(&bars[BAR_P_FULL + 2 * g + (kt & 1)], static_cast<uint32_t>(kt >> 1) & 1u,
-                         ctl);
+          ok = mbar_wait(&bars[BAR_P_FULL + ATT_SBUF * g + b], ph, ctl);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(kt);
-          if (kt + 2 < nWg) {
-            ok = await_kv(kt + 2);
+          issue_pv(kt, b);
+          if (kt + ATT_SBUF < nWg) {
+            ok = await_kv(kt + ATT_SBUF);
             if (!ok) break;
-            issue_s(kt + 2);  // into the buffer P V(kt) has just been issued to read
+            issue_s(kt + ATT_SBUF, b);  // into the buffer P V(kt) has just been issued to read
+          }
+          if (++b == ATT_SBUF) {
+            b = 0;
+            ph ^= 1u;
           }
         } else {
           // past this tile's last key tile: the release below must still
@@ -569,33 +586,14 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const int half = (warp >> 2) & 1;      // key columns 32*half .. 32*half + 31 of each tile
     const int r = tid & (ATT_ROWS - 1);    // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    // this half's 32 columns of S buffer 0 (+64: buffer 1)
-    const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(g * 128 + half * 32);
-    const uint32_t tO = tmem + lane_off + 256u + static_cast<uint32_t>(g * 64 + half * 32);
-    const uint32_t tQ = tmem + lane_off + 384u + static_cast<uint32_t>(g * 32);
+    // this half's 32 columns of S buffer 0 (+64 per buffer)
+    const uint32_t tS0 = tmem + lane_off + static_cast<uint32_t>(g * ATT_SBUF * 64 + half * 32);
+    const uint32_t tO =
+        tmem + lane_off + static_cast<uint32_t>(2 * ATT_SBUF * 64 + g * 64 + half * 32);
     const int i = q0 + g * ATT_ROWS + r;   // query index within the user
     const bool valid = i < n_q;
     const int nW = g == 0 ? nA : nB;
     bool ok = true;
-    if (half == 0) {
-      // this row's query (64 bf16 = 32 columns of packed pairs) into tensor memory
-      uint32_t qv[32];
-      if (valid) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.q + (q_start + i) * p.ld_q + h * ATT_HD);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v4 = src[c];
-          qv[4 * c] = v4.x; qv[4 * c + 1] = v4.y; qv[4 * c + 2] = v4.z; qv[4 * c + 3] = v4.w;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) qv[c] = 0u;
-      }
-      tmem_st32(tQ, qv);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[BAR_Q_FULL]);
-    }
     const uint64_t scale2 = f2_pack(kScale, kScale);
 
     // causal: per-row time-bucket walk and staged position-table copy
@@ -637,16 +635,18 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       }
     };
 
+    int buf = 0;        // S buffer of tile kt (kt mod 3)
+    uint32_t ph = 0;    // its barriers' phase parity at tile kt
     for (int kt = 0; kt < nW; ++kt) {
       const int s = kt % ATT_STAGES;
-      ok = mbar_wait(&bars[BAR_S_FULL + 2 * g + (kt & 1)], static_cast<uint32_t>(kt >> 1) & 1u, ctl);
+      ok = mbar_wait(&bars[BAR_S_FULL + ATT_SBUF * g + buf], ph, ctl);
       // the producer's per-key side data for this stage (already complete)
       if (ok)
         ok = mbar_wait(&bars[BAR_KV_FULL + s], static_cast<uint32_t>(kt / ATT_STAGES) & 1u, ctl);
       ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-collective
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tS = tS0 + static_cast<uint32_t>((kt & 1) * 64);
+      const uint32_t tS = tS0 + static_cast<uint32_t>(buf * 64);
       // 32 keys: TMEM -> registers -> bias, phi2, mask -> P over this half's S
       uint32_t sa[32], pk[16];
       tmem_ld32(tS, sa);
@@ -656,7 +656,11 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       tmem_st16(tS, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[BAR_P_FULL + 2 * g + (kt & 1)]);
+      mbar_arrive(&bars[BAR_P_FULL + ATT_SBUF * g + buf]);
+      if (++buf == ATT_SBUF) {
+        buf = 0;
+        ph ^= 1u;
+      }
     }
 
     // ---------------- epilogue: O / N, LayerNorm partial sums, store

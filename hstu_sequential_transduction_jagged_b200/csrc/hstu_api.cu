@@ -156,7 +156,8 @@ class ProfScope {
 
 // ------------------------------------------------------------------ device info
 
-using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const AttnParams);
+using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const AttnParams);
 
 template <bool CAND, bool PAIRS>
 AttnKernelFn attn_kernel_for(int phi) {
@@ -367,8 +368,9 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
-  CUtensorMap mk, mv;
+  CUtensorMap mq, mk, mv;
   const int64_t hc = static_cast<int64_t>(c->num_heads) * ATT_HD;
+  if ((s = make_map_bf16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS)) != HSTU_OK) return s;
   // with no key rows at all (every history empty) no K/V tile is ever loaded;
   // the maps then describe the query rows so that they stay valid
   const bool no_kv = j.T_kv == 0;
@@ -386,8 +388,6 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.request_ts = j.request_ts;
   p.rab_pos = j.rab_pos;
   p.rab_time = j.rab_time;
-  p.q = static_cast<const __nv_bfloat16*>(j.q);
-  p.ld_q = j.ldq;
   p.q_self = static_cast<const __nv_bfloat16*>(j.q_self);
   p.k_self = static_cast<const __nv_bfloat16*>(j.k_self);
   p.v_self = static_cast<const __nv_bfloat16*>(j.v_self);
@@ -416,7 +416,7 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   const size_t smem = AttnSmem::bytes(p.pos_len, pairs);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
-  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mk, mv, p);
+  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
