@@ -451,8 +451,25 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     int64_t t_req = 0;
     if constexpr (CAND) t_req = p.request_ts[u];
     int issued = 0;
+    // the key timestamps of the next tile are loaded one tile ahead, so that
+    // their global-memory latency overlaps the wait for a free stage and the
+    // current tile's work
+    constexpr int KPL = ATT_KEYS / 32;  // keys per lane per tile
+    int64_t ts_next[KPL];
+    auto load_ts = [&](int kt, int64_t (&t)[KPL]) {
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
+        const int j = kt * ATT_KEYS + lane + 32 * e;
+        t[e] = j < n_kv ? p.timestamps[kv_start + j] : 0;
+      }
+    };
+    if (nk_total > 0) load_ts(0, ts_next);
     for (int kt = 0; kt < nk_total; ++kt) {
       const int s = kt % ATT_STAGES;
+      int64_t ts[KPL];
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) ts[e] = ts_next[e];
+      if (kt + 1 < nk_total) load_ts(kt + 1, ts_next);
       const uint32_t par = (static_cast<uint32_t>(kt / ATT_STAGES) & 1u) ^ 1u;
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&bars[BAR_KV_EMPTY + s], par, ctl) ? 1 : 0;
@@ -465,21 +482,25 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       ++issued;
       uint8_t* key = sKey + s * AttnSmem::kKeyStride;
-      for (int e = 0; e < ATT_KEYS / 32; ++e) {
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) {
         const int c = lane + 32 * e;
         const int j = kt * ATT_KEYS + c;
         if constexpr (CAND) {
           // the whole per-key bias: candidates share position n_kv and time t_req
           float r = 0.0f;
           if (j < n_kv) {
-            const int64_t dt = t_req - p.timestamps[kv_start + j];
-            r = sRv[j] + sTime[time_bucket_search(dt, sThr, p.Tb)];
+            const int64_t dt = t_req - ts[e];
+            const int b = (dt >= 0 && dt < static_cast<int64_t>(INT32_MAX) - 1)
+                              ? time_bucket_octave(static_cast<int32_t>(dt), sOct)
+                              : time_bucket_search(dt, sThr, p.Tb);
+            r = sRv[j] + sTime[b];
           }
           reinterpret_cast<float*>(key)[c] = r;
         } else {
           int32_t rel = INT32_MAX;
           if (j < n_kv) {
-            const int64_t d = p.timestamps[kv_start + j] - t_first;
+            const int64_t d = ts[e] - t_first;
             rel = d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d);
           }
           reinterpret_cast<int32_t*>(key)[c] = rel;
