@@ -234,7 +234,9 @@ enum : int {
 // the whole chunk.  The walk `w` enters at the bucket of the previous key and
 // leaves at the bucket of the last visible key.  Per warp the chunk falls in
 // one of three cases:
-//   every row keeps one bucket      -> one time bias per row;
+//   every row keeps its bucket      -> one time bias per row, `rt_cur`, kept
+//                                      in a register (one compare of the last
+//                                      visible key against the bucket edge);
 //   two buckets B, B+1 in the warp  -> per key: B+1 iff t_j <= t_i - thr[B+1];
 //   more (near the diagonal)        -> per key bucket from the octave table.
 template <int PHI, bool PAIRS>
@@ -242,13 +244,37 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
                                              const float* rvx, const int32_t* kts, int lim,
                                              BucketWalk<int32_t>& w, const float* sTime,
                                              const int64_t* sThr, const int4* sOct,
-                                             uint64_t scale2) {
+                                             uint64_t scale2, float& rt_cur) {
   const unsigned full = 0xffffffffu;
   const bool live = lim >= 0;
   const int last = lim < 31 ? lim : 31;
   // key times of a pair of columns (broadcast shared loads, only off the
   // one-bucket path)
   auto kt_pair = [&](int c) -> int2 { return *reinterpret_cast<const int2*>(kts + c); };
+  auto pos_pair = [&](int c) -> uint64_t {
+    if constexpr (PAIRS) return lds_b64(rvx + c);
+    else return f2_pack(rvx[c], rvx[c + 1]);
+  };
+  auto s_pair = [&](int c) -> uint64_t {
+    return f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+  };
+  // every visible key of every lane still in the lane's current bucket
+  if (__all_sync(full, !live || kts[last] <= w.bound)) {
+    if (live) {
+      const uint64_t rt2 = f2_pack(rt_cur, rt_cur);
+#pragma unroll
+      for (int c = 0; c < 32; c += 2)
+        pk[c >> 1] = phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
+      if (lim < 31) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, lim);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) pk[q] = 0u;
+    }
+    return;
+  }
   int b_first = -1, b_last = 1 << 30;
   bool lane_steady = true;
   if (live) {
@@ -258,14 +284,8 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
     lane_steady = k_last <= w.bound;
     if (!lane_steady) w.step(k_last, sThr);
     b_last = w.b;
+    rt_cur = sTime[b_last];
   }
-  auto pos_pair = [&](int c) -> uint64_t {
-    if constexpr (PAIRS) return lds_b64(rvx + c);
-    else return f2_pack(rvx[c], rvx[c + 1]);
-  };
-  auto s_pair = [&](int c) -> uint64_t {
-    return f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-  };
   if (__all_sync(full, lane_steady)) {
     if (live) {
       const float rt = sTime[b_first];
@@ -619,6 +639,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     // causal: per-row time-bucket walk and staged position-table copy
     BucketWalk<int32_t> w32;
+    float rt_cur = 0.0f;  // time bias of the walk's current bucket
     int copy = 0;
     const float* rv = sRv;
     if constexpr (!CAND) {
@@ -627,6 +648,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                sThr, p.Tb);
       if constexpr (PAIRS) copy = (D - i) & 1;
       rv = sRv + copy * p.pos_len;
+      rt_cur = sTime[w32.b];
     }
 
     // this half's 32 keys of tile kt: S values in `sv`, packed bf16 P pairs to `pk`
@@ -652,7 +674,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // user's end are not stored and skip the work
         const int lim = !valid ? -1 : i - j0;
         causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + half * 32,
-                                 lim, w32, sTime, sThr, sOct, scale2);
+                                 lim, w32, sTime, sThr, sOct, scale2, rt_cur);
       }
     };
 
