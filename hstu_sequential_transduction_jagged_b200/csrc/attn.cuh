@@ -537,9 +537,11 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         static_cast<uint32_t>(kt / ATT_STAGES) & 1u, p.timeout_ns);
     }
   } else if (warp >= ATT_MMA_WARP) {
-    // ---------------- MMA issuers, one thread per query tile
+    // ---------------- MMA issuers, one warp per query tile: the whole warp
+    // runs the loop (waits are warp votes), one elected lane issues
     const int g = warp - ATT_MMA_WARP;
-    if (lane == 0) {
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
       const int nWg = g == 0 ? nA : nB;
@@ -552,13 +554,16 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const uint64_t dK0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_u32(sV), 8192, 1024);
       constexpr uint64_t kStageDesc = ATT_TILE_BYTES >> 4;
-      bool ok = mbar_wait(&bars[BAR_Q_FULL], 0, ctl);
+      auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
+      };
+      bool ok = wait_all(&bars[BAR_Q_FULL], 0);
       tc_fence_after();
-      int kv_ready = 0;  // key tiles whose K/V this thread has seen land
+      int kv_ready = 0;  // key tiles whose K/V this warp has seen land
       auto await_kv = [&](int kt) -> bool {
         while (kv_ready <= kt) {
-          if (!mbar_wait(&bars[BAR_KV_FULL + kv_ready % ATT_STAGES],
-                         static_cast<uint32_t>(kv_ready / ATT_STAGES) & 1u, ctl))
+          if (!wait_all(&bars[BAR_KV_FULL + kv_ready % ATT_STAGES],
+                        static_cast<uint32_t>(kv_ready / ATT_STAGES) & 1u))
             return false;
           tc_fence_after();
           ++kv_ready;
@@ -569,10 +574,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       auto issue_s = [&](int kt, int b) {
         const uint64_t dk = dK0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
         const uint32_t d = tS + static_cast<uint32_t>(b * 64);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < ATT_HD / 16; ++kk)
-          mma_bf16_ss(d, dQ + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(&bars[BAR_S_FULL + ATT_SBUF * g + b]);
+          for (int kk = 0; kk < ATT_HD / 16; ++kk)
+            mma_bf16_ss(d, dQ + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_commit(&bars[BAR_S_FULL + ATT_SBUF * g + b]);
+        }
+        __syncwarp();
       };
       // O += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
       // buffer of tile kt, P of keys 32-63 at columns 32-47
@@ -580,10 +588,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint64_t dv = dV0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
         const uint32_t a = tS + static_cast<uint32_t>(b * 64);
         const uint32_t acc0 = kt > 0 ? 1u : 0u;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < ATT_KEYS / 16; ++kk)
-          mma_bf16_ts(tOg, a + (kk >> 1) * 32 + (kk & 1) * 8, dv + 128 * kk, idesc_pv,
-                      kk > 0 ? 1u : acc0);
+          for (int kk = 0; kk < ATT_KEYS / 16; ++kk)
+            mma_bf16_ts(tOg, a + (kk >> 1) * 32 + (kk & 1) * 8, dv + 128 * kk, idesc_pv,
+                        kk > 0 ? 1u : acc0);
+        }
+        __syncwarp();
       };
       // three tiles ahead: S(0), S(1), S(2) before any P exists
       for (int t = 0; ok && t < ATT_SBUF && t < nWg; ++t) {
@@ -594,7 +605,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint32_t ph = 0;   // phase parity of that buffer's barriers at tile kt
       for (int kt = 0; ok && kt < nk_total; ++kt) {
         if (kt < nWg) {
-          ok = mbar_wait(&bars[BAR_P_FULL + ATT_SBUF * g + b], ph, ctl);
+          ok = wait_all(&bars[BAR_P_FULL + ATT_SBUF * g + b], ph);
           if (!ok) break;
           tc_fence_after();
           issue_pv(kt, b);
@@ -613,11 +624,15 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           ok = await_kv(kt);
           if (!ok) break;
         }
-        mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
+        if (leader) mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
+        __syncwarp();
       }
-      mma_commit(&bars[BAR_O_FULL + g]);
-      // every MMA of this thread must be complete before TMEM is released
-      mma_commit(&bars[BAR_DONE + g]);
+      if (leader) {
+        mma_commit(&bars[BAR_O_FULL + g]);
+        // every MMA of this warp must be complete before TMEM is released
+        mma_commit(&bars[BAR_DONE + g]);
+      }
+      __syncwarp();
       mbar_wait_drain(&bars[BAR_DONE + g], 0, p.timeout_ns);
     }
     __syncwarp();

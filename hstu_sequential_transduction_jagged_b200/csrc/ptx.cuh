@@ -152,6 +152,21 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+// One lane of a converged warp, chosen by the hardware (elect.sync over the
+// full warp).  Elect once and keep the result: tcgen05.commit tracks only the
+// MMAs of the thread that executes it, so one lane must issue all of them.
+// Issuing from an elected lane of a warp that runs the loop together lets the
+// compiler keep the MMA operands warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
