@@ -96,10 +96,16 @@ struct TileIter {
   __device__ __forceinline__ int n() const { return t % n_tiles; }
 };
 
+// Run by a whole warp (waits are warp votes); one elected lane issues every
+// MMA and commit.
 __device__ __forceinline__ void gemm_mma_loop(uint64_t* bars, const uint8_t* sA, const uint8_t* sB,
                                               uint32_t tmem, int total_tiles, int k_blocks,
                                               const WaitCtl& ctl, uint64_t drain_ns) {
   constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_BN, false, false);
+  const bool leader = elect_one();
+  auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
+  };
   int stage = 0;
   uint32_t phase = 0;
   int lt = 0;
@@ -107,28 +113,30 @@ __device__ __forceinline__ void gemm_mma_loop(uint64_t* bars, const uint8_t* sA,
   for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x, ++lt) {
     const int acc = lt & 1;
     const uint32_t acc_par = (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u;
-    ok = mbar_wait(&bars[GB_ACC_EMPTY + acc], acc_par, ctl);
+    ok = wait_all(&bars[GB_ACC_EMPTY + acc], acc_par);
     if (!ok) break;
     tc_fence_after();
     const uint32_t d = tmem + static_cast<uint32_t>(acc * G_BN);
     for (int kb = 0; kb < k_blocks; ++kb) {
-      ok = mbar_wait(&bars[GB_FULL + stage], phase, ctl);
+      ok = wait_all(&bars[GB_FULL + stage], phase);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sA + stage * G_A_BYTES);
-      const uint32_t b0 = smem_u32(sB + stage * G_B_BYTES);
+      const uint64_t da = smem_desc_sw128(smem_u32(sA + stage * G_A_BYTES), 16, 1024);
+      const uint64_t db = smem_desc_sw128(smem_u32(sB + stage * G_B_BYTES), 16, 1024);
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < G_BK / 16; ++kk) {
-        mma_bf16_ss(d, smem_desc_sw128(a0 + kk * 32, 16, 1024),
-                    smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < G_BK / 16; ++kk)
+          mma_bf16_ss(d, da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[GB_EMPTY + stage]);
       }
-      mma_commit(&bars[GB_EMPTY + stage]);
+      __syncwarp();
       if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
     }
-    if (ok) mma_commit(&bars[GB_ACC_FULL + acc]);
+    if (ok && leader) mma_commit(&bars[GB_ACC_FULL + acc]);
+    __syncwarp();
   }
-  mma_commit(&bars[GB_DONE]);
+  if (leader) mma_commit(&bars[GB_DONE]);
+  __syncwarp();
   mbar_wait_drain(&bars[GB_DONE], 0, drain_ns);
 }
 
@@ -200,7 +208,7 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
     __syncwarp();
   } else {
     // epilogue warps 2..5: TMEM lane quarter = warp % 4
@@ -335,7 +343,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
     __syncwarp();
   } else if (warp >= 6) {
     // A-tile producers: Norm(AV) (.) U, bf16, 128B-swizzled K-major layout.
