@@ -55,6 +55,21 @@ __device__ __forceinline__ float apply_act(float x) {
   }
 }
 
+// f1's extra shared memory: per epilogue warp two 4 KB staging buffers of 32
+// rows x 128 bytes (128B-swizzled) for the tensor stores of the output.
+struct F1Smem {
+  static constexpr uint32_t kOut = (GemmSmem::kMisc + 64 + 1023) / 1024 * 1024;
+  static constexpr uint32_t kBufBytes = 32 * 128;
+  static constexpr uint32_t kBytes = kOut + 4 * 2 * kBufBytes + 1024;
+};
+static_assert(F1Smem::kBytes <= 227u * 1024u, "f1 shared memory");
+
+// Tensor maps of the four output column blocks (U, V, Q, K): rows of the
+// block, 128-byte boxes (32 fp32 or 64 bf16 columns) x 32 rows, 128B swizzle.
+struct F1OutMaps {
+  CUtensorMap m[4];
+};
+
 struct F1Params {
   void* dst[4];           // destination of column block b (U, V, Q, K)
   int64_t ld_dst[4];      // row stride of each destination (elements)
@@ -145,6 +160,7 @@ __device__ __forceinline__ void gemm_mma_loop(uint64_t* bars, const uint8_t* sA,
 template <int ACT>
 __global__ void __launch_bounds__(192, 1)
 hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ F1OutMaps out,
                const __grid_constant__ F1Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -211,9 +227,16 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
     __syncwarp();
   } else {
-    // epilogue warps 2..5: TMEM lane quarter = warp % 4
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int row_in_tile = (warp & 3) * 32 + lane;
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4.  Each warp turns its
+    // 32 rows into 128-byte row segments (32 fp32 or 64 bf16 columns) in a
+    // 128B-swizzled staging buffer and writes them with tensor stores; two
+    // buffers alternate, a buffer is refilled once its store has read it.
+    const int q4 = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    uint8_t* stage_base = smem + F1Smem::kOut + q4 * 2 * F1Smem::kBufBytes;
+    uint8_t* my_row = nullptr;  // this lane's row in the current buffer
+    const int sw = lane & 7;    // 16-byte chunk j of row r sits at chunk j ^ (r % 8)
+    int nseg = 0;               // segments this warp has stored
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
@@ -222,8 +245,7 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mt) * G_BM + row_in_tile;
-      const bool row_ok = row < p.M;
+      const int32_t row0 = static_cast<int32_t>(static_cast<int64_t>(mt) * G_BM + q4 * 32);
 #pragma unroll 1
       for (int ch = 0; ch < G_BN / 32; ++ch) {
         uint32_t v[32];
@@ -233,6 +255,7 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int col = nt * G_BN + ch * 32;
         const int blk = col / p.blk_w;
         const int cb = col - blk * p.blk_w;
+        const bool f32 = (p.f32_mask >> blk) & 1u;
         const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
         float z[32];
 #pragma unroll
@@ -243,28 +266,44 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
           z[4 * q + 2] = apply_act<ACT>(__uint_as_float(v[4 * q + 2]) + bb.z);
           z[4 * q + 3] = apply_act<ACT>(__uint_as_float(v[4 * q + 3]) + bb.w);
         }
-        if (row_ok) {
-          if ((p.f32_mask >> blk) & 1u) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dst[blk]) +
-                                                    row * p.ld_dst[blk] + cb);
+        // a bf16 segment takes two 32-column chunks; blocks are 64-column aligned
+        if (f32 || (ch & 1) == 0) {
+          if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
+          __syncwarp();
+          my_row = stage_base + (nseg & 1) * F1Smem::kBufBytes + lane * 128;
+        }
+        if (f32) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dst[blk]) +
-                                                  row * p.ld_dst[blk] + cb);
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(my_row + ((j ^ sw) << 4)) =
+                make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
+        } else {
+          const int j0 = (ch & 1) * 4;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack_bf16x2(z[8 * q], z[8 * q + 1]),
-                                  pack_bf16x2(z[8 * q + 2], z[8 * q + 3]),
-                                  pack_bf16x2(z[8 * q + 4], z[8 * q + 5]),
-                                  pack_bf16x2(z[8 * q + 6], z[8 * q + 7]));
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(my_row + (((j0 + j) ^ sw) << 4)) =
+                make_uint4(pack_bf16x2(z[8 * j], z[8 * j + 1]), pack_bf16x2(z[8 * j + 2], z[8 * j + 3]),
+                           pack_bf16x2(z[8 * j + 4], z[8 * j + 5]),
+                           pack_bf16x2(z[8 * j + 6], z[8 * j + 7]));
+        }
+        if (f32 || (ch & 1) == 1) {
+          fence_proxy_async_smem();  // this lane's writes, before the tensor store reads them
+          __syncwarp();
+          if (lane == 0) {
+            // rows at or past M lie outside the tensor and are not written
+            tma_store_2d(&out.m[blk], stage_base + (nseg & 1) * F1Smem::kBufBytes,
+                         f32 ? cb : cb - 32, row0);
+            bulk_commit();
           }
+          ++nseg;
         }
       }
       tc_fence_before();
       mbar_arrive(&bars[GB_ACC_EMPTY + acc]);
     }
+    // every store must have completed before shared memory is released
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

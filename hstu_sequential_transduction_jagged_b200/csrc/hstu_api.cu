@@ -198,12 +198,13 @@ hstu_status_t device_info(DeviceInfo** out) {
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                att_max));
     const int g = static_cast<int>(GemmSmem::kBytes);
+    const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_SILU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_IDENTITY>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f2_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g));
     d.smem_set = true;
@@ -246,6 +247,24 @@ hstu_status_t make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, in
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// 2-D map for tensor stores of f1's output blocks: fp32 or bf16 [rows, cols]
+// with row stride `ld` elements; box = one 128-byte row segment x 32 rows.
+hstu_status_t make_out_map(CUtensorMap* map, void* base, bool f32, int64_t rows, int64_t cols,
+                           int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return HSTU_ERR_CUDA;
+  const int elt = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * elt};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
@@ -434,9 +453,14 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   if ((s = make_map_bf16(&mw, w1, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
   F1Params p;
   std::memset(&p, 0, sizeof(p));
+  F1OutMaps om;
+  std::memset(&om, 0, sizeof(om));
+  const int64_t blk_w = static_cast<int64_t>(c->num_heads) * ATT_HD;
   for (int b = 0; b < 4; ++b) {
     p.dst[b] = dst[b];
     p.ld_dst[b] = ld_dst[b];
+    if ((s = make_out_map(&om.m[b], dst[b], (f32_mask >> b) & 1u, M, blk_w, ld_dst[b])) != HSTU_OK)
+      return s;
   }
   p.f32_mask = f32_mask;
   p.bias = b1;
@@ -452,13 +476,13 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   ProfScope prof(K_F1, st);
   switch (c->phi1) {
     case HSTU_ACT_RELU:
-      hstu_f1_kernel<HSTU_ACT_RELU><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      hstu_f1_kernel<HSTU_ACT_RELU><<<grid, 192, F1Smem::kBytes, st>>>(mx, mw, om, p);
       break;
     case HSTU_ACT_SILU:
-      hstu_f1_kernel<HSTU_ACT_SILU><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      hstu_f1_kernel<HSTU_ACT_SILU><<<grid, 192, F1Smem::kBytes, st>>>(mx, mw, om, p);
       break;
     default:
-      hstu_f1_kernel<HSTU_ACT_IDENTITY><<<grid, 192, GemmSmem::kBytes, st>>>(mx, mw, p);
+      hstu_f1_kernel<HSTU_ACT_IDENTITY><<<grid, 192, F1Smem::kBytes, st>>>(mx, mw, om, p);
       break;
   }
   HSTU_CHECK_CUDA(cudaGetLastError());
