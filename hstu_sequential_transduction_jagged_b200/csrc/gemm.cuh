@@ -82,6 +82,21 @@ struct F1Params {
   uint64_t timeout_ns;
 };
 
+// f2's extra shared memory: per epilogue warp one 4 KB staging buffer for Y
+// (32 rows x 32 fp32) and one for its bf16 copy (32 rows x 64 bf16), both
+// 128B-swizzled, for tensor stores.
+struct F2Smem {
+  static constexpr uint32_t kOut = (GemmSmem::kRowStats + G_BM * 8 + 1023) / 1024 * 1024;
+  static constexpr uint32_t kBufBytes = 32 * 128;
+  static constexpr uint32_t kBytes = kOut + 4 * 2 * kBufBytes + 1024;
+};
+static_assert(F2Smem::kBytes <= 227u * 1024u, "f2 shared memory");
+
+// Tensor maps of Y (fp32) and of its bf16 copy: 128-byte boxes x 32 rows.
+struct F2OutMaps {
+  CUtensorMap y, y_lp;
+};
+
 struct F2Params {
   const float* av;          // [M, ld_av] fp32 attention output
   const float* u;           // [M, ld_u] fp32 gate
@@ -320,7 +335,8 @@ constexpr int F2_PRODUCER_WARPS = 8;
 constexpr int F2_THREADS = (6 + F2_PRODUCER_WARPS) * 32;
 
 __global__ void __launch_bounds__(F2_THREADS, 1)
-hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ F2Params p) {
+hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ F2OutMaps out,
+               const __grid_constant__ F2Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -490,9 +506,15 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       }
     }
   } else {
-    // epilogue warps 2..5: + b2 + residual, fp32 (and optional bf16) store
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int row_in_tile = (warp & 3) * 32 + lane;
+    // epilogue warps 2..5: + b2 + residual; Y (fp32, 32-column segments) and
+    // its optional bf16 copy (64-column segments) go out through 128B-swizzled
+    // staging buffers and tensor stores
+    const int q4 = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const int row_in_tile = q4 * 32 + lane;
+    uint8_t* buf_y = smem + F2Smem::kOut + q4 * 2 * F2Smem::kBufBytes;
+    uint8_t* buf_l = buf_y + F2Smem::kBufBytes;
+    const int sw = lane & 7;  // 16-byte chunk j of row r sits at chunk j ^ (r % 8)
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
@@ -503,6 +525,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * G_BM + row_in_tile;
       const bool row_ok = row < p.M;
+      const int32_t row0 = static_cast<int32_t>(static_cast<int64_t>(mt) * G_BM + q4 * 32);
 #pragma unroll 1
       for (int ch = 0; ch < G_BN / 32; ++ch) {
         uint32_t v[32];
@@ -511,17 +534,17 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tmem_ld_wait();
         const int col = nt * G_BN + ch * 32;
         if (col >= p.N) continue;  // warp-uniform: the last N tile may be partial
-        if (row_ok) {
-          float y[32];
-          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
+        float y[32];
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 bb = __ldg(b4 + q);
-            y[4 * q + 0] = __uint_as_float(v[4 * q + 0]) + bb.x;
-            y[4 * q + 1] = __uint_as_float(v[4 * q + 1]) + bb.y;
-            y[4 * q + 2] = __uint_as_float(v[4 * q + 2]) + bb.z;
-            y[4 * q + 3] = __uint_as_float(v[4 * q + 3]) + bb.w;
-          }
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = __ldg(b4 + q);
+          y[4 * q + 0] = __uint_as_float(v[4 * q + 0]) + bb.x;
+          y[4 * q + 1] = __uint_as_float(v[4 * q + 1]) + bb.y;
+          y[4 * q + 2] = __uint_as_float(v[4 * q + 2]) + bb.z;
+          y[4 * q + 3] = __uint_as_float(v[4 * q + 3]) + bb.w;
+        }
+        if (row_ok) {
           if (p.x_res != nullptr) {
             const float4* xr = reinterpret_cast<const float4*>(p.x_res + row * p.ld_x + col);
 #pragma unroll
@@ -546,24 +569,42 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               }
             }
           }
-          float4* yo = reinterpret_cast<float4*>(p.y + row * p.ld_y + col);
+        }
+        // both staging buffers are free once the earlier stores have read them
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        uint8_t* ry = buf_y + lane * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            yo[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-          if (p.y_lp != nullptr) {
-            uint4* yl = reinterpret_cast<uint4*>(p.y_lp + row * p.ld_y + col);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(ry + ((j ^ sw) << 4)) =
+              make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+        const bool lp = p.y_lp != nullptr;
+        if (lp) {
+          // this chunk is one half of a 64-column bf16 segment
+          uint8_t* rl = buf_l + lane * 128;
+          const int j0 = (ch & 1) * 4;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              yl[q] = make_uint4(pack_bf16x2(y[8 * q], y[8 * q + 1]),
-                                 pack_bf16x2(y[8 * q + 2], y[8 * q + 3]),
-                                 pack_bf16x2(y[8 * q + 4], y[8 * q + 5]),
-                                 pack_bf16x2(y[8 * q + 6], y[8 * q + 7]));
-          }
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(rl + (((j0 + j) ^ sw) << 4)) =
+                make_uint4(pack_bf16x2(y[8 * j], y[8 * j + 1]), pack_bf16x2(y[8 * j + 2], y[8 * j + 3]),
+                           pack_bf16x2(y[8 * j + 4], y[8 * j + 5]),
+                           pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+        }
+        fence_proxy_async_smem();  // this lane's writes, before the tensor stores read them
+        __syncwarp();
+        if (lane == 0) {
+          // rows at or past M lie outside the tensor and are not written
+          tma_store_2d(&out.y, buf_y, col, row0);
+          if (lp && ((ch & 1) == 1 || col + 32 >= p.N)) tma_store_2d(&out.y_lp, buf_l, col & ~63, row0);
+          bulk_commit();
         }
       }
       tc_fence_before();
       mbar_arrive(&bars[GB_ACC_EMPTY + acc]);
     }
+    // every store must have completed before shared memory is released
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -197,7 +197,6 @@ hstu_status_t device_info(DeviceInfo** out) {
           HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(cand != 0, phi, pairs != 0),
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                att_max));
-    const int g = static_cast<int>(GemmSmem::kBytes);
     const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
@@ -205,8 +204,8 @@ hstu_status_t device_info(DeviceInfo** out) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_IDENTITY>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
-    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f2_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, g));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(F2Smem::kBytes)));
     d.smem_set = true;
   }
   *out = &d;
@@ -501,6 +500,10 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   const int N = c->d_model, K = c->num_heads * c->dv;
   CUtensorMap mw;
   if ((s = make_map_bf16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  F2OutMaps om;
+  std::memset(&om, 0, sizeof(om));
+  if ((s = make_out_map(&om.y, y, true, M, N, ld_y)) != HSTU_OK) return s;
+  if (y_lp != nullptr && (s = make_out_map(&om.y_lp, y_lp, false, M, N, ld_y)) != HSTU_OK) return s;
   F2Params p;
   std::memset(&p, 0, sizeof(p));
   p.av = av;
@@ -528,7 +531,7 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
   ProfScope prof(K_F2, st);
-  hstu_f2_kernel<<<grid, F2_THREADS, GemmSmem::kBytes, st>>>(mw, p);
+  hstu_f2_kernel<<<grid, F2_THREADS, F2Smem::kBytes, st>>>(mw, om, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
