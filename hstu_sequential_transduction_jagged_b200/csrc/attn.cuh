@@ -152,6 +152,21 @@ __device__ __forceinline__ int time_bucket_octave(int32_t dt, const int4* oct) {
   return o.w + (d >= o.x ? 1 : 0) + (d >= o.y ? 1 : 0) + (d >= o.z ? 1 : 0);
 }
 
+// Time bias of 0 <= dt < 2^31 - 1 straight from the octave: `ort[k]` holds the
+// (scaled) biases of the octave's base bucket and of the three buckets after
+// it, so the bias is three compares and selects, with no dependent lookup.
+__device__ __forceinline__ float time_bias_octave(int32_t dt, const int4* oct, const float4* ort) {
+  const int32_t d = dt > 0 ? dt : 0;
+  const int k = 31 - __clz(d + 1);
+  const int4 o = oct[k];
+  const float4 r = ort[k];
+  float v = r.x;
+  v = d >= o.x ? r.y : v;
+  v = d >= o.y ? r.z : v;
+  v = d >= o.z ? r.w : v;
+  return v;
+}
+
 // phi2 applied to a pair given h = (scaled) pre-activation; returns bf16x2.
 // SiLU: tables carry x/2, so p = h + h*tanh(h); ReLU / identity: h = x.
 template <int PHI>
@@ -203,7 +218,8 @@ struct AttnSmem {
   static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * kKeyStride;
   static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
   static constexpr uint32_t kOct = kThr + MAX_TIME_BUCKETS * 8;      // 32 x int4
-  static constexpr uint32_t kBars = kOct + 32 * 16;
+  static constexpr uint32_t kOrt = kOct + 32 * 16;                   // 32 x float4
+  static constexpr uint32_t kBars = kOrt + 32 * 16;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kLnX = kMisc + 64;                        // 2 x 128 float2
   static constexpr uint32_t kPos = kLnX + 2 * ATT_ROWS * 8;
@@ -238,13 +254,13 @@ enum : int {
 //                                      in a register (one compare of the last
 //                                      visible key against the bucket edge);
 //   two buckets B, B+1 in the warp  -> per key: B+1 iff t_j <= t_i - thr[B+1];
-//   more (near the diagonal)        -> per key bucket from the octave table.
+//   more (near the diagonal)        -> per key bias from the octave tables.
 template <int PHI, bool PAIRS>
 __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16],
                                              const float* rvx, const int32_t* kts, int lim,
                                              BucketWalk<int32_t>& w, const float* sTime,
                                              const int64_t* sThr, const int4* sOct,
-                                             uint64_t scale2, float& rt_cur) {
+                                             const float4* sOrt, uint64_t scale2, float& rt_cur) {
   const unsigned full = 0xffffffffu;
   const bool live = lim >= 0;
   const int last = lim < 31 ? lim : 31;
@@ -316,8 +332,8 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
         const int2 k2 = kt_pair(c);
-        const float r0 = sTime[time_bucket_octave(w.ti - k2.x, sOct)];
-        const float r1 = sTime[time_bucket_octave(w.ti - k2.y, sOct)];
+        const float r0 = time_bias_octave(w.ti - k2.x, sOct, sOrt);
+        const float r1 = time_bias_octave(w.ti - k2.y, sOct, sOrt);
         pk[c >> 1] =
             phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
       }
@@ -386,6 +402,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   float* sTime = reinterpret_cast<float*>(smem + AttnSmem::kTimeTab);
   int64_t* sThr = reinterpret_cast<int64_t*>(smem + AttnSmem::kThr);
   int4* sOct = reinterpret_cast<int4*>(smem + AttnSmem::kOct);
+  float4* sOrt = reinterpret_cast<float4*>(smem + AttnSmem::kOrt);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
   float2* sLnX = reinterpret_cast<float2*>(smem + AttnSmem::kLnX);
@@ -447,7 +464,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     sTime[k] = kScale * p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     sThr[k] = p.thr[k];
   }
-  if (tid < 32) sOct[tid] = p.oct[tid];
+  if (tid < 32) {
+    const int4 o = p.oct[tid];
+    sOct[tid] = o;
+    const float* rt = p.rab_time + static_cast<int64_t>(h) * p.Tb;
+    auto tb = [&](int b) { return kScale * rt[min(max(b, 0), p.Tb - 1)]; };
+    sOrt[tid] = make_float4(tb(o.w), tb(o.w + 1), tb(o.w + 2), tb(o.w + 3));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -689,7 +712,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // user's end are not stored and skip the work
         const int lim = !valid ? -1 : i - j0;
         causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + half * 32,
-                                 lim, w32, sTime, sThr, sOct, scale2, rt_cur);
+                                 lim, w32, sTime, sThr, sOct, sOrt, scale2, rt_cur);
       }
     };
 
