@@ -82,15 +82,36 @@ struct F1Params {
   uint64_t timeout_ns;
 };
 
-// f2's extra shared memory: per epilogue warp one 4 KB staging buffer for Y
-// (32 rows x 32 fp32) and one for its bf16 copy (32 rows x 64 bf16), both
-// 128B-swizzled, for tensor stores.
+// f2 works on 128-row tiles that cover up to F2_NW = 512 output columns: two
+// 256-column MMA halves accumulate side by side in tensor memory, so each
+// k-block of the A operand, LayerNorm(AV) (.) U, is built once per row tile
+// (a 256-column tiling builds it once per column tile).  A stage holds the
+// A tile and both W2 halves; the single accumulator uses all 512 columns.
+constexpr int F2_STAGES = 2;
+constexpr int F2_NW = 2 * G_BN;
+constexpr uint32_t F2_B_BYTES = 2 * G_B_BYTES;  // both W2 halves of a k-block: 64 KB
+
 struct F2Smem {
-  static constexpr uint32_t kOut = (GemmSmem::kRowStats + G_BM * 8 + 1023) / 1024 * 1024;
+  static constexpr uint32_t kA = 0;                                // stages x 16 KB
+  static constexpr uint32_t kB = F2_STAGES * G_A_BYTES;            // stages x 64 KB
+  static constexpr uint32_t kBars = kB + F2_STAGES * F2_B_BYTES;   // 16 barriers
+  static constexpr uint32_t kMisc = kBars + 16 * 8;
+  static constexpr uint32_t kRowStats = kMisc + 64;                // 128 x (mean, rstd)
+  // per epilogue warp one 4 KB staging buffer for Y (32 rows x 32 fp32) and one
+  // for its bf16 copy (32 rows x 64 bf16), both 128B-swizzled, for tensor stores
+  static constexpr uint32_t kOut = (kRowStats + G_BM * 8 + 1023) / 1024 * 1024;
   static constexpr uint32_t kBufBytes = 32 * 128;
   static constexpr uint32_t kBytes = kOut + 4 * 2 * kBufBytes + 1024;
 };
 static_assert(F2Smem::kBytes <= 227u * 1024u, "f2 shared memory");
+
+enum : int {
+  F2B_FULL = 0,                          // + stage: W2 bytes + every A-producer warp
+  F2B_EMPTY = F2B_FULL + F2_STAGES,      // + stage
+  F2B_ACC_FULL = F2B_EMPTY + F2_STAGES,
+  F2B_ACC_EMPTY = F2B_ACC_FULL + 1,
+  F2B_DONE = F2B_ACC_EMPTY + 1,
+};
 
 // Tensor maps of Y (fp32) and of its bf16 copy: 128-byte boxes x 32 rows.
 struct F2OutMaps {
@@ -114,7 +135,7 @@ struct F2Params {
   int64_t ld_y;
   int64_t M;
   int32_t N, K, H;
-  int32_t num_m_tiles, num_n_tiles;
+  int32_t num_m_tiles, num_n_tiles;  // f2: num_n_tiles counts groups of F2_NW columns
   uint64_t timeout_ns;
 };
 
@@ -340,26 +361,26 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem + GemmSmem::kA;
-  uint8_t* sB = smem + GemmSmem::kB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmem::kBars);
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + GemmSmem::kMisc);
-  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + GemmSmem::kMisc + 4);
-  float2* sStats = reinterpret_cast<float2*>(smem + GemmSmem::kRowStats);
+  uint8_t* sA = smem + F2Smem::kA;
+  uint8_t* sB = smem + F2Smem::kB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F2Smem::kBars);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + F2Smem::kMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + F2Smem::kMisc + 4);
+  float2* sStats = reinterpret_cast<float2*>(smem + F2Smem::kRowStats);
   const int warp = warp_id(), lane = lane_id();
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int k_blocks = p.K / G_BK;
+  // 256-column MMA halves in column group ng (the last group may have one)
+  auto halves_of = [&](int ng) { return min(2, (p.N - ng * F2_NW + G_BN - 1) / G_BN); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < G_STAGES; ++s) {
-      mbar_init(&bars[GB_FULL + s], 1 + F2_PRODUCER_WARPS);  // TMA of W2 + A-tile producer warps
-      mbar_init(&bars[GB_EMPTY + s], 1);
+    for (int s = 0; s < F2_STAGES; ++s) {
+      mbar_init(&bars[F2B_FULL + s], 1 + F2_PRODUCER_WARPS);  // TMA of W2 + A-tile producer warps
+      mbar_init(&bars[F2B_EMPTY + s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars[GB_ACC_FULL + b], 1);
-      mbar_init(&bars[GB_ACC_EMPTY + b], 128);
-    }
-    mbar_init(&bars[GB_DONE], 1);
+    mbar_init(&bars[F2B_ACC_FULL], 1);
+    mbar_init(&bars[F2B_ACC_EMPTY], 128);
+    mbar_init(&bars[F2B_DONE], 1);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -382,24 +403,67 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       int issued = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const int nt = t % p.num_n_tiles;
+        const int ng = t % p.num_n_tiles;
+        const int nh = halves_of(ng);
         for (int kb = 0; kb < k_blocks; ++kb) {
-          ok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl);
+          ok = mbar_wait(&bars[F2B_EMPTY + stage], phase ^ 1u, ctl);
           if (!ok) break;
-          mbar_arrive_expect_tx(&bars[GB_FULL + stage], G_B_BYTES);
-          tma_load_2d(sB + stage * G_B_BYTES, &tm_w, &bars[GB_FULL + stage], kb * G_BK, nt * G_BN);
+          mbar_arrive_expect_tx(&bars[F2B_FULL + stage], nh * G_B_BYTES);
+          for (int hf = 0; hf < nh; ++hf)
+            tma_load_2d(sB + stage * F2_B_BYTES + hf * G_B_BYTES, &tm_w, &bars[F2B_FULL + stage],
+                        kb * G_BK, ng * F2_NW + hf * G_BN);
           ++issued;
-          if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == F2_STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      for (int k = max(0, issued - G_STAGES); k < issued; ++k)
-        mbar_wait_drain(&bars[GB_FULL + (k % G_STAGES)], static_cast<uint32_t>(k / G_STAGES) & 1u,
+      for (int k = max(0, issued - F2_STAGES); k < issued; ++k)
+        mbar_wait_drain(&bars[F2B_FULL + (k % F2_STAGES)], static_cast<uint32_t>(k / F2_STAGES) & 1u,
                           p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
-    gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    // MMA warp: whole-warp loop, one elected lane issues.  Per k-block both
+    // 256-column halves (tensor-memory columns 0-255 and 256-511).
+    constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_BN, false, false);
+    constexpr uint64_t kHalfDesc = G_B_BYTES >> 4;  // start-address step of the second W2 half
+    const bool leader = elect_one();
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    int lt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++lt) {
+      const int nh = halves_of(t % p.num_n_tiles);
+      // the epilogue has drained the previous tile's accumulator
+      ok = wait_all(&bars[F2B_ACC_EMPTY], (static_cast<uint32_t>(lt) & 1u) ^ 1u);
+      if (!ok) break;
+      tc_fence_after();
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        ok = wait_all(&bars[F2B_FULL + stage], phase);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t da = smem_desc_sw128(smem_u32(sA + stage * G_A_BYTES), 16, 1024);
+        const uint64_t db = smem_desc_sw128(smem_u32(sB + stage * F2_B_BYTES), 16, 1024);
+        if (leader) {
+          for (int hf = 0; hf < nh; ++hf) {
+#pragma unroll
+            for (int kk = 0; kk < G_BK / 16; ++kk)
+              mma_bf16_ss(tmem + static_cast<uint32_t>(hf * G_BN), da + 2 * kk,
+                          db + hf * kHalfDesc + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars[F2B_EMPTY + stage]);
+        }
+        __syncwarp();
+        if (++stage == F2_STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (ok && leader) mma_commit(&bars[F2B_ACC_FULL]);
+      __syncwarp();
+    }
+    if (leader) mma_commit(&bars[F2B_DONE]);
     __syncwarp();
+    mbar_wait_drain(&bars[F2B_DONE], 0, p.timeout_ns);
   } else if (warp >= 6) {
     // A-tile producers: Norm(AV) (.) U, bf16, 128B-swizzled K-major layout.
     // Each warp owns 16 rows of the tile; all of a k-block's loads (4 rows x
@@ -475,7 +539,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           bt[4] = b1.x; bt[5] = b1.y; bt[6] = b1.z; bt[7] = b1.w;
         }
         int wok = 0;
-        if (lane == 0) wok = mbar_wait(&bars[GB_EMPTY + stage], phase ^ 1u, ctl) ? 1 : 0;
+        if (lane == 0) wok = mbar_wait(&bars[F2B_EMPTY + stage], phase ^ 1u, ctl) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, wok, 0) != 0;
         if (!ok) break;
         uint8_t* a_tile = sA + stage * G_A_BYTES;
@@ -501,8 +565,8 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[GB_FULL + stage]);
-        if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+        if (lane == 0) mbar_arrive(&bars[F2B_FULL + stage]);
+        if (++stage == F2_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
   } else {
@@ -517,9 +581,8 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int sw = lane & 7;  // 16-byte chunk j of row r sits at chunk j ^ (r % 8)
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
-      const int mt = t / p.num_n_tiles, nt = t % p.num_n_tiles;
-      const int acc = lt & 1;
-      bool ok = mbar_wait(&bars[GB_ACC_FULL + acc], static_cast<uint32_t>(lt >> 1) & 1u, ctl);
+      const int mt = t / p.num_n_tiles, ng = t % p.num_n_tiles;
+      bool ok = mbar_wait(&bars[F2B_ACC_FULL], static_cast<uint32_t>(lt) & 1u, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -527,13 +590,13 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       const bool row_ok = row < p.M;
       const int32_t row0 = static_cast<int32_t>(static_cast<int64_t>(mt) * G_BM + q4 * 32);
 #pragma unroll 1
-      for (int ch = 0; ch < G_BN / 32; ++ch) {
+      for (int ch = 0; ch < F2_NW / 32; ++ch) {
+        const int col = ng * F2_NW + ch * 32;
+        if (col >= p.N) break;  // warp-uniform: the last column group may be partial
         uint32_t v[32];
         __syncwarp();
-        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(acc * G_BN + ch * 32), v);
+        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(ch * 32), v);
         tmem_ld_wait();
-        const int col = nt * G_BN + ch * 32;
-        if (col >= p.N) continue;  // warp-uniform: the last N tile may be partial
         float y[32];
         const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
 #pragma unroll
@@ -600,7 +663,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars[GB_ACC_EMPTY + acc]);
+      mbar_arrive(&bars[F2B_ACC_EMPTY]);
     }
     // every store must have completed before shared memory is released
     if (lane == 0) bulk_wait_all();

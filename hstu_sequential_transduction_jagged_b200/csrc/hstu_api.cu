@@ -526,7 +526,7 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   p.K = K;
   p.H = c->num_heads;
   p.num_m_tiles = static_cast<int32_t>((M + G_BM - 1) / G_BM);
-  p.num_n_tiles = (N + G_BN - 1) / G_BN;
+  p.num_n_tiles = (N + F2_NW - 1) / F2_NW;  // column groups of up to 512
   p.timeout_ns = kDefaultTimeoutNs;
   const int total = p.num_m_tiles * p.num_n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
