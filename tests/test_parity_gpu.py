@@ -180,6 +180,16 @@ def test_small_bf16_full_per_layer(H):
     _per_layer_check(H, make_case("small-bf16"), "small-bf16 full")
 
 
+@pytest.mark.parametrize("d_model", [64, 320, 768])
+def test_model_widths(H, d_model):
+    """f2's tiles cover up to 512 output columns in two 256-column halves: widths
+    that use one half (64), a partly filled second half (320), or a second
+    column group (768); two layers, so the bf16 copy of Y feeds the next f1."""
+    cfg = make_case("small-bf16").cfg.replace(d_model=d_model, num_heads=2)
+    case = make_case(cfg, seed=26, lengths=[70, 300, 5], num_layers=2)
+    _forward_check(H, case, f"d_model={d_model}")
+
+
 def test_single_layer_kv_cache_and_lp_copy(H):
     case = make_case("small-bf16", seed=25, lengths=[100, 260], num_layers=1)
     t, jag, weights = upload(H, case)
