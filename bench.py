@@ -186,6 +186,40 @@ def traffic_from_profiles(kernel: str):
         return None
 
 
+def pipelined_e2e(torch, n_steps, nb, copy_in, compute, copy_out, stream):
+    """Run `n_steps` host-in / compute / host-out steps with `nb` sets of
+    buffers: the host-to-device copy of step i+1 and the device-to-host copy of
+    step i-1 run on their own streams while step i computes on `stream`.
+    Every step still copies its own inputs from pinned host memory and its own
+    result back.  `copy_in(k)`, `compute(k)` and `copy_out(k)` enqueue on the
+    current stream for buffer set k."""
+    s_in, s_out = torch.cuda.Stream(stream.device), torch.cuda.Stream(stream.device)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nb)]
+    ev_out = [torch.cuda.Event() for _ in range(nb)]
+    for i in range(n_steps):
+        k = i % nb
+        if i >= nb:
+            s_in.wait_event(ev_cmp[k])    # step i-nb has finished reading buffer set k
+        with torch.cuda.stream(s_in):
+            copy_in(k)
+        ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if i >= nb:
+            stream.wait_event(ev_out[k])  # step i-nb's result has left buffer set k
+        with torch.cuda.stream(stream):
+            compute(k)
+        ev_cmp[k].record(stream)
+        s_out.wait_event(ev_cmp[k])
+        with torch.cuda.stream(s_out):
+            copy_out(k)
+        ev_out[k].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+
+
 def run_mfalcon(args, rank, world, local):
     """Time mfalcon_score over every candidate of the M-FALCON workload (the
     history is encoded once beforehand, with its K/V kept per layer)."""
@@ -263,22 +297,45 @@ def run_mfalcon(args, rank, world, local):
         total_ms = float(tt.item())
     ms = total_ms / args.steps
     value = world * M / (ms / 1000.0)
-    # end to end: candidate embeddings in, scores out
+    # end to end: candidate embeddings in, scores out, through the public API.
+    # Serial: copy in, score, copy out, one step after another on one stream.
+    # Pipelined (reported as e2e): two buffer sets, copies of neighbouring steps
+    # overlap the scoring of the current one.
     emb_host = t["cand_emb"].cpu().pin_memory()
-    sc_host = torch.empty(M, dtype=torch.float32).pin_memory()
-    emb_dev = torch.empty_like(t["cand_emb"])
+    NB = 2
+    sc_hosts = [torch.empty(M, dtype=torch.float32).pin_memory() for _ in range(NB)]
+    emb_devs = [torch.empty_like(t["cand_emb"]) for _ in range(NB)]
+    sc_devs = [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(NB)]
 
-    def e2e_step():
-        emb_dev.copy_(emb_host, non_blocking=True)
-        step(emb_dev)
-        sc_host.copy_(scores, non_blocking=True)
+    def score_into(k):
+        H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], emb_devs[k], t["request_ts"],
+                        c.microbatch, c.num_cand, scores=sc_devs[k], workspace=ws_c,
+                        stream=torch.cuda.current_stream())
 
-    e2e_step()
-    torch.cuda.synchronize()
+    def e2e_serial_step():
+        emb_devs[0].copy_(emb_host, non_blocking=True)
+        score_into(0)
+        sc_hosts[0].copy_(sc_devs[0], non_blocking=True)
+
     n_e2e = max(3, min(args.steps, 10))
+    e2e_serial_step()
+    torch.cuda.synchronize()
     a.record(stream)
     for _ in range(n_e2e):
-        e2e_step()
+        e2e_serial_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e_serial_ms = a.elapsed_time(b) / n_e2e
+
+    def run_pipe(n):
+        pipelined_e2e(torch, n, NB, lambda k: emb_devs[k].copy_(emb_host, non_blocking=True),
+                      score_into, lambda k: sc_hosts[k].copy_(sc_devs[k], non_blocking=True),
+                      stream)
+
+    run_pipe(2 * NB)
+    torch.cuda.synchronize()
+    a.record(stream)
+    run_pipe(n_e2e)
     b.record(stream)
     torch.cuda.synchronize()
     e_ms = a.elapsed_time(b) / n_e2e
@@ -307,7 +364,11 @@ def run_mfalcon(args, rank, world, local):
             "clocks": clocks,
             "e2e": {"value": world * M / (e_ms / 1000.0), "unit": "candidates/s",
                     "ms_per_step": e_ms, "h2d_bytes_per_step": int(emb_host.numel() * 2),
-                    "d2h_bytes_per_step": int(M * 4)}}
+                    "d2h_bytes_per_step": int(M * 4),
+                    "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step i-1 "
+                                  "on their own streams overlap step i"},
+            "e2e_serial": {"value": world * M / (e_serial_ms / 1000.0), "unit": "candidates/s",
+                           "ms_per_step": e_serial_ms}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -415,47 +476,80 @@ def main():
     value = world * T / (ms_per_step / 1000.0)
 
     # ---------------- end to end through the public API, host buffers
+    # Every step copies X, offsets and timestamps from pinned host memory and
+    # Y back.  Serial: one step after another on one stream.  Pipelined
+    # (reported as e2e): two buffer sets, the copy-in of step i+1 and the
+    # copy-out of step i-1 overlap the forward of step i.
     e2e = None
+    e2e_serial = None
     if not args.no_e2e:
         x_host = t["x"].cpu().pin_memory()
         off_host = t["offsets"].cpu().pin_memory()
         ts_host = t["timestamps"].cpu().pin_memory()
-        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        x_dev = torch.empty_like(t["x"])
-        off_dev = torch.empty_like(t["offsets"])
-        ts_dev = torch.empty_like(t["timestamps"])
-        jag_e = H.Jagged(off_dev, ts_dev, case.max_len, T)
+        NB = 2
+        y_hosts = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(NB)]
+        x_devs = [torch.empty_like(t["x"]) for _ in range(NB)]
+        off_devs = [torch.empty_like(t["offsets"]) for _ in range(NB)]
+        ts_devs = [torch.empty_like(t["timestamps"]) for _ in range(NB)]
+        y_devs = [torch.empty_like(y) for _ in range(NB)]
+        jags = [H.Jagged(off_devs[k], ts_devs[k], case.max_len, T) for k in range(NB)]
 
-        def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            off_dev.copy_(off_host, non_blocking=True)
-            ts_dev.copy_(ts_host, non_blocking=True)
-            H.forward(cfg, weights, jag_e, x_dev, y_out=y, workspace=ws)
-            y_host.copy_(y, non_blocking=True)
+        def copy_in(k):
+            x_devs[k].copy_(x_host, non_blocking=True)
+            off_devs[k].copy_(off_host, non_blocking=True)
+            ts_devs[k].copy_(ts_host, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
+        def compute(k):
+            H.forward(cfg, weights, jags[k], x_devs[k], y_out=y_devs[k], workspace=ws,
+                      stream=torch.cuda.current_stream())
+
+        def copy_out(k):
+            y_hosts[k].copy_(y_devs[k], non_blocking=True)
+
+        def serial_step():
+            copy_in(0)
+            compute(0)
+            copy_out(0)
+
+        def timed(run, n):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            a.record(stream)
+            run(n)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / n
+            if world > 1:
+                tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                ms = float(tt.item())
+            return ms
+
+        def run_serial(n):
+            for _ in range(n):
+                serial_step()
+
+        def run_pipe(n):
+            pipelined_e2e(torch, n, NB, copy_in, compute, copy_out, stream)
+
         n_e2e = max(3, min(args.steps, 20))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
+        run_serial(2)
         torch.cuda.synchronize()
-        a.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record(stream)
+        e_serial_ms = timed(run_serial, n_e2e)
+        run_pipe(2 * NB)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = timed(run_pipe, n_e2e)
         h2d = (x_host.numel() * x_host.element_size() + off_host.numel() * 8
                + ts_host.numel() * 8)
-        d2h = y_host.numel() * y_host.element_size()
+        d2h = y_hosts[0].numel() * y_hosts[0].element_size()
         e2e = {"value": world * T / (e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step i-1 "
+                             "on their own streams overlap step i"}
+        e2e_serial = {"value": world * T / (e_serial_ms / 1000.0), "unit": "tokens/s",
+                      "ms_per_step": e_serial_ms}
 
     # ---------------- roofline of the dominant kernel (attention), from device events
     peaks, peak_src = load_peaks()
@@ -503,7 +597,7 @@ def main():
                           "pct_of_bf16_peak_sustained": 100 * attn_tflops / peak_sus if attn_tflops else None,
                           "pct_of_bf16_peak_burst": 100 * attn_tflops / peaks["bf16_tflops"] if attn_tflops else None},
             "roofline": roofline, "kernels": kern, "gpu_launches": gpu_launches,
-            "clocks": clocks, "e2e": e2e}
+            "clocks": clocks, "e2e": e2e, "e2e_serial": e2e_serial}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(case)
