@@ -9,19 +9,21 @@
 // inside it; candidate mode (M-FALCON) lets candidate rows see every cached
 // history key and adds each candidate's own key/value in the epilogue.
 //
-// Warp roles (576 threads):
+// Warp roles (608 threads):
 //   warps 0-7   element group A (query tile A): warps 0-3 own key columns
 //               0-31 of every S tile, warps 4-7 columns 32-63; within each
 //               warpgroup thread t owns query row t
 //   warps 8-15  element group B, the same for tile B
-//   warp 16     producer: TMA loads of K, V tiles (128B swizzle) and the
-//               per-key side data (timestamps, or candidate-mode bias)
-//   warp 17     MMA issuer of tile A (one thread) and TMEM owner
-//   warp 18     MMA issuer of tile B (one thread)
-// One issuing thread per query tile: a single thread issuing both tiles'
-// MMAs, with an mbarrier wait in front of every batch, could not keep the
-// tensor pipe fed.  The two issuers touch disjoint tensor memory; a K/V stage
-// is released by one commit from each.
+//   warp 16     producer: TMA loads of the two Q tiles and of the K, V tiles
+//               (128B swizzle, no multicast) and the per-key side data
+//               (int32 times, or the whole candidate-mode bias)
+//   warp 17     MMA issuer of tile A and TMEM owner
+//   warp 18     MMA issuer of tile B
+// Each issuing warp runs its loop together (waits are warp votes) and one
+// lane, elected once, issues every MMA and commit: issued that way the MMA
+// operands stay warp-uniform, and one warp per query tile keeps the tensor
+// pipe fed.  The two issuers touch disjoint tensor memory; a K/V stage is
+// released by one commit from each.
 // Two warpgroups per query tile halve the elements each thread handles per
 // key tile and double the warps that hide tensor-memory, shared-memory and
 // MUFU latency; the work per element is one row-thread's arithmetic either way.
@@ -29,16 +31,16 @@
 // per group (64 fp32 columns each; each half writes its 32 keys of P, bf16
 // pairs, over the first 16 columns of its own 32-column half once they are
 // read) and O_A, O_B (64 fp32 columns each).  S of tile k+3 reuses the buffer
-// of tile k, so it can be issued as soon as P V of tile k is: the MMAs for a
-// tile are issued two tiles before the group needs them, which covers the
+// of tile k, so it is issued right after P V of tile k: the MMAs for a tile
+// are issued two tiles before the group needs them, which covers the
 // issue-to-completion latency of the tensor pipe.  Q_A, Q_B live in shared
-// memory (TMA, 128B swizzle) and S = Q K^T reads both operands from there.
-// Per key tile: S = Q K^T (tcgen05, A from tensor memory), the softmax group
-// reads S row by row, adds the gathered bias, applies phi2 and the mask,
-// writes P (bf16) back over S, then O += P V (tcgen05 with A from tensor
-// memory, V as an MN-major B operand).  The MMAs of one CTA execute in issue
-// order, so S of the next tile is only written after P V has read P.
-// 1/N is applied once to O.
+// memory.
+// Per key tile: S = Q K^T (tcgen05, both operands in shared memory), the
+// element group reads S row by row, adds the gathered bias, applies phi2 and
+// the mask, writes P (bf16) back over S, then O += P V (tcgen05 with A from
+// tensor memory, V as an MN-major B operand).  The MMAs of one issuing thread
+// execute in issue order, so S of tile k+3 is only written after P V of tile
+// k has read P.  1/N is applied once to O.
 //
 // Elementwise work per (query, key, head), SiLU case: x = s + rab, and
 // x*sigmoid(x) = h + h*tanh(h) with h = x/2.  The 1/2 is folded into the bias
@@ -47,9 +49,9 @@
 // two copies offset by one entry, so every thread reads the biases of two
 // adjacent keys with one aligned 8-byte shared load; pairs of keys then go
 // through packed fp32x2 adds and FMAs.  The time bucket only decreases along
-// a row (keys are time-ordered), so a 32-key chunk whose last key still lies
-// in the current bucket needs no per-key work; otherwise a short integer
-// walk over the bucket edges runs per key.
+// a row (keys are time-ordered), so a 32-key chunk whose last visible key
+// still lies in each row's current bucket takes the row's cached time bias;
+// otherwise the chunk is resolved per key (see causal_chunk).
 #pragma once
 
 #include "ptx.cuh"
