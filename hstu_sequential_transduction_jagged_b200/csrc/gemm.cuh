@@ -8,10 +8,15 @@
 //        LayerNorm-and-gate computed by producer warps directly into the
 //        swizzled shared-memory A tile, so Norm(AV) (.) U never reaches HBM.
 //
-// Both are persistent tcgen05 GEMMs: 128 x 256 output tiles, 64-wide K steps
-// through a 4-stage shared-memory ring fed by TMA (128B swizzle), fp32
-// accumulators double-buffered in tensor memory (2 x 256 columns) so the
-// epilogue of one tile overlaps the main loop of the next.
+// Both are persistent tcgen05 GEMMs with 64-wide K steps through a shared-
+// memory ring fed by TMA (128B swizzle), an MMA warp that issues from one
+// elected lane, and epilogue warps that stage 128-byte output row segments in
+// swizzled shared memory for TMA tensor stores.  f1 uses 128 x 256 tiles, 4
+// stages and two tensor-memory accumulators (2 x 256 columns), so the
+// epilogue of one tile overlaps the main loop of the next.  f2 uses 128-row
+// tiles covering up to 512 output columns (two 256-column halves side by side
+// in tensor memory), so its A operand is built once per row tile, with 2
+// stages and a single accumulator.
 #pragma once
 
 #include "ptx.cuh"
