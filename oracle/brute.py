@@ -7,7 +7,8 @@ either one shows up as a disagreement.
 
 Follows the review of "Actions Speak Louder than Words" (xllm-io paper-review
 of arXiv 2402.17152), section 三 核心公式 Eq. 1-3, with the same readings as
-`oracle.hstu` (SiLU/ReLU/identity phi2, 1/n_u, LayerNorm over H*dv,
+`oracle.hstu` (SiLU/ReLU/identity phi2 with 1/n_u, or the softmax ablation
+over the visible keys; LayerNorm over H*dv,
 ln(dt+1)/0.301 time buckets, min(i-j, P-1) position buckets, residual).
 """
 from __future__ import annotations
@@ -66,15 +67,25 @@ def layer(x, offsets, ts, w1, b1, w2, b2, rab_pos, rab_time, H, dqk, dv,
             # Eq. 2 for row i, every head
             o = [0.0] * hv
             for h in range(H):
+                pre = []
                 for j in range(i + 1):
                     dot = 0.0
                     for t in range(dqk):
                         dot += Q[i][h * dqk + t] * K[j][h * dqk + t]
                     bp = min(i - j, P - 1)
                     bt = _tbucket(ts[s + i] - ts[s + j], Tb)
-                    a = _act(dot + rab_pos[h][bp] + rab_time[h][bt], phi2) / n
+                    pre.append(dot + rab_pos[h][bp] + rab_time[h][bt])
+                if phi2 == "softmax":
+                    # ablation: softmax over the visible keys j <= i, no 1/n
+                    top = max(pre)
+                    ex = [math.exp(val - top) for val in pre]
+                    tot = sum(ex)
+                    weights = [val / tot for val in ex]
+                else:
+                    weights = [_act(val, phi2) / n for val in pre]
+                for j in range(i + 1):
                     for t in range(dv):
-                        o[h * dv + t] += a * V[j][h * dv + t]
+                        o[h * dv + t] += weights[j] * V[j][h * dv + t]
             # Eq. 3: LayerNorm over all heads, gate with U, project, residual
             mean = sum(o) / hv
             var = sum((val - mean) * (val - mean) for val in o) / hv

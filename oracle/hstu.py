@@ -29,6 +29,11 @@ documented constant here, never hidden):
   * Norm is LayerNorm over the H*dv concatenated heads of one token, biased
     variance, eps = 1e-5, optional affine (gamma, beta).
   * Residual: Y = X + f2(...).  No pre-norm, no final norm.
+  * phi2 = "softmax" is the ablation "HSTU (-rab, Softmax)" of the review's
+    section 六 (消融实验, HSTU 组件消融) and section 五 (industrial streaming
+    table): the pointwise phi2 and its 1/N are replaced by a row-wise softmax
+    over the visible keys of the same pre-activation Q K^T + rab (no extra
+    scale; "-rab" is the same with zero bias tables).
   * M-FALCON: a candidate sits at position n_u with timestamp t_req, attends to
     the user's cached history rows (keys/values of every layer) and to itself
     (position bucket 0, time bucket 0); its score is <y_c^(L), e_c>.  Its
@@ -99,9 +104,27 @@ def rab_matrix(ts_q: np.ndarray, ts_k: np.ndarray, pos_q: np.ndarray, pos_k: np.
     return rab_pos_h[bp] + rab_time_h[bt]
 
 
+def attention_weights(s: np.ndarray, mask: np.ndarray, phi2: str, n_norm: int) -> np.ndarray:
+    """Attention weights from the pre-activations s = Q K^T + rab of one head.
+
+    Pointwise phi2 (Eq. 2): a_ij = phi2(s_ij) / N for visible keys, 0 otherwise.
+    Softmax ablation: a_ij = exp(s_ij) / sum over visible j' of exp(s_ij') for
+    visible keys (a row with no visible key gets all zeros); N is not used.
+    """
+    if phi2 == "softmax":
+        z = np.where(mask, s, -np.inf)
+        m = z.max(axis=1, keepdims=True)
+        m = np.where(np.isfinite(m), m, 0.0)
+        e = np.where(mask, np.exp(np.where(mask, s, 0.0) - m), 0.0)
+        den = e.sum(axis=1, keepdims=True)
+        return e / np.where(den > 0.0, den, 1.0)
+    return np.where(mask, phi(s, phi2), 0.0) / float(n_norm)
+
+
 def user_attention(q, k, v, ts, rab_pos, rab_time, n_norm: int, H: int, dqk: int, dv: int,
                    phi2: str = "silu") -> np.ndarray:
-    """Eq. 2 for one user: causal pointwise attention, per head, divided by N.
+    """Eq. 2 for one user: causal pointwise attention, per head, divided by N
+    (or the softmax ablation, see attention_weights).
 
     q, k: [n, H*dqk]; v: [n, H*dv]; ts: [n] int64; returns AV [n, H*dv].
     """
@@ -116,7 +139,7 @@ def user_attention(q, k, v, ts, rab_pos, rab_time, n_norm: int, H: int, dqk: int
         kh = k[:, h * dqk:(h + 1) * dqk]
         vh = v[:, h * dv:(h + 1) * dv]
         s = qh @ kh.T + rab_matrix(ts, ts, pos, pos, rab_pos[h], rab_time[h])
-        a = np.where(mask, phi(s, phi2), 0.0) / float(n_norm)
+        a = attention_weights(s, mask, phi2, n_norm)
         out[:, h * dv:(h + 1) * dv] = a @ vh
     return out
 
@@ -209,12 +232,14 @@ def history_kv(x, offsets, timestamps, layers, cfg):
 
 
 def mfalcon_scores(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_emb,
-                   request_ts, microbatch: int, kv=None) -> np.ndarray:
+                   request_ts, microbatch: int, kv=None, return_rows: bool = False):
     """M-FALCON: score every candidate against its user's cached history.
 
     Candidates of a user are taken b_m at a time; inside a microbatch each
     candidate's row only sees the history keys/values and its own key/value,
     so the microbatch size changes the schedule, not the result.
+    `kv` = (per-layer K list, per-layer V list) replaces the history encode.
+    With return_rows the final residual-stream rows y_c^(L) are returned too.
     """
     H, dqk, dv = cfg.num_heads, cfg.dqk, cfg.dv
     if kv is None:
@@ -223,6 +248,7 @@ def mfalcon_scores(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_
         ks, vs = kv
     e_all = _f64(cand_emb)
     scores = np.zeros(e_all.shape[0])
+    rows = np.zeros_like(e_all)
     B = len(offsets) - 1
     for uu in range(B):
         hs, he = int(offsets[uu]), int(offsets[uu + 1])
@@ -253,12 +279,17 @@ def mfalcon_scores(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_
                     own_k = k[:, h * dqk:(h + 1) * dqk]
                     own_v = v[:, h * dv:(h + 1) * dv]
                     s_self = np.einsum("cd,cd->c", qh, own_k) + rp[h, 0] + rt[h, 0]
-                    o = phi(s_hist, cfg.phi2) @ vh + phi(s_self, cfg.phi2)[:, None] * own_v
-                    av[:, h * dv:(h + 1) * dv] = o / float(max(n_u, 1))
+                    # keys of a candidate row: the n_u history rows, then itself
+                    s_all = np.concatenate([s_hist, s_self[:, None]], axis=1)
+                    a = attention_weights(s_all, np.ones(s_all.shape, dtype=bool), cfg.phi2,
+                                          max(n_u, 1))
+                    o = a[:, :n_u] @ vh + a[:, n_u:n_u + 1] * own_v
+                    av[:, h * dv:(h + 1) * dv] = o
                 xc, _ = output(xc, av, u, w2, b2, cfg.ln_eps, _f64(layer.ln_gamma),
                                _f64(layer.ln_beta))
             scores[mb:mend] = np.einsum("cd,cd->c", xc, e)
-    return scores
+            rows[mb:mend] = xc
+    return (scores, rows) if return_rows else scores
 
 
 def score_alone(hist_x, offsets, timestamps, layers, cfg, cand_offsets, cand_emb,

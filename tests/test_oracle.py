@@ -126,29 +126,95 @@ def test_closed_form_linear_recurrence(n):
             assert np.allclose(av[i, sl], q[i, sl] @ state / N, rtol=1e-11, atol=1e-12)
 
 
-def test_jagged_equals_padded_and_masked():
-    case = make_case(_tiny_cfg(), seed=3, lengths=[5, 1, 9, 3])
+@pytest.mark.parametrize("phi2", ["silu", "softmax"])
+def test_jagged_equals_padded_and_masked(phi2):
+    """Jagged users equal a padded batch with a key-padding mask.  The padding
+    sits BEFORE each user's rows (left padding), where the causal mask alone
+    would let every real row see it: only the key-padding mask removes the
+    garbage keys, positions count from the user's first real row and N = n_u.
+    A jagged implementation that leaked across users, miscounted positions or
+    used the padded length as N would differ."""
+    case = make_case(_tiny_cfg(phi2=phi2), seed=3, lengths=[5, 1, 9, 3])
     cfg, lw = case.cfg, case.layers[0]
     x = case.x.astype(np.float64)
     ref = O.layer_fwd(x, case.offsets, case.timestamps, lw, cfg)["av"]
-    maxlen = case.max_len
+    Lp = case.max_len + 4
     rng = np.random.default_rng(0)
+    H, dqk, dv = cfg.num_heads, cfg.dqk, cfg.dv
+    rp, rt = lw.rab_pos.astype(float), lw.rab_time.astype(float)
     for uu in range(len(case.offsets) - 1):
         s, e = case.offsets[uu], case.offsets[uu + 1]
         n = e - s
-        pad = rng.standard_normal((maxlen, cfg.d_model)) * 100.0  # garbage padding
-        pad[:n] = x[s:e]
-        ts = np.concatenate([case.timestamps[s:e], rng.integers(0, 10**9, maxlen - n)])
-        u, v, q, k = O.projection(pad, lw.w1.astype(float), lw.b1.astype(float),
-                                  cfg.num_heads, cfg.dqk, cfg.dv)
-        av = O.user_attention(q, k, v, ts, lw.rab_pos.astype(float), lw.rab_time.astype(float),
-                              n, cfg.num_heads, cfg.dqk, cfg.dv, cfg.phi2)
-        assert np.array_equal(av[:n], ref[s:e])
+        padn = Lp - n
+        seq = np.concatenate([rng.standard_normal((padn, cfg.d_model)) * 100.0, x[s:e]])
+        ts = np.concatenate([rng.integers(0, 10**9, padn), case.timestamps[s:e]])
+        pos = np.arange(Lp) - padn                      # real rows at positions 0..n-1
+        real = pos >= 0
+        mask = (pos[None, :] <= pos[:, None]) & real[None, :]
+        u, v, q, k = O.projection(seq, lw.w1.astype(float), lw.b1.astype(float), H, dqk, dv)
+        av = np.zeros((Lp, H * dv))
+        for h in range(H):
+            sh = (q[:, h * dqk:(h + 1) * dqk] @ k[:, h * dqk:(h + 1) * dqk].T
+                  + O.rab_matrix(ts, ts, pos, pos, rp[h], rt[h]))
+            a = O.attention_weights(sh, mask, phi2, n)
+            av[:, h * dv:(h + 1) * dv] = a @ v[:, h * dv:(h + 1) * dv]
+        assert np.allclose(av[padn:], ref[s:e], rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one():
+    """Softmax ablation: the weights of each row sum to 1 over its visible keys,
+    so with V = 1 every output entry is exactly 1 (up to rounding), whatever Q, K, rab."""
+    rng = np.random.default_rng(21)
+    n, H, dh = 13, 2, 4
+    q, k = rng.standard_normal((n, H * dh)) * 3, rng.standard_normal((n, H * dh)) * 3
+    v = np.ones((n, H * dh))
+    ts = np.sort(rng.integers(0, 10**7, n))
+    rp, rt = rng.standard_normal((H, 20)), rng.standard_normal((H, 40))
+    av = O.user_attention(q, k, v, ts, rp, rt, n, H, dh, dh, "softmax")
+    assert np.allclose(av, 1.0, rtol=0, atol=1e-13)
+
+
+def test_softmax_equals_torch_attention():
+    """Softmax ablation against torch's scaled_dot_product_attention (float64,
+    scale 1, additive bias = rab plus -inf above the diagonal)."""
+    import torch
+    rng = np.random.default_rng(22)
+    n, H, dh = 11, 3, 4
+    q, k, v = (rng.standard_normal((n, H * dh)) for _ in range(3))
+    ts = np.sort(rng.integers(0, 10**6, n))
+    rp, rt = rng.standard_normal((H, 6)), rng.standard_normal((H, 32))
+    av = O.user_attention(q, k, v, ts, rp, rt, n, H, dh, dh, "softmax")
+    pos = np.arange(n)
+    for h in range(H):
+        bias = O.rab_matrix(ts, ts, pos, pos, rp[h], rt[h])
+        bias = np.where(pos[None, :] <= pos[:, None], bias, -np.inf)
+        sl = slice(h * dh, (h + 1) * dh)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[None, None, :, sl]), torch.from_numpy(k[None, None, :, sl]),
+            torch.from_numpy(v[None, None, :, sl]), attn_mask=torch.from_numpy(bias[None, None]),
+            scale=1.0)[0, 0].numpy()
+        assert np.allclose(av[:, sl], want, rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_invariant_to_constant_bias():
+    """Adding one constant to every rab entry leaves the softmax weights unchanged
+    (and changes the pointwise result, which has no such invariance)."""
+    rng = np.random.default_rng(23)
+    n, H, dh = 9, 1, 4
+    q, k, v = (rng.standard_normal((n, H * dh)) for _ in range(3))
+    ts = np.sort(rng.integers(0, 10**6, n))
+    rp, rt = rng.standard_normal((H, 5)), rng.standard_normal((H, 30))
+    a = O.user_attention(q, k, v, ts, rp, rt, n, H, dh, dh, "softmax")
+    b = O.user_attention(q, k, v, ts, rp + 0.7, rt, n, H, dh, dh, "softmax")
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+    c = O.user_attention(q, k, v, ts, rp, rt, n, H, dh, dh, "silu")
+    d = O.user_attention(q, k, v, ts, rp + 0.7, rt, n, H, dh, dh, "silu")
+    assert not np.allclose(c, d)
 
 
 # --------------------------------------------------------------------------- whole layer
 
-@pytest.mark.parametrize("phi2", ["silu", "relu", "identity"])
+@pytest.mark.parametrize("phi2", ["silu", "relu", "identity", "softmax"])
 @pytest.mark.parametrize("affine", [False, True])
 def test_brute_force_equals_vectorised(phi2, affine):
     cfg = _tiny_cfg(phi2=phi2)
@@ -243,8 +309,10 @@ def _mf_case(seed=7, lengths=(6, 1, 0, 11), m=5):
     return make_case(cfg, seed=seed, lengths=list(lengths))
 
 
-def test_mfalcon_equals_scoring_alone():
+@pytest.mark.parametrize("phi2", ["silu", "softmax"])
+def test_mfalcon_equals_scoring_alone(phi2):
     case = _mf_case()
+    case.cfg = case.cfg.replace(phi2=phi2)
     cfg = case.cfg
     sc = O.mfalcon_scores(case.x, case.offsets, case.timestamps, case.layers, cfg,
                           case.cand_offsets, case.cand_emb, case.request_ts, 2)
