@@ -11,7 +11,10 @@ shards with no collective: weak scaling).
 Prints one JSON line (rank 0).  `value` is whole-job tokens/s with inputs
 resident in HBM; `e2e` is the same metric through the public API with the
 inputs copied from pinned host memory and the output copied back inside the
-timed region.  `--impl reference` times the float64 CPU oracle instead.
+timed region.  At N = 1 the line also carries `workloads`: the other
+configurations (tiny fp32, small bf16, Stochastic Length, M-FALCON scoring)
+timed the same way, each with its own roofline.  `--impl reference` times the
+float64 CPU oracle instead.
 """
 from __future__ import annotations
 
@@ -40,6 +43,13 @@ WORKLOAD_TEXT = {
                "cached history, 2048 candidates per user in microbatches of 256",
 }
 MFALCON_METRIC = "M-FALCON candidate scores/sec at 1 B200 (cached history K/V)"
+# The attention launches of these workloads last about a millisecond inside
+# steps of a few milliseconds, far from the seconds-long matmul loop that
+# defines the sustained figure, so their roofline uses the burst peak.
+PEAK_RULE = ("burst: the kernel is timed per launch (~0.05-1.2 ms) inside short steps; "
+             "the sustained figure belongs to a seconds-long loop")
+# fp32 FFMA peak for the fp32 SIMT workload: 148 SMs x 128 FMA/clk x 2 flop x clock
+FP32_LANES_PER_SM = 128
 
 
 def load_peaks():
@@ -53,14 +63,25 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 
+def gpu_selector(torch, local: int) -> str:
+    """nvidia-smi id of the GPU torch calls cuda:local.  nvidia-smi ignores
+    CUDA_VISIBLE_DEVICES, so the CUDA ordinal is not an NVML index: select by
+    UUID (or PCI bus id when the UUID is unavailable)."""
+    props = torch.cuda.get_device_properties(local)
+    u = str(getattr(props, "uuid", "") or "")
+    if u:
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
         self.proc = None
         self.path = None
 
@@ -78,7 +99,8 @@ class ClockSampler:
 
     def stop(self) -> dict:
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "gpu": self.gpu}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -92,46 +114,71 @@ class ClockSampler:
                     rows.append(parts)
         os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "gpu": self.gpu}
         sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
         mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "gpu": self.gpu}
 
 
 # ----------------------------------------------------------------------------- oracle baseline
 
-def oracle_sample(case, target_s: float = 15.0):
-    """Time the float64 oracle on a causal prefix of user 0 (both layers).
-
-    Rows 0..m-1 of a user depend only on its first m tokens, so the prefix is
-    an exact piece of the workload; m is grown until one run takes about
-    target_s seconds (or the whole user is covered)."""
-    from oracle import hstu as O
-    import numpy as np
-    n0 = int(case.offsets[1] - case.offsets[0])
-    m = min(512, n0)
-    while True:
-        t0 = time.perf_counter()
-        O.forward(case.x, case.offsets, case.timestamps, case.layers, case.cfg,
-                  users=[0], prefix=[m])
-        dt = time.perf_counter() - t0
-        if m >= n0 or dt >= target_s * 0.5:
-            break
-        # causal work grows about quadratically in the prefix length
-        m = min(n0, int(m * min(4.0, max(1.2, math.sqrt(target_s / max(dt, 1e-3))))))
+def _oracle_cores():
     cores = os.cpu_count()
     try:
         from threadpoolctl import threadpool_info
         threads = max((i.get("num_threads", 0) for i in threadpool_info()), default=cores)
     except Exception:
         threads = cores
-    return {"value": m / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"float64 oracle, user 0 causal prefix of {m} of {n0} tokens, "
-                      f"all {case.cfg.num_layers} layers, {dt:.1f} s",
-            "host_cpu_count": cores, "seconds": dt}
+    return threads, cores
+
+
+def oracle_extrapolated(case, target_s: float = 15.0):
+    """The float64 oracle's rate on the whole workload, extrapolated from two
+    timed causal prefixes of user 0.
+
+    Rows 0..m-1 of a user depend only on its first m tokens, so a prefix is an
+    exact piece of the workload.  The oracle's cost per user is a per-token
+    term (projection, LayerNorm, f2) plus a per-(query, key) term (it forms
+    dense n x n matrices per head): t(m) = a m + b m^2.  Prefixes m and m/2 are
+    timed (all layers), a and b solved, and t = sum_u (a n_u + b n_u^2) gives
+    the whole-workload time.  Labelled extrapolated."""
+    from oracle import hstu as O
+    n0 = int(case.offsets[1] - case.offsets[0])
+
+    def run(m):
+        t0 = time.perf_counter()
+        O.forward(case.x, case.offsets, case.timestamps, case.layers, case.cfg,
+                  users=[0], prefix=[m])
+        return time.perf_counter() - t0
+
+    m = min(256, n0)
+    dt = run(m)
+    while m < n0 and dt < 0.45 * target_s:
+        m = min(n0, int(m * min(4.0, max(1.25, math.sqrt(0.6 * target_s / max(dt, 1e-3))))))
+        dt = run(m)
+    m1 = max(1, m // 2)
+    dt1 = run(m1)
+    # t = a m + b m^2 through both points (b >= 0, a >= 0)
+    if m1 == m:
+        a, b = dt / m, 0.0
+    else:
+        b = max(0.0, (dt / m - dt1 / m1) / (m - m1))
+        a = max(0.0, dt / m - b * m)
+    n = case.lengths.astype(float)
+    t_full = float(sum(a * x + b * x * x for x in n))
+    tokens = float(n.sum())
+    threads, cores = _oracle_cores()
+    return {"value": tokens / t_full, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "extrapolated": True,
+            "sample": f"float64 oracle on causal prefixes of user 0 ({m1} and {m} of {n0} tokens, "
+                      f"all {case.cfg.num_layers} layers: {dt1:.2f} s and {dt:.2f} s); "
+                      f"t(m) = a m + b m^2 fitted (a={a:.3e} s/token, b={b:.3e} s/pair) and "
+                      f"extrapolated to the whole workload ({int(tokens)} tokens, "
+                      f"{len(n)} users): {t_full:.0f} s",
+            "host_cpu_count": cores, "seconds_timed": dt + dt1, "seconds_extrapolated": t_full}
 
 
 def run_reference(args, rank, world):
@@ -140,26 +187,25 @@ def run_reference(args, rank, world):
         return
     from gen import make_case
     case = make_case(args.workload)
-    samples = []
     for _ in range(args.warmup):
-        oracle_sample(case, target_s=2.0)
-    for _ in range(args.steps):
-        samples.append(oracle_sample(case, target_s=args.ref_seconds))
-    v = sum(s["value"] for s in samples) / len(samples)
+        oracle_extrapolated(case, target_s=1.0)
+    samples = [oracle_extrapolated(case, target_s=args.ref_seconds) for _ in range(args.steps)]
+    vals = sorted(s["value"] for s in samples)
+    v = vals[len(vals) // 2]
     last = samples[-1]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000.0 * last["seconds"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": 1000.0 * last["seconds_extrapolated"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload)},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": last["cores"],
-                             "kind": "oracle", "sample": last["sample"]},
+                             "kind": "oracle", "extrapolated": True, "sample": last["sample"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ----------------------------------------------------------------------------- main arm
+# ----------------------------------------------------------------------------- helpers
 
 def traffic_from_profiles(kernel: str):
     """DRAM bytes per launch of `kernel` from a committed ncu summary, if its
@@ -220,160 +266,317 @@ def pipelined_e2e(torch, n_steps, nb, copy_in, compute, copy_out, stream):
     stream.wait_stream(s_out)
 
 
-def run_mfalcon(args, rank, world, local):
+class Ctx:
+    """Per-process GPU context shared by the workload measurements."""
+
+    def __init__(self, args, rank, world, local):
+        import torch
+        import torch.distributed as dist
+        from hstu_sequential_transduction_jagged_b200 import build as hbuild
+        from hstu_sequential_transduction_jagged_b200 import hstu as H
+        self.torch, self.dist, self.H = torch, dist, H
+        self.args, self.rank, self.world, self.local = args, rank, world, local
+        torch.cuda.set_device(local)
+        self.dev = torch.device("cuda", local)
+        if world > 1:
+            from datetime import timedelta
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=self.dev)
+        if rank == 0:
+            hbuild.build()
+        if world > 1:
+            dist.barrier()
+        self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=self.dev)  # > L2
+        self.stream = torch.cuda.current_stream()
+        self.peaks, self.peak_src = load_peaks()
+        self.gpu_id = gpu_selector(torch, local)
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed_steps(self, step, steps, sample_clocks=True):
+        """`steps` calls of step(), each bracketed by CUDA events on the launching
+        stream, an L2 flush (256 MiB write) before each outside the events.
+        Returns (per-step ms list, library per-kernel times, clocks)."""
+        torch, H = self.torch, self.H
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        sampler = ClockSampler(self.gpu_id) if sample_clocks else None
+        if sampler:
+            sampler.start()
+        if self.world > 1:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        H.profiler_start()
+        for i in range(steps):
+            self.flush.zero_()
+            evs[i][0].record(self.stream)
+            step()
+            evs[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        kernels = H.profiler_stop()
+        if self.world > 1:
+            self.dist.barrier()
+        clocks = sampler.stop() if sampler else None
+        assert H.device_status() == 0
+        return [a.elapsed_time(b) for a, b in evs], kernels, clocks
+
+
+def _median(xs):
+    s = sorted(xs)
+    n = len(s)
+    return s[n // 2] if n % 2 else 0.5 * (s[n // 2 - 1] + s[n // 2])
+
+
+def _kernel_table(kernels):
+    tot = max(1e-9, sum(v[1] for v in kernels.values()))
+    return {k: {"launches": n, "ms_per_launch": m / n, "share": m / tot}
+            for k, (n, m) in kernels.items()}
+
+
+def _roofline(ctx, kernels, name, flop, kernel_label, bound="tensor"):
+    n, ms = kernels.get(name, (0, 0.0))
+    if not n:
+        return None
+    per = ms / n
+    achieved = flop / (per / 1000.0) / 1e12
+    if bound == "alu":
+        # fp32 SIMT kernels: FFMA lanes x 2 flop x max SM clock
+        peak = 148 * FP32_LANES_PER_SM * 2 * ctx.peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        src = "derived: 148 SMs x 128 fp32 FMA lanes x 2 flop x max SM clock"
+    else:
+        peak = ctx.peaks["bf16_tflops"]
+        src = f"{ctx.peak_src} bf16 dense, burst ({PEAK_RULE})"
+    out = {"kernel": kernel_label, "bound": bound, "achieved": achieved, "peak": peak,
+           "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": src,
+           "algorithmic_flop_per_launch": flop, "ms_per_launch": per}
+    if bound == "tensor":
+        sus = ctx.peaks.get("bf16_tflops_sustained")
+        if sus:
+            out["frac_of_sustained"] = achieved / sus
+    return out
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batch=None):
+    """Time hstu_forward over one workload; returns a dict (value, rooflines...)."""
+    torch, H = ctx.torch, ctx.H
+    from gen import make_case, algorithmic_counts
+    from gen.device import case_tensors
+    case = make_case(name, batch=batch)
+    c = case.cfg
+    counts = algorithmic_counts(case)
+    t = case_tensors(case, ctx.dev)
+    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
+    weights = [H.LayerWeights(**lw) for lw in t["layers"]]
+    cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets,
+                        dqk=c.dqk, dv=c.dv, phi1=c.phi1, phi2=c.phi2, ln_eps=c.ln_eps,
+                        dtype=c.dtype)
+    L, T = c.num_layers, case.total_tokens
+    ws = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=ctx.dev)
+    y = torch.empty((T, c.d_model), dtype=torch.float32, device=ctx.dev)
+
+    def step():
+        H.forward(cfg, weights, jag, t["x"], y_out=y, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    step_ms, kernels, clocks = ctx.timed_steps(step, steps, sample_clocks)
+    total = ctx.max_over_ranks(sum(step_ms))
+    ms = total / steps
+    value = ctx.world * T / (ms / 1000.0)
+    world = ctx.world
+    bf16 = c.dtype == "bf16"
+    attn_name = "attention" if bf16 else "fp32_attention"
+    roof = _roofline(ctx, kernels, attn_name, counts["attn_flop_per_layer"],
+                     "hstu_attn_kernel (causal)" if bf16 else "hstu_f32_attn_kernel (causal)",
+                     "tensor" if bf16 else "alu")
+    if roof is not None and name == "long-bf16":
+        roof["traffic"] = traffic_from_profiles("attention")
+    kern = _kernel_table(kernels)
+    for kname, key in (("f1_gemm", "f1_flop_per_layer"), ("f2_gemm", "f2_flop_per_layer")):
+        if kname in kern:
+            per = kern[kname]["ms_per_launch"]
+            kern[kname]["tflops"] = counts[key] / (per / 1000.0) / 1e12
+            kern[kname]["frac_of_bf16_burst"] = kern[kname]["tflops"] / ctx.peaks["bf16_tflops"]
+    if "f2_gemm" in kern:
+        # algorithmic bytes of f2: AV and U (fp32), residual (fp32 after layer 0), Y fp32 + bf16 copy
+        d, hv = c.d_model, c.num_heads * c.dv
+        byt = T * (hv * 4 * 2 + d * 4 + d * 4 + d * 2) + d * hv * 2
+        kern["f2_gemm"]["algorithmic_bytes"] = byt
+        kern["f2_gemm"]["gbs"] = byt / (kern["f2_gemm"]["ms_per_launch"] / 1000.0) / 1e9
+        kern["f2_gemm"]["frac_of_hbm"] = kern["f2_gemm"]["gbs"] / ctx.peaks["hbm_gbs"]
+    out = {"metric": "tokens/s", "value": value, "unit": "tokens/s",
+           "workload": WORKLOAD_TEXT[name], "ms_per_step": ms,
+           "ms_per_step_median": _median(step_ms), "tokens_per_step": world * T,
+           "layer_tokens_per_s": value * L, "layers": L, "dtype": c.dtype,
+           "roofline": roof, "kernels": kern, "gpu_launches": sum(n for n, _ in kernels.values()),
+           "clocks": clocks, "_case": case}
+    if with_e2e:
+        out.update(forward_e2e(ctx, case, t, cfg, weights, ws, y, steps))
+    return out
+
+
+def forward_e2e(ctx, case, t, cfg, weights, ws, y, steps):
+    """Same forward through the public API with host buffers: X, offsets and
+    timestamps copied from pinned host memory and Y copied back, every step.
+    Serial: one step after another.  Pipelined (reported as e2e): two buffer
+    sets, the copy-in of step i+1 and copy-out of step i-1 overlap step i."""
+    torch, H = ctx.torch, ctx.H
+    T = case.total_tokens
+    x_host = t["x"].cpu().pin_memory()
+    off_host = t["offsets"].cpu().pin_memory()
+    ts_host = t["timestamps"].cpu().pin_memory()
+    NB = 2
+    y_hosts = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(NB)]
+    x_devs = [torch.empty_like(t["x"]) for _ in range(NB)]
+    off_devs = [torch.empty_like(t["offsets"]) for _ in range(NB)]
+    ts_devs = [torch.empty_like(t["timestamps"]) for _ in range(NB)]
+    y_devs = [torch.empty_like(y) for _ in range(NB)]
+    jags = [H.Jagged(off_devs[k], ts_devs[k], case.max_len, T) for k in range(NB)]
+
+    def copy_in(k):
+        x_devs[k].copy_(x_host, non_blocking=True)
+        off_devs[k].copy_(off_host, non_blocking=True)
+        ts_devs[k].copy_(ts_host, non_blocking=True)
+
+    def compute(k):
+        H.forward(cfg, weights, jags[k], x_devs[k], y_out=y_devs[k], workspace=ws,
+                  stream=torch.cuda.current_stream())
+
+    def copy_out(k):
+        y_hosts[k].copy_(y_devs[k], non_blocking=True)
+
+    def run_serial(n):
+        for _ in range(n):
+            copy_in(0)
+            compute(0)
+            copy_out(0)
+
+    def run_pipe(n):
+        pipelined_e2e(torch, n, NB, copy_in, compute, copy_out, ctx.stream)
+
+    def timed(run, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ctx.world > 1:
+            ctx.dist.barrier()
+        torch.cuda.synchronize()
+        a.record(ctx.stream)
+        run(n)
+        b.record(ctx.stream)
+        torch.cuda.synchronize()
+        return ctx.max_over_ranks(a.elapsed_time(b) / n)
+
+    n_e2e = max(3, min(steps, 20))
+    run_serial(2)
+    torch.cuda.synchronize()
+    e_serial_ms = timed(run_serial, n_e2e)
+    run_pipe(2 * NB)
+    torch.cuda.synchronize()
+    e_ms = timed(run_pipe, n_e2e)
+    h2d = x_host.numel() * x_host.element_size() + off_host.numel() * 8 + ts_host.numel() * 8
+    d2h = y_hosts[0].numel() * y_hosts[0].element_size()
+    w = ctx.world
+    return {"e2e": {"value": w * T / (e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e_ms,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step i-1 "
+                                  "on their own streams overlap step i"},
+            "e2e_serial": {"value": w * T / (e_serial_ms / 1000.0), "unit": "tokens/s",
+                           "ms_per_step": e_serial_ms}}
+
+
+def measure_mfalcon(ctx, steps, warmup, with_e2e, sample_clocks=True, batch=None):
     """Time mfalcon_score over every candidate of the M-FALCON workload (the
     history is encoded once beforehand, with its K/V kept per layer)."""
     import numpy as np
-    import torch
-    import torch.distributed as dist
+    torch, H = ctx.torch, ctx.H
     from gen import make_case
     from gen.device import case_tensors
-    from hstu_sequential_transduction_jagged_b200 import build as hbuild
-    from hstu_sequential_transduction_jagged_b200 import hstu as H
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    if rank == 0:
-        hbuild.build()
-    if world > 1:
-        dist.barrier()
-    case = make_case("mfalcon", batch=args.batch)
+    case = make_case("mfalcon", batch=batch)
     c = case.cfg
-    t = case_tensors(case, dev)
+    t = case_tensors(case, ctx.dev)
     jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
     weights = [H.LayerWeights(**lw) for lw in t["layers"]]
     cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets)
     L, T, hv = c.num_layers, case.total_tokens, c.num_heads * 64
     M = t["cand_emb"].shape[0]
-    kv = torch.empty((L, T, 2 * hv), dtype=torch.bfloat16, device=dev)
-    ws_h = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=dev)
-    ws_c = torch.empty(H.mfalcon_workspace_bytes(cfg, M), dtype=torch.uint8, device=dev)
-    scores = torch.empty(M, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
-    # history encode (timed on its own)
+    kv = torch.empty((L, T, 2 * hv), dtype=torch.bfloat16, device=ctx.dev)
+    ws_h = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=ctx.dev)
+    ws_c = torch.empty(H.mfalcon_workspace_bytes(cfg, M), dtype=torch.uint8, device=ctx.dev)
+    scores = torch.empty(M, dtype=torch.float32, device=ctx.dev)
     for _ in range(2):
         H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv, workspace=ws_h)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    a.record(stream)
+    a.record(ctx.stream)
     H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv, workspace=ws_h)
-    b.record(stream)
+    b.record(ctx.stream)
     torch.cuda.synchronize()
     hist_ms = a.elapsed_time(b)
 
-    def step(emb):
-        H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], emb, t["request_ts"],
+    def step():
+        H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], t["cand_emb"], t["request_ts"],
                         c.microbatch, c.num_cand, scores=scores, workspace=ws_c)
 
-    for _ in range(args.warmup):
-        step(t["cand_emb"])
+    for _ in range(warmup):
+        step()
     torch.cuda.synchronize()
     assert H.device_status() == 0
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    H.profiler_start()
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        step(t["cand_emb"])
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    kernels = H.profiler_stop()
-    clocks = sampler.stop()
-    assert H.device_status() == 0
-    total_ms = sum(x.elapsed_time(y) for x, y in evs)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    ms = total_ms / args.steps
-    value = world * M / (ms / 1000.0)
-    # end to end: candidate embeddings in, scores out, through the public API.
-    # Serial: copy in, score, copy out, one step after another on one stream.
-    # Pipelined (reported as e2e): two buffer sets, copies of neighbouring steps
-    # overlap the scoring of the current one.
-    emb_host = t["cand_emb"].cpu().pin_memory()
-    NB = 2
-    sc_hosts = [torch.empty(M, dtype=torch.float32).pin_memory() for _ in range(NB)]
-    emb_devs = [torch.empty_like(t["cand_emb"]) for _ in range(NB)]
-    sc_devs = [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(NB)]
-
-    def score_into(k):
-        H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], emb_devs[k], t["request_ts"],
-                        c.microbatch, c.num_cand, scores=sc_devs[k], workspace=ws_c,
-                        stream=torch.cuda.current_stream())
-
-    def e2e_serial_step():
-        emb_devs[0].copy_(emb_host, non_blocking=True)
-        score_into(0)
-        sc_hosts[0].copy_(sc_devs[0], non_blocking=True)
-
-    n_e2e = max(3, min(args.steps, 10))
-    e2e_serial_step()
-    torch.cuda.synchronize()
-    a.record(stream)
-    for _ in range(n_e2e):
-        e2e_serial_step()
-    b.record(stream)
-    torch.cuda.synchronize()
-    e_serial_ms = a.elapsed_time(b) / n_e2e
-
-    def run_pipe(n):
-        pipelined_e2e(torch, n, NB, lambda k: emb_devs[k].copy_(emb_host, non_blocking=True),
-                      score_into, lambda k: sc_hosts[k].copy_(sc_devs[k], non_blocking=True),
-                      stream)
-
-    run_pipe(2 * NB)
-    torch.cuda.synchronize()
-    a.record(stream)
-    run_pipe(n_e2e)
-    b.record(stream)
-    torch.cuda.synchronize()
-    e_ms = a.elapsed_time(b) / n_e2e
-    peaks, peak_src = load_peaks()
-    peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    step_ms, kernels, clocks = ctx.timed_steps(step, steps, sample_clocks)
+    ms = ctx.max_over_ranks(sum(step_ms)) / steps
+    value = ctx.world * M / (ms / 1000.0)
     n_u = case.lengths.astype(np.float64)
     cand_flop = float(((n_u + 1) * c.num_cand).sum()) * c.num_heads * 256  # per layer
-    ca_n, ca_ms = kernels.get("mfalcon_attention", (0, 0.0))
-    ca_tf = cand_flop / (ca_ms / ca_n / 1000.0) / 1e12 if ca_n else None
-    kern = {k: {"launches": n, "ms_per_launch": m / n} for k, (n, m) in kernels.items()}
-    line = {"metric": MFALCON_METRIC, "value": value, "unit": "candidates/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT["mfalcon"], "candidates_per_step": world * M,
-                       "history_tokens": T, "layers": L, "microbatch": c.microbatch,
-                       "l2": "flushed between timed steps (256 MiB write outside the events)",
-                       "parallelism": f"dp{world}: users sharded, no collective"},
-            "history_encode_ms": hist_ms,
-            "roofline": {"kernel": "hstu_attn_kernel (candidate)", "bound": "tensor",
-                         "achieved": ca_tf, "peak": peak_sus, "unit": "TFLOP/s",
-                         "frac": ca_tf / peak_sus if ca_tf else None, "traffic": None,
-                         "peak_source": f"{peak_src} bf16 dense, sustained",
-                         "algorithmic_flop_per_launch": cand_flop},
-            "kernels": kern, "gpu_launches": sum(n for n, _ in kernels.values()),
-            "clocks": clocks,
-            "e2e": {"value": world * M / (e_ms / 1000.0), "unit": "candidates/s",
-                    "ms_per_step": e_ms, "h2d_bytes_per_step": int(emb_host.numel() * 2),
-                    "d2h_bytes_per_step": int(M * 4),
-                    "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step i-1 "
-                                  "on their own streams overlap step i"},
-            "e2e_serial": {"value": world * M / (e_serial_ms / 1000.0), "unit": "candidates/s",
-                           "ms_per_step": e_serial_ms}}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    roof = _roofline(ctx, kernels, "mfalcon_attention", cand_flop, "hstu_attn_kernel (candidate)")
+    out = {"metric": MFALCON_METRIC, "value": value, "unit": "candidates/s",
+           "workload": WORKLOAD_TEXT["mfalcon"], "ms_per_step": ms,
+           "ms_per_step_median": _median(step_ms), "candidates_per_step": ctx.world * M,
+           "history_tokens": T, "layers": L, "microbatch": c.microbatch,
+           "history_encode_ms": hist_ms, "roofline": roof, "kernels": _kernel_table(kernels),
+           "gpu_launches": sum(n for n, _ in kernels.values()), "clocks": clocks}
+    if with_e2e:
+        emb_host = t["cand_emb"].cpu().pin_memory()
+        NB = 2
+        sc_hosts = [torch.empty(M, dtype=torch.float32).pin_memory() for _ in range(NB)]
+        emb_devs = [torch.empty_like(t["cand_emb"]) for _ in range(NB)]
+        sc_devs = [torch.empty(M, dtype=torch.float32, device=ctx.dev) for _ in range(NB)]
+
+        def score_into(k):
+            H.mfalcon_score(cfg, weights, jag, kv, t["cand_offsets"], emb_devs[k],
+                            t["request_ts"], c.microbatch, c.num_cand, scores=sc_devs[k],
+                            workspace=ws_c, stream=torch.cuda.current_stream())
+
+        def run_pipe(n):
+            pipelined_e2e(torch, n, NB, lambda k: emb_devs[k].copy_(emb_host, non_blocking=True),
+                          score_into, lambda k: sc_hosts[k].copy_(sc_devs[k], non_blocking=True),
+                          ctx.stream)
+
+        n_e2e = max(3, min(steps, 10))
+        run_pipe(2 * NB)
+        torch.cuda.synchronize()
+        a.record(ctx.stream)
+        run_pipe(n_e2e)
+        b.record(ctx.stream)
+        torch.cuda.synchronize()
+        e_ms = ctx.max_over_ranks(a.elapsed_time(b) / n_e2e)
+        out["e2e"] = {"value": ctx.world * M / (e_ms / 1000.0), "unit": "candidates/s",
+                      "ms_per_step": e_ms, "h2d_bytes_per_step": int(emb_host.numel() * 2),
+                      "d2h_bytes_per_step": int(M * 4),
+                      "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step "
+                                    "i-1 on their own streams overlap step i"}
+    return out
+
+
+# ----------------------------------------------------------------------------- main
+
+def _public(d):
+    return {k: v for k, v in d.items() if not k.startswith("_")}
 
 
 def main():
@@ -385,6 +588,8 @@ def main():
     ap.add_argument("--workload", default="long-bf16", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations (profiling runs)")
     ap.add_argument("--ref-seconds", type=float, default=15.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="fewer users than the workload (profiling runs only)")
@@ -399,213 +604,60 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+
+    ctx = Ctx(args, rank, world, local)
     if args.workload == "mfalcon":
-        run_mfalcon(args, rank, world, local)
-        return
-
-    import numpy as np
-    import torch
-    import torch.distributed as dist
-    from gen import make_case, algorithmic_counts
-    from gen.device import case_tensors
-    from hstu_sequential_transduction_jagged_b200 import build as hbuild
-    from hstu_sequential_transduction_jagged_b200 import hstu as H
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+        r = measure_mfalcon(ctx, args.steps, args.warmup, not args.no_e2e, batch=args.batch)
+        line = {"metric": MFALCON_METRIC, "value": r["value"], "unit": "candidates/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD_TEXT["mfalcon"],
+                           "candidates_per_step": r["candidates_per_step"],
+                           "l2": "flushed between timed steps (256 MiB write outside the events)",
+                           "parallelism": f"dp{world}: users sharded, no collective"}}
+        line.update({k: v for k, v in r.items() if k not in line and k != "metric"})
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    else:
+        r = measure_forward(ctx, args.workload, args.steps, args.warmup, not args.no_e2e,
+                            batch=args.batch)
+        case = r["_case"]
+        line = {"metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+                "ms_per_step_median": r["ms_per_step_median"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": case.cfg.dtype,
+                "data": "synthetic",
+                "config": {"workload": WORKLOAD_TEXT[args.workload],
+                           "global_batch": world * len(case.lengths), "seq_len": case.max_len,
+                           "tokens_per_step": world * case.total_tokens,
+                           "layers": case.cfg.num_layers,
+                           "l2": "flushed between timed steps (256 MiB write outside the events)",
+                           "parallelism": f"dp{world}: users sharded, no collective"},
+                "layer_tokens_per_s": r["layer_tokens_per_s"], "roofline": r["roofline"],
+                "kernels": r["kernels"], "gpu_launches": r["gpu_launches"],
+                "clocks": r["clocks"], "e2e": r.get("e2e"), "e2e_serial": r.get("e2e_serial")}
+        if r["roofline"]:
+            line["attention"] = {"tflops": r["roofline"]["achieved"],
+                                 "pct_of_bf16_peak_burst": 100 * r["roofline"]["frac"],
+                                 "pct_of_bf16_peak_sustained":
+                                     100 * r["roofline"].get("frac_of_sustained", 0.0)}
+        if world == 1 and not args.no_workloads and args.batch is None:
+            subs = {}
+            for name in ("small-bf16", "sl-bf16", "tiny-fp32"):
+                if name == args.workload:
+                    continue
+                subs[name] = _public(measure_forward(ctx, name, min(args.steps, 20), args.warmup,
+                                                     False, sample_clocks=(name == "sl-bf16")))
+            subs["mfalcon"] = measure_mfalcon(ctx, min(args.steps, 20), args.warmup, True)
+            line["workloads"] = subs
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_extrapolated(case)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=dev)
-    if rank == 0:
-        hbuild.build()
-    if world > 1:
-        dist.barrier()
-
-    case = make_case(args.workload, batch=args.batch)
-    cfgd = case.cfg
-    counts = algorithmic_counts(case)
-    t = case_tensors(case, dev)
-    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
-    weights = [H.LayerWeights(**lw) for lw in t["layers"]]
-    cfg = H.LayerConfig(cfgd.d_model, cfgd.num_heads, cfgd.num_pos_buckets, cfgd.num_time_buckets,
-                        dqk=cfgd.dqk, dv=cfgd.dv, phi1=cfgd.phi1, phi2=cfgd.phi2,
-                        ln_eps=cfgd.ln_eps, dtype=cfgd.dtype)
-    L = cfgd.num_layers
-    T = case.total_tokens
-    ws = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=dev)
-    y = torch.empty((T, cfgd.d_model), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
-    stream = torch.cuda.current_stream()
-
-    def step(x_in):
-        H.forward(cfg, weights, jag, x_in, y_out=y, workspace=ws)
-
-    for _ in range(args.warmup):
-        step(t["x"])
-    torch.cuda.synchronize()
-    assert H.device_status() == 0
-
-    # ---------------- timed region: inputs resident in HBM, L2 flushed between steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    H.profiler_start()
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        step(t["x"])
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    kernels = H.profiler_stop()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    assert H.device_status() == 0
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1000.0)
-
-    # ---------------- end to end through the public API, host buffers
-    # Every step copies X, offsets and timestamps from pinned host memory and
-    # Y back.  Serial: one step after another on one stream.  Pipelined
-    # (reported as e2e): two buffer sets, the copy-in of step i+1 and the
-    # copy-out of step i-1 overlap the forward of step i.
-    e2e = None
-    e2e_serial = None
-    if not args.no_e2e:
-        x_host = t["x"].cpu().pin_memory()
-        off_host = t["offsets"].cpu().pin_memory()
-        ts_host = t["timestamps"].cpu().pin_memory()
-        NB = 2
-        y_hosts = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(NB)]
-        x_devs = [torch.empty_like(t["x"]) for _ in range(NB)]
-        off_devs = [torch.empty_like(t["offsets"]) for _ in range(NB)]
-        ts_devs = [torch.empty_like(t["timestamps"]) for _ in range(NB)]
-        y_devs = [torch.empty_like(y) for _ in range(NB)]
-        jags = [H.Jagged(off_devs[k], ts_devs[k], case.max_len, T) for k in range(NB)]
-
-        def copy_in(k):
-            x_devs[k].copy_(x_host, non_blocking=True)
-            off_devs[k].copy_(off_host, non_blocking=True)
-            ts_devs[k].copy_(ts_host, non_blocking=True)
-
-        def compute(k):
-            H.forward(cfg, weights, jags[k], x_devs[k], y_out=y_devs[k], workspace=ws,
-                      stream=torch.cuda.current_stream())
-
-        def copy_out(k):
-            y_hosts[k].copy_(y_devs[k], non_blocking=True)
-
-        def serial_step():
-            copy_in(0)
-            compute(0)
-            copy_out(0)
-
-        def timed(run, n):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            if world > 1:
-                dist.barrier()
-            torch.cuda.synchronize()
-            a.record(stream)
-            run(n)
-            b.record(stream)
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / n
-            if world > 1:
-                tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                ms = float(tt.item())
-            return ms
-
-        def run_serial(n):
-            for _ in range(n):
-                serial_step()
-
-        def run_pipe(n):
-            pipelined_e2e(torch, n, NB, copy_in, compute, copy_out, stream)
-
-        n_e2e = max(3, min(args.steps, 20))
-        run_serial(2)
-        torch.cuda.synchronize()
-        e_serial_ms = timed(run_serial, n_e2e)
-        run_pipe(2 * NB)
-        torch.cuda.synchronize()
-        e_ms = timed(run_pipe, n_e2e)
-        h2d = (x_host.numel() * x_host.element_size() + off_host.numel() * 8
-               + ts_host.numel() * 8)
-        d2h = y_hosts[0].numel() * y_hosts[0].element_size()
-        e2e = {"value": world * T / (e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "pipelining": "2 buffer sets; copy-in of step i+1 and copy-out of step i-1 "
-                             "on their own streams overlap step i"}
-        e2e_serial = {"value": world * T / (e_serial_ms / 1000.0), "unit": "tokens/s",
-                      "ms_per_step": e_serial_ms}
-
-    # ---------------- roofline of the dominant kernel (attention), from device events
-    peaks, peak_src = load_peaks()
-    attn_launches, attn_ms = kernels.get("attention", (0, 0.0))
-    attn_flop = counts["attn_flop_per_layer"]  # algorithmic: causal pairs x H x 256
-    attn_tflops = attn_flop / (attn_ms / attn_launches / 1000.0) / 1e12 if attn_launches else None
-    peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    roofline = {"kernel": "hstu_attn_kernel (causal)", "bound": "tensor",
-                "achieved": attn_tflops, "peak": peak_sus, "unit": "TFLOP/s",
-                "frac": (attn_tflops / peak_sus) if attn_tflops else None,
-                "traffic": traffic_from_profiles("attention"),
-                "peak_source": f"{peak_src} bf16 dense, sustained (kernel timed inside a long step)",
-                "algorithmic_flop_per_launch": attn_flop,
-                "ms_per_launch": attn_ms / attn_launches if attn_launches else None}
-    kern = {}
-    for name, (n, ms) in kernels.items():
-        ent = {"launches": n, "ms_per_launch": ms / n, "share": ms / max(1e-9, sum(
-            v[1] for v in kernels.values()))}
-        if name == "f1_gemm":
-            ent["tflops"] = counts["f1_flop_per_layer"] / (ms / n / 1000.0) / 1e12
-            ent["frac_of_peak"] = ent["tflops"] / peak_sus
-        if name == "f2_gemm":
-            ent["tflops"] = counts["f2_flop_per_layer"] / (ms / n / 1000.0) / 1e12
-            ent["frac_of_peak"] = ent["tflops"] / peak_sus
-            # algorithmic bytes: AV, U (fp32), X residual (bf16 or fp32), Y fp32 (+bf16), W2
-            T_, d, hv = T, cfgd.d_model, cfgd.num_heads * cfgd.dv
-            byt = T_ * (hv * 4 * 2 + d * 4 + d * 4 + d * 2) + d * hv * 2
-            ent["gbs_approx"] = byt / (ms / n / 1000.0) / 1e9
-        if name == "attention":
-            ent["tflops"] = attn_tflops
-        kern[name] = ent
-    gpu_launches = sum(n for n, _ in kernels.values())
-
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": cfgd.dtype, "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT[args.workload], "global_batch": world * case.cfg.batch
-                       if args.workload != "sl-bf16" else world * len(case.lengths),
-                       "seq_len": case.max_len, "tokens_per_step": world * T, "layers": L,
-                       "l2": "flushed between timed steps (256 MiB write outside the events)",
-                       "parallelism": f"dp{world}: users sharded, no collective"},
-            "layer_tokens_per_s": value * L,
-            "attention": {"tflops": attn_tflops,
-                          "pct_of_bf16_peak_sustained": 100 * attn_tflops / peak_sus if attn_tflops else None,
-                          "pct_of_bf16_peak_burst": 100 * attn_tflops / peaks["bf16_tflops"] if attn_tflops else None},
-            "roofline": roofline, "kernels": kern, "gpu_launches": gpu_launches,
-            "clocks": clocks, "e2e": e2e, "e2e_serial": e2e_serial}
-
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample(case)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+        ctx.dist.barrier()
+        ctx.dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -87,6 +87,7 @@ struct AttnParams {
   int64_t ld_av;
   float* ln_part;              // [T_q, H, 2] (sum, centred sum of squares) or nullptr
   int32_t B, H, P, Tb;
+  int32_t max_q, max_kv;       // host-declared length bounds the launch is sized for
   int32_t num_qpairs;
   int32_t pos_len;             // floats per staged copy of the position table
   int32_t phi2;
@@ -244,21 +245,23 @@ enum : int {
 
 // ---------------------------------------------------------------- causal chunk
 
-// One 32-key chunk of one causal row: S values in `sv` -> packed bf16 P in `pk`.
-// `rvx` points at the staged position table entry of column 0 (entries for
-// consecutive columns are consecutive), `kts` at the chunk's key times
-// (seconds since the user's first event, 16-byte aligned).  Columns above
-// `lim` are masked (P = 0) and never move the time-bucket walk; lim < 0 masks
-// the whole chunk.  The walk `w` enters at the bucket of the previous key and
-// leaves at the bucket of the last visible key.  Per warp the chunk falls in
-// one of three cases:
+// One 32-key chunk of one causal row: the pre-activations h = scale * (s + rab)
+// of its key pairs are handed to `sink(c, h2)` (columns c, c + 1 packed as an
+// fp32 pair), in live lanes only.  `rvx` points at the staged position table
+// entry of column 0 (entries for consecutive columns are consecutive), `kts`
+// at the chunk's key times (seconds since the user's first event, 16-byte
+// aligned).  Columns above `lim` are masked by the caller and never move the
+// time-bucket walk; lim < 0 marks a lane with no visible key in the chunk
+// (the sink is not called).  The walk `w` enters at the bucket of the previous
+// key and leaves at the bucket of the last visible key.  Per warp the chunk
+// falls in one of three cases:
 //   every row keeps its bucket      -> one time bias per row, `rt_cur`, kept
 //                                      in a register (one compare of the last
 //                                      visible key against the bucket edge);
 //   two buckets B, B+1 in the warp  -> per key: B+1 iff t_j <= t_i - thr[B+1];
 //   more (near the diagonal)        -> per key bias from the octave tables.
-template <int PHI, bool PAIRS>
-__device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16],
+template <bool PAIRS, class Sink>
+__device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], Sink&& sink,
                                              const float* rvx, const int32_t* kts, int lim,
                                              BucketWalk<int32_t>& w, const float* sTime,
                                              const int64_t* sThr, const int4* sOct,
@@ -281,15 +284,7 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
     if (live) {
       const uint64_t rt2 = f2_pack(rt_cur, rt_cur);
 #pragma unroll
-      for (int c = 0; c < 32; c += 2)
-        pk[c >> 1] = phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
-      if (lim < 31) {
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, lim);
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < 16; ++q) pk[q] = 0u;
+      for (int c = 0; c < 32; c += 2) sink(c, f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
     }
     return;
   }
@@ -309,8 +304,7 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
       const float rt = sTime[b_first];
       const uint64_t rt2 = f2_pack(rt, rt);
 #pragma unroll
-      for (int c = 0; c < 32; c += 2)
-        pk[c >> 1] = phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
+      for (int c = 0; c < 32; c += 2) sink(c, f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), rt2)));
     }
   } else {
     const int B_hi = __reduce_max_sync(full, b_first);
@@ -326,8 +320,7 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
           const int2 k2 = kt_pair(c);
           const float r0 = (k2.x <= edge) ? rt_hi : rt_lo;
           const float r1 = (k2.y <= edge) ? rt_hi : rt_lo;
-          pk[c >> 1] =
-              phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
+          sink(c, f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
         }
       }
     } else if (live) {
@@ -336,12 +329,23 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], uint32_t 
         const int2 k2 = kt_pair(c);
         const float r0 = time_bias_octave(w.ti - k2.x, sOct, sOrt);
         const float r1 = time_bias_octave(w.ti - k2.y, sOct, sOrt);
-        pk[c >> 1] =
-            phi_pair<PHI>(f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
+        sink(c, f2_fma(s_pair(c), scale2, f2_add(pos_pair(c), f2_pack(r0, r1))));
       }
     }
   }
-  if (!live) {
+}
+
+// Pointwise phi2 of one causal chunk: packed bf16 P in `pk`, masked above `lim`.
+template <int PHI, bool PAIRS>
+__device__ __forceinline__ void causal_chunk_pointwise(const uint32_t (&sv)[32], uint32_t (&pk)[16],
+                                                       const float* rvx, const int32_t* kts, int lim,
+                                                       BucketWalk<int32_t>& w, const float* sTime,
+                                                       const int64_t* sThr, const int4* sOct,
+                                                       const float4* sOrt, uint64_t scale2,
+                                                       float& rt_cur) {
+  causal_chunk<PAIRS>(sv, [&](int c, uint64_t h2) { pk[c >> 1] = phi_pair<PHI>(h2); }, rvx, kts,
+                      lim, w, sTime, sThr, sOct, sOrt, scale2, rt_cur);
+  if (lim < 0) {
 #pragma unroll
     for (int q = 0; q < 16; ++q) pk[q] = 0u;
   } else if (lim < 31) {
@@ -374,6 +378,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   } else {
     q_start = kv_start;
     n_q = n_kv;
+  }
+  // The grid and the staged position table are sized from the host-declared
+  // maximum lengths; a user longer than declared would leave rows unwritten
+  // or read past the staged table, so it is reported and nothing runs.
+  if (n_q > p.max_q || n_kv > p.max_kv || n_q < 0 || n_kv < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_status(HSTU_ERR_DEVICE_CHECK);
+    return;  // uniform across the CTA, before any allocation
   }
   const int q0 = qp * 2 * ATT_ROWS;
   if (q0 >= n_q) return;  // uniform across the CTA, before any allocation
@@ -713,8 +724,9 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // last visible column: keys after the row are masked; rows past the
         // user's end are not stored and skip the work
         const int lim = !valid ? -1 : i - j0;
-        causal_chunk<PHI, PAIRS>(sv, pk, rv + xc, reinterpret_cast<const int32_t*>(key) + half * 32,
-                                 lim, w32, sTime, sThr, sOct, sOrt, scale2, rt_cur);
+        causal_chunk_pointwise<PHI, PAIRS>(sv, pk, rv + xc,
+                                           reinterpret_cast<const int32_t*>(key) + half * 32, lim,
+                                           w32, sTime, sThr, sOct, sOrt, scale2, rt_cur);
       }
     };
 

@@ -90,6 +90,7 @@ struct F32AttnParams {
   int64_t ld_av;
   int32_t B, H, P, Tb, phi2;
   int32_t cand;
+  int32_t max_q, max_kv;  // host-declared length bounds the grid is sized for
   int64_t thr[MAX_TIME_BUCKETS];
 };
 
@@ -111,6 +112,10 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
   const int n_kv = static_cast<int>(p.kv_offsets[u + 1] - kv0);
   const int64_t q0g = p.cand ? p.q_offsets[u] : kv0;
   const int n_q = p.cand ? static_cast<int>(p.q_offsets[u + 1] - q0g) : n_kv;
+  if (n_q > p.max_q || n_kv > p.max_kv || n_q < 0 || n_kv < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(HSTU_ERR_DEVICE_CHECK);
+    return;
+  }
   const int r0 = blockIdx.x * 32;
   if (r0 >= n_q) return;
   for (int e = threadIdx.x; e < p.Tb; e += blockDim.x) sthr[e] = p.thr[e];

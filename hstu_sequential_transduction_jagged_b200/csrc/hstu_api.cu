@@ -297,6 +297,8 @@ hstu_status_t check_jag(const hstu_jagged_t* j) {
   if (j->batch > 0 && j->offsets == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
   if (j->total_tokens > 0 && (j->timestamps == nullptr || j->batch == 0))
     return HSTU_ERR_INVALID_ARGUMENT;
+  // a batch with rows has a user of length >= 1; the kernels are sized from max_len
+  if (j->total_tokens > 0 && j->max_len == 0) return HSTU_ERR_INVALID_ARGUMENT;
   if (j->max_len > kMaxLen || j->batch > 65535) return HSTU_ERR_UNSUPPORTED;
   if (j->total_tokens > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
   return HSTU_OK;
@@ -418,6 +420,8 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.H = c->num_heads;
   p.P = c->num_pos_buckets;
   p.Tb = c->num_time_buckets;
+  p.max_q = j.max_q_len;
+  p.max_kv = j.max_kv_len;
   p.num_qpairs = (j.max_q_len + 2 * ATT_ROWS - 1) / (2 * ATT_ROWS);
   // largest staged-table origin D over the CTAs, plus the diagonal overhang
   const size_t dmax = CAND ? static_cast<size_t>(j.max_kv_len)
@@ -596,6 +600,8 @@ hstu_status_t launch_f32_attn(const AttnJob& j, cudaStream_t st) {
   p.Tb = c->num_time_buckets;
   p.phi2 = c->phi2;
   p.cand = j.q_offsets != nullptr ? 1 : 0;
+  p.max_q = j.max_q_len;
+  p.max_kv = j.max_kv_len;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
   dim3 grid((j.max_q_len + 31) / 32, c->num_heads, j.batch);
   ProfScope prof(K_F32_ATTN, st);
@@ -801,6 +807,93 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
   return launch_attn_bf16<false>(j, st);
 }
 
+hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
+                                const void* q, const void* k, const void* v, const float* rab_pos,
+                                const float* rab_time, float* av_out, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (jag->total_tokens == 0 || jag->batch == 0) return HSTU_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || rab_pos == nullptr ||
+      rab_time == nullptr || av_out == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(av_out))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  const int64_t hv = static_cast<int64_t>(cfg->num_heads) * ATT_HD;
+  AttnJob j;
+  std::memset(&j, 0, sizeof(j));
+  j.cfg = cfg;
+  j.kv_offsets = jag->offsets;
+  j.timestamps = jag->timestamps;
+  j.batch = jag->batch;
+  j.max_q_len = j.max_kv_len = jag->max_len;
+  j.T_q = j.T_kv = jag->total_tokens;
+  j.q = q; j.ldq = hv;
+  j.k = k; j.ldk = hv;
+  j.v = v; j.ldv = hv;
+  j.rab_pos = rab_pos;
+  j.rab_time = rab_time;
+  j.ld_av = hv;
+  j.timeout_ns = kDefaultTimeoutNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == HSTU_FP32) {
+    j.av = av_out;
+    return launch_f32_attn(j, st);
+  }
+  j.av_f32 = av_out;
+  return launch_attn_bf16<false>(j, st);
+}
+
+hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* history,
+                               const void* k_hist, const void* v_hist,
+                               const int64_t* cand_offsets, int64_t num_cand, int32_t max_cand,
+                               const void* q, const void* k, const void* v,
+                               const int64_t* request_ts, const float* rab_pos,
+                               const float* rab_time, float* av_out, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(history)) != HSTU_OK) return s;
+  if (num_cand < 0 || max_cand < 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (num_cand == 0 || history->batch == 0) return HSTU_OK;
+  if (max_cand == 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (max_cand > kMaxLen || num_cand > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
+  if (cand_offsets == nullptr || q == nullptr || k == nullptr || v == nullptr ||
+      request_ts == nullptr || rab_pos == nullptr || rab_time == nullptr || av_out == nullptr ||
+      (history->total_tokens > 0 && (k_hist == nullptr || v_hist == nullptr)))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_hist) ||
+      !aligned16(v_hist) || !aligned16(av_out))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  const int64_t hv = static_cast<int64_t>(cfg->num_heads) * ATT_HD;
+  AttnJob j;
+  std::memset(&j, 0, sizeof(j));
+  j.cfg = cfg;
+  j.kv_offsets = history->offsets;
+  j.q_offsets = cand_offsets;
+  j.timestamps = history->timestamps;
+  j.request_ts = request_ts;
+  j.batch = history->batch;
+  j.max_q_len = max_cand;
+  j.max_kv_len = history->max_len;
+  j.T_q = num_cand;
+  j.T_kv = history->total_tokens;
+  j.q = q; j.ldq = hv;
+  j.k = k_hist; j.ldk = hv;
+  j.v = v_hist; j.ldv = hv;
+  j.q_self = q; j.k_self = k; j.v_self = v; j.ld_self = hv;
+  j.rab_pos = rab_pos;
+  j.rab_time = rab_time;
+  j.ld_av = hv;
+  j.timeout_ns = kDefaultTimeoutNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == HSTU_FP32) {
+    j.av = av_out;
+    return launch_f32_attn(j, st);
+  }
+  j.av_f32 = av_out;
+  return launch_attn_bf16<true>(j, st);
+}
+
 hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
                              const hstu_jagged_t* jag, const void* x_in, const float* x_res,
                              float* y_out, void* y_out_lp, void* kv_cache_out, void* workspace,
@@ -897,8 +990,8 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                             const hstu_layer_weights_t* weights, const hstu_jagged_t* history,
                             const void* kv_cache, const int64_t* cand_offsets, int64_t num_cand,
                             int32_t max_cand, const void* cand_emb, const int64_t* request_ts,
-                            int32_t microbatch, float* scores, void* workspace, size_t ws_bytes,
-                            void* stream) {
+                            int32_t microbatch, float* scores, float* cand_y_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
   hstu_status_t s;
   if ((s = check_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(history)) != HSTU_OK) return s;
@@ -908,11 +1001,13 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
     if ((s = check_weights(cfg, &weights[l])) != HSTU_OK) return s;
   if (num_cand == 0 || history->batch == 0) return HSTU_OK;
   if (max_cand > kMaxLen) return HSTU_ERR_UNSUPPORTED;
+  if (max_cand == 0) return HSTU_ERR_INVALID_ARGUMENT;  // num_cand > 0 here
   if (num_cand > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
   if (cand_offsets == nullptr || cand_emb == nullptr || request_ts == nullptr ||
       scores == nullptr || (history->total_tokens > 0 && kv_cache == nullptr))
     return HSTU_ERR_INVALID_ARGUMENT;
-  if (!aligned16(cand_emb) || !aligned16(kv_cache) || !aligned16(workspace))
+  if (!aligned16(cand_emb) || !aligned16(kv_cache) || !aligned16(workspace) ||
+      !aligned16(cand_y_out))
     return HSTU_ERR_INVALID_ARGUMENT;
   if (workspace == nullptr || ws_bytes < hstu_mfalcon_workspace_bytes(cfg, num_cand))
     return HSTU_ERR_WORKSPACE_TOO_SMALL;
@@ -951,7 +1046,8 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
     j.v = cache_l + static_cast<size_t>(hv) * e;
     j.ldv = 2 * hv;
     const float* xres = (l == 0) ? nullptr : yf[(l - 1) & 1];
-    float* yo = yf[l & 1];
+    // the last layer writes the caller's buffer when one is given
+    float* yo = (l == num_layers - 1 && cand_y_out != nullptr) ? cand_y_out : yf[l & 1];
     if (cfg->dtype == HSTU_FP32) {
       const float* xin = (l == 0) ? static_cast<const float*>(cand_emb) : yf[(l - 1) & 1];
       s = layer_fp32(cfg, &weights[l], j, xin, xres, M, yo, nullptr, ws, true, st);
@@ -961,7 +1057,7 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
     }
     if (s != HSTU_OK) return s;
   }
-  const float* yfin = yf[(num_layers - 1) & 1];
+  const float* yfin = cand_y_out != nullptr ? cand_y_out : yf[(num_layers - 1) & 1];
   const unsigned blocks = static_cast<unsigned>((M * 32 + 255) / 256);
   ProfScope prof(K_SCORE, st);
   if (cfg->dtype == HSTU_FP32)

@@ -63,6 +63,9 @@ EXPORTS = {
                                      [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64]),
     "hstu_mfalcon_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int64]),
     "hstu_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "hstu_attn_fwd_f32": (ctypes.c_int, [ctypes.c_void_p] * 9),
+    "mfalcon_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64, ctypes.c_int32]
+                         + [ctypes.c_void_p] * 8),
     "hstu_layer_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hstu_layer_fwd_static": (ctypes.c_int, [ctypes.c_void_p] * 9),
     "hstu_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32] + [ctypes.c_void_p] * 6
@@ -71,7 +74,8 @@ EXPORTS = {
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
-                                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.c_void_p]),
     "hstu_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "hstu_profiler_start": (ctypes.c_int, []),
     "hstu_profiler_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]),
@@ -215,6 +219,34 @@ def attn_fwd(cfg: LayerConfig, jag: Jagged, q, k, v, rab_pos, rab_time, av_out=N
     return av_out
 
 
+def attn_fwd_f32(cfg: LayerConfig, jag: Jagged, q, k, v, rab_pos, rab_time, av_out=None,
+                 stream=None) -> torch.Tensor:
+    """Eq. 2 over a jagged batch with the result in fp32: AV[T, H*dv] float32."""
+    if av_out is None:
+        av_out = torch.empty((jag.total_tokens, cfg.num_heads * cfg.dv), dtype=torch.float32,
+                             device=q.device)
+    c, j = cfg.c(), jag.c()
+    _check(lib().hstu_attn_fwd_f32(ctypes.byref(c), ctypes.byref(j), _p(q), _p(k), _p(v),
+                                   _p(rab_pos), _p(rab_time), _p(av_out), _stream(stream)),
+           "hstu_attn_fwd_f32")
+    return av_out
+
+
+def mfalcon_attn_fwd(cfg: LayerConfig, history: Jagged, k_hist, v_hist, cand_offsets,
+                     max_cand: int, q, k, v, request_ts, rab_pos, rab_time, av_out=None,
+                     stream=None) -> torch.Tensor:
+    """Candidate-mode attention alone (history keys/values plus self): AV [M, H*dv] fp32."""
+    M = q.shape[0]
+    if av_out is None:
+        av_out = torch.empty((M, cfg.num_heads * cfg.dv), dtype=torch.float32, device=q.device)
+    c, j = cfg.c(), history.c()
+    _check(lib().mfalcon_attn_fwd(ctypes.byref(c), ctypes.byref(j), _p(k_hist), _p(v_hist),
+                                  _p(cand_offsets), M, max_cand, _p(q), _p(k), _p(v),
+                                  _p(request_ts), _p(rab_pos), _p(rab_time), _p(av_out),
+                                  _stream(stream)), "mfalcon_attn_fwd")
+    return av_out
+
+
 def layer_fwd(cfg: LayerConfig, w: LayerWeights, jag: Jagged, x_in, x_res=None, y_out=None,
               y_out_lp=None, kv_cache_out=None, workspace=None, stream=None) -> torch.Tensor:
     """One HSTU layer; returns the fp32 residual-stream output Y [T, d]."""
@@ -266,8 +298,9 @@ def forward(cfg: LayerConfig, weights: Sequence[LayerWeights], jag: Jagged, x_in
 
 def mfalcon_score(cfg: LayerConfig, weights: Sequence[LayerWeights], history: Jagged, kv_cache,
                   cand_offsets, cand_emb, request_ts, microbatch: int, max_cand: int,
-                  scores=None, workspace=None, stream=None) -> torch.Tensor:
-    """M-FALCON candidate scores [num_cand] fp32."""
+                  scores=None, cand_y_out=None, workspace=None, stream=None) -> torch.Tensor:
+    """M-FALCON candidate scores [num_cand] fp32.  With `cand_y_out` ([num_cand, d]
+    float32) each candidate's final residual-stream row is written there too."""
     dev = cand_emb.device
     M = cand_emb.shape[0]
     L = len(weights)
@@ -278,7 +311,8 @@ def mfalcon_score(cfg: LayerConfig, weights: Sequence[LayerWeights], history: Ja
     c, j = cfg.c(), history.c()
     _check(lib().mfalcon_score(ctypes.byref(c), L, arr, ctypes.byref(j), _p(kv_cache),
                                _p(cand_offsets), M, max_cand, _p(cand_emb), _p(request_ts),
-                               microbatch, _p(scores), _p(ws), ws.numel(), _stream(stream)),
+                               microbatch, _p(scores), _p(cand_y_out), _p(ws), ws.numel(),
+                               _stream(stream)),
            "mfalcon_score")
     return scores
 

@@ -72,7 +72,9 @@ typedef enum { HSTU_ACT_IDENTITY = 0, HSTU_ACT_RELU = 1, HSTU_ACT_SILU = 2 } hst
 typedef struct {
   int32_t batch;              /* B >= 0 */
   int64_t total_tokens;       /* T == offsets[B], known to the caller (no device read) */
-  int32_t max_len;            /* >= max_u (offsets[u+1] - offsets[u]) */
+  int32_t max_len;            /* >= max_u (offsets[u+1] - offsets[u]); >= 1 when T > 0.
+                                 Kernels are sized from it: a longer user is reported
+                                 as HSTU_ERR_DEVICE_CHECK and its rows are not computed */
   const int64_t* offsets;     /* device [B+1], offsets[0] = 0, non-decreasing */
   const int64_t* timestamps;  /* device [T], int64 seconds */
 } hstu_jagged_t;
@@ -131,6 +133,44 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
                             void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Eq. 2 alone with an fp32 result: the same computation as hstu_attn_fwd, with
+ * AV written in fp32 (the precision the layer path hands to Norm(.) of Eq. 3)
+ * instead of being rounded to cfg->dtype.
+ *   q, k, v  device [T, H*64] in cfg->dtype; av_out device [T, H*64] fp32.
+ *   rab_pos device [H, P] fp32, rab_time device [H, Tb] fp32.
+ * Needs no workspace.  Rows of av_out belonging to users are written.  A user
+ * longer than jag->max_len is reported as HSTU_ERR_DEVICE_CHECK in the device
+ * status word and its rows are not written.
+ */
+hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
+                                const void* q, const void* k, const void* v,
+                                const float* rab_pos, const float* rab_time, float* av_out,
+                                void* stream);
+
+/*
+ * Eq. 2 in candidate mode alone (the attention step of M-FALCON, section 三,
+ * M-FALCON 推理算法): every candidate row c of user u sits at position n_u with
+ * timestamp request_ts[u] and attends to all n_u cached history keys/values of
+ * u and to its own key/value (position bucket 0, time bucket 0):
+ *   AV_c = ( sum_j phi2(q_c.k_j + rab_pos[h, min(n_u - j, P-1)]
+ *                        + rab_time[h, bt(t_req - t_j)]) v_j
+ *            + phi2(q_c.k_c + rab_pos[h, 0] + rab_time[h, 0]) v_c ) / max(n_u, 1).
+ *   history      jagged history (offsets, timestamps, max_len >= every n_u).
+ *   k_hist, v_hist device [T_hist, H*64] in cfg->dtype (cached keys/values).
+ *   cand_offsets device [B+1]; num_cand rows in all, max_cand >= each count.
+ *   q, k, v      device [num_cand, H*64] in cfg->dtype: the candidates' own rows.
+ *   request_ts   device [B] int64.  av_out device [num_cand, H*64] fp32.
+ * Needs no workspace.  Lengths beyond max_len / max_cand are reported as
+ * HSTU_ERR_DEVICE_CHECK in the device status word.
+ */
+hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* history,
+                               const void* k_hist, const void* v_hist,
+                               const int64_t* cand_offsets, int64_t num_cand, int32_t max_cand,
+                               const void* q, const void* k, const void* v,
+                               const int64_t* request_ts, const float* rab_pos,
+                               const float* rab_time, float* av_out, void* stream);
+
+/*
  * One HSTU layer (Eq. 1-3 and the residual) over a jagged batch.
  *   x_in        device [T, d] in cfg dtype: the layer input fed to f1.
  *   x_res       device [T, d] fp32 residual input, or NULL to use x_in.
@@ -174,13 +214,19 @@ hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
  *   microbatch   b_m >= 1.  Microbatches run concurrently as tiles of one
  *                launch; scores do not depend on b_m.
  *   scores       device [num_cand] fp32.
+ *   cand_y_out   device [num_cand, d] fp32, or NULL: receives y_c, each
+ *                candidate's final residual-stream row (the vector the score
+ *                is taken against).
+ *   workspace    ws_bytes >= hstu_mfalcon_workspace_bytes(cfg, num_cand).
+ * A history or candidate count beyond max_len / max_cand is reported as
+ * HSTU_ERR_DEVICE_CHECK in the device status word.
  */
 hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                             const hstu_layer_weights_t* weights, const hstu_jagged_t* history,
                             const void* kv_cache, const int64_t* cand_offsets, int64_t num_cand,
                             int32_t max_cand, const void* cand_emb, const int64_t* request_ts,
-                            int32_t microbatch, float* scores, void* workspace, size_t ws_bytes,
-                            void* stream);
+                            int32_t microbatch, float* scores, float* cand_y_out, void* workspace,
+                            size_t ws_bytes, void* stream);
 
 /* Per-kernel timing.  Between hstu_profiler_start() and hstu_profiler_stop()
  * every kernel the library launches is bracketed by CUDA events recorded on

@@ -28,3 +28,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    path = os.environ.get("HSTU_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        import json
+        from hstu_testutil import PARITY_LOG
+    except Exception:
+        return
+    with open(path, "w") as f:
+        json.dump(PARITY_LOG, f, indent=1)
