@@ -506,7 +506,7 @@ def measure_mfalcon(ctx, steps, warmup, with_e2e, sample_clocks=True, batch=None
     cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets)
     L, T, hv = c.num_layers, case.total_tokens, c.num_heads * 64
     M = t["cand_emb"].shape[0]
-    kv = torch.empty((L, T, 2 * hv), dtype=torch.bfloat16, device=ctx.dev)
+    kv = torch.empty((L, T, 2 * hv), dtype=cfg.cache_dtype, device=ctx.dev)
     ws_h = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=ctx.dev)
     ws_c = torch.empty(H.mfalcon_workspace_bytes(cfg, M), dtype=torch.uint8, device=ctx.dev)
     scores = torch.empty(M, dtype=torch.float32, device=ctx.dev)

@@ -6,7 +6,7 @@ import torch
 
 from .inputs import Case
 
-_TORCH = {"bf16": torch.bfloat16, "fp32": torch.float32}
+_TORCH = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
 
 
 def tensor(a: np.ndarray, dtype, device) -> torch.Tensor:

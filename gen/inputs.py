@@ -143,9 +143,16 @@ def round_bf16(a) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).reshape(a32.shape)
 
 
+def round_fp16(a) -> np.ndarray:
+    """Round to the nearest IEEE half (ties to even); returns float32 values."""
+    return np.asarray(a, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
 def to_dtype(a, dtype: str) -> np.ndarray:
     if dtype == "bf16":
         return round_bf16(a)
+    if dtype == "fp16":
+        return round_fp16(a)
     if dtype == "fp32":
         return np.ascontiguousarray(a, dtype=np.float32)
     raise ValueError(dtype)

@@ -78,18 +78,18 @@ struct AttnParams {
   const int64_t* request_ts;   // [B] (candidate mode)
   const float* rab_pos;        // [H, P]
   const float* rab_time;       // [H, Tb]
-  const __nv_bfloat16* q_self; // candidate mode: candidate Q, K, V rows (self term)
-  const __nv_bfloat16* k_self;
-  const __nv_bfloat16* v_self;
+  const void* q_self;          // candidate mode: candidate Q, K, V rows (self term),
+  const void* k_self;          // in the kernel's operand type (bf16 or fp16)
+  const void* v_self;
   int64_t ld_self;             // row stride (elements) of q_self/k_self/v_self
-  __nv_bfloat16* av;           // [T_q, ld_av] bf16 output, or
+  void* av;                    // [T_q, ld_av] output in the operand type, or
   float* av_f32;               // [T_q, ld_av] fp32 output (the layer path feeds LayerNorm)
   int64_t ld_av;
   float* ln_part;              // [T_q, H, 2] (sum, centred sum of squares) or nullptr
   int32_t B, H, P, Tb;
   int32_t max_q, max_kv;       // host-declared length bounds the launch is sized for
   int32_t num_qpairs;
-  int32_t pos_len;             // floats per staged copy of the position table
+  int32_t pos_len;             // entries per staged copy of the position table
   int32_t phi2;
   uint64_t timeout_ns;
   int64_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0)
@@ -170,21 +170,38 @@ __device__ __forceinline__ float time_bias_octave(int32_t dt, const int4* oct, c
   return v;
 }
 
-// phi2 applied to a pair given h = (scaled) pre-activation; returns bf16x2.
+// phi2 applied to a pair given h = (scaled) pre-activation, in fp32; returns
+// the pair of P values as bf16x2, or as fp16x2 when F16.
 // SiLU: tables carry x/2, so p = h + h*tanh(h); ReLU / identity: h = x.
-template <int PHI>
+template <int PHI, bool F16>
 __device__ __forceinline__ uint32_t phi_pair(uint64_t h2) {
+  auto to16 = [](uint64_t v) -> uint32_t {
+    if constexpr (F16) return f2_to_h2(v);
+    else return f2_to_bf16x2(v);
+  };
   if constexpr (PHI == HSTU_ACT_SILU) {
     float h0, h1;
     f2_unpack(h2, h0, h1);
     const uint64_t t2 = f2_pack(tanh_approx(h0), tanh_approx(h1));
-    return f2_to_bf16x2(f2_fma(h2, t2, h2));
+    return to16(f2_fma(h2, t2, h2));
   } else if constexpr (PHI == HSTU_ACT_RELU) {
     float h0, h1;
     f2_unpack(h2, h0, h1);
-    return pack_bf16x2(fmaxf(h0, 0.0f), fmaxf(h1, 0.0f));
+    return to16(f2_pack(fmaxf(h0, 0.0f), fmaxf(h1, 0.0f)));
   } else {
-    return f2_to_bf16x2(h2);
+    return to16(h2);
+  }
+}
+
+// phi2 of an fp16x2 pair of (scaled) pre-activations; SiLU: p = h + h*tanh(h).
+template <int PHI>
+__device__ __forceinline__ uint32_t phi_h2(uint32_t h) {
+  if constexpr (PHI == HSTU_ACT_SILU) {
+    return h2_fma(h, h2_tanh(h), h);
+  } else if constexpr (PHI == HSTU_ACT_RELU) {
+    return h2_max(h, 0u);
+  } else {
+    return h;
   }
 }
 
@@ -226,8 +243,10 @@ struct AttnSmem {
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kLnX = kMisc + 64;                        // 2 x 128 float2
   static constexpr uint32_t kPos = kLnX + 2 * ATT_ROWS * 8;
-  static constexpr uint32_t bytes(int pos_len, bool pairs) {
-    return kPos + static_cast<uint32_t>(pos_len) * 4u * (pairs ? 2u : 1u) + 1024u;  // + align slack
+  // pos_len entries per copy of `elt` bytes each (fp32, or fp16 for the
+  // causal fp16-operand kernel), two copies with paired reads
+  static constexpr uint32_t bytes(int pos_len, bool pairs, uint32_t elt = 4u) {
+    return kPos + static_cast<uint32_t>(pos_len) * elt * (pairs ? 2u : 1u) + 1024u;  // + align slack
   }
 };
 
@@ -246,15 +265,16 @@ enum : int {
 // ---------------------------------------------------------------- causal chunk
 
 // One 32-key chunk of one causal row: the pre-activations h = scale * (s + rab)
-// of its key pairs are handed to `sink(c, h2)` (columns c, c + 1 packed as an
-// fp32 pair), in live lanes only.  `rvx` points at the staged position table
-// entry of column 0 (entries for consecutive columns are consecutive), `kts`
-// at the chunk's key times (seconds since the user's first event, 16-byte
-// aligned).  Columns above `lim` are masked by the caller and never move the
-// time-bucket walk; lim < 0 marks a lane with no visible key in the chunk
-// (the sink is not called).  The walk `w` enters at the bucket of the previous
-// key and leaves at the bucket of the last visible key.  Per warp the chunk
-// falls in one of three cases:
+// of its key pairs are handed to `sink(c, h2)` (columns c, c + 1 as an fp32
+// pair) in live lanes only.  `rvx` points at the staged position table entry
+// of column 0 (entries for consecutive columns are consecutive; with PAIRS the
+// entry pair of an even column is one aligned 8-byte load), `kts` at the
+// chunk's key times (seconds since the user's first event, 16-byte aligned).
+// Columns above `lim` are masked by the caller and never move the time-bucket
+// walk; lim < 0 marks a lane with no visible key in the chunk (the sink is not
+// called).  The walk `w` enters at the bucket of the previous key and leaves
+// at the bucket of the last visible key.  Per warp the chunk falls in one of
+// three cases:
 //   every row keeps its bucket      -> one time bias per row, `rt_cur`, kept
 //                                      in a register (one compare of the last
 //                                      visible key against the bucket edge);
@@ -335,16 +355,18 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], Sink&& si
   }
 }
 
-// Pointwise phi2 of one causal chunk: packed bf16 P in `pk`, masked above `lim`.
-template <int PHI, bool PAIRS>
+// Pointwise phi2 of one causal chunk: packed 16-bit P (bf16, or fp16 when F16)
+// in `pk`, masked above `lim`.
+template <int PHI, bool PAIRS, bool F16>
 __device__ __forceinline__ void causal_chunk_pointwise(const uint32_t (&sv)[32], uint32_t (&pk)[16],
                                                        const float* rvx, const int32_t* kts, int lim,
                                                        BucketWalk<int32_t>& w, const float* sTime,
                                                        const int64_t* sThr, const int4* sOct,
                                                        const float4* sOrt, uint64_t scale2,
                                                        float& rt_cur) {
-  causal_chunk<PAIRS>(sv, [&](int c, uint64_t h2) { pk[c >> 1] = phi_pair<PHI>(h2); }, rvx, kts,
-                      lim, w, sTime, sThr, sOct, sOrt, scale2, rt_cur);
+  causal_chunk<PAIRS>(
+      sv, [&](int c, uint64_t h) { pk[c >> 1] = phi_pair<PHI, F16>(h); }, rvx, kts, lim, w, sTime,
+      sThr, sOct, sOrt, scale2, rt_cur);
   if (lim < 0) {
 #pragma unroll
     for (int q = 0; q < 16; ++q) pk[q] = 0u;
@@ -356,7 +378,10 @@ __device__ __forceinline__ void causal_chunk_pointwise(const uint32_t (&sv)[32],
 
 // ---------------------------------------------------------------- kernel
 
-template <bool CAND, int PHI, bool PAIRS>
+// F16: Q, K, V (and so P) are fp16 instead of bf16.  The causal element math
+// is fp32 either way; candidate mode with fp16 operands runs it on packed fp16
+// pairs (its per-key bias is precomputed, so the chain is short).
+template <bool CAND, int PHI, bool PAIRS, bool F16>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v,
@@ -552,7 +577,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                               : time_bucket_search(dt, sThr, p.Tb);
             r = sRv[j] + sTime[b];
           }
-          reinterpret_cast<float*>(key)[c] = r;
+          if constexpr (F16) reinterpret_cast<__half*>(key)[c] = __float2half_rn(r);
+          else reinterpret_cast<float*>(key)[c] = r;
         } else {
           int32_t rel = INT32_MAX;
           if (j < n_kv) {
@@ -578,8 +604,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int g = warp - ATT_MMA_WARP;
     {
       const bool leader = elect_one();
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(ATT_ROWS, ATT_KEYS, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(ATT_ROWS, ATT_HD, false, true);
+      constexpr uint32_t idesc_qk = idesc_16_f32(ATT_ROWS, ATT_KEYS, false, false, F16);
+      constexpr uint32_t idesc_pv = idesc_16_f32(ATT_ROWS, ATT_HD, false, true, F16);
       const int nWg = g == 0 ? nA : nB;
       // tensor memory: S buffers (P over them) and O of this tile
       const uint32_t tS = tmem + static_cast<uint32_t>(g * ATT_SBUF * 64);
@@ -687,6 +713,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int nW = g == 0 ? nA : nB;
     bool ok = true;
     const uint64_t scale2 = f2_pack(kScale, kScale);
+    const uint32_t scale_h2 = h2_splat(kScale);
 
     // causal: per-row time-bucket walk and staged position-table copy
     BucketWalk<int32_t> w32;
@@ -702,17 +729,27 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       rt_cur = sTime[w32.b];
     }
 
-    // this half's 32 keys of tile kt: S values in `sv`, packed bf16 P pairs to `pk`
+    // this half's 32 keys of tile kt: S values in `sv`, packed 16-bit P pairs to `pk`
     auto chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int kt, int s) {
       const uint8_t* key = sKey + s * AttnSmem::kKeyStride;
       const int j0 = kt * ATT_KEYS + half * 32;  // key index of column 0
       if constexpr (CAND) {
-        const float* kr = reinterpret_cast<const float*>(key) + half * 32;
+        if constexpr (F16) {
+          const __half* kr = reinterpret_cast<const __half*>(key) + half * 32;
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                     scale2, lds_b64(kr + c));
-          pk[c >> 1] = phi_pair<PHI>(h2);
+          for (int c = 0; c < 32; c += 2) {
+            const uint32_t s16 =
+                f2_to_h2(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])));
+            pk[c >> 1] = phi_h2<PHI>(h2_fma(s16, scale_h2, lds_b32(kr + c)));
+          }
+        } else {
+          const float* kr = reinterpret_cast<const float*>(key) + half * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const uint64_t h2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                       scale2, lds_b64(kr + c));
+            pk[c >> 1] = phi_pair<PHI, false>(h2);
+          }
         }
         const int last = n_kv - 1 - j0;  // last live column
         if (last < 31) {
@@ -720,13 +757,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
         }
       } else {
-        const int xc = D - i + j0 + copy;  // table index at column 0
         // last visible column: keys after the row are masked; rows past the
         // user's end are not stored and skip the work
         const int lim = !valid ? -1 : i - j0;
-        causal_chunk_pointwise<PHI, PAIRS>(sv, pk, rv + xc,
-                                           reinterpret_cast<const int32_t*>(key) + half * 32, lim,
-                                           w32, sTime, sThr, sOct, sOrt, scale2, rt_cur);
+        const int32_t* kts = reinterpret_cast<const int32_t*>(key) + half * 32;
+        const int xc = D - i + j0 + copy;  // table index at column 0
+        causal_chunk_pointwise<PHI, PAIRS, F16>(sv, pk, rv + xc, kts, lim, w32, sTime, sThr, sOct,
+                                                sOrt, scale2, rt_cur);
       }
     };
 
@@ -783,20 +820,26 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (valid) {
         if constexpr (CAND) {
           // the candidate's own key/value: position bucket 0, time bucket 0
-          const __nv_bfloat16* qs = p.q_self + row * p.ld_self + h * ATT_HD;
-          const __nv_bfloat16* ks = p.k_self + row * p.ld_self + h * ATT_HD;
-          const __nv_bfloat16* vs = p.v_self + row * p.ld_self + h * ATT_HD + half * HC;
+          const uint16_t* qs = static_cast<const uint16_t*>(p.q_self) + row * p.ld_self + h * ATT_HD;
+          const uint16_t* ks = static_cast<const uint16_t*>(p.k_self) + row * p.ld_self + h * ATT_HD;
+          const uint16_t* vs =
+              static_cast<const uint16_t*>(p.v_self) + row * p.ld_self + h * ATT_HD + half * HC;
+          // a packed pair of the operand type as two floats
+          auto to_f2 = [](uint32_t w) -> float2 {
+            if constexpr (F16) return __half22float2(*reinterpret_cast<const __half2*>(&w));
+            else return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+          };
           float dot = 0.0f;
 #pragma unroll
           for (int c = 0; c < ATT_HD; c += 8) {
-            uint4 qa = *reinterpret_cast<const uint4*>(qs + c);
-            uint4 ka = *reinterpret_cast<const uint4*>(ks + c);
-            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qa);
-            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&ka);
+            const uint4 qa = *reinterpret_cast<const uint4*>(qs + c);
+            const uint4 ka = *reinterpret_cast<const uint4*>(ks + c);
+            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w};
+            const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-              float2 qf = __bfloat1622float2(q2[t]);
-              float2 kf = __bfloat1622float2(k2[t]);
+              const float2 qf = to_f2(qw[t]);
+              const float2 kf = to_f2(kw[t]);
               dot = fmaf(qf.x, kf.x, dot);
               dot = fmaf(qf.y, kf.y, dot);
             }
@@ -806,11 +849,11 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const float ps = apply_phi<PHI>(dot + rab0);
 #pragma unroll
           for (int c = 0; c < HC; c += 8) {
-            uint4 va = *reinterpret_cast<const uint4*>(vs + c);
-            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&va);
+            const uint4 va = *reinterpret_cast<const uint4*>(vs + c);
+            const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-              float2 vf = __bfloat1622float2(v2[t]);
+              const float2 vf = to_f2(vw[t]);
               o[c + 2 * t] = fmaf(ps, vf.x, o[c + 2 * t]);
               o[c + 2 * t + 1] = fmaf(ps, vf.y, o[c + 2 * t + 1]);
             }
@@ -834,14 +877,18 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int c = 0; c < HC; c += 4)
             dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
         } else {
-          __nv_bfloat16* dst = p.av + row * p.ld_av + h * ATT_HD + half * HC;
+          uint16_t* dst = static_cast<uint16_t*>(p.av) + row * p.ld_av + h * ATT_HD + half * HC;
+          auto pack = [](float a, float b) -> uint32_t {
+            if constexpr (F16) return pack_h2(a, b);
+            else return pack_bf16x2(a, b);
+          };
 #pragma unroll
           for (int c = 0; c < HC; c += 8) {
             uint4 pkt;
-            pkt.x = pack_bf16x2(o[c + 0], o[c + 1]);
-            pkt.y = pack_bf16x2(o[c + 2], o[c + 3]);
-            pkt.z = pack_bf16x2(o[c + 4], o[c + 5]);
-            pkt.w = pack_bf16x2(o[c + 6], o[c + 7]);
+            pkt.x = pack(o[c + 0], o[c + 1]);
+            pkt.y = pack(o[c + 2], o[c + 3]);
+            pkt.z = pack(o[c + 4], o[c + 5]);
+            pkt.w = pack(o[c + 6], o[c + 7]);
             *reinterpret_cast<uint4*>(dst + c) = pkt;
           }
         }

@@ -78,7 +78,8 @@ struct F1OutMaps {
 struct F1Params {
   void* dst[4];           // destination of column block b (U, V, Q, K)
   int64_t ld_dst[4];      // row stride of each destination (elements)
-  uint32_t f32_mask;      // bit b set: block b is stored as fp32, else bf16
+  uint32_t f32_mask;      // bit b set: block b is stored as fp32
+  uint32_t f16_mask;      // bit b set: block b is stored as fp16 (else bf16)
   const float* bias;      // [N]
   int64_t M;
   int32_t N, K;
@@ -297,6 +298,7 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int blk = col / p.blk_w;
         const int cb = col - blk * p.blk_w;
         const bool f32 = (p.f32_mask >> blk) & 1u;
+        const bool h16 = (p.f16_mask >> blk) & 1u;
         const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
         float z[32];
 #pragma unroll
@@ -320,12 +322,12 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]);
         } else {
           const int j0 = (ch & 1) * 4;
+          auto pk2 = [h16](float a, float b) { return h16 ? pack_h2(a, b) : pack_bf16x2(a, b); };
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             *reinterpret_cast<uint4*>(my_row + (((j0 + j) ^ sw) << 4)) =
-                make_uint4(pack_bf16x2(z[8 * j], z[8 * j + 1]), pack_bf16x2(z[8 * j + 2], z[8 * j + 3]),
-                           pack_bf16x2(z[8 * j + 4], z[8 * j + 5]),
-                           pack_bf16x2(z[8 * j + 6], z[8 * j + 7]));
+                make_uint4(pk2(z[8 * j], z[8 * j + 1]), pk2(z[8 * j + 2], z[8 * j + 3]),
+                           pk2(z[8 * j + 4], z[8 * j + 5]), pk2(z[8 * j + 6], z[8 * j + 7]));
         }
         if (f32 || (ch & 1) == 1) {
           fence_proxy_async_smem();  // this lane's writes, before the tensor store reads them

@@ -159,18 +159,24 @@ class ProfScope {
 using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                              const AttnParams);
 
-template <bool CAND, bool PAIRS>
+template <bool CAND, bool PAIRS, bool F16>
 AttnKernelFn attn_kernel_for(int phi) {
   switch (phi) {
-    case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS>;
-    case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS>;
-    default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS>;
+    case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS, F16>;
+    case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS, F16>;
+    default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS, F16>;
   }
 }
 
-AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs) {
-  if (cand) return pairs ? attn_kernel_for<true, true>(phi) : attn_kernel_for<true, false>(phi);
-  return pairs ? attn_kernel_for<false, true>(phi) : attn_kernel_for<false, false>(phi);
+template <bool F16>
+AttnKernelFn attn_kernel_ptr_t(bool cand, int phi, bool pairs) {
+  if (cand)
+    return pairs ? attn_kernel_for<true, true, F16>(phi) : attn_kernel_for<true, false, F16>(phi);
+  return pairs ? attn_kernel_for<false, true, F16>(phi) : attn_kernel_for<false, false, F16>(phi);
+}
+
+AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16) {
+  return f16 ? attn_kernel_ptr_t<true>(cand, phi, pairs) : attn_kernel_ptr_t<false>(cand, phi, pairs);
 }
 
 struct DeviceInfo {
@@ -194,9 +200,10 @@ hstu_status_t device_info(DeviceInfo** out) {
     for (int cand = 0; cand < 2; ++cand)
       for (int phi = 0; phi < 3; ++phi)
         for (int pairs = 0; pairs < 2; ++pairs)
-          HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(cand != 0, phi, pairs != 0),
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               att_max));
+          for (int f16 = 0; f16 < 2; ++f16)
+            HSTU_CHECK_CUDA(cudaFuncSetAttribute(
+                attn_kernel_ptr(cand != 0, phi, pairs != 0, f16 != 0),
+                cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
     const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
@@ -233,26 +240,29 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [rows, cols] matrix with row stride `ld`
-// elements; box = box_cols x box_rows; 128-byte swizzle.
-hstu_status_t make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
-                            int64_t ld, int box_cols, int box_rows) {
+// 2-D map over a row-major [rows, cols] matrix of 16-bit elements (bf16, or
+// fp16 when f16) with row stride `ld` elements; box = box_cols x box_rows;
+// 128-byte swizzle.
+hstu_status_t make_map_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                          int64_t ld, int box_cols, int box_rows, bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return HSTU_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
-// 2-D map for tensor stores of f1's output blocks: fp32 or bf16 [rows, cols]
-// with row stride `ld` elements; box = one 128-byte row segment x 32 rows.
+// 2-D map for tensor stores of f1's output blocks: fp32, bf16 or fp16
+// [rows, cols] with row stride `ld` elements; box = one 128-byte row segment x
+// 32 rows.
 hstu_status_t make_out_map(CUtensorMap* map, void* base, bool f32, int64_t rows, int64_t cols,
-                           int64_t ld) {
+                           int64_t ld, bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return HSTU_ERR_CUDA;
   const int elt = f32 ? 4 : 2;
@@ -260,8 +270,10 @@ hstu_status_t make_out_map(CUtensorMap* map, void* base, bool f32, int64_t rows,
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * elt};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt), 32};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const CUtensorMapDataType dt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                     : (f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  CUresult r = fn(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
@@ -281,7 +293,8 @@ hstu_status_t check_cfg(const hstu_layer_cfg_t* c) {
   if (c->phi1 < HSTU_ACT_IDENTITY || c->phi1 > HSTU_ACT_SILU || c->phi2 < HSTU_ACT_IDENTITY ||
       c->phi2 > HSTU_ACT_SILU)
     return HSTU_ERR_INVALID_ARGUMENT;
-  if (c->dtype != HSTU_BF16 && c->dtype != HSTU_FP32) return HSTU_ERR_INVALID_ARGUMENT;
+  if (c->dtype != HSTU_BF16 && c->dtype != HSTU_FP32 && c->dtype != HSTU_FP16)
+    return HSTU_ERR_INVALID_ARGUMENT;
   if (!(c->ln_eps >= 0.0f)) return HSTU_ERR_INVALID_ARGUMENT;
   if (c->dqk != ATT_HD || c->dv != ATT_HD) return HSTU_ERR_UNSUPPORTED;
   if (c->d_model % 64 != 0) return HSTU_ERR_UNSUPPORTED;
@@ -289,6 +302,13 @@ hstu_status_t check_cfg(const hstu_layer_cfg_t* c) {
     return HSTU_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(c->num_heads) * ATT_HD > 8192) return HSTU_ERR_UNSUPPORTED;
   return HSTU_OK;
+}
+
+// Layer entry points: bf16 or fp32 storage (fp16 is an attention-operand type only).
+hstu_status_t check_layer_cfg(const hstu_layer_cfg_t* c) {
+  hstu_status_t s = check_cfg(c);
+  if (s != HSTU_OK) return s;
+  return c->dtype == HSTU_FP16 ? HSTU_ERR_UNSUPPORTED : HSTU_OK;
 }
 
 hstu_status_t check_jag(const hstu_jagged_t* j) {
@@ -379,10 +399,12 @@ struct AttnJob {
   float* av_f32;                // fp32 output (layer path)
   float* ln_part;
   uint64_t timeout_ns;
+  bool f16;                     // Q, K, V (and P) in fp16 instead of bf16
 };
 
+// Tensor-core attention over 16-bit operands (bf16, or fp16 when j.f16).
 template <bool CAND>
-hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
+hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   const hstu_layer_cfg_t* c = j.cfg;
   if (j.batch == 0 || j.T_q == 0 || j.max_q_len == 0) return HSTU_OK;
   DeviceInfo* di = nullptr;
@@ -390,15 +412,15 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   if (s != HSTU_OK) return s;
   CUtensorMap mq, mk, mv;
   const int64_t hc = static_cast<int64_t>(c->num_heads) * ATT_HD;
-  if ((s = make_map_bf16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS, j.f16)) != HSTU_OK) return s;
   // with no key rows at all (every history empty) no K/V tile is ever loaded;
   // the maps then describe the query rows so that they stay valid
   const bool no_kv = j.T_kv == 0;
-  if ((s = make_map_bf16(&mk, no_kv ? j.q : j.k, no_kv ? j.T_q : j.T_kv, hc,
-                         no_kv ? j.ldq : j.ldk, ATT_HD, ATT_KEYS)) != HSTU_OK)
+  if ((s = make_map_16(&mk, no_kv ? j.q : j.k, no_kv ? j.T_q : j.T_kv, hc,
+                       no_kv ? j.ldq : j.ldk, ATT_HD, ATT_KEYS, j.f16)) != HSTU_OK)
     return s;
-  if ((s = make_map_bf16(&mv, no_kv ? j.q : j.v, no_kv ? j.T_q : j.T_kv, hc,
-                         no_kv ? j.ldq : j.ldv, ATT_HD, ATT_KEYS)) != HSTU_OK)
+  if ((s = make_map_16(&mv, no_kv ? j.q : j.v, no_kv ? j.T_q : j.T_kv, hc,
+                       no_kv ? j.ldq : j.ldv, ATT_HD, ATT_KEYS, j.f16)) != HSTU_OK)
     return s;
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -408,11 +430,11 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   p.request_ts = j.request_ts;
   p.rab_pos = j.rab_pos;
   p.rab_time = j.rab_time;
-  p.q_self = static_cast<const __nv_bfloat16*>(j.q_self);
-  p.k_self = static_cast<const __nv_bfloat16*>(j.k_self);
-  p.v_self = static_cast<const __nv_bfloat16*>(j.v_self);
+  p.q_self = j.q_self;
+  p.k_self = j.k_self;
+  p.v_self = j.v_self;
   p.ld_self = j.ld_self;
-  p.av = static_cast<__nv_bfloat16*>(j.av);
+  p.av = j.av;
   p.av_f32 = j.av_f32;
   p.ld_av = j.ld_av;
   p.ln_part = j.ln_part;
@@ -429,31 +451,35 @@ hstu_status_t launch_attn_bf16(const AttnJob& j, cudaStream_t st) {
   // per-copy length = 16 (mod 32) floats: the two copies' 8-byte pair reads
   // by neighbouring lanes then fall in disjoint shared-memory banks
   p.pos_len = static_cast<int32_t>(align_up(dmax + ATT_ROWS + 2, 32) + 16);
+  const uint32_t pos_elt = 4u;
   p.phi2 = c->phi2;
   p.timeout_ns = j.timeout_ns;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
   if (!compute_octaves(c->num_time_buckets, p.thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
   dim3 grid(c->num_heads, j.batch, p.num_qpairs);
-  const bool pairs = AttnSmem::bytes(p.pos_len, true) <= 227u * 1024u;
-  const size_t smem = AttnSmem::bytes(p.pos_len, pairs);
+  const bool pairs = AttnSmem::bytes(p.pos_len, true, pos_elt) <= 227u * 1024u;
+  const size_t smem = AttnSmem::bytes(p.pos_len, pairs, pos_elt);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
-  attn_kernel_ptr(CAND, c->phi2, pairs)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+  attn_kernel_ptr(CAND, c->phi2, pairs, j.f16)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
 
+// f32_mask / f16_mask bit b: column block b (U, V, Q, K) is stored as fp32 /
+// fp16; otherwise bf16.
 hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t ldx, int64_t M,
                              const void* w1, const float* b1, void* const dst[4],
-                             const int64_t ld_dst[4], uint32_t f32_mask, cudaStream_t st) {
+                             const int64_t ld_dst[4], uint32_t f32_mask, uint32_t f16_mask,
+                             cudaStream_t st) {
   if (M == 0) return HSTU_OK;
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
   const int N = n1_of(c), K = c->d_model;
   CUtensorMap mx, mw;
-  if ((s = make_map_bf16(&mx, x, M, K, ldx, G_BK, G_BM)) != HSTU_OK) return s;
-  if ((s = make_map_bf16(&mw, w1, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mx, x, M, K, ldx, G_BK, G_BM)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mw, w1, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
   F1Params p;
   std::memset(&p, 0, sizeof(p));
   F1OutMaps om;
@@ -462,10 +488,12 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   for (int b = 0; b < 4; ++b) {
     p.dst[b] = dst[b];
     p.ld_dst[b] = ld_dst[b];
-    if ((s = make_out_map(&om.m[b], dst[b], (f32_mask >> b) & 1u, M, blk_w, ld_dst[b])) != HSTU_OK)
+    if ((s = make_out_map(&om.m[b], dst[b], (f32_mask >> b) & 1u, M, blk_w, ld_dst[b],
+                          (f16_mask >> b) & 1u)) != HSTU_OK)
       return s;
   }
   p.f32_mask = f32_mask;
+  p.f16_mask = f16_mask;
   p.bias = b1;
   p.M = M;
   p.N = N;
@@ -503,7 +531,7 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   if (s != HSTU_OK) return s;
   const int N = c->d_model, K = c->num_heads * c->dv;
   CUtensorMap mw;
-  if ((s = make_map_bf16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
   F2OutMaps om;
   std::memset(&om, 0, sizeof(om));
   if ((s = make_out_map(&om.y, y, true, M, N, ld_y)) != HSTU_OK) return s;
@@ -659,17 +687,19 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
                          float* y_out, void* y_lp, void* kv_cache, const LayerWs& ws, bool cand,
                          cudaStream_t st) {
   const int hv = c->num_heads * ATT_HD, d = c->d_model;
-  __nv_bfloat16* vqk = static_cast<__nv_bfloat16*>(ws.z);
-  // f1 column blocks U, V, Q, K -> U (fp32), V, Q, K (bf16; K/V into the cache if given)
+  __half* vqk = static_cast<__half*>(ws.z);
+  // f1 column blocks U, V, Q, K -> U (fp32), V, Q, K (fp16; K/V into the cache
+  // if given).  The attention operands are fp16: the same tensor-core rate as
+  // bf16 with 8x finer rounding of Q, K, V and P.
   void* dst[4] = {ws.u, vqk, vqk + hv, vqk + 2 * hv};
   int64_t ldd[4] = {hv, 3 * hv, 3 * hv, 3 * hv};
   if (kv_cache != nullptr) {
-    __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(kv_cache);
+    __half* kv = static_cast<__half*>(kv_cache);
     dst[1] = kv + hv;  // V
     dst[3] = kv;       // K
     ldd[1] = ldd[3] = 2 * hv;
   }
-  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, 1u, st);
+  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, 1u, 0xEu, st);
   if (s != HSTU_OK) return s;
   AttnJob j = base;
   j.q = dst[2];
@@ -686,7 +716,8 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
   j.av_f32 = static_cast<float*>(ws.av);
   j.ld_av = hv;
   j.ln_part = static_cast<float*>(ws.extra);
-  s = cand ? launch_attn_bf16<true>(j, st) : launch_attn_bf16<false>(j, st);
+  j.f16 = true;
+  s = cand ? launch_attn_tc<true>(j, st) : launch_attn_tc<false>(j, st);
   if (s != HSTU_OK) return s;
   return launch_f2_bf16(c, w, static_cast<const float*>(ws.av), hv, ws.u, hv,
                         static_cast<const float*>(ws.extra), x_res, x_in, d, y_out, y_lp, d, T,
@@ -748,18 +779,18 @@ const char* hstu_status_string(hstu_status_t s) {
 }
 
 size_t hstu_layer_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total_tokens) {
-  if (check_cfg(cfg) != HSTU_OK || total_tokens < 0) return 0;
+  if (check_layer_cfg(cfg) != HSTU_OK || total_tokens < 0) return 0;
   return layer_ws_bytes(cfg, total_tokens);
 }
 
 size_t hstu_forward_workspace_bytes(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                                     int64_t total_tokens) {
-  if (check_cfg(cfg) != HSTU_OK || total_tokens < 0 || num_layers < 1) return 0;
+  if (check_layer_cfg(cfg) != HSTU_OK || total_tokens < 0 || num_layers < 1) return 0;
   return layer_ws_bytes(cfg, total_tokens) + stream_ws_bytes(cfg, total_tokens);
 }
 
 size_t hstu_mfalcon_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t num_cand) {
-  if (check_cfg(cfg) != HSTU_OK || num_cand < 0) return 0;
+  if (check_layer_cfg(cfg) != HSTU_OK || num_cand < 0) return 0;
   return layer_ws_bytes(cfg, num_cand) + stream_ws_bytes(cfg, num_cand);
 }
 
@@ -804,7 +835,8 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
   j.timeout_ns = kDefaultTimeoutNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == HSTU_FP32) return launch_f32_attn(j, st);
-  return launch_attn_bf16<false>(j, st);
+  j.f16 = cfg->dtype == HSTU_FP16;
+  return launch_attn_tc<false>(j, st);
 }
 
 hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
@@ -841,7 +873,8 @@ hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t
     return launch_f32_attn(j, st);
   }
   j.av_f32 = av_out;
-  return launch_attn_bf16<false>(j, st);
+  j.f16 = cfg->dtype == HSTU_FP16;
+  return launch_attn_tc<false>(j, st);
 }
 
 hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* history,
@@ -891,7 +924,8 @@ hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t*
     return launch_f32_attn(j, st);
   }
   j.av_f32 = av_out;
-  return launch_attn_bf16<true>(j, st);
+  j.f16 = cfg->dtype == HSTU_FP16;
+  return launch_attn_tc<true>(j, st);
 }
 
 hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
@@ -899,7 +933,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
                              float* y_out, void* y_out_lp, void* kv_cache_out, void* workspace,
                              size_t ws_bytes, void* stream) {
   hstu_status_t s;
-  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_layer_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(jag)) != HSTU_OK) return s;
   if ((s = check_weights(cfg, w)) != HSTU_OK) return s;
   const int64_t T = jag->total_tokens;
@@ -936,7 +970,7 @@ hstu_status_t hstu_layer_fwd_static(const hstu_layer_cfg_t* cfg, const hstu_laye
                                     const float* x_res, float* y_out, void* y_out_lp,
                                     void* kv_cache_out, void* stream) {
   hstu_status_t s;
-  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_layer_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(jag)) != HSTU_OK) return s;
   if (layer_ws_bytes(cfg, jag->total_tokens) > HSTU_STATIC_SCRATCH_BYTES)
     return HSTU_ERR_WORKSPACE_TOO_SMALL;
@@ -951,7 +985,7 @@ hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                            const void* x_in, float* y_out, void* kv_cache_out, void* workspace,
                            size_t ws_bytes, void* stream) {
   hstu_status_t s;
-  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_layer_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(jag)) != HSTU_OK) return s;
   if (num_layers < 1 || weights == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
   for (int l = 0; l < num_layers; ++l)
@@ -993,7 +1027,7 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                             int32_t microbatch, float* scores, float* cand_y_out, void* workspace,
                             size_t ws_bytes, void* stream) {
   hstu_status_t s;
-  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_layer_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(history)) != HSTU_OK) return s;
   if (num_layers < 1 || weights == nullptr || microbatch < 1 || num_cand < 0 || max_cand < 0)
     return HSTU_ERR_INVALID_ARGUMENT;
@@ -1037,6 +1071,7 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
   base.T_q = M;
   base.T_kv = history->total_tokens;
   base.timeout_ns = kDefaultTimeoutNs;
+  base.f16 = true;  // bf16 layers keep their cached K/V in fp16
   for (int l = 0; l < num_layers; ++l) {
     const uint8_t* cache_l = static_cast<const uint8_t*>(kv_cache) + cache_layer * l;
     AttnJob j = base;

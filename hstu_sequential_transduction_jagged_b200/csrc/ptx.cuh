@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "status.cuh"
 
@@ -309,16 +310,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 accumulation; A and B are
+// both bf16 (f16 = false) or both fp16 (f16 = true).
+__host__ __device__ constexpr uint32_t idesc_16_f32(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                    bool f16) {
   return (1u << 4)                                  // D format: f32
-         | (1u << 7)                                // A format: bf16
-         | (1u << 10)                               // B format: bf16
+         | ((f16 ? 0u : 1u) << 7)                   // A format: 0 f16, 1 bf16
+         | ((f16 ? 0u : 1u) << 10)                  // B format: 0 f16, 1 bf16
          | ((a_mn_major ? 1u : 0u) << 15)           // A major
          | ((b_mn_major ? 1u : 0u) << 16)           // B major
          | ((static_cast<uint32_t>(N) >> 3) << 17)  // N / 8
          | ((static_cast<uint32_t>(M) >> 4) << 24); // M / 16
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
+                                                      bool b_mn_major) {
+  return idesc_16_f32(M, N, a_mn_major, b_mn_major, false);
 }
 
 // ------------------------------------------------------------------ misc
@@ -365,6 +372,64 @@ __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------- packed fp16 pairs
+// A uint32_t holds two fp16 values: the low half is the lower column.
+
+// fp16x2 from an fp32 pair (low <- lo, high <- hi), round to nearest, values
+// beyond the fp16 range saturate to +-65504 instead of becoming infinite.
+__device__ __forceinline__ uint32_t f2_to_h2(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_tanh(uint32_t a) {
+  uint32_t r;
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_ex2(uint32_t a) {
+  uint32_t r;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(a));
+  return r;
+}
+// Both halves of an fp16x2 as fp32.
+__device__ __forceinline__ void h2_to_f(uint32_t v, float& lo, float& hi) {
+  unsigned short a, b;
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(a), "=h"(b) : "r"(v));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(a));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(b));
+}
+__device__ __forceinline__ uint32_t h2_splat(float x) { return pack_h2(x, x); }
+// Two fp16 values from 16-bit shared-memory entries into one fp16x2.
+__device__ __forceinline__ uint32_t h2_join(unsigned short lo, unsigned short hi) {
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+__device__ __forceinline__ uint32_t lds_b32(const void* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

@@ -18,8 +18,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhstu.so")
 
 ACT = {"identity": 0, "relu": 1, "silu": 2}
-DTYPE = {"bf16": 0, "fp32": 1}
-TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32}
+DTYPE = {"bf16": 0, "fp32": 1, "fp16": 2}
+TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32, "fp16": torch.float16}
+# dtype of the per-layer key/value cache of a layer configured with `dtype`
+CACHE_DTYPE = {"bf16": torch.float16, "fp32": torch.float32}
 STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARGUMENT", 2: "HSTU_ERR_UNSUPPORTED",
           3: "HSTU_ERR_CUDA", 4: "HSTU_ERR_WORKSPACE_TOO_SMALL", 5: "HSTU_ERR_DEVICE_TIMEOUT",
           6: "HSTU_ERR_DEVICE_CHECK"}
@@ -140,6 +142,11 @@ class LayerConfig:
     @property
     def torch_dtype(self):
         return TORCH_DTYPE[self.dtype]
+
+    @property
+    def cache_dtype(self):
+        """dtype of the K/V cache hstu_layer_fwd / hstu_forward write."""
+        return CACHE_DTYPE[self.dtype]
 
     @property
     def n1(self) -> int:

@@ -22,6 +22,8 @@
  *   - Norm = LayerNorm over the H*dv concatenated heads of a token, biased
  *     variance, eps from the config, optional affine;
  *   - Y = X + f2(...): the residual stream is fp32.
+ *   - bf16 layers compute attention on fp16 Q, K, V and P (f1 writes them in
+ *     fp16; values saturate at +-65504), with fp32 accumulation.
  *
  * Conventions for every entry point:
  *   - Pointers marked "device" must point to memory of the current CUDA
@@ -63,7 +65,11 @@ typedef enum {
   HSTU_ERR_DEVICE_CHECK = 6        /* a device-side input check failed */
 } hstu_status_t;
 
-typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1 } hstu_dtype_t;
+/* Storage types.  Layers run in bf16 (tensor cores) or fp32 (SIMT); FP16 is
+ * accepted by the attention-only entry points (hstu_attn_fwd*,
+ * mfalcon_attn_fwd) for fp16 Q, K, V, the operand type the bf16 layers use
+ * for their attention internally. */
+typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1, HSTU_FP16 = 2 } hstu_dtype_t;
 
 typedef enum { HSTU_ACT_IDENTITY = 0, HSTU_ACT_RELU = 1, HSTU_ACT_SILU = 2 } hstu_act_t;
 
@@ -177,9 +183,12 @@ hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t*
  *   y_out       device [T, d] fp32: X + f2(Norm(AV) (.) U).
  *   y_out_lp    device [T, d] in cfg dtype (a rounded copy of y_out for the
  *               next layer's f1), or NULL.
- *   kv_cache_out device [T, 2, H, 64] in cfg dtype (per row: K of every head,
+ *   kv_cache_out device [T, 2, H, 64] (per row: K of every head,
  *               then V of every head), or NULL.  When given, this layer's K
- *               and V rows are kept there for M-FALCON.
+ *               and V rows are kept there for M-FALCON.  bf16 layers keep
+ *               K and V in fp16 (their attention operands are fp16: the
+ *               same tensor-core rate as bf16 with 8x finer rounding);
+ *               fp32 layers in fp32.
  *   workspace   device, ws_bytes >= hstu_layer_workspace_bytes(cfg, T).
  * x_in, y_out and y_out_lp must not overlap.
  */
@@ -192,7 +201,8 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
  * A stack of num_layers HSTU layers (the residual stream stays fp32).
  *   weights      host array [num_layers] of per-layer weight structs.
  *   x_in         device [T, d] in cfg dtype.  y_out device [T, d] fp32.
- *   kv_cache_out device [num_layers][T, 2, H, 64] in cfg dtype, or NULL.
+ *   kv_cache_out device [num_layers][T, 2, H, 64] (fp16 for bf16 layers, fp32
+ *                for fp32 layers), or NULL.
  *   workspace    ws_bytes >= hstu_forward_workspace_bytes(cfg, num_layers, T).
  */
 hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
@@ -207,7 +217,8 @@ hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
  * user's cached history keys/values and to itself only.  score_c = <y_c, e_c>
  * where y_c is its final fp32 residual-stream row.
  *   history      jagged history (offsets/timestamps of the cached rows).
- *   kv_cache     device [num_layers][T_hist, 2, H, 64] from hstu_forward.
+ *   kv_cache     device [num_layers][T_hist, 2, H, 64] from hstu_forward (fp16
+ *                for bf16 layers, fp32 for fp32 layers).
  *   cand_offsets device [B+1] candidate row ranges per user; num_cand = total
  *                rows, max_cand >= the largest per-user count.
  *   cand_emb     device [num_cand, d] in cfg dtype.  request_ts device [B].

@@ -50,16 +50,15 @@ def assert_close(got, want, what="", max_abs=MAX_ABS, rel_l2=REL_L2, scaled=Fals
     return ma, rl
 
 
-def check_scores(got, want, emb, L, what):
-    """M-FALCON scores s_c = <y_c, e_c>.  About ||e_c||^2 (~d) of each score is
-    the input itself, so the comparison is made on the part the layers add,
-    s_c - <e_c, e_c> (computed in float64 from the inputs, the same on both
-    sides): rel-L2 <= 5e-3.  And the score error divided by ||e_c|| is the error
-    of y_c along the unit vector e_c / ||e_c||, i.e. one coordinate of y_c in an
-    orthonormal basis; it is held to the per-coordinate bound of y_c itself
-    (2e-2 per layer, 2e-2 sqrt(L) for an L-layer stack).  The rel-L2 bound of
-    the layer part is 5e-3 for one layer and 5e-3 sqrt(L) for a stack, the
-    random-walk growth of independent per-layer rounding errors."""
+def check_scores(got, want, emb, what):
+    """M-FALCON scores s_c = <y_c, e_c>.  The raw scores meet rel-L2 <= 5e-3 with
+    a wide margin, because about ||e_c||^2 (~d) of each score is the input
+    itself; so the comparison that can fail is made on the part the layers
+    add, s_c - <e_c, e_c> (computed in float64 from the inputs, the same on
+    both sides): rel-L2 <= 5e-3.  The max-abs bound is translated to the score
+    through e_c: the score error divided by ||e_c|| is the error of y_c along
+    the unit vector e_c / ||e_c||, one coordinate of y_c in an orthonormal
+    basis, and it is held to the per-coordinate bound of y_c itself (2e-2)."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     e = np.asarray(emb, dtype=np.float64)
@@ -67,8 +66,7 @@ def check_scores(got, want, emb, L, what):
     _, rl = errors(got - ee, want - ee)
     proj = np.abs(got - want) / np.maximum(np.linalg.norm(e, axis=1), 1e-30)
     pm = float(proj.max()) if proj.size else 0.0
-    bound = MAX_ABS * np.sqrt(L)
-    bound_rel = REL_L2 * np.sqrt(L)
+    bound, bound_rel = MAX_ABS, REL_L2
     record(what, pm, rl, bound, bound_rel, "score: max |ds|/||e_c||; rel-L2 of s - <e,e>")
     _, raw_rel = errors(got, want)
     record(what + " (raw scores)", float(np.abs(got - want).max()) if got.size else 0.0, raw_rel,
@@ -101,7 +99,7 @@ def upload(H, case, device="cuda"):
 
 
 def upload_attn(H, ac, device="cuda"):
-    dt = torch.bfloat16 if ac.dtype == "bf16" else torch.float32
+    dt = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[ac.dtype]
     offs = tensor(ac.offsets, torch.int64, device)
     ts = tensor(ac.timestamps, torch.int64, device)
     lens = np.diff(ac.offsets)

@@ -11,7 +11,8 @@ float64 oracle:
 
   * Q = 0, so S = Q K^T = 0 exactly, and phi2 is the identity or ReLU (with
     non-negative biases both give P = rab exactly; the values are small
-    integers, exact in bf16);
+    integers, exact in fp16 and bf16).  The operands are fp16 -- the kernel
+    the bf16 layers run -- unless a test names bf16;
   * V is one-hot by key residue: V[j, c] = 1 iff j mod 64 == c, so
     AV[i, c] * n_u = sum over keys j <= i with j = c (mod 64) of rab_ij, an
     integer below 2^24, which fp32 accumulation and the 1/n_u scale keep to
@@ -104,7 +105,7 @@ def _onehot_v(offsets, heads):
     return np.tile(v, (1, heads))
 
 
-def _run_causal(H, ts_users, P, Tb, rab_pos, rab_time, phi2):
+def _run_causal(H, ts_users, P, Tb, rab_pos, rab_time, phi2, dtype="fp16"):
     heads = rab_pos.shape[0]
     lens = [len(t) for t in ts_users]
     offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
@@ -112,11 +113,12 @@ def _run_causal(H, ts_users, P, Tb, rab_pos, rab_time, phi2):
     ts = np.concatenate(ts_users).astype(np.int64)
     jag = H.Jagged(tensor(offs, torch.int64, "cuda"), tensor(ts, torch.int64, "cuda"),
                    max(lens), T)
-    q = torch.zeros((T, heads * 64), dtype=torch.bfloat16, device="cuda")
+    tdt = H.TORCH_DTYPE[dtype]
+    q = torch.zeros((T, heads * 64), dtype=tdt, device="cuda")
     k = torch.zeros_like(q)
-    v = tensor(_onehot_v(offs, heads), torch.bfloat16, "cuda")
+    v = tensor(_onehot_v(offs, heads), tdt, "cuda")
     cfg = H.LayerConfig(d_model=64, num_heads=heads, num_pos_buckets=P, num_time_buckets=Tb,
-                        phi2=phi2)
+                        phi2=phi2, dtype=dtype)
     av = H.attn_fwd_f32(cfg, jag, q, k, v, tensor(rab_pos, torch.float32, "cuda"),
                         tensor(rab_time, torch.float32, "cuda"))
     assert H.device_status() == 0
@@ -138,11 +140,11 @@ def _time_tables(heads, Tb, ks):
     return rt
 
 
-def _check_time(H, ts_users, Tb, ks, phi2, P=8192):
+def _check_time(H, ts_users, Tb, ks, phi2, P=8192, dtype="fp16"):
     heads = 1 + len(ks)
     rt = _time_tables(heads, Tb, ks)
     rp = np.zeros((heads, P), dtype=np.float32)
-    offs, av = _run_causal(H, ts_users, P, Tb, rp, rt, phi2)
+    offs, av = _run_causal(H, ts_users, P, Tb, rp, rt, phi2, dtype)
     for u, ts in enumerate(ts_users):
         n = len(ts)
         if n == 0:
@@ -150,18 +152,18 @@ def _check_time(H, ts_users, Tb, ks, phi2, P=8192):
         got = _as_integers(av[offs[u]:offs[u + 1]], n, f"user {u}")
         want = _time_sums(ts, Tb, ks)
         bad = np.argwhere(got != want)
-        assert bad.size == 0, f"user {u} (n={n}, Tb={Tb}, phi2={phi2}): first mismatch " \
+        assert bad.size == 0, f"user {u} (n={n}, Tb={Tb}, phi2={phi2}, {dtype}): first mismatch " \
                               f"(row, head, residue) {tuple(bad[0])}"
 
 
-def _check_pos(H, lens, P, ks, phi2, Tb=128):
+def _check_pos(H, lens, P, ks, phi2, Tb=128, dtype="fp16"):
     heads = 1 + len(ks)
     rp = _pos_fn(P, ks).astype(np.float32)
     rt = np.zeros((heads, Tb), dtype=np.float32)
     rng = np.random.default_rng(11)
     ts_users = [TS0 + np.floor(np.cumsum(rng.exponential(3600, n))).astype(np.int64)
                 for n in lens]
-    offs, av = _run_causal(H, ts_users, P, Tb, rp, rt, phi2)
+    offs, av = _run_causal(H, ts_users, P, Tb, rp, rt, phi2, dtype)
     for u, n in enumerate(lens):
         if n == 0:
             continue
@@ -173,13 +175,14 @@ def _check_pos(H, lens, P, ks, phi2, Tb=128):
 
 # ------------------------------------------------------------------ causal kernel
 
-@pytest.mark.parametrize("phi2", ["identity", "relu"])
-def test_time_buckets_long_lognormal_timeline(H, phi2):
+@pytest.mark.parametrize("phi2,dtype", [("identity", "fp16"), ("relu", "fp16"),
+                                        ("identity", "bf16")])
+def test_time_buckets_long_lognormal_timeline(H, phi2, dtype):
     """The long-sequence workload's timelines (8 users x 8192, log-normal gaps,
     Tb 128): every (row, key) time bucket of the kernel equals the oracle's."""
     case = make_case("long-bf16", num_layers=1)
     ts_users = [case.timestamps[case.offsets[u]:case.offsets[u + 1]] for u in range(case.cfg.batch)]
-    _check_time(H, ts_users, 128, [2, 10, 25, 40, 50, 56, 60], phi2)
+    _check_time(H, ts_users, 128, [2, 10, 25, 40, 50, 56, 60], phi2, dtype=dtype)
 
 
 @pytest.mark.parametrize("Tb", [32, 128])
@@ -214,9 +217,11 @@ def test_time_buckets_bucket_edges(H):
     _check_time(H, ts_users, 128, [1, 2, 3, 10, 30, 50, 61], "identity")
 
 
-def test_position_buckets_paired_table(H):
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_position_buckets_paired_table(H, dtype):
     """Position buckets on the paired (two staggered copies) table path."""
-    _check_pos(H, [8192, 1, 700, 2049], 8192, [1, 2, 63, 64, 1000, 4095, 8191], "identity")
+    _check_pos(H, [8192, 1, 700, 2049], 8192, [1, 2, 63, 64, 1000, 4095, 8191], "identity",
+               dtype=dtype)
 
 
 def test_position_buckets_clamped(H):
@@ -224,16 +229,19 @@ def test_position_buckets_clamped(H):
     _check_pos(H, [3000, 450], 300, [1, 2, 64, 150, 298, 299, 300], "relu")
 
 
-def test_position_buckets_single_copy_path(H):
-    """One user at the longest supported length (16384): the position table no
-    longer fits twice in shared memory and the single-copy path runs."""
-    _check_pos(H, [16384], 16384, [1, 2, 63, 4096, 9000, 16000, 16383], "identity")
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_position_buckets_longest_sequence(H, dtype):
+    """One user at the longest supported length (16384).  With bf16 operands
+    the fp32 position table no longer fits twice in shared memory and the
+    single-copy path runs; the fp16 table (fp16 operands) still fits twice."""
+    _check_pos(H, [16384], 16384, [1, 2, 63, 4096, 9000, 16000, 16383], "identity", dtype=dtype)
 
 
-def test_time_buckets_single_copy_path(H):
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_time_buckets_longest_sequence(H, dtype):
     rng = np.random.default_rng(14)
     ts_users = [TS0 + np.floor(np.cumsum(rng.lognormal(7.0, 2.0, 16384))).astype(np.int64)]
-    _check_time(H, ts_users, 128, [2, 10, 25, 40, 50, 56, 60], "identity", P=16384)
+    _check_time(H, ts_users, 128, [2, 10, 25, 40, 50, 56, 60], "identity", P=16384, dtype=dtype)
 
 
 # ------------------------------------------------------------------ candidate mode (M-FALCON)
@@ -246,7 +254,7 @@ def _cand_case(rng, hist_lens, cand_lens):
     return ts_users, req
 
 
-def _run_cand(H, ts_users, req, cand_lens, P, Tb, rab_pos, rab_time):
+def _run_cand(H, ts_users, req, cand_lens, P, Tb, rab_pos, rab_time, dtype="fp16"):
     heads = rab_pos.shape[0]
     hl = [len(t) for t in ts_users]
     hoffs = np.concatenate([[0], np.cumsum(hl)]).astype(np.int64)
@@ -255,13 +263,14 @@ def _run_cand(H, ts_users, req, cand_lens, P, Tb, rab_pos, rab_time):
     ts = np.concatenate(ts_users).astype(np.int64)
     jag = H.Jagged(tensor(hoffs, torch.int64, "cuda"), tensor(ts, torch.int64, "cuda"),
                    max(hl), T)
-    kh = torch.zeros((max(T, 1), heads * 64), dtype=torch.bfloat16, device="cuda")
-    vh = tensor(_onehot_v(hoffs, heads), torch.bfloat16, "cuda")
-    q = torch.zeros((M, heads * 64), dtype=torch.bfloat16, device="cuda")
+    tdt = H.TORCH_DTYPE[dtype]
+    kh = torch.zeros((max(T, 1), heads * 64), dtype=tdt, device="cuda")
+    vh = tensor(_onehot_v(hoffs, heads), tdt, "cuda")
+    q = torch.zeros((M, heads * 64), dtype=tdt, device="cuda")
     k = torch.zeros_like(q)
     v = torch.zeros_like(q)  # the self term adds nothing
     cfg = H.LayerConfig(d_model=64, num_heads=heads, num_pos_buckets=P, num_time_buckets=Tb,
-                        phi2="identity")
+                        phi2="identity", dtype=dtype)
     av = H.mfalcon_attn_fwd(cfg, jag, kh, vh, tensor(coffs, torch.int64, "cuda"),
                             max(cand_lens), q, k, v, tensor(req, torch.int64, "cuda"),
                             tensor(rab_pos, torch.float32, "cuda"),
@@ -270,7 +279,8 @@ def _run_cand(H, ts_users, req, cand_lens, P, Tb, rab_pos, rab_time):
     return coffs, av.cpu().numpy().reshape(M, heads, 64).astype(np.float64)
 
 
-def test_candidate_mode_buckets(H):
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_candidate_mode_buckets(H, dtype):
     """Candidate rows sit at position n_u with time t_req: their bucket against
     history key j is min(n_u - j, P - 1) and bt(t_req - t_j)."""
     rng = np.random.default_rng(15)
@@ -282,9 +292,10 @@ def test_candidate_mode_buckets(H):
     heads = 8
     rt = _time_tables(heads, Tb, ks_t)
     coffs, av_t = _run_cand(H, ts_users, req, cands, P, Tb,
-                            np.zeros((heads, P), np.float32), rt)
+                            np.zeros((heads, P), np.float32), rt, dtype)
     rp = _pos_fn(P, ks_p).astype(np.float32)
-    _, av_p = _run_cand(H, ts_users, req, cands, P, Tb, rp, np.zeros((heads, Tb), np.float32))
+    _, av_p = _run_cand(H, ts_users, req, cands, P, Tb, rp, np.zeros((heads, Tb), np.float32),
+                        dtype)
     fp = _pos_fn(P, ks_p)
     for u, n in enumerate(hist):
         rows = slice(coffs[u], coffs[u + 1])

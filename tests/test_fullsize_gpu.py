@@ -27,9 +27,7 @@ def _prefix_check(case, y, user, m, what):
     want, _ = O.forward(case.x, case.offsets, case.timestamps, case.layers, cfg,
                         users=[user], prefix=[m])
     s = int(case.offsets[user])
-    L = cfg.num_layers
-    assert_close(y[s:s + m], want[s:s + m], f"{what} user {user} rows 0..{m - 1}",
-                 max_abs=2e-2 * np.sqrt(L))
+    assert_close(y[s:s + m], want[s:s + m], f"{what} user {user} rows 0..{m - 1}")
 
 
 def _single_user_rows(H, case, t, cfg, weights, user):
@@ -141,7 +139,7 @@ def test_mfalcon_full_size_sampled(H):
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
     L, T, hv = case.cfg.num_layers, case.total_tokens, case.cfg.num_heads * 64
-    kv = torch.empty((L, T, 2 * hv), dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty((L, T, 2 * hv), dtype=cfg.cache_dtype, device="cuda")
     H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv)
     M = case.cand_emb.shape[0]
     y = torch.empty((M, case.cfg.d_model), dtype=torch.float32, device="cuda")
@@ -168,7 +166,6 @@ def test_mfalcon_full_size_sampled(H):
                                   return_rows=True)
         got_y.append(yn[rows]); want_y.append(wy)
         got_s.append(sc[rows]); want_s.append(ws); emb.append(case.cand_emb[rows])
-    assert_close(np.concatenate(got_y), np.concatenate(want_y), "mfalcon full-size final rows",
-                 max_abs=2e-2 * np.sqrt(L))
-    check_scores(np.concatenate(got_s), np.concatenate(want_s), np.concatenate(emb), L,
+    assert_close(np.concatenate(got_y), np.concatenate(want_y), "mfalcon full-size final rows")
+    check_scores(np.concatenate(got_s), np.concatenate(want_s), np.concatenate(emb),
                  "mfalcon full-size scores")

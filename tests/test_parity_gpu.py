@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from gen import make_case, round_bf16, to_dtype
+from gen import make_case, round_bf16, round_fp16, to_dtype
 from gen.device import tensor
 from gen.inputs import make_attn_case
 from oracle import hstu as O
@@ -63,12 +63,15 @@ def test_rab_index_bit_exact(H):
 ATTN_LENGTHS = [1, 127, 128, 129, 255, 256, 257, 700, 0, 64]
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("phi2", ["silu", "relu", "identity"])
-def test_attention_parity(H, phi2):
+def test_attention_parity(H, phi2, dtype):
+    """Attention alone for both operand types: fp16 is what the bf16 layers run
+    (f1 writes fp16 Q, K, V), bf16 serves bf16 inputs given directly."""
     P, Tb, heads = 512, 128, 2
-    ac = make_attn_case(ATTN_LENGTHS, heads, P, Tb, seed=5)
+    ac = make_attn_case(ATTN_LENGTHS, heads, P, Tb, seed=5, dtype=dtype)
     cfg = H.LayerConfig(d_model=128, num_heads=heads, num_pos_buckets=P, num_time_buckets=Tb,
-                        phi2=phi2)
+                        phi2=phi2, dtype=dtype)
     jag, q, k, v, rp, rt = upload_attn(H, ac)
     av = H.attn_fwd(cfg, jag, q, k, v, rp, rt).float().cpu().numpy()
     _status_ok(H)
@@ -80,15 +83,17 @@ def test_attention_parity(H, phi2):
                                 ac.v[s:e].astype(np.float64), ac.timestamps[s:e],
                                 ac.rab_pos.astype(np.float64), ac.rab_time.astype(np.float64),
                                 e - s, heads, 64, 64, phi2)
-        assert_close(av[s:e], want, f"user {u} (n={e - s}) phi2={phi2}", scaled=True)
+        assert_close(av[s:e], want, f"user {u} (n={e - s}) phi2={phi2} {dtype}", scaled=True)
 
 
-def test_attention_position_clamp_and_large_bias(H):
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_attention_position_clamp_and_large_bias(H, dtype):
     """P smaller than the sequence (clamped position buckets) and a bias large
     enough that a wrong gather is visible."""
     P, Tb, heads = 48, 16, 1
-    ac = make_attn_case([300, 5, 190], heads, P, Tb, seed=8, rab_std=0.5)
-    cfg = H.LayerConfig(d_model=64, num_heads=heads, num_pos_buckets=P, num_time_buckets=Tb)
+    ac = make_attn_case([300, 5, 190], heads, P, Tb, seed=8, rab_std=0.5, dtype=dtype)
+    cfg = H.LayerConfig(d_model=64, num_heads=heads, num_pos_buckets=P, num_time_buckets=Tb,
+                        dtype=dtype)
     jag, q, k, v, rp, rt = upload_attn(H, ac)
     av = H.attn_fwd(cfg, jag, q, k, v, rp, rt).float().cpu().numpy()
     for u in range(3):
@@ -103,15 +108,14 @@ def test_attention_position_clamp_and_large_bias(H):
 # ------------------------------------------------------------------ whole layers
 
 def _forward_check(H, case, what, check_delta=True):
-    """Whole stack: rel-L2 <= 5e-3 and max-abs <= 2e-2 * sqrt(L) (independent
-    per-layer rounding errors accumulate as a random walk through the residual)."""
+    """Whole stack at the stated bound: max abs <= 2e-2 and rel-L2 <= 5e-3
+    against the float64 oracle, plus the layer delta Y - X on its own."""
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
     y = H.forward(cfg, weights, jag, t["x"]).cpu().numpy()
     _status_ok(H)
     want, _ = O.forward(case.x, case.offsets, case.timestamps, case.layers, case.cfg)
-    L = case.cfg.num_layers
-    ma, rl = assert_close(y, want, what, max_abs=2e-2 * np.sqrt(L))
+    ma, rl = assert_close(y, want, what)
     if check_delta:
         # the change Y - X on its own, so the residual cannot hide errors
         x = case.x.astype(np.float64)
@@ -197,7 +201,7 @@ def test_single_layer_kv_cache_and_lp_copy(H):
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
     T, d, hv = case.total_tokens, case.cfg.d_model, case.cfg.num_heads * 64
-    kv = torch.zeros((T, 2 * hv), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((T, 2 * hv), dtype=cfg.cache_dtype, device="cuda")
     ylp = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
     y = H.layer_fwd(cfg, weights[0], jag, t["x"], y_out_lp=ylp, kv_cache_out=kv)
     want = O.layer_fwd(case.x, case.offsets, case.timestamps, case.layers[0], case.cfg)
@@ -252,7 +256,7 @@ def _mfalcon_run(H, case, microbatch, rows=False):
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
     L, T, hv = case.cfg.num_layers, case.total_tokens, case.cfg.num_heads * 64
-    kv = torch.empty((L, max(T, 1), 2 * hv), dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty((L, max(T, 1), 2 * hv), dtype=cfg.cache_dtype, device="cuda")
     H.forward(cfg, weights, jag, t["x"], kv_cache_out=kv)
     y = None
     if rows:
@@ -275,19 +279,20 @@ def test_mfalcon_parity(H):
                                     case.cand_offsets, case.cand_emb, case.request_ts, 64,
                                     return_rows=True)
     L = case.cfg.num_layers
-    assert_close(y, want_y, "mfalcon final rows", max_abs=2e-2 * np.sqrt(L))
+    assert_close(y, want_y, "mfalcon final rows")
     e = case.cand_emb.astype(np.float64)
     dma, drl = errors(y - e, want_y - e)
     record("mfalcon final rows delta y-e", dma, drl, None, 2e-2)
     assert drl <= 2e-2, f"delta rel_l2={drl:.3e}"
-    check_scores(sc, want, case.cand_emb, L, "mfalcon scores")
+    check_scores(sc, want, case.cand_emb, "mfalcon scores")
 
 
 def test_mfalcon_per_layer(H):
     """Every M-FALCON layer on its own at the stated bound (max abs 2e-2,
     rel-L2 5e-3): layer l gets the oracle's layer l-1 candidate rows and the
-    oracle's layer-l history keys/values, both rounded to bf16 and given to
-    both sides, so differences come from the GPU arithmetic of that layer."""
+    oracle's layer-l history keys/values, rounded to bf16 (rows) and fp16 (the
+    cache's type) and given to both sides, so differences come from the GPU
+    arithmetic of that layer."""
     case = _mfalcon_case(33, [300, 0, 129, 1000], m=150, layers=4)
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
@@ -297,11 +302,11 @@ def test_mfalcon_per_layer(H):
     M = cur.shape[0]
     for l, lw in enumerate(case.layers):
         xt = round_bf16(cur)
-        kt, vt = round_bf16(ks[l]), round_bf16(vs[l])
+        kt, vt = round_fp16(ks[l]), round_fp16(vs[l])  # the cache holds fp16
         want_s, want_y = O.mfalcon_scores(None, case.offsets, case.timestamps, [lw], case.cfg,
                                           case.cand_offsets, xt, case.request_ts, 64,
                                           kv=([kt], [vt]), return_rows=True)
-        kv = tensor(np.concatenate([kt, vt], axis=1)[None], torch.bfloat16, "cuda")
+        kv = tensor(np.concatenate([kt, vt], axis=1)[None], cfg.cache_dtype, "cuda")
         y = torch.empty((M, d), dtype=torch.float32, device="cuda")
         sc = H.mfalcon_score(cfg, [weights[l]], jag, kv, t["cand_offsets"],
                              tensor(xt, torch.bfloat16, "cuda"), t["request_ts"], 64,
@@ -310,7 +315,7 @@ def test_mfalcon_per_layer(H):
         yn = y.cpu().numpy()
         assert_close(yn, want_y, f"mfalcon layer {l} rows")
         assert_close(yn - xt, want_y - xt, f"mfalcon layer {l} delta", max_abs=2e-2, rel_l2=2e-2)
-        check_scores(sc.cpu().numpy(), want_s, xt, 1, f"mfalcon layer {l} scores")
+        check_scores(sc.cpu().numpy(), want_s, xt, f"mfalcon layer {l} scores")
         cur = want_y
 
 
