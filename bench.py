@@ -41,7 +41,25 @@ WORKLOAD_TEXT = {
     "tiny-fp32": "1 HSTU layer fp32, d_model 64, 1 head x 64, 4 users, lengths U{8..64}",
     "mfalcon": "M-FALCON ranking: 4 HSTU layers bf16, d_model 512, 8 heads x 64, 16 users x 4096 "
                "cached history, 2048 candidates per user in microbatches of 256",
+    "long-bf16-softmax": "the long-sequence workload with the (-rab, Softmax) ablation: softmax "
+                         "over the visible keys instead of the pointwise phi2, zero bias tables",
 }
+# workloads that are another workload with a changed configuration:
+# name -> (base workload, config changes, zero the rab tables)
+VARIANTS = {"long-bf16-softmax": ("long-bf16", {"phi2": "softmax"}, True)}
+
+
+def make_workload(name, batch=None):
+    from gen import make_case
+    base, changes, zero_rab = VARIANTS.get(name, (name, {}, False))
+    case = make_case(base, batch=batch)
+    if changes:
+        case = make_case(case.cfg.replace(**changes), seed=case.seed, batch=batch)
+    if zero_rab:
+        for lw in case.layers:
+            lw.rab_pos[:] = 0.0
+            lw.rab_time[:] = 0.0
+    return case
 MFALCON_METRIC = "M-FALCON candidate scores/sec at 1 B200 (cached history K/V)"
 # The attention launches of these workloads last about a millisecond inside
 # steps of a few milliseconds, far from the seconds-long matmul loop that
@@ -185,8 +203,7 @@ def run_reference(args, rank, world):
     """The reference arm: the float64 oracle on the host cores (rank 0 only)."""
     if rank != 0:
         return
-    from gen import make_case
-    case = make_case(args.workload)
+    case = make_workload(args.workload)
     for _ in range(args.warmup):
         oracle_extrapolated(case, target_s=1.0)
     samples = [oracle_extrapolated(case, target_s=args.ref_seconds) for _ in range(args.steps)]
@@ -365,9 +382,9 @@ def _roofline(ctx, kernels, name, flop, kernel_label, bound="tensor"):
 def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batch=None):
     """Time hstu_forward over one workload; returns a dict (value, rooflines...)."""
     torch, H = ctx.torch, ctx.H
-    from gen import make_case, algorithmic_counts
+    from gen import algorithmic_counts
     from gen.device import case_tensors
-    case = make_case(name, batch=batch)
+    case = make_workload(name, batch=batch)
     c = case.cfg
     counts = algorithmic_counts(case)
     t = case_tensors(case, ctx.dev)
@@ -644,7 +661,7 @@ def main():
                                      100 * r["roofline"].get("frac_of_sustained", 0.0)}
         if world == 1 and not args.no_workloads and args.batch is None:
             subs = {}
-            for name in ("small-bf16", "sl-bf16", "tiny-fp32"):
+            for name in ("small-bf16", "sl-bf16", "tiny-fp32", "long-bf16-softmax"):
                 if name == args.workload:
                     continue
                 subs[name] = _public(measure_forward(ctx, name, min(args.steps, 20), args.warmup,

@@ -112,28 +112,33 @@ __device__ __forceinline__ int time_bucket_search(int64_t dt, const int64_t* thr
 // Bucket of t_i - t_j for one query row as j walks forward through keys with
 // non-decreasing timestamps: the bucket can only go down, so each step is a
 // compare against the current lower edge and an occasional decrement.
-// T is int64_t (absolute seconds) or int32_t (seconds since the user's first
-// event, used when the user's whole span fits).
+// T is int64_t (absolute seconds, with the int64 threshold table) or int32_t
+// (seconds since the user's first event, used when the user's whole span
+// fits, with the threshold table clamped to int32: every bucket the walk
+// visits has a threshold at most t_i < 2^31, so the clamp changes no bound).
 template <typename T>
 struct BucketWalk {
+  using TT = T;  // threshold table entry type
   int b;
   T ti;
   T bound;  // keys with t_j <= bound are still in bucket >= b
 
-  __device__ __forceinline__ void init(T t_row, T t_first_key, const int64_t* thr, int Tb) {
+  __device__ __forceinline__ void init(T t_row, T t_first_key, const int64_t* thr64, const TT* thr,
+                                       int Tb) {
     ti = t_row;
-    b = time_bucket_search(static_cast<int64_t>(t_row) - static_cast<int64_t>(t_first_key), thr, Tb);
+    b = time_bucket_search(static_cast<int64_t>(t_row) - static_cast<int64_t>(t_first_key), thr64,
+                           Tb);
     set_bound(thr);
   }
-  __device__ __forceinline__ void set_bound(const int64_t* thr) {
+  __device__ __forceinline__ void set_bound(const TT* thr) {
     if constexpr (sizeof(T) == 8) {
       bound = (b == 0) ? INT64_MAX : ti - thr[b];
     } else {
-      bound = (b == 0) ? INT32_MAX : static_cast<T>(static_cast<int64_t>(ti) - thr[b]);
+      bound = (b == 0) ? INT32_MAX : ti - thr[b];  // ti >= 0, thr[b] in [0, INT32_MAX]
     }
   }
   // Advance to a key with timestamp tj; returns true when the bucket changed.
-  __device__ __forceinline__ bool step(T tj, const int64_t* thr) {
+  __device__ __forceinline__ bool step(T tj, const TT* thr) {
     bool changed = false;
     while (tj > bound) {
       --b;
@@ -217,8 +222,13 @@ __device__ __forceinline__ float apply_phi(float x) {
   }
 }
 
+// Scale folded into the staged bias tables and applied to S: SiLU works on
+// x/2 (x sigmoid(x) = h + h tanh(h), h = x/2); softmax on x log2(e), so that
+// exp(x - m) = 2^(h - m') with the MUFU's exp2.
 template <int PHI>
-__host__ __device__ constexpr float phi_scale() { return PHI == HSTU_ACT_SILU ? 0.5f : 1.0f; }
+__host__ __device__ constexpr float phi_scale() {
+  return PHI == HSTU_ACT_SILU ? 0.5f : (PHI == HSTU_ACT_SOFTMAX ? 1.4426950408889634f : 1.0f);
+}
 
 // Zero the keys of a bf16 pair at columns c, c+1 that are above `last`.
 __device__ __forceinline__ uint32_t mask_pair(uint32_t w, int c, int last) {
@@ -237,12 +247,14 @@ struct AttnSmem {
   static constexpr uint32_t kKeyStride = ATT_KEYS * 4;                // bytes per stage
   static constexpr uint32_t kTimeTab = kKeyInfo + ATT_STAGES * kKeyStride;
   static constexpr uint32_t kThr = kTimeTab + MAX_TIME_BUCKETS * 4;
-  static constexpr uint32_t kOct = kThr + MAX_TIME_BUCKETS * 8;      // 32 x int4
+  static constexpr uint32_t kThr32 = kThr + MAX_TIME_BUCKETS * 8;   // int32 copy, clamped
+  static constexpr uint32_t kOct = kThr32 + MAX_TIME_BUCKETS * 4;    // 32 x int4
   static constexpr uint32_t kOrt = kOct + 32 * 16;                   // 32 x float4
   static constexpr uint32_t kBars = kOrt + 32 * 16;
   static constexpr uint32_t kMisc = kBars + 32 * 8;
   static constexpr uint32_t kLnX = kMisc + 64;                        // 2 x 128 float2
-  static constexpr uint32_t kPos = kLnX + 2 * ATT_ROWS * 8;
+  static constexpr uint32_t kML = kLnX + 2 * ATT_ROWS * 8;           // 4 x 128 float2
+  static constexpr uint32_t kPos = kML + 4 * ATT_ROWS * 8;
   // pos_len entries per copy of `elt` bytes each (fp32, or fp16 for the
   // causal fp16-operand kernel), two copies with paired reads
   static constexpr uint32_t bytes(int pos_len, bool pairs, uint32_t elt = 4u) {
@@ -284,7 +296,7 @@ template <bool PAIRS, class Sink>
 __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], Sink&& sink,
                                              const float* rvx, const int32_t* kts, int lim,
                                              BucketWalk<int32_t>& w, const float* sTime,
-                                             const int64_t* sThr, const int4* sOct,
+                                             const int32_t* sThr, const int4* sOct,
                                              const float4* sOrt, uint64_t scale2, float& rt_cur) {
   const unsigned full = 0xffffffffu;
   const bool live = lim >= 0;
@@ -332,9 +344,9 @@ __device__ __forceinline__ void causal_chunk(const uint32_t (&sv)[32], Sink&& si
     if (B_hi - B_lo == 1) {
       if (live) {
         const float rt_hi = sTime[B_hi], rt_lo = sTime[B_lo];
-        const int64_t e = static_cast<int64_t>(w.ti) - sThr[B_hi];
-        const int32_t edge =
-            e < static_cast<int64_t>(INT32_MIN) ? INT32_MIN : static_cast<int32_t>(e);
+        // keys with t_j <= edge are in bucket B_hi (ti >= 0 and the clamped
+        // threshold <= INT32_MAX, so the difference does not overflow)
+        const int32_t edge = w.ti - sThr[B_hi];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           const int2 k2 = kt_pair(c);
@@ -361,7 +373,7 @@ template <int PHI, bool PAIRS, bool F16>
 __device__ __forceinline__ void causal_chunk_pointwise(const uint32_t (&sv)[32], uint32_t (&pk)[16],
                                                        const float* rvx, const int32_t* kts, int lim,
                                                        BucketWalk<int32_t>& w, const float* sTime,
-                                                       const int64_t* sThr, const int4* sOct,
+                                                       const int32_t* sThr, const int4* sOct,
                                                        const float4* sOrt, uint64_t scale2,
                                                        float& rt_cur) {
   causal_chunk<PAIRS>(
@@ -426,6 +438,12 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     nB = has_b ? (q0 + 2 * ATT_ROWS) / ATT_KEYS : 0;
   }
   const int nk_total = nA > nB ? nA : nB;
+  // The softmax ablation takes two passes over the key tiles: the first finds
+  // each row's max and sum, the second writes P and runs P V.  Stage index
+  // si = pass * nk_total + tile.
+  constexpr bool kSoftmax = PHI == HSTU_ACT_SOFTMAX;
+  constexpr int kPasses = kSoftmax ? 2 : 1;
+  const int n_stages = kPasses * nk_total;
 
   // causal rows read position offsets i - j in [-127, q0 + 255]; candidates
   // read n_kv - j in [1, n_kv].  The staged table holds scale * rab_pos at
@@ -439,11 +457,13 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* sKey = smem + AttnSmem::kKeyInfo;
   float* sTime = reinterpret_cast<float*>(smem + AttnSmem::kTimeTab);
   int64_t* sThr = reinterpret_cast<int64_t*>(smem + AttnSmem::kThr);
+  int32_t* sThr32 = reinterpret_cast<int32_t*>(smem + AttnSmem::kThr32);
   int4* sOct = reinterpret_cast<int4*>(smem + AttnSmem::kOct);
   float4* sOrt = reinterpret_cast<float4*>(smem + AttnSmem::kOrt);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + AttnSmem::kMisc);
   float2* sLnX = reinterpret_cast<float2*>(smem + AttnSmem::kLnX);
+  float2* sML = reinterpret_cast<float2*>(smem + AttnSmem::kML);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 4);
   float* sRv = reinterpret_cast<float*>(smem + AttnSmem::kPos);
 
@@ -501,6 +521,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   for (int k = tid; k < p.Tb; k += ATT_THREADS) {
     sTime[k] = kScale * p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     sThr[k] = p.thr[k];
+    sThr32[k] = p.thr[k] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(p.thr[k]) : INT32_MAX;
   }
   if (tid < 32) {
     const int4 o = p.oct[tid];
@@ -544,22 +565,26 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         t[e] = j < n_kv ? p.timestamps[kv_start + j] : 0;
       }
     };
-    if (nk_total > 0) load_ts(0, ts_next);
-    for (int kt = 0; kt < nk_total; ++kt) {
-      const int s = kt % ATT_STAGES;
+    if (n_stages > 0) load_ts(0, ts_next);
+    for (int si = 0; si < n_stages; ++si) {
+      const int kt = si % nk_total;                // key tile
+      const bool last_pass = si >= (kPasses - 1) * nk_total;
+      const int s = si % ATT_STAGES;
       int64_t ts[KPL];
 #pragma unroll
       for (int e = 0; e < KPL; ++e) ts[e] = ts_next[e];
-      if (kt + 1 < nk_total) load_ts(kt + 1, ts_next);
-      const uint32_t par = (static_cast<uint32_t>(kt / ATT_STAGES) & 1u) ^ 1u;
+      if (si + 1 < n_stages) load_ts((si + 1) % nk_total, ts_next);
+      const uint32_t par = (static_cast<uint32_t>(si / ATT_STAGES) & 1u) ^ 1u;
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&bars[BAR_KV_EMPTY + s], par, ctl) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars[BAR_KV_FULL + s], 2 * ATT_TILE_BYTES);
+        // V is only read by P V, in the last pass
+        mbar_arrive_expect_tx(&bars[BAR_KV_FULL + s], (last_pass ? 2 : 1) * ATT_TILE_BYTES);
         const int32_t row = static_cast<int32_t>(kv_start + kt * ATT_KEYS);
         tma_load_2d(sK + s * ATT_TILE_BYTES, &tm_k, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
-        tma_load_2d(sV + s * ATT_TILE_BYTES, &tm_v, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
+        if (last_pass)
+          tma_load_2d(sV + s * ATT_TILE_BYTES, &tm_v, &bars[BAR_KV_FULL + s], h * ATT_HD, row);
       }
       ++issued;
       uint8_t* key = sKey + s * AttnSmem::kKeyStride;
@@ -644,10 +669,10 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         __syncwarp();
       };
-      // O += P(kt) V(kt); P of keys 0-31 sits at columns 0-15 of the S
-      // buffer of tile kt, P of keys 32-63 at columns 32-47
-      auto issue_pv = [&](int kt, int b) {
-        const uint64_t dv = dV0 + static_cast<uint64_t>(kt % ATT_STAGES) * kStageDesc;
+      // O += P(kt) V(kt) from stage si; P of keys 0-31 sits at columns 0-15
+      // of the S buffer, P of keys 32-63 at columns 32-47
+      auto issue_pv = [&](int kt, int si, int b) {
+        const uint64_t dv = dV0 + static_cast<uint64_t>(si % ATT_STAGES) * kStageDesc;
         const uint32_t a = tS + static_cast<uint32_t>(b * 64);
         const uint32_t acc0 = kt > 0 ? 1u : 0u;
         if (leader) {
@@ -658,24 +683,36 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         __syncwarp();
       };
-      // three tiles ahead: S(0), S(1), S(2) before any P exists
-      for (int t = 0; ok && t < ATT_SBUF && t < nWg; ++t) {
-        ok = await_kv(t);
-        if (ok) issue_s(t, t);
+      // This tile's items: its nWg key tiles, once per pass; item gi reads
+      // stage stage_of(gi).  (With two passes the look-ahead of three items
+      // reaches at most nB - nA + 3 = 5 stages past the current one, inside
+      // the ring of ATT_STAGES.)
+      const int n_items = kPasses * nWg;
+      auto stage_of = [&](int gi) -> int {
+        return gi < nWg ? gi : nk_total + (gi - nWg);
+      };
+      // three items ahead: S of items 0, 1, 2 before any P exists
+      for (int t = 0; ok && t < ATT_SBUF && t < n_items; ++t) {
+        ok = await_kv(stage_of(t));
+        if (ok) issue_s(stage_of(t), t);
       }
-      int b = 0;         // buffer of tile kt
-      uint32_t ph = 0;   // phase parity of that buffer's barriers at tile kt
-      for (int kt = 0; ok && kt < nk_total; ++kt) {
+      int b = 0;         // buffer of item gi
+      uint32_t ph = 0;   // phase parity of that buffer's barriers at item gi
+      int gi = 0;
+      for (int si = 0; ok && si < n_stages; ++si) {
+        const int kt = si % nk_total;
         if (kt < nWg) {
           ok = wait_all(&bars[BAR_P_FULL + ATT_SBUF * g + b], ph);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(kt, b);
-          if (kt + ATT_SBUF < nWg) {
-            ok = await_kv(kt + ATT_SBUF);
+          if (si >= (kPasses - 1) * nk_total) issue_pv(kt, si, b);  // last pass: P V
+          if (gi + ATT_SBUF < n_items) {
+            const int sn = stage_of(gi + ATT_SBUF);
+            ok = await_kv(sn);
             if (!ok) break;
-            issue_s(kt + ATT_SBUF, b);  // into the buffer P V(kt) has just been issued to read
+            issue_s(sn, b);  // into the buffer P V(kt) has just been issued to read
           }
+          ++gi;
           if (++b == ATT_SBUF) {
             b = 0;
             ph ^= 1u;
@@ -683,10 +720,10 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         } else {
           // past this tile's last key tile: the release below must still
           // follow the stage's load, so it counts toward this tile's phase
-          ok = await_kv(kt);
+          ok = await_kv(si);
           if (!ok) break;
         }
-        if (leader) mma_commit(&bars[BAR_KV_EMPTY + kt % ATT_STAGES]);
+        if (leader) mma_commit(&bars[BAR_KV_EMPTY + si % ATT_STAGES]);
         __syncwarp();
       }
       if (leader) {
@@ -723,7 +760,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if constexpr (!CAND) {
       const int64_t d = (valid ? p.timestamps[kv_start + i] : t_first) - t_first;
       w32.init(d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d), 0,
-               sThr, p.Tb);
+               sThr, sThr32, p.Tb);
       if constexpr (PAIRS) copy = (D - i) & 1;
       rv = sRv + copy * p.pos_len;
       rt_cur = sTime[w32.b];
@@ -762,37 +799,196 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int lim = !valid ? -1 : i - j0;
         const int32_t* kts = reinterpret_cast<const int32_t*>(key) + half * 32;
         const int xc = D - i + j0 + copy;  // table index at column 0
-        causal_chunk_pointwise<PHI, PAIRS, F16>(sv, pk, rv + xc, kts, lim, w32, sTime, sThr, sOct,
-                                                sOrt, scale2, rt_cur);
+        causal_chunk_pointwise<PHI, PAIRS, F16>(sv, pk, rv + xc, kts, lim, w32, sTime, sThr32,
+                                                sOct, sOrt, scale2, rt_cur);
       }
     };
 
-    int buf = 0;        // S buffer of tile kt (kt mod 3)
-    uint32_t ph = 0;    // its barriers' phase parity at tile kt
-    for (int kt = 0; kt < nW; ++kt) {
-      const int s = kt % ATT_STAGES;
-      ok = mbar_wait(&bars[BAR_S_FULL + ATT_SBUF * g + buf], ph, ctl);
-      // the producer's per-key side data for this stage (already complete)
-      if (ok)
-        ok = mbar_wait(&bars[BAR_KV_FULL + s], static_cast<uint32_t>(kt / ATT_STAGES) & 1u, ctl);
-      ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-collective
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tS = tS0 + static_cast<uint32_t>(buf * 64);
-      // 32 keys: TMEM -> registers -> bias, phi2, mask -> P over this half's S
-      uint32_t sa[32], pk[16];
-      tmem_ld32(tS, sa);
-      tmem_ld_wait(sa);
-      chunk(sa, pk, kt, s);
-      __syncwarp();
-      tmem_st16(tS, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars[BAR_P_FULL + ATT_SBUF * g + buf]);
-      if (++buf == ATT_SBUF) {
-        buf = 0;
-        ph ^= 1u;
+    // candidate mode: the candidate's own key/value enters with position
+    // bucket 0 and time bucket 0
+    const int64_t row = q_start + i;
+    auto to_f2 = [](uint32_t w) -> float2 {  // a packed pair of the operand type
+      if constexpr (F16) return __half22float2(*reinterpret_cast<const __half2*>(&w));
+      else return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+    };
+    auto self_dot = [&]() -> float {
+      const uint16_t* qs = static_cast<const uint16_t*>(p.q_self) + row * p.ld_self + h * ATT_HD;
+      const uint16_t* ks = static_cast<const uint16_t*>(p.k_self) + row * p.ld_self + h * ATT_HD;
+      float dot = 0.0f;
+#pragma unroll
+      for (int c = 0; c < ATT_HD; c += 8) {
+        const uint4 qa = *reinterpret_cast<const uint4*>(qs + c);
+        const uint4 ka = *reinterpret_cast<const uint4*>(ks + c);
+        const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 qf = to_f2(qw[t]);
+          const float2 kf = to_f2(kw[t]);
+          dot = fmaf(qf.x, kf.x, dot);
+          dot = fmaf(qf.y, kf.y, dot);
+        }
       }
+      return dot;
+    };
+    auto self_rab = [&]() -> float {
+      return p.rab_pos[static_cast<int64_t>(h) * p.P] + p.rab_time[static_cast<int64_t>(h) * p.Tb];
+    };
+
+    // ---- softmax ablation: running max and sum of 2^h over this half's keys
+    // (h = (s + rab) log2 e); the first pass only reads S, the second writes
+    // P = 2^(h - m - log2 l)
+    float sm_m = -INFINITY, sm_l = 0.0f;
+    float h_self = -INFINITY;  // candidate mode: the own key's pre-activation
+    if constexpr (kSoftmax && CAND) {
+      if (valid) h_self = kScale * (self_dot() + self_rab());
+      if (half == 0 && valid) {
+        sm_m = h_self;
+        sm_l = 1.0f;
+      }
+    }
+    // fold the scaled pre-activations of one chunk (pairs in hh, columns
+    // above `last` invisible) into (sm_m, sm_l)
+    auto softmax_accumulate = [&](const uint64_t (&hh)[16], int last) {
+      if (last < 0) return;
+      float cm = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float a, bb;
+        f2_unpack(hh[q], a, bb);
+        if (2 * q <= last) cm = fmaxf(cm, a);
+        if (2 * q + 1 <= last) cm = fmaxf(cm, bb);
+      }
+      if (cm > sm_m) {
+        sm_l *= ex2_approx(sm_m - cm);
+        sm_m = cm;
+      }
+      const uint64_t neg = f2_pack(-sm_m, -sm_m);
+      float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float a, bb;
+        f2_unpack(f2_add(hh[q], neg), a, bb);
+        const float e0 = ex2_approx(a), e1 = ex2_approx(bb);
+        acc0 += (2 * q <= last) ? e0 : 0.0f;
+        acc1 += (2 * q + 1 <= last) ? e1 : 0.0f;
+      }
+      sm_l += acc0 + acc1;
+    };
+    // pre-activations of keys 32*half .. 32*half + 31 of tile kt (fp32 pairs)
+    // and the last visible column
+    auto chunk_h = [&](const uint32_t (&sv)[32], uint64_t (&hh)[16], int kt, int s) -> int {
+      const uint8_t* key = sKey + s * AttnSmem::kKeyStride;
+      const int j0 = kt * ATT_KEYS + half * 32;
+      if constexpr (CAND) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          uint64_t bias;
+          if constexpr (F16) {
+            const float2 bf = __half22float2(
+                *reinterpret_cast<const __half2*>(reinterpret_cast<const __half*>(key) + half * 32 + c));
+            bias = f2_pack(bf.x, bf.y);
+          } else {
+            bias = lds_b64(reinterpret_cast<const float*>(key) + half * 32 + c);
+          }
+          hh[c >> 1] = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), scale2, bias);
+        }
+        return valid ? min(31, n_kv - 1 - j0) : -1;
+      } else {
+        const int lim = !valid ? -1 : i - j0;
+        causal_chunk<PAIRS>(
+            sv, [&](int c, uint64_t hv) { hh[c >> 1] = hv; }, rv + (D - i + j0 + copy),
+            reinterpret_cast<const int32_t*>(key) + half * 32, lim, w32, sTime, sThr32, sOct,
+            sOrt, scale2, rt_cur);
+        return lim < 31 ? lim : 31;
+      }
+    };
+
+    int buf = 0;        // S buffer of the current item (item index mod 3)
+    uint32_t ph = 0;    // its barriers' phase parity
+    // one pass over this tile's nW key tiles; stage of tile kt in pass `pass`
+    // is pass * nk_total + kt
+    auto run_pass = [&](int pass) {
+      for (int kt = 0; kt < nW; ++kt) {
+        const int si = pass * nk_total + kt;
+        const int s = si % ATT_STAGES;
+        ok = mbar_wait(&bars[BAR_S_FULL + ATT_SBUF * g + buf], ph, ctl);
+        // the producer's per-key side data for this stage (already complete)
+        if (ok)
+          ok = mbar_wait(&bars[BAR_KV_FULL + s], static_cast<uint32_t>(si / ATT_STAGES) & 1u, ctl);
+        ok = __all_sync(0xffffffffu, ok);  // TMEM loads below are warp-collective
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tS0 + static_cast<uint32_t>(buf * 64);
+        // 32 keys: TMEM -> registers -> bias, phi2, mask -> P over this half's S
+        uint32_t sa[32];
+        tmem_ld32(tS, sa);
+        tmem_ld_wait(sa);
+        if (kSoftmax && pass == 0) {
+          uint64_t hh[16];
+          const int last = chunk_h(sa, hh, kt, s);
+          softmax_accumulate(hh, last);
+        } else if constexpr (kSoftmax) {
+          uint64_t hh[16];
+          const int last = chunk_h(sa, hh, kt, s);
+          uint32_t pk[16];
+          const uint64_t neg = f2_pack(-sm_m, -sm_m);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            float a, bb;
+            f2_unpack(f2_add(hh[q], neg), a, bb);
+            const uint64_t e2 = f2_pack(ex2_approx(a), ex2_approx(bb));
+            if constexpr (F16) pk[q] = f2_to_h2(e2);
+            else pk[q] = f2_to_bf16x2(e2);
+          }
+          if (last < 0) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = 0u;
+          } else if (last < 31) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
+          }
+          __syncwarp();
+          tmem_st16(tS, pk);
+          tmem_st_wait();
+        } else {
+          uint32_t pk[16];
+          chunk(sa, pk, kt, s);
+          __syncwarp();
+          tmem_st16(tS, pk);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[BAR_P_FULL + ATT_SBUF * g + buf]);
+        if (++buf == ATT_SBUF) {
+          buf = 0;
+          ph ^= 1u;
+        }
+      }
+    };
+    if constexpr (kSoftmax) {
+      run_pass(0);
+      // merge the two halves' (max, sum) of each row; every thread of the
+      // group's 256 reaches this barrier (a failed wait only skips work)
+      sML[(g * 2 + half) * ATT_ROWS + r] = make_float2(sm_m, sm_l);
+      named_barrier_sync(1 + g, 2 * ATT_ROWS);
+      const float2 other = sML[(g * 2 + (half ^ 1)) * ATT_ROWS + r];
+      const float m = fmaxf(sm_m, other.x);
+      float l = 0.0f;
+      if (m > -INFINITY) l = sm_l * ex2_approx(sm_m - m) + other.y * ex2_approx(other.x - m);
+      // P = 2^(h - m) / l = 2^(h - (m + log2 l)); rows with no visible key keep P = 0
+      sm_m = l > 0.0f ? m + lg2_approx(l) : INFINITY;
+      named_barrier_sync(1 + g, 2 * ATT_ROWS);  // both halves have read before reuse
+      if constexpr (!CAND) {
+        // the second pass walks the time buckets from the first key again
+        const int64_t d = (valid ? p.timestamps[kv_start + i] : t_first) - t_first;
+        w32.init(d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d),
+                 0, sThr, sThr32, p.Tb);
+        rt_cur = sTime[w32.b];
+      }
+      if (ok) run_pass(1);
+    } else {
+      run_pass(0);
     }
 
     // ---------------- epilogue: O / N, LayerNorm partial sums, store
@@ -804,7 +1000,6 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (ok && nW > 0) ok = mbar_wait(&bars[BAR_O_FULL + g], 0, ctl);
     ok = __all_sync(0xffffffffu, ok);
     float hsum = 0.0f, hm2 = 0.0f;
-    const int64_t row = q_start + i;
     if (ok) {
       if (nW > 0) {
         tc_fence_after();
@@ -820,33 +1015,11 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (valid) {
         if constexpr (CAND) {
           // the candidate's own key/value: position bucket 0, time bucket 0
-          const uint16_t* qs = static_cast<const uint16_t*>(p.q_self) + row * p.ld_self + h * ATT_HD;
-          const uint16_t* ks = static_cast<const uint16_t*>(p.k_self) + row * p.ld_self + h * ATT_HD;
           const uint16_t* vs =
               static_cast<const uint16_t*>(p.v_self) + row * p.ld_self + h * ATT_HD + half * HC;
-          // a packed pair of the operand type as two floats
-          auto to_f2 = [](uint32_t w) -> float2 {
-            if constexpr (F16) return __half22float2(*reinterpret_cast<const __half2*>(&w));
-            else return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-          };
-          float dot = 0.0f;
-#pragma unroll
-          for (int c = 0; c < ATT_HD; c += 8) {
-            const uint4 qa = *reinterpret_cast<const uint4*>(qs + c);
-            const uint4 ka = *reinterpret_cast<const uint4*>(ks + c);
-            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w};
-            const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float2 qf = to_f2(qw[t]);
-              const float2 kf = to_f2(kw[t]);
-              dot = fmaf(qf.x, kf.x, dot);
-              dot = fmaf(qf.y, kf.y, dot);
-            }
-          }
-          const float rab0 = (p.rab_pos[static_cast<int64_t>(h) * p.P] +
-                              p.rab_time[static_cast<int64_t>(h) * p.Tb]);
-          const float ps = apply_phi<PHI>(dot + rab0);
+          float ps;
+          if constexpr (kSoftmax) ps = ex2_approx(h_self - sm_m);  // already divided by the sum
+          else ps = apply_phi<PHI>(self_dot() + self_rab());
 #pragma unroll
           for (int c = 0; c < HC; c += 8) {
             const uint4 va = *reinterpret_cast<const uint4*>(vs + c);
@@ -859,7 +1032,9 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
           }
         }
-        const float inv_n = 1.0f / static_cast<float>(CAND ? max(n_kv, 1) : n_kv);
+        // pointwise phi2 divides by N = n_u; softmax weights are normalised already
+        const float inv_n =
+            kSoftmax ? 1.0f : 1.0f / static_cast<float>(CAND ? max(n_kv, 1) : n_kv);
 #pragma unroll
         for (int c = 0; c < HC; ++c) {
           o[c] *= inv_n;
@@ -924,8 +1099,12 @@ __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_
                                             int max_len, int32_t* pos_idx, int32_t* time_idx,
                                             const __grid_constant__ AttnParams p) {
   __shared__ int64_t sThr[MAX_TIME_BUCKETS];
+  __shared__ int32_t sThr32[MAX_TIME_BUCKETS];
   __shared__ int4 sOct[32];
-  for (int k = threadIdx.x; k < Tb; k += blockDim.x) sThr[k] = p.thr[k];
+  for (int k = threadIdx.x; k < Tb; k += blockDim.x) {
+    sThr[k] = p.thr[k];
+    sThr32[k] = p.thr[k] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(p.thr[k]) : INT32_MAX;
+  }
   if (threadIdx.x < 32) sOct[threadIdx.x] = p.oct[threadIdx.x];
   __syncthreads();
   const int u = blockIdx.y;
@@ -939,13 +1118,13 @@ __global__ void hstu_debug_rab_index_kernel(const int64_t* offsets, const int64_
   const bool ts32 = timestamps[s + n - 1] - t0 < static_cast<int64_t>(INT32_MAX) - 1;
   BucketWalk<int32_t> w32;
   BucketWalk<int64_t> w64;
-  if (ts32) w32.init(static_cast<int32_t>(timestamps[s + i] - t0), 0, sThr, Tb);
-  else w64.init(timestamps[s + i], t0, sThr, Tb);
+  if (ts32) w32.init(static_cast<int32_t>(timestamps[s + i] - t0), 0, sThr, sThr32, Tb);
+  else w64.init(timestamps[s + i], t0, sThr, sThr, Tb);
   for (int j = 0; j < n; ++j) {
     if (j <= i) {
       int b;
       if (ts32) {
-        w32.step(static_cast<int32_t>(timestamps[s + j] - t0), sThr);
+        w32.step(static_cast<int32_t>(timestamps[s + j] - t0), sThr32);
         b = w32.b;
       } else {
         w64.step(timestamps[s + j], sThr);

@@ -133,6 +133,34 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
   const int key_end = p.cand ? n_kv : min(n_kv, r0 + 32);
   const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
   const float* rt = p.rab_time + static_cast<int64_t>(h) * p.Tb;
+  // The softmax ablation takes two passes: the first finds the row's max m
+  // and sum l of exp(x - m) over its visible keys (the candidate's own key
+  // included), the second accumulates exp(x - m) / l times V.
+  const bool softmax = p.phi2 == HSTU_ACT_SOFTMAX;
+  float sm_m = -INFINITY, sm_l = 0.0f, x_self = 0.0f;
+  if (softmax && p.cand && i < n_q) {
+    const int64_t row = q0g + i;
+    float s = 0.0f;
+    for (int c = 0; c < 64; ++c)
+      s = fmaf(p.q_self[row * p.ld_self + h * 64 + c], p.k_self[row * p.ld_self + h * 64 + c], s);
+    x_self = s + rp[0] + rt[0];
+    if (qt == 0) {
+      sm_m = x_self;
+      sm_l = 1.0f;
+    }
+  }
+  for (int pass = softmax ? 0 : 1; pass < 2; ++pass) {
+  if (pass == 1 && softmax) {
+    // merge the four threads of the row
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, sm_m, o);
+      const float ol = __shfl_xor_sync(0xffffffffu, sm_l, o);
+      const float m = fmaxf(sm_m, om);
+      sm_l = (m == -INFINITY) ? 0.0f : sm_l * expf(sm_m - m) + ol * expf(om - m);
+      sm_m = m;
+    }
+  }
   for (int j0 = 0; j0 < key_end; j0 += 32) {
     __syncthreads();
     for (int e = threadIdx.x; e < 32 * 64; e += 128) {
@@ -153,29 +181,49 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
         for (int c = 0; c < 64; ++c) s = fmaf(sq[r][c], sk[jj][c], s);
         const int bp = min(pos_row - j, p.P - 1);
         const int bt = time_bucket_search(t_row - p.timestamps[kv0 + j], sthr, p.Tb);
-        pval = phi_runtime(s + rp[bp] + rt[bt], p.phi2);
+        const float x = s + rp[bp] + rt[bt];
+        if (!softmax) {
+          pval = phi_runtime(x, p.phi2);
+        } else if (pass == 0) {
+          if (x > sm_m) {
+            sm_l = sm_l * expf(sm_m - x) + 1.0f;
+            sm_m = x;
+          } else {
+            sm_l += expf(x - sm_m);
+          }
+        } else {
+          pval = expf(x - sm_m) / sm_l;
+        }
       }
       sp[r][jj] = pval;
     }
     __syncthreads();
-    for (int jj = 0; jj < 32; ++jj) {
-      const float pv = sp[r][jj];
+    if (pass == 1) {
+      for (int jj = 0; jj < 32; ++jj) {
+        const float pv = sp[r][jj];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) o[c] = fmaf(pv, sv[jj][qt * 16 + c], o[c]);
+        for (int c = 0; c < 16; ++c) o[c] = fmaf(pv, sv[jj][qt * 16 + c], o[c]);
+      }
     }
+  }
   }
   if (i >= n_q) return;
   const int64_t row = q0g + i;
   if (p.cand) {
-    float s = 0.0f;
-    for (int c = 0; c < 64; ++c)
-      s = fmaf(p.q_self[row * p.ld_self + h * 64 + c], p.k_self[row * p.ld_self + h * 64 + c], s);
-    const float ps = phi_runtime(s + rp[0] + rt[0], p.phi2);
+    float ps;
+    if (softmax) {
+      ps = expf(x_self - sm_m) / sm_l;
+    } else {
+      float s = 0.0f;
+      for (int c = 0; c < 64; ++c)
+        s = fmaf(p.q_self[row * p.ld_self + h * 64 + c], p.k_self[row * p.ld_self + h * 64 + c], s);
+      ps = phi_runtime(s + rp[0] + rt[0], p.phi2);
+    }
 #pragma unroll
     for (int c = 0; c < 16; ++c)
       o[c] = fmaf(ps, p.v_self[row * p.ld_self + h * 64 + qt * 16 + c], o[c]);
   }
-  const float inv_n = 1.0f / static_cast<float>(p.cand ? max(n_kv, 1) : n_kv);
+  const float inv_n = softmax ? 1.0f : 1.0f / static_cast<float>(p.cand ? max(n_kv, 1) : n_kv);
 #pragma unroll
   for (int c = 0; c < 16; ++c) p.av[row * p.ld_av + h * 64 + qt * 16 + c] = o[c] * inv_n;
 }

@@ -80,6 +80,7 @@ struct F1Params {
   int64_t ld_dst[4];      // row stride of each destination (elements)
   uint32_t f32_mask;      // bit b set: block b is stored as fp32
   uint32_t f16_mask;      // bit b set: block b is stored as fp16 (else bf16)
+  int32_t ab_f16;         // X and W1 are fp16 (else bf16)
   const float* bias;      // [N]
   int64_t M;
   int32_t N, K;
@@ -137,7 +138,9 @@ struct F2Params {
   const __nv_bfloat16* x_lp;
   int64_t ld_x;
   float* y;                 // [M, ld_y] fp32
-  __nv_bfloat16* y_lp;      // [M, ld_y] or nullptr
+  void* y_lp;               // [M, ld_y] bf16 (fp16 when ylp_f16), or nullptr
+  int32_t ylp_f16;
+  int32_t ab_f16;           // the A tile (Norm(AV) (.) U) and W2 are fp16 (else bf16)
   int64_t ld_y;
   int64_t M;
   int32_t N, K, H;
@@ -157,8 +160,8 @@ struct TileIter {
 // MMA and commit.
 __device__ __forceinline__ void gemm_mma_loop(uint64_t* bars, const uint8_t* sA, const uint8_t* sB,
                                               uint32_t tmem, int total_tiles, int k_blocks,
-                                              const WaitCtl& ctl, uint64_t drain_ns) {
-  constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_BN, false, false);
+                                              const WaitCtl& ctl, uint64_t drain_ns, bool f16) {
+  const uint32_t idesc = idesc_16_f32(G_BM, G_BN, false, false, f16);
   const bool leader = elect_one();
   auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
@@ -266,7 +269,7 @@ hstu_f1_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     }
     __syncwarp();
   } else if (warp == 1) {
-    gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns);
+    gemm_mma_loop(bars, sA, sB, tmem, total, k_blocks, ctl, p.timeout_ns, p.ab_f16 != 0);
     __syncwarp();
   } else {
     // epilogue warps 2..5: TMEM lane quarter = warp % 4.  Each warp turns its
@@ -431,7 +434,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   } else if (warp == 1) {
     // MMA warp: whole-warp loop, one elected lane issues.  Per k-block both
     // 256-column halves (tensor-memory columns 0-255 and 256-511).
-    constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_BN, false, false);
+    const uint32_t idesc = idesc_16_f32(G_BM, G_BN, false, false, p.ab_f16 != 0);
     constexpr uint64_t kHalfDesc = G_B_BYTES >> 4;  // start-address step of the second W2 half
     const bool leader = elect_one();
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
@@ -564,7 +567,7 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const float g0 = fmaf((af[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]) * uf[2 * e];
             const float g1 =
                 fmaf((af[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
-            w4[e] = pack_bf16x2(g0, g1);
+            w4[e] = p.ab_f16 ? pack_h2(g0, g1) : pack_bf16x2(g0, g1);
           }
           // rows past the end carry zeros (their stats are zero and the data too)
           *reinterpret_cast<uint4*>(a_tile + r * 128 + ((c16 ^ (r & 7)) << 4)) =
@@ -649,6 +652,8 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           *reinterpret_cast<float4*>(ry + ((j ^ sw) << 4)) =
               make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
         const bool lp = p.y_lp != nullptr;
+        const bool lp16 = p.ylp_f16 != 0;
+        auto pk2 = [lp16](float a, float b) { return lp16 ? pack_h2(a, b) : pack_bf16x2(a, b); };
         if (lp) {
           // this chunk is one half of a 64-column bf16 segment
           uint8_t* rl = buf_l + lane * 128;
@@ -656,9 +661,8 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             *reinterpret_cast<uint4*>(rl + (((j0 + j) ^ sw) << 4)) =
-                make_uint4(pack_bf16x2(y[8 * j], y[8 * j + 1]), pack_bf16x2(y[8 * j + 2], y[8 * j + 3]),
-                           pack_bf16x2(y[8 * j + 4], y[8 * j + 5]),
-                           pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+                make_uint4(pk2(y[8 * j], y[8 * j + 1]), pk2(y[8 * j + 2], y[8 * j + 3]),
+                           pk2(y[8 * j + 4], y[8 * j + 5]), pk2(y[8 * j + 6], y[8 * j + 7]));
         }
         fence_proxy_async_smem();  // this lane's writes, before the tensor stores read them
         __syncwarp();
@@ -682,6 +686,37 @@ hstu_f2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ weight conversion
+
+// dst[i] = fp16(src[i]) for bf16 src: exact for every bf16 value inside the
+// fp16 normal range (both carry 8 bits of significand or more); values below
+// 2^-14 keep fp16's subnormal spacing of 2^-24.  n is a multiple of 8 and
+// both pointers are 16-byte aligned.
+__global__ void hstu_bf16_to_f16_kernel(const uint4* src, uint4* dst, int64_t n8) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      o[e] = pack_h2(f.x, f.y);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// dst[i] = fp16(src[i]) for fp32 src (round to nearest, saturating at
+// +-65504); n is a multiple of 8, both pointers 16-byte aligned.
+__global__ void hstu_f32_to_f16_kernel(const float4* src, uint4* dst, int64_t n8) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const float4 a = src[2 * i], b = src[2 * i + 1];
+    dst[i] = make_uint4(pack_h2(a.x, a.y), pack_h2(a.z, a.w), pack_h2(b.x, b.y), pack_h2(b.z, b.w));
   }
 }
 

@@ -100,11 +100,11 @@ const int64_t* thresholds_for(int Tb) {
 // ------------------------------------------------------------------ profiler
 
 enum KernelKind : int {
-  K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_COUNT
+  K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
-                                           "fp32_attention",    "fp32_ln_gate"};
+                                           "fp32_attention",    "fp32_ln_gate", "weight_cvt"};
 
 struct Profiler {
   std::mutex mu;
@@ -164,6 +164,7 @@ AttnKernelFn attn_kernel_for(int phi) {
   switch (phi) {
     case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS, F16>;
     case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS, F16>;
+    case HSTU_ACT_SOFTMAX: return hstu_attn_kernel<CAND, HSTU_ACT_SOFTMAX, PAIRS, F16>;
     default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS, F16>;
   }
 }
@@ -198,7 +199,7 @@ hstu_status_t device_info(DeviceInfo** out) {
   if (!d.smem_set) {
     const int att_max = 227 * 1024;
     for (int cand = 0; cand < 2; ++cand)
-      for (int phi = 0; phi < 3; ++phi)
+      for (int phi = 0; phi < 4; ++phi)
         for (int pairs = 0; pairs < 2; ++pairs)
           for (int f16 = 0; f16 < 2; ++f16)
             HSTU_CHECK_CUDA(cudaFuncSetAttribute(
@@ -291,7 +292,7 @@ hstu_status_t check_cfg(const hstu_layer_cfg_t* c) {
       c->num_pos_buckets <= 0 || c->num_time_buckets <= 0)
     return HSTU_ERR_INVALID_ARGUMENT;
   if (c->phi1 < HSTU_ACT_IDENTITY || c->phi1 > HSTU_ACT_SILU || c->phi2 < HSTU_ACT_IDENTITY ||
-      c->phi2 > HSTU_ACT_SILU)
+      c->phi2 > HSTU_ACT_SOFTMAX)
     return HSTU_ERR_INVALID_ARGUMENT;
   if (c->dtype != HSTU_BF16 && c->dtype != HSTU_FP32 && c->dtype != HSTU_FP16)
     return HSTU_ERR_INVALID_ARGUMENT;
@@ -334,19 +335,31 @@ int n1_of(const hstu_layer_cfg_t* c) { return 2 * c->num_heads * (c->dqk + c->dv
 //              [T, H, 2] fp32.  AV and U stay fp32 because LayerNorm removes the
 //              large common mean of AV and would magnify bf16 rounding there.
 //   fp32 path: Z [T, n1] fp32, AV [T, H*dv] fp32, G [T, H*dv] fp32.
+//   bf16 path, also: fp16 copies of W1 [n1, d] and W2 [d, H*dv] (the GEMM
+//              operands paired with fp16 activations).
 struct LayerWs {
   void* z;      // bf16: VQK; fp32: Z
   float* u;     // bf16 path: U fp32
   void* av;
   void* extra;  // bf16: LN partials; fp32: G
+  __half* w1h;  // bf16 path: fp16 W1
+  __half* w2h;  // bf16 path: fp16 W2
+  __half* x16;  // bf16 path: fp16 copy of the fp32 layer input (x_in = NULL)
 };
+
+size_t weights_f16_bytes(const hstu_layer_cfg_t* c) {
+  const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
+  const size_t d = static_cast<size_t>(c->d_model);
+  return align_up(static_cast<size_t>(n1_of(c)) * d * 2, 256) + align_up(d * hv * 2, 256);
+}
 
 size_t layer_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
   const size_t t = static_cast<size_t>(T);
   const size_t hv = static_cast<size_t>(c->num_heads) * c->dv;
   if (c->dtype == HSTU_BF16)
     return align_up(t * 3 * hv * 2, 256) + 2 * align_up(t * hv * 4, 256) +
-           align_up(t * c->num_heads * 2 * sizeof(float), 256);
+           align_up(t * c->num_heads * 2 * sizeof(float), 256) + weights_f16_bytes(c) +
+           align_up(t * static_cast<size_t>(c->d_model) * 2, 256);
   return align_up(t * n1_of(c) * 4, 256) + 2 * align_up(t * hv * 4, 256);
 }
 
@@ -367,7 +380,37 @@ LayerWs carve_layer(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
   w.av = p;
   p += align_up(t * hv * 4, 256);
   w.extra = p;
+  w.w1h = w.w2h = w.x16 = nullptr;
+  if (c->dtype == HSTU_BF16) {
+    p += align_up(t * c->num_heads * 2 * sizeof(float), 256);
+    w.w1h = reinterpret_cast<__half*>(p);
+    p += align_up(static_cast<size_t>(n1_of(c)) * c->d_model * 2, 256);
+    w.w2h = reinterpret_cast<__half*>(p);
+    p += align_up(static_cast<size_t>(c->d_model) * hv * 2, 256);
+    w.x16 = reinterpret_cast<__half*>(p);
+  }
   return w;
+}
+
+hstu_status_t convert_f32_to_f16(const float* src, __half* dst, int64_t n, cudaStream_t st) {
+  const int64_t n8 = n / 8;  // n = T * d_model, d_model a multiple of 64
+  const int blocks = static_cast<int>(std::min<int64_t>((n8 + 255) / 256, 4096));
+  ProfScope prof(K_CVT, st);
+  hstu_f32_to_f16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
+                                                  reinterpret_cast<uint4*>(dst), n8);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t convert_bf16_to_f16(const void* src, __half* dst, int64_t n, cudaStream_t st) {
+  // n is a multiple of 64 for every weight matrix here (d and H*64 are)
+  const int64_t n8 = n / 8;
+  const int blocks = static_cast<int>(std::min<int64_t>((n8 + 255) / 256, 1024));
+  ProfScope prof(K_CVT, st);
+  hstu_bf16_to_f16_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                   reinterpret_cast<uint4*>(dst), n8);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
 }
 
 // residual-stream buffers of a multi-layer pass: 2 x fp32 [T, d] + 2 x low-precision [T, d]
@@ -471,15 +514,15 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
 hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t ldx, int64_t M,
                              const void* w1, const float* b1, void* const dst[4],
                              const int64_t ld_dst[4], uint32_t f32_mask, uint32_t f16_mask,
-                             cudaStream_t st) {
+                             bool ab_f16, cudaStream_t st) {
   if (M == 0) return HSTU_OK;
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
   const int N = n1_of(c), K = c->d_model;
   CUtensorMap mx, mw;
-  if ((s = make_map_16(&mx, x, M, K, ldx, G_BK, G_BM)) != HSTU_OK) return s;
-  if ((s = make_map_16(&mw, w1, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mx, x, M, K, ldx, G_BK, G_BM, ab_f16)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mw, w1, N, K, K, G_BK, G_BN, ab_f16)) != HSTU_OK) return s;
   F1Params p;
   std::memset(&p, 0, sizeof(p));
   F1OutMaps om;
@@ -494,6 +537,7 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   }
   p.f32_mask = f32_mask;
   p.f16_mask = f16_mask;
+  p.ab_f16 = ab_f16 ? 1 : 0;
   p.bias = b1;
   p.M = M;
   p.N = N;
@@ -520,22 +564,26 @@ hstu_status_t launch_f1_bf16(const hstu_layer_cfg_t* c, const void* x, int64_t l
   return HSTU_OK;
 }
 
+// w2 is bf16 as given, or its fp16 copy (ab_f16: the A tile is then built in
+// fp16 too); y_lp is written in fp16 when ylp_f16.
 hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
-                             const float* av, int64_t ld_av, const float* u, int64_t ld_u,
-                             const float* ln_part, const float* x_res, const void* x_lp,
-                             int64_t ld_x, float* y, void* y_lp, int64_t ld_y, int64_t M,
-                             cudaStream_t st) {
+                             const void* w2, bool ab_f16, const float* av, int64_t ld_av,
+                             const float* u, int64_t ld_u, const float* ln_part,
+                             const float* x_res, const void* x_lp, int64_t ld_x, float* y,
+                             void* y_lp, bool ylp_f16, int64_t ld_y, int64_t M, cudaStream_t st) {
   if (M == 0) return HSTU_OK;
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
   const int N = c->d_model, K = c->num_heads * c->dv;
   CUtensorMap mw;
-  if ((s = make_map_16(&mw, w->w2, N, K, K, G_BK, G_BN)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mw, w2, N, K, K, G_BK, G_BN, ab_f16)) != HSTU_OK) return s;
   F2OutMaps om;
   std::memset(&om, 0, sizeof(om));
   if ((s = make_out_map(&om.y, y, true, M, N, ld_y)) != HSTU_OK) return s;
-  if (y_lp != nullptr && (s = make_out_map(&om.y_lp, y_lp, false, M, N, ld_y)) != HSTU_OK) return s;
+  if (y_lp != nullptr &&
+      (s = make_out_map(&om.y_lp, y_lp, false, M, N, ld_y, ylp_f16)) != HSTU_OK)
+    return s;
   F2Params p;
   std::memset(&p, 0, sizeof(p));
   p.av = av;
@@ -551,7 +599,9 @@ hstu_status_t launch_f2_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights
   p.x_lp = static_cast<const __nv_bfloat16*>(x_lp);
   p.ld_x = ld_x;
   p.y = y;
-  p.y_lp = static_cast<__nv_bfloat16*>(y_lp);
+  p.y_lp = y_lp;
+  p.ylp_f16 = ylp_f16 ? 1 : 0;
+  p.ab_f16 = ab_f16 ? 1 : 0;
   p.ld_y = ld_y;
   p.M = M;
   p.N = N;
@@ -682,11 +732,26 @@ hstu_status_t layer_fp32(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
 }
 
 // One layer on the bf16 tensor-core path.
+//   x_f16   x_in is fp16 (a residual-stream copy handed over by the previous
+//           layer of a stack; then x_res must be given): f1 runs on fp16 X and
+//           an fp16 copy of W1.  Otherwise x_in is the caller's bf16 and f1 runs
+//           on bf16 X and W1 as given.
+//   ylp_f16 the rounded copy of Y (y_lp) is fp16, else bf16.
+// f2 always runs on fp16: its A tile Norm(AV) (.) U is built in fp16 and W2 is
+// converted.  fp16 has the same tensor-core rate as bf16 and 8x finer
+// rounding; bf16 weights convert to fp16 exactly inside fp16's normal range.
 hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
-                         const AttnJob& base, const void* x_in, const float* x_res, int64_t T,
-                         float* y_out, void* y_lp, void* kv_cache, const LayerWs& ws, bool cand,
-                         cudaStream_t st) {
+                         const AttnJob& base, const void* x_in, bool x_f16, const float* x_res,
+                         int64_t T, float* y_out, void* y_lp, bool ylp_f16, void* kv_cache,
+                         const LayerWs& ws, bool cand, cudaStream_t st) {
   const int hv = c->num_heads * ATT_HD, d = c->d_model;
+  if (x_f16 && x_res == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  hstu_status_t s;
+  if (x_f16 && (s = convert_bf16_to_f16(w->w1, ws.w1h, static_cast<int64_t>(n1_of(c)) * d, st)) !=
+                   HSTU_OK)
+    return s;
+  if ((s = convert_bf16_to_f16(w->w2, ws.w2h, static_cast<int64_t>(d) * hv, st)) != HSTU_OK)
+    return s;
   __half* vqk = static_cast<__half*>(ws.z);
   // f1 column blocks U, V, Q, K -> U (fp32), V, Q, K (fp16; K/V into the cache
   // if given).  The attention operands are fp16: the same tensor-core rate as
@@ -699,7 +764,8 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
     dst[3] = kv;       // K
     ldd[1] = ldd[3] = 2 * hv;
   }
-  hstu_status_t s = launch_f1_bf16(c, x_in, d, T, w->w1, w->b1, dst, ldd, 1u, 0xEu, st);
+  s = launch_f1_bf16(c, x_in, d, T, x_f16 ? static_cast<const void*>(ws.w1h) : w->w1, w->b1, dst,
+                     ldd, 1u, 0xEu, x_f16, st);
   if (s != HSTU_OK) return s;
   AttnJob j = base;
   j.q = dst[2];
@@ -719,9 +785,9 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
   j.f16 = true;
   s = cand ? launch_attn_tc<true>(j, st) : launch_attn_tc<false>(j, st);
   if (s != HSTU_OK) return s;
-  return launch_f2_bf16(c, w, static_cast<const float*>(ws.av), hv, ws.u, hv,
-                        static_cast<const float*>(ws.extra), x_res, x_in, d, y_out, y_lp, d, T,
-                        st);
+  return launch_f2_bf16(c, w, ws.w2h, true, static_cast<const float*>(ws.av), hv, ws.u, hv,
+                        static_cast<const float*>(ws.extra), x_res, x_in, d, y_out, y_lp,
+                        ylp_f16, d, T, st);
 }
 
 hstu_status_t check_weights(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w) {
@@ -938,7 +1004,9 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
   if ((s = check_weights(cfg, w)) != HSTU_OK) return s;
   const int64_t T = jag->total_tokens;
   if (T == 0 || jag->batch == 0) return HSTU_OK;
-  if (x_in == nullptr || y_out == nullptr) return HSTU_ERR_INVALID_ARGUMENT;
+  // x_in may be NULL when the fp32 residual x_res is given (bf16 layers)
+  if ((x_in == nullptr && (x_res == nullptr || cfg->dtype != HSTU_BF16)) || y_out == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(x_res) || !aligned16(y_out) || !aligned16(y_out_lp) ||
       !aligned16(kv_cache_out) || !aligned16(workspace))
     return HSTU_ERR_INVALID_ARGUMENT;
@@ -962,7 +1030,14 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
                                       cudaMemcpyDeviceToDevice, st));
     return s;
   }
-  return layer_bf16(cfg, w, base, x_in, x_res, T, y_out, y_out_lp, kv_cache_out, ws, false, st);
+  if (x_in == nullptr) {
+    // f1 reads the fp32 residual input rounded to fp16 (as between the layers of a stack)
+    if ((s = convert_f32_to_f16(x_res, ws.x16, T * cfg->d_model, st)) != HSTU_OK) return s;
+    return layer_bf16(cfg, w, base, ws.x16, true, x_res, T, y_out, y_out_lp, false, kv_cache_out,
+                      ws, false, st);
+  }
+  return layer_bf16(cfg, w, base, x_in, false, x_res, T, y_out, y_out_lp, false, kv_cache_out, ws,
+                    false, st);
 }
 
 hstu_status_t hstu_layer_fwd_static(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
@@ -1005,16 +1080,33 @@ hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
   float* yf[2] = {reinterpret_cast<float*>(sp), reinterpret_cast<float*>(sp + fbytes)};
   void* yl[2] = {sp + 2 * fbytes, sp + 2 * fbytes + lbytes};
   const size_t cache_layer = static_cast<size_t>(T) * 2 * cfg->num_heads * ATT_HD * elt(cfg);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnJob base;
+  std::memset(&base, 0, sizeof(base));
+  base.cfg = cfg;
+  base.kv_offsets = jag->offsets;
+  base.timestamps = jag->timestamps;
+  base.batch = jag->batch;
+  base.max_q_len = base.max_kv_len = jag->max_len;
+  base.T_q = base.T_kv = T;
+  base.timeout_ns = kDefaultTimeoutNs;
+  const LayerWs ws = carve_layer(cfg, T, workspace);
   for (int l = 0; l < num_layers; ++l) {
     const bool last = (l == num_layers - 1);
-    const void* xin = (l == 0) ? x_in : (cfg->dtype == HSTU_BF16 ? yl[(l - 1) & 1]
-                                                                  : static_cast<void*>(yf[(l - 1) & 1]));
     const float* xres = (l == 0) ? nullptr : yf[(l - 1) & 1];
     float* yo = last ? y_out : yf[l & 1];
-    void* ylp = (last || cfg->dtype == HSTU_FP32) ? nullptr : yl[l & 1];
     void* kv = kv_cache_out == nullptr ? nullptr
                                        : static_cast<uint8_t*>(kv_cache_out) + cache_layer * l;
-    s = hstu_layer_fwd(cfg, &weights[l], jag, xin, xres, yo, ylp, kv, workspace, lw, stream);
+    if (cfg->dtype == HSTU_BF16) {
+      // between layers the residual stream's rounded copy is fp16
+      const void* xin = (l == 0) ? x_in : yl[(l - 1) & 1];
+      s = layer_bf16(cfg, &weights[l], base, xin, l > 0, xres, T, yo, last ? nullptr : yl[l & 1],
+                     true, kv, ws, false, st);
+    } else {
+      const float* xin = (l == 0) ? static_cast<const float*>(x_in) : yf[(l - 1) & 1];
+      s = layer_fp32(cfg, &weights[l], base, xin, xres, T, yo, static_cast<float*>(kv), ws, false,
+                     st);
+    }
     if (s != HSTU_OK) return s;
   }
   return HSTU_OK;
@@ -1088,7 +1180,8 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
       s = layer_fp32(cfg, &weights[l], j, xin, xres, M, yo, nullptr, ws, true, st);
     } else {
       const void* xin = (l == 0) ? cand_emb : yl[(l - 1) & 1];
-      s = layer_bf16(cfg, &weights[l], j, xin, xres, M, yo, yl[l & 1], nullptr, ws, true, st);
+      s = layer_bf16(cfg, &weights[l], j, xin, l > 0, xres, M, yo, yl[l & 1], true, nullptr, ws,
+                     true, st);
     }
     if (s != HSTU_OK) return s;
   }

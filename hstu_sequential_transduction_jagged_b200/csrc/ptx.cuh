@@ -341,6 +341,18 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
+// 2^x and log2(x) on the MUFU (approximate, flush-to-zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Packed fp32 pair arithmetic (two lanes of a 64-bit register).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhstu.so")
 
-ACT = {"identity": 0, "relu": 1, "silu": 2}
+ACT = {"identity": 0, "relu": 1, "silu": 2, "softmax": 3}
 DTYPE = {"bf16": 0, "fp32": 1, "fp16": 2}
 TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32, "fp16": torch.float16}
 # dtype of the per-layer key/value cache of a layer configured with `dtype`
@@ -256,8 +256,10 @@ def mfalcon_attn_fwd(cfg: LayerConfig, history: Jagged, k_hist, v_hist, cand_off
 
 def layer_fwd(cfg: LayerConfig, w: LayerWeights, jag: Jagged, x_in, x_res=None, y_out=None,
               y_out_lp=None, kv_cache_out=None, workspace=None, stream=None) -> torch.Tensor:
-    """One HSTU layer; returns the fp32 residual-stream output Y [T, d]."""
-    dev = x_in.device
+    """One HSTU layer; returns the fp32 residual-stream output Y [T, d].  For bf16
+    layers x_in may be None when x_res (fp32) is given: f1 then reads x_res
+    rounded to fp16."""
+    dev = (x_in if x_in is not None else x_res).device
     if y_out is None:
         y_out = torch.empty((jag.total_tokens, cfg.d_model), dtype=torch.float32, device=dev)
     nbytes = layer_workspace_bytes(cfg, jag.total_tokens)
@@ -278,7 +280,7 @@ def layer_fwd_static(cfg: LayerConfig, w: LayerWeights, jag: Jagged, x_in, x_res
     (STATIC_SCRATCH_BYTES per GPU) is used, so the C call itself allocates nothing."""
     if y_out is None:
         y_out = torch.empty((jag.total_tokens, cfg.d_model), dtype=torch.float32,
-                            device=x_in.device)
+                            device=(x_in if x_in is not None else x_res).device)
     c, j, wc = cfg.c(), jag.c(), w.c()
     _check(lib().hstu_layer_fwd_static(ctypes.byref(c), ctypes.byref(wc), ctypes.byref(j),
                                        _p(x_in), _p(x_res), _p(y_out), _p(y_out_lp),

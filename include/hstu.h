@@ -23,7 +23,13 @@
  *     variance, eps from the config, optional affine;
  *   - Y = X + f2(...): the residual stream is fp32.
  *   - bf16 layers compute attention on fp16 Q, K, V and P (f1 writes them in
- *     fp16; values saturate at +-65504), with fp32 accumulation.
+ *     fp16; values saturate at +-65504), with fp32 accumulation, and f2 on
+ *     fp16 operands (Norm(AV) (.) U, and an fp16 copy of W2 made in the
+ *     workspace each call).  Inside hstu_forward and mfalcon_score the layers
+ *     after the first take an fp16 copy of the fp32 residual stream, with an
+ *     fp16 copy of W1.  fp16 runs at the bf16 tensor-core rate with 8x finer
+ *     rounding; bf16 weights convert to fp16 exactly inside fp16's normal
+ *     range.
  *
  * Conventions for every entry point:
  *   - Pointers marked "device" must point to memory of the current CUDA
@@ -71,7 +77,17 @@ typedef enum {
  * for their attention internally. */
 typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1, HSTU_FP16 = 2 } hstu_dtype_t;
 
-typedef enum { HSTU_ACT_IDENTITY = 0, HSTU_ACT_RELU = 1, HSTU_ACT_SILU = 2 } hstu_act_t;
+/* Pointwise nonlinearities.  HSTU_ACT_SOFTMAX is accepted for phi2 only: the
+ * "HSTU (-rab, Softmax)" ablation of the review's section 六 (HSTU component
+ * ablation table), a row-wise softmax over the visible keys of the same
+ * pre-activation Q K^T + rab, replacing phi2 and its 1/N (pass zero bias
+ * tables for "-rab"). */
+typedef enum {
+  HSTU_ACT_IDENTITY = 0,
+  HSTU_ACT_RELU = 1,
+  HSTU_ACT_SILU = 2,
+  HSTU_ACT_SOFTMAX = 3
+} hstu_act_t;
 
 /* A jagged batch of per-user, time-ordered action sequences (the "unified
  * time series" x_0..x_{n-1} of each user, section 二/三 of the review). */
@@ -93,7 +109,7 @@ typedef struct {
   int32_t num_pos_buckets;    /* P */
   int32_t num_time_buckets;   /* Tb */
   int32_t phi1;               /* hstu_act_t, ReLU per Eq. 1 */
-  int32_t phi2;               /* hstu_act_t, SiLU by default */
+  int32_t phi2;               /* hstu_act_t, SiLU by default (or SOFTMAX) */
   float ln_eps;               /* LayerNorm epsilon (1e-5) */
   int32_t dtype;              /* hstu_dtype_t of X, W1, W2 and all bf16 intermediates */
 } hstu_layer_cfg_t;
@@ -178,7 +194,10 @@ hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t*
 
 /*
  * One HSTU layer (Eq. 1-3 and the residual) over a jagged batch.
- *   x_in        device [T, d] in cfg dtype: the layer input fed to f1.
+ *   x_in        device [T, d] in cfg dtype: the layer input fed to f1.  For
+ *               bf16 layers it may be NULL when x_res is given: f1 then reads
+ *               x_res rounded to fp16 (with an fp16 copy of W1), the way the
+ *               layers after the first of hstu_forward run.
  *   x_res       device [T, d] fp32 residual input, or NULL to use x_in.
  *   y_out       device [T, d] fp32: X + f2(Norm(AV) (.) U).
  *   y_out_lp    device [T, d] in cfg dtype (a rounded copy of y_out for the

@@ -57,8 +57,8 @@ def _per_layer_prefix_check(H, case, users, prefix, what):
     """Each layer at the stated tolerance (max abs 2e-2, rel-L2 5e-3) on the
     full batch, in the launch configuration of the forward: layer l runs over
     every user with the oracle's layer l-1 output in the checked prefix rows
-    (fp32 residual, bf16 copy for f1) and the GPU's own layer l-1 output
-    elsewhere.  Rows before m of a user depend on its first m inputs only
+    and the GPU's own layer l-1 output elsewhere, as the fp32 residual input
+    that f1 reads rounded to fp16 (x_in = None, as inside a stack).  Rows before m of a user depend on its first m inputs only
     (the mask is causal and N = n_u is fixed), so the prefix rows of layer l
     are compared with the oracle's layer l on the same inputs."""
     t, jag, weights = upload(H, case)
@@ -74,7 +74,7 @@ def _per_layer_prefix_check(H, case, users, prefix, what):
         if l > 0:
             x_res = y_gpu.clone()
             x_res[rows_t] = tensor(cur_o[rows].astype(np.float32), torch.float32, "cuda")
-            x_lp = x_res.to(cfg.torch_dtype)
+            x_lp = None
         y_gpu = H.layer_fwd(cfg, weights[l], jag, x_lp, x_res=x_res)
         assert H.device_status() == 0
         got = y_gpu[rows_t].cpu().numpy()

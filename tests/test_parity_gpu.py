@@ -64,7 +64,7 @@ ATTN_LENGTHS = [1, 127, 128, 129, 255, 256, 257, 700, 0, 64]
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
-@pytest.mark.parametrize("phi2", ["silu", "relu", "identity"])
+@pytest.mark.parametrize("phi2", ["silu", "relu", "identity", "softmax"])
 def test_attention_parity(H, phi2, dtype):
     """Attention alone for both operand types: fp16 is what the bf16 layers run
     (f1 writes fp16 Q, K, V), bf16 serves bf16 inputs given directly."""
@@ -127,8 +127,9 @@ def _forward_check(H, case, what, check_delta=True):
 
 def _per_layer_check(H, case, what):
     """Every layer on its own at the stated tolerance (max-abs 2e-2, rel-L2 5e-3):
-    layer l gets the oracle's layer l-1 output as input (fp32 residual, bf16 copy
-    for f1), the way the GPU's own previous layer hands it over."""
+    layer l gets the oracle's layer l-1 output as its fp32 residual input, and
+    f1 reads it rounded to fp16 (x_in = None), the way the GPU's own previous
+    layer hands it over inside a stack."""
     t, jag, weights = upload(H, case)
     cfg = config_of(H, case.cfg)
     cur = case.x.astype(np.float64)
@@ -137,8 +138,8 @@ def _per_layer_check(H, case, what):
         if l == 0:
             x_in, x_res = t["x"], None
         else:
-            x_in = tensor(to_dtype(cur, case.cfg.dtype), cfg.torch_dtype, "cuda")
             x_res = tensor(cur.astype(np.float32), torch.float32, "cuda")
+            x_in = None if case.cfg.dtype == "bf16" else x_res
         y = H.layer_fwd(cfg, weights[l], jag, x_in, x_res=x_res).cpu().numpy()
         _status_ok(H)
         assert_close(y, want, f"{what} layer {l}")
@@ -160,11 +161,36 @@ def test_small_bf16_full_workload(H):
     _forward_check(H, case, "small-bf16 full")
 
 
-@pytest.mark.parametrize("phi2", ["relu", "identity"])
+@pytest.mark.parametrize("phi2", ["relu", "identity", "softmax"])
 def test_small_bf16_other_phi2(H, phi2):
     cfg = make_case("small-bf16").cfg.replace(phi2=phi2)
     case = make_case(cfg, seed=22, lengths=[200, 33, 400])
     _forward_check(H, case, f"small-bf16 phi2={phi2}")
+
+
+def test_softmax_ablation_without_rab(H):
+    """The "HSTU (-rab, Softmax)" ablation: softmax phi2 with zero bias tables,
+    whole 2-layer stack and each layer at the stated bound."""
+    cfg = make_case("small-bf16").cfg.replace(phi2="softmax")
+    case = make_case(cfg, seed=28, lengths=[300, 1, 129, 512, 64])
+    for lw in case.layers:
+        lw.rab_pos[:] = 0.0
+        lw.rab_time[:] = 0.0
+    _forward_check(H, case, "softmax -rab")
+    _per_layer_check(H, case, "softmax -rab")
+
+
+def test_softmax_sl_bf16_per_layer(H):
+    """Softmax ablation on the Stochastic Length shapes (d 512, 8 heads, 4 layers)."""
+    cfg = make_case("sl-bf16").cfg.replace(phi2="softmax")
+    case = make_case(cfg, seed=29, lengths=[1, 300, 1100, 2500])
+    _forward_check(H, case, "softmax sl-bf16")
+    _per_layer_check(H, case, "softmax sl-bf16")
+
+
+def test_softmax_tiny_fp32(H):
+    case = make_case(make_case("tiny-fp32").cfg.replace(phi2="softmax"), seed=30)
+    _forward_check(H, case, "softmax tiny-fp32")
 
 
 def test_layernorm_affine(H):
@@ -285,6 +311,23 @@ def test_mfalcon_parity(H):
     record("mfalcon final rows delta y-e", dma, drl, None, 2e-2)
     assert drl <= 2e-2, f"delta rel_l2={drl:.3e}"
     check_scores(sc, want, case.cand_emb, "mfalcon scores")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_mfalcon_softmax(H, dtype):
+    """M-FALCON with the softmax ablation: a candidate's softmax runs over its
+    user's history keys and its own key."""
+    cfg = make_case("mfalcon").cfg.replace(num_cand=70, phi2="softmax")
+    if dtype == "fp32":
+        cfg = cfg.replace(dtype="fp32", d_model=64, num_heads=1)
+    case = make_case(cfg, seed=34, lengths=[300, 0, 129, 700], num_layers=2)
+    sc, y = _mfalcon_run(H, case, 32, rows=True)
+    _status_ok(H)
+    want, want_y = O.mfalcon_scores(case.x, case.offsets, case.timestamps, case.layers, case.cfg,
+                                    case.cand_offsets, case.cand_emb, case.request_ts, 32,
+                                    return_rows=True)
+    assert_close(y, want_y, f"mfalcon softmax {dtype} final rows")
+    check_scores(sc, want, case.cand_emb, f"mfalcon softmax {dtype} scores")
 
 
 def test_mfalcon_per_layer(H):
