@@ -508,6 +508,47 @@ def forward_e2e(ctx, case, t, cfg, weights, ws, y, steps):
                            "ms_per_step": e_serial_ms}}
 
 
+def measure_sl_sampler(ctx, steps, warmup):
+    """Time the GPU Stochastic Length sampler on the sl-bf16 batch before
+    subsampling: 64 users with full timelines of 4096 events, d_model 512 bf16
+    rows gathered.  The gather is HBM-bound: algorithmic bytes are the kept
+    rows read and written plus their index and timestamp (8 bytes each, read
+    and written)."""
+    torch, H = ctx.torch, ctx.H
+    from gen import make_case
+    from gen.device import case_tensors
+    cfg = make_case("sl-bf16").cfg.replace(len_kind="fixed")
+    case = make_case(cfg, seed=3, num_layers=1)
+    t = case_tensors(case, ctx.dev)
+    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
+    seeds = iter(range(10 ** 6))
+
+    def step():
+        H.stochastic_length(jag, cfg.sl_alpha, 7, next(seeds), x=t["x"])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    step_ms, kernels, _ = ctx.timed_steps(step, steps, sample_clocks=False)
+    ms = sum(step_ms) / steps
+    out = H.stochastic_length(jag, cfg.sl_alpha, 7, 0, x=t["x"])
+    T_out = int(out["offsets"][-1].item())
+    row = cfg.d_model * 2
+    n_g, ms_g = kernels.get("sl_gather", (0, 0.0))
+    byt = T_out * (2 * row + 2 * 8 + 2 * 8)
+    gbs = byt / (ms_g / n_g / 1000.0) / 1e9 if n_g else None
+    return {"metric": "events kept/s", "value": T_out / (ms / 1000.0), "unit": "events/s",
+            "workload": "Stochastic Length (alpha 1.6) of 64 users x 4096 events, d_model 512 "
+                        "bf16 rows gathered", "ms_per_step": ms, "events_in": case.total_tokens,
+            "events_kept_example": T_out, "kernels": _kernel_table(kernels),
+            "gpu_launches": sum(n for n, _ in kernels.values()),
+            "roofline": None if gbs is None else {
+                "kernel": "hstu_sl_gather_kernel", "bound": "hbm", "achieved": gbs,
+                "peak": ctx.peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                "traffic": None, "algorithmic_bytes_per_launch": byt,
+                "ms_per_launch": ms_g / n_g}}
+
+
 def measure_mfalcon(ctx, steps, warmup, with_e2e, sample_clocks=True, batch=None):
     """Time mfalcon_score over every candidate of the M-FALCON workload (the
     history is encoded once beforehand, with its K/V kept per layer)."""
@@ -667,6 +708,7 @@ def main():
                 subs[name] = _public(measure_forward(ctx, name, min(args.steps, 20), args.warmup,
                                                      False, sample_clocks=(name == "sl-bf16")))
             subs["mfalcon"] = measure_mfalcon(ctx, min(args.steps, 20), args.warmup, True)
+            subs["sl-sampler"] = measure_sl_sampler(ctx, min(args.steps, 20), args.warmup)
             line["workloads"] = subs
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_extrapolated(case)

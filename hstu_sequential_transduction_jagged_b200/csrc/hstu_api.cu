@@ -17,6 +17,7 @@
 #include "attn.cuh"
 #include "fp32_path.cuh"
 #include "gemm.cuh"
+#include "sl.cuh"
 
 using namespace hstu;
 
@@ -100,11 +101,13 @@ const int64_t* thresholds_for(int Tb) {
 // ------------------------------------------------------------------ profiler
 
 enum KernelKind : int {
-  K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT, K_COUNT
+  K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT,
+  K_SL, K_SL_GATHER, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
-                                           "fp32_attention",    "fp32_ln_gate", "weight_cvt"};
+                                           "fp32_attention",    "fp32_ln_gate", "weight_cvt",
+                                           "sl_select",         "sl_gather"};
 
 struct Profiler {
   std::mutex mu;
@@ -214,6 +217,9 @@ hstu_status_t device_info(DeviceInfo** out) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(F2Smem::kBytes)));
+    HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_sl_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SL_MAX_LEN * static_cast<int>(sizeof(uint64_t))));
     d.smem_set = true;
   }
   *out = &d;
@@ -1195,6 +1201,49 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
     hstu_score_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
         yfin, d, static_cast<const __nv_bfloat16*>(cand_emb), d, M, d, scores);
   HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_stochastic_length(const hstu_jagged_t* full, const void* x_full,
+                                     int32_t row_bytes, float alpha, uint64_t seed, uint64_t step,
+                                     int64_t* offsets_out, int32_t* lengths_out,
+                                     int32_t* max_len_out, int64_t* kept_index_out,
+                                     int64_t* timestamps_out, void* x_out, void* stream) {
+  hstu_status_t s;
+  if ((s = check_jag(full)) != HSTU_OK) return s;
+  if (!(alpha > 0.0f) || !std::isfinite(alpha)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (offsets_out == nullptr || lengths_out == nullptr || kept_index_out == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (timestamps_out != nullptr && full->total_tokens > 0 && full->timestamps == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if ((x_full == nullptr) != (x_out == nullptr)) return HSTU_ERR_INVALID_ARGUMENT;
+  if (x_full != nullptr &&
+      (row_bytes <= 0 || row_bytes % 16 != 0 || !aligned16(x_full) || !aligned16(x_out)))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (full->max_len > SL_MAX_LEN) return HSTU_ERR_UNSUPPORTED;
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != HSTU_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int32_t B = full->batch;
+  {
+    ProfScope prof(K_SL, st);
+    if (B > 0)
+      hstu_sl_lengths_kernel<<<(B + 255) / 256, 256, 0, st>>>(full->offsets, B, 1.0 / alpha, seed,
+                                                             step, lengths_out);
+    hstu_sl_scan_kernel<<<1, SL_SCAN_THREADS, 0, st>>>(lengths_out, B, offsets_out, max_len_out);
+    if (B > 0 && full->max_len > 0)
+      hstu_sl_select_kernel<<<B, SL_SELECT_THREADS, full->max_len * sizeof(uint64_t), st>>>(
+          full->offsets, full->timestamps, lengths_out, offsets_out, full->max_len,
+          full->total_tokens, seed, step, kept_index_out, timestamps_out);
+    HSTU_CHECK_CUDA(cudaGetLastError());
+  }
+  if (x_full != nullptr && B > 0 && full->total_tokens > 0) {
+    ProfScope prof(K_SL_GATHER, st);
+    hstu_sl_gather_kernel<<<di->sm_count * 8, 256, 0, st>>>(
+        offsets_out, B, full->total_tokens, kept_index_out, static_cast<const uint4*>(x_full),
+        static_cast<uint4*>(x_out), row_bytes / 16);
+    HSTU_CHECK_CUDA(cudaGetLastError());
+  }
   return HSTU_OK;
 }
 

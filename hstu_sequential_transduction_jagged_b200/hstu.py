@@ -78,6 +78,9 @@ EXPORTS = {
                                      ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                      ctypes.c_void_p]),
+    "hstu_stochastic_length": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                              ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64]
+                               + [ctypes.c_void_p] * 7),
     "hstu_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "hstu_profiler_start": (ctypes.c_int, []),
     "hstu_profiler_stop": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]),
@@ -324,6 +327,31 @@ def mfalcon_score(cfg: LayerConfig, weights: Sequence[LayerWeights], history: Ja
                                _stream(stream)),
            "mfalcon_score")
     return scores
+
+
+def stochastic_length(jag: Jagged, alpha: float, seed: int, step: int, x=None, stream=None):
+    """Stochastic Length subsampling on the GPU.  Returns a dict with the output
+    offsets [B+1], lengths [B], max_len [1], kept_index [T_full] (first T_out
+    valid), timestamps [T_full] and, when x is given, the gathered rows
+    [T_full, ...] (first T_out valid).  T_out = offsets[B] stays on the device."""
+    dev = jag.offsets.device
+    B, T = jag.batch, jag.total_tokens
+    out = {"offsets": torch.empty(B + 1, dtype=torch.int64, device=dev),
+           "lengths": torch.empty(max(B, 1), dtype=torch.int32, device=dev),
+           "max_len": torch.zeros(1, dtype=torch.int32, device=dev),
+           "kept_index": torch.empty(max(T, 1), dtype=torch.int64, device=dev),
+           "timestamps": torch.empty(max(T, 1), dtype=torch.int64, device=dev)}
+    row_bytes = 0
+    if x is not None:
+        out["x"] = torch.empty((max(T, 1),) + tuple(x.shape[1:]), dtype=x.dtype, device=dev)
+        row_bytes = x[0].numel() * x.element_size() if T else 16
+    j = jag.c()
+    _check(lib().hstu_stochastic_length(ctypes.byref(j), _p(x), row_bytes, alpha, seed, step,
+                                        _p(out["offsets"]), _p(out["lengths"]),
+                                        _p(out["max_len"]), _p(out["kept_index"]),
+                                        _p(out["timestamps"]), _p(out.get("x")),
+                                        _stream(stream)), "hstu_stochastic_length")
+    return out
 
 
 def device_status(stream=None) -> int:

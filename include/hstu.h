@@ -258,6 +258,37 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
                             int32_t microbatch, float* scores, float* cand_y_out, void* workspace,
                             size_t ws_bytes, void* stream);
 
+/*
+ * Stochastic Length (review section 三, Stochastic Length): every user's n
+ * events are shortened to L = min(n, ceil(n u^(1/alpha))), u ~ Uniform(0, 1],
+ * keeping a uniformly random subset of L events in time order.
+ * Randomness: Philox4x64-10 (Salmon et al., SC 2011) with key (seed, 0);
+ * user u's length uses counter (0, u, step, 0) and u = ((x >> 11) + 1) 2^-53
+ * from its first output word x; position p's rank key is the first output
+ * word of counter (p, u, step, 1); the kept subset is the L smallest rank
+ * keys (equal keys: the lower position).  The length is decided in fp64.
+ *   full          the input batch (offsets and timestamps on the device;
+ *                 max_len <= 16384).
+ *   x_full        device [T_full] rows of row_bytes bytes each (any element
+ *                 type; row_bytes a multiple of 16), or NULL with x_out NULL.
+ *   alpha > 0; seed, step select the random stream (use the training step
+ *                 as `step` to draw fresh subsets each step).
+ *   offsets_out   device [B+1]: the output batch's offsets; offsets_out[B]
+ *                 is its total T_out (read it back to size the next call).
+ *   lengths_out   device int32 [B]: L per user.
+ *   max_len_out   device int32 [1] or NULL: the largest L.
+ *   kept_index_out device int64 [T_full]: for output row r < T_out, the row
+ *                 of the input it copies.
+ *   timestamps_out device int64 [T_full] or NULL; x_out device [T_full] rows
+ *                 or NULL: the kept rows' timestamps and rows.
+ * Allocates nothing; four launches on `stream`.
+ */
+hstu_status_t hstu_stochastic_length(const hstu_jagged_t* full, const void* x_full,
+                                     int32_t row_bytes, float alpha, uint64_t seed, uint64_t step,
+                                     int64_t* offsets_out, int32_t* lengths_out,
+                                     int32_t* max_len_out, int64_t* kept_index_out,
+                                     int64_t* timestamps_out, void* x_out, void* stream);
+
 /* Per-kernel timing.  Between hstu_profiler_start() and hstu_profiler_stop()
  * every kernel the library launches is bracketed by CUDA events recorded on
  * its own stream (device time, no host synchronisation while running).
