@@ -37,9 +37,25 @@ def _tbucket(dt, Tb):
     return max(0, min(Tb - 1, b))
 
 
+def _visible(i, j, n_us, n_r, t):
+    """Generalised (MTGR-style) mask, row by row: U+S seen by all and seeing only
+    U+S, R causal, a candidate seeing U+S, the R events up to its time, itself."""
+    r_end = n_us + n_r
+    if j < n_us:
+        return True
+    if i < n_us:
+        return False
+    if i < r_end:
+        return j <= i
+    if j < r_end:
+        return t[j] <= t[i]
+    return j == i
+
+
 def layer(x, offsets, ts, w1, b1, w2, b2, rab_pos, rab_time, H, dqk, dv,
-          phi1="relu", phi2="silu", eps=1e-5, gamma=None, beta=None):
-    """One layer with explicit loops.  All arguments are nested lists / scalars."""
+          phi1="relu", phi2="silu", eps=1e-5, gamma=None, beta=None, segments=None):
+    """One layer with explicit loops.  All arguments are nested lists / scalars;
+    `segments` [[n_us, n_r], ...] selects the generalised masks (else causal)."""
     T = len(x)
     d = len(x[0]) if T else 0
     n1 = len(w1)
@@ -63,29 +79,34 @@ def layer(x, offsets, ts, w1, b1, w2, b2, rab_pos, rab_time, H, dqk, dv,
         V = [r[hv:2 * hv] for r in z]
         Q = [r[2 * hv:2 * hv + H * dqk] for r in z]
         K = [r[2 * hv + H * dqk:2 * hv + 2 * H * dqk] for r in z]
+        tu = ts[s:e]
         for i in range(n):
             # Eq. 2 for row i, every head
+            if segments is None:
+                keys = list(range(i + 1))
+            else:
+                keys = [j for j in range(n) if _visible(i, j, segments[uu][0], segments[uu][1], tu)]
             o = [0.0] * hv
             for h in range(H):
                 pre = []
-                for j in range(i + 1):
+                for j in keys:
                     dot = 0.0
                     for t in range(dqk):
                         dot += Q[i][h * dqk + t] * K[j][h * dqk + t]
-                    bp = min(i - j, P - 1)
+                    bp = min(abs(i - j), P - 1)
                     bt = _tbucket(ts[s + i] - ts[s + j], Tb)
                     pre.append(dot + rab_pos[h][bp] + rab_time[h][bt])
                 if phi2 == "softmax":
-                    # ablation: softmax over the visible keys j <= i, no 1/n
+                    # ablation: softmax over the visible keys, no 1/n
                     top = max(pre)
                     ex = [math.exp(val - top) for val in pre]
                     tot = sum(ex)
                     weights = [val / tot for val in ex]
                 else:
                     weights = [_act(val, phi2) / n for val in pre]
-                for j in range(i + 1):
+                for idx, j in enumerate(keys):
                     for t in range(dv):
-                        o[h * dv + t] += weights[j] * V[j][h * dv + t]
+                        o[h * dv + t] += weights[idx] * V[j][h * dv + t]
             # Eq. 3: LayerNorm over all heads, gate with U, project, residual
             mean = sum(o) / hv
             var = sum((val - mean) * (val - mean) for val in o) / hv

@@ -34,6 +34,16 @@ documented constant here, never hidden):
     table): the pointwise phi2 and its 1/N are replaced by a row-wise softmax
     over the visible keys of the same pre-activation Q K^T + rab (no extra
     scale; "-rab" is the same with zero bias tables).
+  * Generalised (MTGR-style) masks, from the RecSysChannel digest of "MTGR:
+    Industrial-Scale Generative Recommendation Framework in Meituan" (Dynamic
+    Masking): a user's tokens are ordered U+S (profile and long history),
+    then R (short history), then C (candidates), with n_us and n_r given per
+    user.  U+S keys are visible to every row, U+S rows see only U+S
+    (both directions); R rows are causal; a candidate sees U+S, the R events
+    at or before its own timestamp ("the preceding part of R") and itself,
+    not the other candidates.  Positions are the token indices; the position
+    bucket of a key after the row (inside U+S) is min(|i - j|, P - 1); the
+    time bucket of a negative difference is 0.  N = n_u, all the user's tokens.
   * M-FALCON: a candidate sits at position n_u with timestamp t_req, attends to
     the user's cached history rows (keys/values of every layer) and to itself
     (position bucket 0, time bucket 0); its score is <y_c^(L), e_c>.  Its
@@ -99,7 +109,8 @@ def rab_matrix(ts_q: np.ndarray, ts_k: np.ndarray, pos_q: np.ndarray, pos_k: np.
     P, Tb = rab_pos_h.shape[0], rab_time_h.shape[0]
     dpos = pos_q[:, None] - pos_k[None, :]
     dts = ts_q[:, None].astype(np.int64) - ts_k[None, :].astype(np.int64)
-    bp = pos_bucket(np.maximum(dpos, 0), P)
+    # |i - j|: keys after the row only occur inside the bidirectional U+S block
+    bp = pos_bucket(np.abs(dpos), P)
     bt = time_bucket(dts, Tb)
     return rab_pos_h[bp] + rab_time_h[bt]
 
@@ -121,10 +132,31 @@ def attention_weights(s: np.ndarray, mask: np.ndarray, phi2: str, n_norm: int) -
     return np.where(mask, phi(s, phi2), 0.0) / float(n_norm)
 
 
+def segment_mask(ts, n_us: int, n_r: int) -> np.ndarray:
+    """Visibility of the generalised (MTGR-style) mask for one user: rows i,
+    keys j over the user's n tokens ordered U+S, R, C."""
+    ts = np.asarray(ts, dtype=np.int64)
+    n = len(ts)
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    r_end = n_us + n_r
+    key_us = j < n_us
+    key_r = (j >= n_us) & (j < r_end)
+    row_us = i < n_us
+    row_r = (i >= n_us) & (i < r_end)
+    row_c = i >= r_end
+    vis = key_us & (row_us | row_r | row_c)              # U+S: visible to all
+    vis |= row_r & key_r & (j <= i)                       # R: causal
+    vis |= row_c & key_r & (ts[None, :] <= ts[:, None])   # C: R events up to its time
+    vis |= row_c & (j == i)                               # C: itself only
+    return vis
+
+
 def user_attention(q, k, v, ts, rab_pos, rab_time, n_norm: int, H: int, dqk: int, dv: int,
-                   phi2: str = "silu") -> np.ndarray:
+                   phi2: str = "silu", mask=None) -> np.ndarray:
     """Eq. 2 for one user: causal pointwise attention, per head, divided by N
-    (or the softmax ablation, see attention_weights).
+    (or the softmax ablation, see attention_weights); `mask` (bool [n, n])
+    replaces the causal mask (the generalised masks of segment_mask).
 
     q, k: [n, H*dqk]; v: [n, H*dv]; ts: [n] int64; returns AV [n, H*dv].
     """
@@ -133,7 +165,8 @@ def user_attention(q, k, v, ts, rab_pos, rab_time, n_norm: int, H: int, dqk: int
     if n == 0:
         return out
     pos = np.arange(n)
-    mask = np.tril(np.ones((n, n), dtype=bool))
+    if mask is None:
+        mask = np.tril(np.ones((n, n), dtype=bool))
     for h in range(H):
         qh = q[:, h * dqk:(h + 1) * dqk]
         kh = k[:, h * dqk:(h + 1) * dqk]
@@ -167,13 +200,15 @@ def _f64(a):
 
 
 def layer_fwd(x, offsets, timestamps, layer, cfg, *, keep_stages: bool = True,
-              users: Optional[Sequence[int]] = None, prefix: Optional[Sequence[int]] = None):
+              users: Optional[Sequence[int]] = None, prefix: Optional[Sequence[int]] = None,
+              segments=None):
     """One HSTU layer over a jagged batch.
 
     Returns a dict with Y [T, d] and (if keep_stages) U, V, Q, K, AV, G = Norm(AV) (.) U.
     `users` restricts work to some users (other rows are left NaN); `prefix[i]`
     computes only the first prefix[i] rows of users[i] (valid because the layer
-    is causal and N = n_u does not depend on the prefix).
+    is causal and N = n_u does not depend on the prefix).  `segments` ([B, 2]:
+    n_us, n_r per user) selects the generalised masks (no prefix then).
     """
     x = _f64(x)
     H, dqk, dv = cfg.num_heads, cfg.dqk, cfg.dv
@@ -197,7 +232,11 @@ def layer_fwd(x, offsets, timestamps, layer, cfg, *, keep_stages: bool = True,
             continue
         xu = x[s:e]
         u, v, q, k = projection(xu, w1, b1, H, dqk, dv, cfg.phi1)
-        av = user_attention(q, k, v, timestamps[s:e], rp, rt, n_u, H, dqk, dv, cfg.phi2)
+        mask = None
+        if segments is not None:
+            assert prefix is None
+            mask = segment_mask(timestamps[s:e], int(segments[uu][0]), int(segments[uu][1]))
+        av = user_attention(q, k, v, timestamps[s:e], rp, rt, n_u, H, dqk, dv, cfg.phi2, mask)
         y, g = output(xu, av, u, w2, b2, cfg.ln_eps, gamma, beta)
         res["y"][s:e] = y
         if keep_stages:
@@ -207,13 +246,13 @@ def layer_fwd(x, offsets, timestamps, layer, cfg, *, keep_stages: bool = True,
 
 
 def forward(x, offsets, timestamps, layers, cfg, *, keep_stages: bool = False,
-            users=None, prefix=None):
+            users=None, prefix=None, segments=None):
     """Stack of HSTU layers (the residual stream is carried in float64)."""
     cur = _f64(x)
     stages = []
     for layer in layers:
         r = layer_fwd(cur, offsets, timestamps, layer, cfg, keep_stages=keep_stages,
-                      users=users, prefix=prefix)
+                      users=users, prefix=prefix, segments=segments)
         stages.append(r)
         cur = r["y"]
     return cur, stages

@@ -377,3 +377,77 @@ def test_planted_mistakes_are_caught(monkeypatch):
     y_bru = brute.layer(case.x.astype(float).tolist(), H=cfg.num_heads, dqk=cfg.dqk, dv=cfg.dv,
                         phi2=cfg.phi2, **_brute_args(case, lw))
     assert not np.allclose(y_bad, np.array(y_bru), rtol=1e-9)
+
+
+# --------------------------------------------------------------------------- generalised masks
+
+def _seg_case(phi2="silu", lens=(9, 1, 12, 6), seed=41):
+    case = make_case(_tiny_cfg(phi2=phi2, num_pos_buckets=5), seed=seed, lengths=list(lens))
+    return case
+
+
+@pytest.mark.parametrize("phi2", ["silu", "identity", "softmax"])
+def test_segments_all_history_is_causal(phi2):
+    """n_us = 0 and n_r = n (no profile, no candidates) is the causal layer."""
+    case = _seg_case(phi2)
+    segs = [[0, int(n)] for n in case.lengths]
+    a = O.layer_fwd(case.x, case.offsets, case.timestamps, case.layers[0], case.cfg)["y"]
+    b = O.layer_fwd(case.x, case.offsets, case.timestamps, case.layers[0], case.cfg,
+                    segments=segs)["y"]
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("phi2", ["silu", "softmax"])
+def test_segments_brute_force_equals_vectorised(phi2):
+    case = _seg_case(phi2)
+    segs = [[3, 4], [1, 0], [4, 5], [0, 2]]  # n_c = 2, 0, 3, 4
+    lw = case.layers[0]
+    ts = case.timestamps.copy()
+    s0, e0 = case.offsets[2], case.offsets[3]
+    ts[s0:e0] = np.sort(ts[s0:e0])
+    ts[e0 - 3:e0] = ts[s0 + 6]  # candidates timed inside R: they see only part of it
+    y_vec = O.layer_fwd(case.x, case.offsets, ts, lw, case.cfg, segments=segs)["y"]
+    y_bru = brute.layer(case.x.astype(float).tolist(), H=case.cfg.num_heads, dqk=case.cfg.dqk,
+                        dv=case.cfg.dv, phi1=case.cfg.phi1, phi2=phi2, eps=case.cfg.ln_eps,
+                        segments=segs, **{**_brute_args(case, lw), "ts": [int(t) for t in ts]})
+    assert np.allclose(y_vec, np.array(y_bru), rtol=1e-12, atol=1e-12)
+
+
+def _av(case, ts, segs, x=None):
+    x = case.x if x is None else x
+    return O.layer_fwd(x, case.offsets, ts, case.layers[0], case.cfg, segments=segs)["av"]
+
+
+def test_segments_visibility_invariants():
+    """U+S rows ignore R and C; R rows ignore later R and C; a candidate ignores
+    the other candidates and the R events after its time."""
+    case = _seg_case("silu", lens=(14,))
+    n_us, n_r = 4, 6  # rows 0-3 U+S, 4-9 R, 10-13 C
+    segs = [[n_us, n_r]]
+    ts = np.sort(case.timestamps.copy())
+    ts[10:] = ts[7]  # candidates at the time of R row 7: they see R rows 4..7
+    base = _av(case, ts, segs)
+    rng = np.random.default_rng(1)
+
+    def perturbed(rows):
+        x = case.x.copy()
+        x[rows] += rng.standard_normal((len(rows), x.shape[1]))
+        return _av(case, ts, segs, x)
+    a = perturbed(list(range(4, 14)))            # every R and C token
+    assert np.array_equal(a[:4], base[:4])
+    b = perturbed([8, 9, 10, 11, 12, 13])         # R rows 8, 9 and the candidates
+    assert np.array_equal(b[:8], base[:8])
+    c = perturbed([8, 9, 11, 12, 13])             # later R and the other candidates
+    assert np.array_equal(c[10], base[10])
+    assert not np.array_equal(perturbed([7])[10], base[10])   # R row 7 is visible to it
+    assert not np.array_equal(perturbed([10])[10], base[10])  # and so is itself
+
+
+def test_segment_mask_rules():
+    ts = np.array([0, 0, 5, 10, 20, 30, 15, 30, 1], dtype=np.int64)
+    m = O.segment_mask(ts, 2, 4)  # U+S 0-1, R 2-5, C 6-8
+    assert m[0].tolist() == [1, 1, 0, 0, 0, 0, 0, 0, 0]
+    assert m[3].tolist() == [1, 1, 1, 1, 0, 0, 0, 0, 0]
+    assert m[6].tolist() == [1, 1, 1, 1, 0, 0, 1, 0, 0]   # t = 15: R events at 5 and 10
+    assert m[7].tolist() == [1, 1, 1, 1, 1, 1, 0, 1, 0]   # t = 30: all of R
+    assert m[8].tolist() == [1, 1, 0, 0, 0, 0, 0, 0, 1]   # t = 1: no R event yet
