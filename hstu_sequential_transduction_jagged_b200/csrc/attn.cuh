@@ -78,10 +78,12 @@ struct AttnParams {
   const int64_t* request_ts;   // [B] (candidate mode)
   const float* rab_pos;        // [H, P]
   const float* rab_time;       // [H, Tb]
-  const void* q_self;          // candidate mode: candidate Q, K, V rows (self term),
-  const void* k_self;          // in the kernel's operand type (bf16 or fp16)
-  const void* v_self;
-  int64_t ld_self;             // row stride (elements) of q_self/k_self/v_self
+  const void* q_self;          // rows' own Q, K, V for the self term (candidate mode,
+  const void* k_self;          // and candidate rows of the generalised masks), in the
+  const void* v_self;          // kernel's operand type (bf16 or fp16)
+  int64_t ld_qs, ld_ks, ld_vs; // their row strides (elements)
+  const int32_t* segments;     // [B, 2] (n_us, n_r) per user: generalised masks, or nullptr
+  int32_t max_static;          // bound on n_us (staged position range)
   void* av;                    // [T_q, ld_av] output in the operand type, or
   float* av_f32;               // [T_q, ld_av] fp32 output (the layer path feeds LayerNorm)
   int64_t ld_av;
@@ -423,9 +425,31 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_status(HSTU_ERR_DEVICE_CHECK);
     return;  // uniform across the CTA, before any allocation
   }
+  // Generalised (MTGR-style) masks: the user's tokens are U+S (n_us), R (n_r),
+  // then candidates.  Every row sees a prefix of the keys (U+S rows: the U+S
+  // block; R rows: up to themselves; candidate rows: U+S and the R events up
+  // to their own time) and candidate rows also themselves, added like the
+  // candidate-mode self term.
+  const bool masked = !CAND && p.segments != nullptr;
+  int n_us = 0, r_end = n_kv;  // plain causal: every row is an R row
+  if (masked) {
+    n_us = p.segments[2 * u];
+    const int n_r = p.segments[2 * u + 1];
+    if (n_us < 0 || n_r < 0 || n_us + n_r > n_kv || n_us > p.max_static) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_status(HSTU_ERR_DEVICE_CHECK);
+      return;  // uniform across the CTA, before any allocation
+    }
+    r_end = n_us + n_r;
+  }
   const int q0 = qp * 2 * ATT_ROWS;
   if (q0 >= n_q) return;  // uniform across the CTA, before any allocation
   const bool has_b = (q0 + ATT_ROWS) < n_q;
+
+  // The softmax ablation takes two passes over the key tiles: the first finds
+  // each row's max and sum, the second writes P and runs P V.  Stage index
+  // si = pass * nk_total + tile.
+  constexpr bool kSoftmax = PHI == HSTU_ACT_SOFTMAX;
+  constexpr int kPasses = kSoftmax ? 2 : 1;
 
   // number of key tiles each query tile consumes
   int nA, nB;
@@ -433,16 +457,29 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int nk = (n_kv + ATT_KEYS - 1) / ATT_KEYS;
     nA = nk;
     nB = has_b ? nk : 0;
-  } else {
+  } else if (!masked) {
     nA = (q0 + ATT_ROWS) / ATT_KEYS;      // keys 0 .. q0 + 127
     nB = has_b ? (q0 + 2 * ATT_ROWS) / ATT_KEYS : 0;
+  } else {
+    // exclusive end of the keys any row in [r0, r0 + 128) sees
+    auto tile_end = [&](int r0) -> int {
+      if (r0 >= n_q) return 0;
+      const int r1 = min(r0 + ATT_ROWS, n_q);
+      int e = 0;
+      if (r0 < n_us) e = n_us;                                   // U+S rows
+      if (r1 > n_us && r0 < r_end) e = max(e, min(r1, r_end));   // R rows
+      if (r1 > r_end) e = max(e, r_end);                         // candidate rows
+      return e;
+    };
+    nA = (tile_end(q0) + ATT_KEYS - 1) / ATT_KEYS;
+    nB = (tile_end(q0 + ATT_ROWS) + ATT_KEYS - 1) / ATT_KEYS;
+    // two passes look three items ahead across the pass boundary; the ring
+    // of stages holds that only while tile A takes at most two fewer key
+    // tiles than tile B, so tile A then walks tile B's (masked) tiles too
+    if (kSoftmax && has_b && nB - nA > 2) nA = nB;
+    if (kSoftmax && has_b && nA - nB > 2) nB = nA;
   }
   const int nk_total = nA > nB ? nA : nB;
-  // The softmax ablation takes two passes over the key tiles: the first finds
-  // each row's max and sum, the second writes P and runs P V.  Stage index
-  // si = pass * nk_total + tile.
-  constexpr bool kSoftmax = PHI == HSTU_ACT_SOFTMAX;
-  constexpr int kPasses = kSoftmax ? 2 : 1;
   const int n_stages = kPasses * nk_total;
 
   // causal rows read position offsets i - j in [-127, q0 + 255]; candidates
@@ -508,13 +545,16 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   {
     const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
-    const int xend = min(p.pos_len, D + ATT_ROWS + 2);
+    // offsets i - j down to -(keys after the row a chunk reads): 127 + 2 in
+    // causal mode, up to the U+S block (+ a chunk) with the generalised masks;
+    // the bucket of an offset d is min(|d|, P - 1)
+    const int xend = min(p.pos_len, D + (masked ? max(ATT_ROWS, p.max_static + 2 * 32) : ATT_ROWS) + 2);
     for (int x = tid; x < xend; x += ATT_THREADS) {
       const int d0 = D - x;  // copy 0 holds offset D - x
-      sRv[x] = (d0 >= 0) ? kScale * rp[min(d0, p.P - 1)] : 0.0f;
+      sRv[x] = kScale * rp[min(abs(d0), p.P - 1)];
       if constexpr (PAIRS) {
         const int d1 = D + 1 - x;  // copy 1 holds offset D + 1 - x
-        sRv[p.pos_len + x] = (d1 >= 0) ? kScale * rp[min(d1, p.P - 1)] : 0.0f;
+        sRv[p.pos_len + x] = kScale * rp[min(abs(d1), p.P - 1)];
       }
     }
   }
@@ -757,13 +797,33 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float rt_cur = 0.0f;  // time bias of the walk's current bucket
     int copy = 0;
     const float* rv = sRv;
+    // keys this row sees: the prefix [0, vis_end), and itself when self_row
+    int vis_end = i + 1;
+    bool self_row = false;
     if constexpr (!CAND) {
       const int64_t d = (valid ? p.timestamps[kv_start + i] : t_first) - t_first;
+      if (valid && d >= static_cast<int64_t>(INT32_MAX) - 1) record_status(HSTU_ERR_DEVICE_CHECK);
       w32.init(d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d), 0,
                sThr, sThr32, p.Tb);
       if constexpr (PAIRS) copy = (D - i) & 1;
       rv = sRv + copy * p.pos_len;
       rt_cur = sTime[w32.b];
+      if (masked && valid) {
+        if (i < n_us) {
+          vis_end = n_us;
+        } else if (i >= r_end) {
+          // a candidate: the R events at or before its own time (R is time-ordered)
+          const int64_t t_i = p.timestamps[kv_start + i];
+          int lo = n_us, hi = r_end;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (p.timestamps[kv_start + mid] <= t_i) lo = mid + 1;
+            else hi = mid;
+          }
+          vis_end = lo;
+          self_row = true;
+        }
+      }
     }
 
     // this half's 32 keys of tile kt: S values in `sv`, packed 16-bit P pairs to `pk`
@@ -794,9 +854,9 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int c = 0; c < 32; c += 2) pk[c >> 1] = mask_pair(pk[c >> 1], c, last);
         }
       } else {
-        // last visible column: keys after the row are masked; rows past the
-        // user's end are not stored and skip the work
-        const int lim = !valid ? -1 : i - j0;
+        // last visible column: keys past the row's visible prefix are masked;
+        // rows past the user's end are not stored and skip the work
+        const int lim = !valid ? -1 : vis_end - 1 - j0;
         const int32_t* kts = reinterpret_cast<const int32_t*>(key) + half * 32;
         const int xc = D - i + j0 + copy;  // table index at column 0
         causal_chunk_pointwise<PHI, PAIRS, F16>(sv, pk, rv + xc, kts, lim, w32, sTime, sThr32,
@@ -812,8 +872,8 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       else return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
     };
     auto self_dot = [&]() -> float {
-      const uint16_t* qs = static_cast<const uint16_t*>(p.q_self) + row * p.ld_self + h * ATT_HD;
-      const uint16_t* ks = static_cast<const uint16_t*>(p.k_self) + row * p.ld_self + h * ATT_HD;
+      const uint16_t* qs = static_cast<const uint16_t*>(p.q_self) + row * p.ld_qs + h * ATT_HD;
+      const uint16_t* ks = static_cast<const uint16_t*>(p.k_self) + row * p.ld_ks + h * ATT_HD;
       float dot = 0.0f;
 #pragma unroll
       for (int c = 0; c < ATT_HD; c += 8) {
@@ -840,7 +900,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // P = 2^(h - m - log2 l)
     float sm_m = -INFINITY, sm_l = 0.0f;
     float h_self = -INFINITY;  // candidate mode: the own key's pre-activation
-    if constexpr (kSoftmax && CAND) {
+    if (kSoftmax && (CAND || self_row)) {
       if (valid) h_self = kScale * (self_dot() + self_rab());
       if (half == 0 && valid) {
         sm_m = h_self;
@@ -895,7 +955,7 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         return valid ? min(31, n_kv - 1 - j0) : -1;
       } else {
-        const int lim = !valid ? -1 : i - j0;
+        const int lim = !valid ? -1 : vis_end - 1 - j0;
         causal_chunk<PAIRS>(
             sv, [&](int c, uint64_t hv) { hh[c >> 1] = hv; }, rv + (D - i + j0 + copy),
             reinterpret_cast<const int32_t*>(key) + half * 32, lim, w32, sTime, sThr32, sOct,
@@ -1013,10 +1073,10 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int c = 0; c < HC; ++c) o[c] = 0.0f;
       }
       if (valid) {
-        if constexpr (CAND) {
+        if (CAND || self_row) {
           // the candidate's own key/value: position bucket 0, time bucket 0
           const uint16_t* vs =
-              static_cast<const uint16_t*>(p.v_self) + row * p.ld_self + h * ATT_HD + half * HC;
+              static_cast<const uint16_t*>(p.v_self) + row * p.ld_vs + h * ATT_HD + half * HC;
           float ps;
           if constexpr (kSoftmax) ps = ex2_approx(h_self - sm_m);  // already divided by the sum
           else ps = apply_phi<PHI>(self_dot() + self_rab());

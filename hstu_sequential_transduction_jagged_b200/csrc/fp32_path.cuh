@@ -91,6 +91,7 @@ struct F32AttnParams {
   int32_t B, H, P, Tb, phi2;
   int32_t cand;
   int32_t max_q, max_kv;  // host-declared length bounds the grid is sized for
+  const int32_t* segments;  // [B, 2] (n_us, n_r): generalised masks, or nullptr
   int64_t thr[MAX_TIME_BUCKETS];
 };
 
@@ -127,10 +128,35 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
   const int i = r0 + r;  // query index within the user
   const int64_t t_row = p.cand ? p.request_ts[u] : ((i < n_q) ? p.timestamps[kv0 + i] : 0);
   const int pos_row = p.cand ? n_kv : i;
+  // keys this row sees: the prefix [0, vis_end), and itself when self_row
+  // (candidate mode, or a candidate row of the generalised masks)
+  int vis_end = i + 1;
+  bool self_row = p.cand != 0;
+  const bool masked = !p.cand && p.segments != nullptr;
+  if (masked) {
+    const int n_us = p.segments[2 * u], n_r = p.segments[2 * u + 1];
+    if (n_us < 0 || n_r < 0 || n_us + n_r > n_kv) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(HSTU_ERR_DEVICE_CHECK);
+      return;
+    }
+    const int r_end = n_us + n_r;
+    if (i < n_us) {
+      vis_end = n_us;
+    } else if (i >= r_end && i < n_q) {
+      int lo = n_us, hi = r_end;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (p.timestamps[kv0 + mid] <= t_row) lo = mid + 1;
+        else hi = mid;
+      }
+      vis_end = lo;
+      self_row = true;
+    }
+  }
   float o[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) o[c] = 0.0f;
-  const int key_end = p.cand ? n_kv : min(n_kv, r0 + 32);
+  const int key_end = (p.cand || masked) ? n_kv : min(n_kv, r0 + 32);
   const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
   const float* rt = p.rab_time + static_cast<int64_t>(h) * p.Tb;
   // The softmax ablation takes two passes: the first finds the row's max m
@@ -138,11 +164,14 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
   // included), the second accumulates exp(x - m) / l times V.
   const bool softmax = p.phi2 == HSTU_ACT_SOFTMAX;
   float sm_m = -INFINITY, sm_l = 0.0f, x_self = 0.0f;
-  if (softmax && p.cand && i < n_q) {
-    const int64_t row = q0g + i;
+  // the row's own query and key (self term)
+  const int64_t row_s = q0g + i;
+  const float* qs = p.cand ? p.q_self + row_s * p.ld_self : p.q + row_s * p.ldq;
+  const float* ks = p.cand ? p.k_self + row_s * p.ld_self : p.k + row_s * p.ldk;
+  const float* vs = p.cand ? p.v_self + row_s * p.ld_self : p.v + row_s * p.ldv;
+  if (softmax && self_row && i < n_q) {
     float s = 0.0f;
-    for (int c = 0; c < 64; ++c)
-      s = fmaf(p.q_self[row * p.ld_self + h * 64 + c], p.k_self[row * p.ld_self + h * 64 + c], s);
+    for (int c = 0; c < 64; ++c) s = fmaf(qs[h * 64 + c], ks[h * 64 + c], s);
     x_self = s + rp[0] + rt[0];
     if (qt == 0) {
       sm_m = x_self;
@@ -175,11 +204,11 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
       const int jj = qt * 8 + kk;
       const int j = j0 + jj;
       float pval = 0.0f;
-      const bool live = (j < n_kv) && (p.cand || j <= i) && (i < n_q);
+      const bool live = (j < n_kv) && (p.cand || j < vis_end) && (i < n_q);
       if (live) {
         float s = 0.0f;
         for (int c = 0; c < 64; ++c) s = fmaf(sq[r][c], sk[jj][c], s);
-        const int bp = min(pos_row - j, p.P - 1);
+        const int bp = min(abs(pos_row - j), p.P - 1);
         const int bt = time_bucket_search(t_row - p.timestamps[kv0 + j], sthr, p.Tb);
         const float x = s + rp[bp] + rt[bt];
         if (!softmax) {
@@ -209,19 +238,17 @@ __global__ void __launch_bounds__(128) hstu_f32_attn_kernel(const __grid_constan
   }
   if (i >= n_q) return;
   const int64_t row = q0g + i;
-  if (p.cand) {
+  if (self_row) {
     float ps;
     if (softmax) {
       ps = expf(x_self - sm_m) / sm_l;
     } else {
       float s = 0.0f;
-      for (int c = 0; c < 64; ++c)
-        s = fmaf(p.q_self[row * p.ld_self + h * 64 + c], p.k_self[row * p.ld_self + h * 64 + c], s);
+      for (int c = 0; c < 64; ++c) s = fmaf(qs[h * 64 + c], ks[h * 64 + c], s);
       ps = phi_runtime(s + rp[0] + rt[0], p.phi2);
     }
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      o[c] = fmaf(ps, p.v_self[row * p.ld_self + h * 64 + qt * 16 + c], o[c]);
+    for (int c = 0; c < 16; ++c) o[c] = fmaf(ps, vs[h * 64 + qt * 16 + c], o[c]);
   }
   const float inv_n = softmax ? 1.0f : 1.0f / static_cast<float>(p.cand ? max(n_kv, 1) : n_kv);
 #pragma unroll

@@ -327,6 +327,8 @@ hstu_status_t check_jag(const hstu_jagged_t* j) {
   // a batch with rows has a user of length >= 1; the kernels are sized from max_len
   if (j->total_tokens > 0 && j->max_len == 0) return HSTU_ERR_INVALID_ARGUMENT;
   if (j->max_len > kMaxLen || j->batch > 65535) return HSTU_ERR_UNSUPPORTED;
+  if (j->segments != nullptr && (j->max_static < 0 || j->max_static > kMaxLen))
+    return HSTU_ERR_INVALID_ARGUMENT;
   if (j->total_tokens > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
   return HSTU_OK;
 }
@@ -442,6 +444,8 @@ struct AttnJob {
   const void* k; int64_t ldk;
   const void* v; int64_t ldv;
   const void* q_self; const void* k_self; const void* v_self; int64_t ld_self;
+  const int32_t* segments;      // generalised masks (causal mode), or nullptr
+  int32_t max_static;
   const float* rab_pos;
   const float* rab_time;
   void* av; int64_t ld_av;      // bf16 [.., ld_av] output (attention alone)
@@ -479,10 +483,20 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   p.request_ts = j.request_ts;
   p.rab_pos = j.rab_pos;
   p.rab_time = j.rab_time;
-  p.q_self = j.q_self;
-  p.k_self = j.k_self;
-  p.v_self = j.v_self;
-  p.ld_self = j.ld_self;
+  if (!CAND && j.segments != nullptr) {
+    // candidate rows of the generalised masks add their own key/value: read
+    // from the tensors being attended
+    p.q_self = j.q; p.ld_qs = j.ldq;
+    p.k_self = j.k; p.ld_ks = j.ldk;
+    p.v_self = j.v; p.ld_vs = j.ldv;
+    p.segments = j.segments;
+    p.max_static = j.max_static;
+  } else {
+    p.q_self = j.q_self;
+    p.k_self = j.k_self;
+    p.v_self = j.v_self;
+    p.ld_qs = p.ld_ks = p.ld_vs = j.ld_self;
+  }
   p.av = j.av;
   p.av_f32 = j.av_f32;
   p.ld_av = j.ld_av;
@@ -499,7 +513,12 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
                            : align_up(static_cast<size_t>(j.max_q_len), 2 * ATT_ROWS);
   // per-copy length = 16 (mod 32) floats: the two copies' 8-byte pair reads
   // by neighbouring lanes then fall in disjoint shared-memory banks
-  p.pos_len = static_cast<int32_t>(align_up(dmax + ATT_ROWS + 2, 32) + 16);
+  // the staged offsets reach 127 + 2 past a row (causal), or the U+S block
+  // plus two chunks (generalised masks)
+  const size_t extra = (!CAND && j.segments != nullptr)
+                           ? std::max<size_t>(ATT_ROWS, static_cast<size_t>(j.max_static) + 64)
+                           : ATT_ROWS;
+  p.pos_len = static_cast<int32_t>(align_up(dmax + extra + 2, 32) + 16);
   const uint32_t pos_elt = 4u;
   p.phi2 = c->phi2;
   p.timeout_ns = j.timeout_ns;
@@ -684,6 +703,7 @@ hstu_status_t launch_f32_attn(const AttnJob& j, cudaStream_t st) {
   p.Tb = c->num_time_buckets;
   p.phi2 = c->phi2;
   p.cand = j.q_offsets != nullptr ? 1 : 0;
+  p.segments = p.cand ? nullptr : j.segments;
   p.max_q = j.max_q_len;
   p.max_kv = j.max_kv_len;
   std::memcpy(p.thr, thresholds_for(c->num_time_buckets), sizeof(int64_t) * c->num_time_buckets);
@@ -893,6 +913,8 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
   std::memset(&j, 0, sizeof(j));
   j.cfg = cfg;
   j.kv_offsets = jag->offsets;
+  j.segments = jag->segments;
+  j.max_static = jag->max_static;
   j.timestamps = jag->timestamps;
   j.batch = jag->batch;
   j.max_q_len = j.max_kv_len = jag->max_len;
@@ -928,6 +950,8 @@ hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t
   std::memset(&j, 0, sizeof(j));
   j.cfg = cfg;
   j.kv_offsets = jag->offsets;
+  j.segments = jag->segments;
+  j.max_static = jag->max_static;
   j.timestamps = jag->timestamps;
   j.batch = jag->batch;
   j.max_q_len = j.max_kv_len = jag->max_len;
@@ -959,6 +983,7 @@ hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t*
   if ((s = check_cfg(cfg)) != HSTU_OK) return s;
   if ((s = check_jag(history)) != HSTU_OK) return s;
   if (num_cand < 0 || max_cand < 0) return HSTU_ERR_INVALID_ARGUMENT;
+  if (history->segments != nullptr) return HSTU_ERR_UNSUPPORTED;
   if (num_cand == 0 || history->batch == 0) return HSTU_OK;
   if (max_cand == 0) return HSTU_ERR_INVALID_ARGUMENT;
   if (max_cand > kMaxLen || num_cand > (int64_t(1) << 31) - 1) return HSTU_ERR_UNSUPPORTED;
@@ -1021,6 +1046,8 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weigh
   std::memset(&base, 0, sizeof(base));
   base.cfg = cfg;
   base.kv_offsets = jag->offsets;
+  base.segments = jag->segments;
+  base.max_static = jag->max_static;
   base.timestamps = jag->timestamps;
   base.batch = jag->batch;
   base.max_q_len = base.max_kv_len = jag->max_len;
@@ -1091,6 +1118,8 @@ hstu_status_t hstu_forward(const hstu_layer_cfg_t* cfg, int32_t num_layers,
   std::memset(&base, 0, sizeof(base));
   base.cfg = cfg;
   base.kv_offsets = jag->offsets;
+  base.segments = jag->segments;
+  base.max_static = jag->max_static;
   base.timestamps = jag->timestamps;
   base.batch = jag->batch;
   base.max_q_len = base.max_kv_len = jag->max_len;
@@ -1129,6 +1158,7 @@ hstu_status_t mfalcon_score(const hstu_layer_cfg_t* cfg, int32_t num_layers,
   if ((s = check_jag(history)) != HSTU_OK) return s;
   if (num_layers < 1 || weights == nullptr || microbatch < 1 || num_cand < 0 || max_cand < 0)
     return HSTU_ERR_INVALID_ARGUMENT;
+  if (history->segments != nullptr) return HSTU_ERR_UNSUPPORTED;
   for (int l = 0; l < num_layers; ++l)
     if ((s = check_weights(cfg, &weights[l])) != HSTU_OK) return s;
   if (num_cand == 0 || history->batch == 0) return HSTU_OK;

@@ -36,7 +36,8 @@ class HSTUError(RuntimeError):
 class JaggedT(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("total_tokens", ctypes.c_int64),
                 ("max_len", ctypes.c_int32), ("offsets", ctypes.c_void_p),
-                ("timestamps", ctypes.c_void_p)]
+                ("timestamps", ctypes.c_void_p), ("segments", ctypes.c_void_p),
+                ("max_static", ctypes.c_int32)]
 
 
 class LayerCfgT(ctypes.Structure):
@@ -162,6 +163,8 @@ class Jagged:
     timestamps: torch.Tensor   # int64 [T] on the device
     max_len: int
     total_tokens: int
+    segments: Optional[torch.Tensor] = None  # int32 [B, 2] (n_us, n_r): generalised masks
+    max_static: int = 0                      # >= every n_us
 
     @property
     def batch(self) -> int:
@@ -169,7 +172,9 @@ class Jagged:
 
     def c(self) -> JaggedT:
         return JaggedT(self.batch, self.total_tokens, self.max_len, self.offsets.data_ptr(),
-                       self.timestamps.data_ptr() if self.timestamps.numel() else None)
+                       self.timestamps.data_ptr() if self.timestamps.numel() else None,
+                       None if self.segments is None else self.segments.data_ptr(),
+                       self.max_static)
 
 
 @dataclass

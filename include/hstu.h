@@ -99,6 +99,19 @@ typedef struct {
                                  as HSTU_ERR_DEVICE_CHECK and its rows are not computed */
   const int64_t* offsets;     /* device [B+1], offsets[0] = 0, non-decreasing */
   const int64_t* timestamps;  /* device [T], int64 seconds */
+  /* Generalised masks (the Dynamic Masking of MTGR, RecSysChannel digest of
+   * "MTGR: Industrial-Scale Generative Recommendation Framework in Meituan"),
+   * or NULL for the plain causal mask.  device int32 [B, 2]: (n_us, n_r) per
+   * user, whose tokens are then ordered U+S (n_us: profile and long history),
+   * R (n_r: short history), candidates (the rest).  U+S keys are visible to
+   * every row and U+S rows see only U+S (both directions); R rows are causal;
+   * a candidate sees U+S, the R events at or before its own timestamp and
+   * itself, not the other candidates.  The position bucket of a key after
+   * the row is min(|i - j|, P - 1); N stays n_u.  Timestamps must be
+   * non-decreasing over U+S and R; candidates' timestamps are free.  Not
+   * accepted by the M-FALCON entry points. */
+  const int32_t* segments;
+  int32_t max_static;         /* >= every n_us when segments is given */
 } hstu_jagged_t;
 
 typedef struct {
