@@ -43,10 +43,15 @@ WORKLOAD_TEXT = {
                "cached history, 2048 candidates per user in microbatches of 256",
     "long-bf16-softmax": "the long-sequence workload with the (-rab, Softmax) ablation: softmax "
                          "over the visible keys instead of the pointwise phi2, zero bias tables",
+    "long-bf16-mtgr": "the long-sequence workload with generalised (MTGR-style) masks: per user "
+                      "1024 U+S tokens, 6144 R tokens, 1024 candidates timed across R",
+    "sl-sampler": "GPU Stochastic Length sampler on 64 users x 4096 events (alpha 1.6), d_model "
+                  "512 bf16 rows gathered",
 }
 # workloads that are another workload with a changed configuration:
 # name -> (base workload, config changes, zero the rab tables)
-VARIANTS = {"long-bf16-softmax": ("long-bf16", {"phi2": "softmax"}, True)}
+VARIANTS = {"long-bf16-softmax": ("long-bf16", {"phi2": "softmax"}, True),
+            "long-bf16-mtgr": ("long-bf16", {}, False)}
 
 
 def make_workload(name, batch=None):
@@ -59,7 +64,40 @@ def make_workload(name, batch=None):
         for lw in case.layers:
             lw.rab_pos[:] = 0.0
             lw.rab_time[:] = 0.0
+    if name == "long-bf16-mtgr":
+        # U+S 1024, R 6144, candidates 1024 with timestamps spread over R's span
+        import numpy as np
+        rng = np.random.default_rng(7)
+        n_us, n_r = 1024, 6144
+        segs = []
+        for u in range(len(case.lengths)):
+            s0, n = int(case.offsets[u]), int(case.lengths[u])
+            lo, hi = case.timestamps[s0 + n_us], case.timestamps[s0 + n_us + n_r - 1]
+            case.timestamps[s0 + n_us + n_r:s0 + n] = np.sort(rng.integers(lo, hi + 1, n - n_us - n_r))
+            segs.append([n_us, n_r])
+        case.extra["segments"] = np.array(segs, dtype=np.int32)
     return case
+
+
+def visible_pairs(case) -> int:
+    """Causal pairs, or the visible (query, key) pairs of the generalised masks."""
+    import numpy as np
+    segs = case.extra.get("segments")
+    n = case.lengths.astype(np.int64)
+    if segs is None:
+        return int((n * (n + 1) // 2).sum())
+    total = 0
+    for u, seg in enumerate(segs):
+        n_us, n_r = int(seg[0]), int(seg[1])
+        s0, nu = int(case.offsets[u]), int(n[u])
+        r_end = n_us + n_r
+        ts = case.timestamps[s0:s0 + nu]
+        total += n_us * n_us                                         # U+S rows
+        total += int(np.arange(n_us + 1, r_end + 1).sum())           # R rows: i + 1
+        r_vis = np.searchsorted(ts[n_us:r_end], ts[r_end:], side="right")
+        total += int((n_us + r_vis + 1).sum())                       # candidates
+    return total
+
 MFALCON_METRIC = "M-FALCON candidate scores/sec at 1 B200 (cached history K/V)"
 # The attention launches of these workloads last about a millisecond inside
 # steps of a few milliseconds, far from the seconds-long matmul loop that
@@ -387,8 +425,12 @@ def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batc
     case = make_workload(name, batch=batch)
     c = case.cfg
     counts = algorithmic_counts(case)
+    counts["attn_flop_per_layer"] = visible_pairs(case) * c.num_heads * (2 * c.dqk + 2 * c.dv)
     t = case_tensors(case, ctx.dev)
-    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens)
+    segs = case.extra.get("segments")
+    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, case.total_tokens,
+                   None if segs is None else torch.from_numpy(segs).to(ctx.dev),
+                   0 if segs is None else int(segs[:, 0].max()))
     weights = [H.LayerWeights(**lw) for lw in t["layers"]]
     cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets,
                         dqk=c.dqk, dv=c.dv, phi1=c.phi1, phi2=c.phi2, ln_eps=c.ln_eps,
@@ -664,7 +706,12 @@ def main():
         return
 
     ctx = Ctx(args, rank, world, local)
-    if args.workload == "mfalcon":
+    if args.workload == "sl-sampler":
+        r = measure_sl_sampler(ctx, args.steps, args.warmup)
+        if rank == 0:
+            print(json.dumps({**r, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "higher_is_better": True, "data": "synthetic"}), flush=True)
+    elif args.workload == "mfalcon":
         r = measure_mfalcon(ctx, args.steps, args.warmup, not args.no_e2e, batch=args.batch)
         line = {"metric": MFALCON_METRIC, "value": r["value"], "unit": "candidates/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -702,7 +749,8 @@ def main():
                                      100 * r["roofline"].get("frac_of_sustained", 0.0)}
         if world == 1 and not args.no_workloads and args.batch is None:
             subs = {}
-            for name in ("small-bf16", "sl-bf16", "tiny-fp32", "long-bf16-softmax"):
+            for name in ("small-bf16", "sl-bf16", "tiny-fp32", "long-bf16-softmax",
+                         "long-bf16-mtgr"):
                 if name == args.workload:
                     continue
                 subs[name] = _public(measure_forward(ctx, name, min(args.steps, 20), args.warmup,

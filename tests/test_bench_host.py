@@ -150,3 +150,23 @@ def test_traffic_lookup_follows_source_hash(tmp_path, monkeypatch):
     assert bench.traffic_from_profiles("k") == 1234.0
     src.write_text("kernel v2\n")
     assert bench.traffic_from_profiles("k") is None
+
+
+def test_visible_pair_count_matches_the_mask():
+    """bench.py's algorithmic pair count for masked workloads equals the number
+    of visible (query, key) pairs of the oracle's mask."""
+    import numpy as np
+    from gen import make_case
+    from oracle import hstu as O
+    bench = _bench()
+    case = make_case("small-bf16", seed=3, lengths=[300, 77, 129])
+    assert bench.visible_pairs(case) == sum(n * (n + 1) // 2 for n in (300, 77, 129))
+    segs = np.array([[40, 200], [0, 77], [129, 0]], dtype=np.int32)
+    ts = case.timestamps.copy()
+    ts[240:300] = np.sort(np.random.default_rng(0).integers(ts[40], ts[239] + 1, 60))
+    case.timestamps = ts
+    case.extra["segments"] = segs
+    want = sum(int(O.segment_mask(ts[case.offsets[u]:case.offsets[u + 1]], a, b).sum())
+               for u, (a, b) in enumerate(segs))
+    got = bench.visible_pairs(case)
+    assert isinstance(got, int) and got == want
