@@ -224,8 +224,12 @@ __global__ void __launch_bounds__(SL_SELECT_THREADS) hstu_sl_select_kernel(
   }
 }
 
-// x_out[r] = x[kept_index[r]] for r < offsets_out[B]: one warp per row,
-// 16-byte copies, grid-strided over the rows.
+// x_out[r] = x[kept_index[r]] for r < offsets_out[B]: a warp copies four rows
+// at a time (16-byte accesses, every load of the four rows issued before the
+// first store, so enough bytes are in flight to cover the memory latency),
+// grid-strided over the rows.
+constexpr int SL_GATHER_ROWS = 4;
+
 __global__ void __launch_bounds__(256) hstu_sl_gather_kernel(const int64_t* offsets_out, int32_t B,
                                                              int64_t T_full,
                                                              const int64_t* kept_index,
@@ -238,13 +242,32 @@ __global__ void __launch_bounds__(256) hstu_sl_gather_kernel(const int64_t* offs
   }
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < total;
-       r += warps) {
-    const int64_t k = kept_index[r];
-    if (k < 0 || k >= T_full) continue;  // a user the selection skipped (reported there)
-    const uint4* src = x + k * row_vec;
-    uint4* dst = x_out + r * row_vec;
-    for (int c = lane; c < row_vec; c += 32) dst[c] = src[c];
+  const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  for (int64_t r0 = w0 * SL_GATHER_ROWS; r0 < total; r0 += warps * SL_GATHER_ROWS) {
+    int64_t src[SL_GATHER_ROWS];
+#pragma unroll
+    for (int q = 0; q < SL_GATHER_ROWS; ++q) {
+      const int64_t r = r0 + q;
+      const int64_t k = r < total ? kept_index[r] : -1;
+      src[q] = (k >= 0 && k < T_full) ? k : -1;  // -1: past the end, or a user the selection skipped
+    }
+    for (int c0 = 0; c0 < row_vec; c0 += 64) {
+      uint4 v[SL_GATHER_ROWS][2];
+#pragma unroll
+      for (int q = 0; q < SL_GATHER_ROWS; ++q)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c0 + e * 32 + lane;
+          if (src[q] >= 0 && c < row_vec) v[q][e] = x[src[q] * row_vec + c];
+        }
+#pragma unroll
+      for (int q = 0; q < SL_GATHER_ROWS; ++q)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = c0 + e * 32 + lane;
+          if (src[q] >= 0 && c < row_vec) x_out[(r0 + q) * row_vec + c] = v[q][e];
+        }
+    }
   }
 }
 
