@@ -47,6 +47,8 @@ WORKLOAD_TEXT = {
                       "1024 U+S tokens, 6144 R tokens, 1024 candidates timed across R",
     "sl-sampler": "GPU Stochastic Length sampler on 64 users x 4096 events (alpha 1.6), d_model "
                   "512 bf16 rows gathered",
+    "long-bf16-fused": "the long-sequence workload with f2 inside the attention kernel "
+                       "(HSTU_FLAG_FUSED_F2: the last head CTA of each query tile pair runs it)",
 }
 # workloads that are another workload with a changed configuration:
 # name -> (base workload, config changes, zero the rab tables)
@@ -422,7 +424,8 @@ def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batc
     torch, H = ctx.torch, ctx.H
     from gen import algorithmic_counts
     from gen.device import case_tensors
-    case = make_workload(name, batch=batch)
+    fused = name.endswith("-fused")
+    case = make_workload(name[:-len("-fused")] if fused else name, batch=batch)
     c = case.cfg
     counts = algorithmic_counts(case)
     counts["attn_flop_per_layer"] = visible_pairs(case) * c.num_heads * (2 * c.dqk + 2 * c.dv)
@@ -434,7 +437,7 @@ def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batc
     weights = [H.LayerWeights(**lw) for lw in t["layers"]]
     cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets,
                         dqk=c.dqk, dv=c.dv, phi1=c.phi1, phi2=c.phi2, ln_eps=c.ln_eps,
-                        dtype=c.dtype)
+                        dtype=c.dtype, fused_f2=fused)
     L, T = c.num_layers, case.total_tokens
     ws = torch.empty(H.forward_workspace_bytes(cfg, L, T), dtype=torch.uint8, device=ctx.dev)
     y = torch.empty((T, c.d_model), dtype=torch.float32, device=ctx.dev)
@@ -452,12 +455,23 @@ def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batc
     value = ctx.world * T / (ms / 1000.0)
     world = ctx.world
     bf16 = c.dtype == "bf16"
-    attn_name = "attention" if bf16 else "fp32_attention"
-    roof = _roofline(ctx, kernels, attn_name, counts["attn_flop_per_layer"],
-                     "hstu_attn_kernel (causal)" if bf16 else "hstu_f32_attn_kernel (causal)",
-                     "tensor" if bf16 else "alu")
-    if roof is not None and name == "long-bf16":
-        roof["traffic"] = traffic_from_profiles("attention")
+    if bf16 and "attention_f2_fused" in kernels:
+        # the layer-fused kernel: attention plus f2 (Norm(AV) (.) U, W2, residual)
+        roof = _roofline(ctx, kernels, "attention_f2_fused",
+                         counts["attn_flop_per_layer"] + counts["f2_flop_per_layer"],
+                         "hstu_attn_kernel (causal, layer-fused f2)", "tensor")
+        if roof is not None:
+            roof["algorithmic_flop_attention"] = counts["attn_flop_per_layer"]
+            roof["algorithmic_flop_f2"] = counts["f2_flop_per_layer"]
+            if name == "long-bf16":
+                roof["traffic"] = traffic_from_profiles("attention_f2_fused")
+    else:
+        attn_name = "attention" if bf16 else "fp32_attention"
+        roof = _roofline(ctx, kernels, attn_name, counts["attn_flop_per_layer"],
+                         "hstu_attn_kernel (causal)" if bf16 else "hstu_f32_attn_kernel (causal)",
+                         "tensor" if bf16 else "alu")
+        if roof is not None and name == "long-bf16":
+            roof["traffic"] = traffic_from_profiles("attention")
     kern = _kernel_table(kernels)
     for kname, key in (("f1_gemm", "f1_flop_per_layer"), ("f2_gemm", "f2_flop_per_layer")):
         if kname in kern:
@@ -743,14 +757,15 @@ def main():
                 "kernels": r["kernels"], "gpu_launches": r["gpu_launches"],
                 "clocks": r["clocks"], "e2e": r.get("e2e"), "e2e_serial": r.get("e2e_serial")}
         if r["roofline"]:
-            line["attention"] = {"tflops": r["roofline"]["achieved"],
+            line["attention"] = {"kernel": r["roofline"]["kernel"],
+                                 "tflops": r["roofline"]["achieved"],
                                  "pct_of_bf16_peak_burst": 100 * r["roofline"]["frac"],
                                  "pct_of_bf16_peak_sustained":
                                      100 * r["roofline"].get("frac_of_sustained", 0.0)}
         if world == 1 and not args.no_workloads and args.batch is None:
             subs = {}
-            for name in ("small-bf16", "sl-bf16", "tiny-fp32", "long-bf16-softmax",
-                         "long-bf16-mtgr"):
+            for name in ("long-bf16-fused", "small-bf16", "sl-bf16", "tiny-fp32",
+                         "long-bf16-softmax", "long-bf16-mtgr"):
                 if name == args.workload:
                     continue
                 subs[name] = _public(measure_forward(ctx, name, min(args.steps, 20), args.warmup,

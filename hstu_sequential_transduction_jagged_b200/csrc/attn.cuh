@@ -71,6 +71,28 @@ constexpr uint32_t ATT_TILE_BYTES = ATT_KEYS * ATT_HD * 2;  // one K or V tile: 
 constexpr uint32_t ATT_Q_BYTES = ATT_ROWS * ATT_HD * 2;     // one Q tile: 16 KB
 constexpr int ATT_SBUF = 3;                                 // S buffers per query tile
 
+// Layer-fused f2 (causal layer path): the last of the H head CTAs of a query
+// tile pair to finish builds Norm(AV) (.) U of the pair's rows and runs
+// Y = X + (Norm(AV) (.) U) W2^T + b2 for them before it exits.
+struct TailParams {
+  int32_t* count;              // [B * num_qpairs] arrivals per tile pair, zero before the launch
+  const float* u;              // [T, ld_u] U (fp32)
+  int64_t ld_u;
+  const float* x_res;          // [T, ld_x] fp32 residual, or nullptr:
+  const __nv_bfloat16* x_lp;   //   bf16 residual
+  int64_t ld_x;
+  const float* b2;             // [N]
+  const float* gamma;          // [K] or nullptr (1)
+  const float* beta;           // [K] or nullptr (0)
+  float eps;
+  float* y;                    // [T, ld_y] fp32
+  void* y_lp;                  // [T, ld_y] fp16 (ylp_f16) or bf16 copy, or nullptr
+  int32_t ylp_f16;
+  int64_t ld_y;
+  int32_t N;                   // d_model (<= 512)
+  int32_t K;                   // H * 64 (<= 512)
+};
+
 struct AttnParams {
   const int64_t* kv_offsets;   // [B+1] key/value rows per user (query rows too in causal mode)
   const int64_t* q_offsets;    // [B+1] candidate rows per user (candidate mode)
@@ -96,6 +118,7 @@ struct AttnParams {
   uint64_t timeout_ns;
   int64_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0)
   int4 oct[32];                   // per octave k of dt+1: {t1, t2, t3, bucket(2^k - 1)}
+  TailParams tail;                // FUSED kernels only
 };
 
 // ---------------------------------------------------------------- time buckets
@@ -253,12 +276,23 @@ struct AttnSmem {
   static constexpr uint32_t kOct = kThr32 + MAX_TIME_BUCKETS * 4;    // 32 x int4
   static constexpr uint32_t kOrt = kOct + 32 * 16;                   // 32 x float4
   static constexpr uint32_t kBars = kOrt + 32 * 16;
-  static constexpr uint32_t kMisc = kBars + 32 * 8;
+  static constexpr uint32_t kMisc = kBars + 48 * 8;
   static constexpr uint32_t kLnX = kMisc + 64;                        // 2 x 128 float2
   static constexpr uint32_t kML = kLnX + 2 * ATT_ROWS * 8;           // 4 x 128 float2
   static constexpr uint32_t kPos = kML + 4 * ATT_ROWS * 8;
   // pos_len entries per copy of `elt` bytes each (fp32, or fp16 for the
   // causal fp16-operand kernel), two copies with paired reads
+  // fused f2 tail, after the attention is done: a ring of four 32 KB W2 boxes
+  // (256 rows x 64 columns, fp16) over Q, K and V, and a ring of three 16 KB
+  // A blocks (128 rows x 64 columns of Norm(AV) (.) U, fp16) after the side data
+  static constexpr uint32_t kTailBox = 256 * 64 * 2;
+  static constexpr int kTailWStages = 4;
+  static constexpr uint32_t kTailW = 0;
+  static constexpr uint32_t kTailABlock = ATT_ROWS * 128;
+  static constexpr int kTailAStages = 3;
+  static constexpr uint32_t kTailA = (kPos + 1023u) & ~1023u;
+  static constexpr uint32_t kTailBytes = kTailA + kTailAStages * kTailABlock + 1024u;  // + align slack
+  static_assert(kTailW + kTailWStages * kTailBox <= kKeyInfo, "tail W2 ring overlaps the side data");
   static constexpr uint32_t bytes(int pos_len, bool pairs, uint32_t elt = 4u) {
     return kPos + static_cast<uint32_t>(pos_len) * elt * (pairs ? 2u : 1u) + 1024u;  // + align slack
   }
@@ -273,8 +307,16 @@ enum : int {
   BAR_P_FULL = BAR_S_FULL + 2 * ATT_SBUF,  // + ATT_SBUF * group + buffer
   BAR_O_FULL = BAR_P_FULL + 2 * ATT_SBUF,  // + group
   BAR_DONE = BAR_O_FULL + 2,               // + group
-  BAR_COUNT = BAR_DONE + 2
+  // fused f2 tail
+  BAR_T_A_FULL = BAR_DONE + 2,             // + stage: an A block is built
+  BAR_T_A_EMPTY = BAR_T_A_FULL + 3,        // + stage: its MMAs completed
+  BAR_T_W_FULL = BAR_T_A_EMPTY + 3,        // + stage: a W2 box landed
+  BAR_T_W_EMPTY = BAR_T_W_FULL + 4,        // + stage: its MMAs completed
+  BAR_T_ACC_FULL = BAR_T_W_EMPTY + 4,      // the tile's accumulator is complete
+  BAR_T_DONE = BAR_T_ACC_FULL + 1,
+  BAR_COUNT = BAR_T_DONE + 1
 };
+static_assert(BAR_COUNT <= 48, "barrier slots");
 
 // ---------------------------------------------------------------- causal chunk
 
@@ -390,16 +432,259 @@ __device__ __forceinline__ void causal_chunk_pointwise(const uint32_t (&sv)[32],
   }
 }
 
+// ---------------------------------------------------------------- fused f2 tail
+
+// Y = X + (Norm(AV) (.) U) W2^T + b2 for the query rows [q0, q0 + 256) of user
+// u (rows at or past n_q are skipped), run by the whole CTA after its
+// attention, one 128-row tile after the other:
+//   element warps (threads 0..511) build the fp16 A operand one 64-column
+//     block at a time into a ring of three (all loads of a block are issued
+//     before its slot is awaited), then run the epilogue from tensor memory;
+//   the producer warp streams the fp16 W2 boxes (256 output columns x 64) by
+//     TMA through a ring of four;
+//   the first MMA warp issues, per block, the MMAs of both 256-column halves
+//     into tensor memory columns 0..N-1.
+// AV and the LayerNorm partial sums of the other heads were written by other
+// CTAs of this launch and are read through L2 (ld.global.cg).
+__device__ __forceinline__ void attn_f2_tail(const CUtensorMap* tm_w2, const AttnParams& p,
+                                             uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                                             int64_t q_start, int q0, int n_q,
+                                             const WaitCtl& ctl) {
+  const TailParams& t = p.tail;
+  const int warp = warp_id(), lane = lane_id(), tid = threadIdx.x;
+  uint8_t* sA = smem + AttnSmem::kTailA;
+  uint8_t* sW = smem + AttnSmem::kTailW;
+  float2* sStats = reinterpret_cast<float2*>(smem + AttnSmem::kLnX);
+  constexpr int kWS = AttnSmem::kTailWStages, kAS = AttnSmem::kTailAStages;
+  constexpr uint32_t kBox = AttnSmem::kTailBox, kABlk = AttnSmem::kTailABlock;
+  const int n_mt = (q0 + ATT_ROWS < n_q) ? 2 : 1;
+  const int k_blocks = t.K / 64;
+  const int halves = (t.N + 255) / 256;
+
+  if (warp == ATT_PRODUCER_WARP) {
+    if (lane == 0) {
+      tma_prefetch_desc(tm_w2);
+      int st = 0, issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int mt = 0; ok && mt < n_mt; ++mt)
+        for (int kb = 0; ok && kb < k_blocks; ++kb)
+          for (int hf = 0; hf < halves; ++hf) {
+            ok = mbar_wait(&bars[BAR_T_W_EMPTY + st], ph ^ 1u, ctl);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&bars[BAR_T_W_FULL + st], kBox);
+            tma_load_2d(sW + st * kBox, tm_w2, &bars[BAR_T_W_FULL + st], kb * 64, hf * 256);
+            ++issued;
+            if (++st == kWS) { st = 0; ph ^= 1u; }
+          }
+      // the boxes still in flight land before shared memory is released
+      for (int k = max(0, issued - kWS); k < issued; ++k)
+        mbar_wait_drain(&bars[BAR_T_W_FULL + (k % kWS)], static_cast<uint32_t>(k / kWS) & 1u,
+                        ctl.limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == ATT_MMA_WARP) {
+    const bool leader = elect_one();
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
+    };
+    int ws = 0, as = 0;
+    uint32_t wph = 0, aph = 0;
+    bool ok = true;
+    for (int mt = 0; ok && mt < n_mt; ++mt) {
+      for (int kb = 0; ok && kb < k_blocks; ++kb) {
+        ok = wait_all(&bars[BAR_T_A_FULL + as], aph);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t da = smem_desc_sw128(smem_u32(sA + as * kABlk), 16, 1024);
+        for (int hf = 0; hf < halves; ++hf) {
+          ok = wait_all(&bars[BAR_T_W_FULL + ws], wph);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dw = smem_desc_sw128(smem_u32(sW + ws * kBox), 16, 1024);
+          const int n = min(256, t.N - hf * 256);
+          const uint32_t idesc = idesc_16_f32(ATT_ROWS, n, false, false, true);
+          if (leader) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + static_cast<uint32_t>(hf * 256), da + 2 * kk, dw + 2 * kk, idesc,
+                          (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&bars[BAR_T_W_EMPTY + ws]);
+          }
+          __syncwarp();
+          if (++ws == kWS) { ws = 0; wph ^= 1u; }
+        }
+        if (leader) mma_commit(&bars[BAR_T_A_EMPTY + as]);
+        __syncwarp();
+        if (++as == kAS) { as = 0; aph ^= 1u; }
+      }
+      if (ok && leader) mma_commit(&bars[BAR_T_ACC_FULL]);
+      __syncwarp();
+    }
+    if (leader) mma_commit(&bars[BAR_T_DONE]);
+    __syncwarp();
+    mbar_wait_drain(&bars[BAR_T_DONE], 0, ctl.limit_ns);
+  } else if (tid < 16 * 32) {
+    const float inv_k = 1.0f / static_cast<float>(t.K);
+    const int q4 = warp & 3;    // tensor-memory lane quarter
+    const int cg = warp >> 2;   // 128-column group of the epilogue
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    int as = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    for (int mt = 0; mt < n_mt; ++mt) {
+      const int base = q0 + mt * ATT_ROWS;
+      // per-row LayerNorm statistics from the heads' partial sums
+      if (tid < ATT_ROWS) {
+        float mean = 0.0f, rstd = 0.0f;
+        if (base + tid < n_q) {
+          const float2* lp = reinterpret_cast<const float2*>(p.ln_part) + (q_start + base + tid) * p.H;
+          float tot = 0.0f;
+          for (int hh = 0; hh < p.H; ++hh) tot += __ldcg(&lp[hh].x);
+          mean = tot * inv_k;
+          float m2 = 0.0f;
+          for (int hh = 0; hh < p.H; ++hh) {
+            const float2 v = __ldcg(&lp[hh]);
+            const float dm = v.x * (1.0f / 64.0f) - mean;
+            m2 += v.y + 64.0f * dm * dm;
+          }
+          rstd = rsqrtf(m2 * inv_k + t.eps);
+        }
+        sStats[tid] = make_float2(mean, rstd);
+      }
+      named_barrier_sync(3, 16 * 32);
+      // A blocks: 128 rows x 8 chunks of 8 columns; this thread's two chunks
+      // (rows tid/8 and tid/8 + 64, chunk tid%8) of every block
+      const int j = tid & 7;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        const int col = kb * 64 + j * 8;
+        float4 av[2][2], uv[2][2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int r = (tid >> 3) + h2 * 64;
+          if (base + r < n_q) {
+            const int64_t row = q_start + base + r;
+            const float4* ap = reinterpret_cast<const float4*>(p.av_f32 + row * p.ld_av + col);
+            const float4* up = reinterpret_cast<const float4*>(t.u + row * t.ld_u + col);
+            av[h2][0] = __ldcg(ap);
+            av[h2][1] = __ldcg(ap + 1);
+            uv[h2][0] = up[0];
+            uv[h2][1] = up[1];
+          } else {
+            av[h2][0] = av[h2][1] = uv[h2][0] = uv[h2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float gm[8], bt[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          gm[e] = t.gamma != nullptr ? __ldg(t.gamma + col + e) : 1.0f;
+          bt[e] = t.beta != nullptr ? __ldg(t.beta + col + e) : 0.0f;
+        }
+        if (ok) ok = mbar_wait(&bars[BAR_T_A_EMPTY + as], aph ^ 1u, ctl);
+        uint8_t* blk = sA + as * kABlk;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int r = (tid >> 3) + h2 * 64;
+          const float2 sr = sStats[r];
+          const float af[8] = {av[h2][0].x, av[h2][0].y, av[h2][0].z, av[h2][0].w,
+                               av[h2][1].x, av[h2][1].y, av[h2][1].z, av[h2][1].w};
+          const float uf[8] = {uv[h2][0].x, uv[h2][0].y, uv[h2][0].z, uv[h2][0].w,
+                               uv[h2][1].x, uv[h2][1].y, uv[h2][1].z, uv[h2][1].w};
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g0 = fmaf((af[2 * e] - sr.x) * sr.y, gm[2 * e], bt[2 * e]) * uf[2 * e];
+            const float g1 =
+                fmaf((af[2 * e + 1] - sr.x) * sr.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
+            w[e] = pack_h2(g0, g1);
+          }
+          // rows past the end carry zeros (their statistics and data are zero)
+          if (ok)
+            *reinterpret_cast<uint4*>(blk + r * 128 + ((j ^ (r & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();  // the previous tile's tensor-memory reads, before the MMAs reuse it
+        mbar_arrive(&bars[BAR_T_A_FULL + as]);
+        if (++as == kAS) { as = 0; aph ^= 1u; }
+      }
+      // epilogue: + b2 + residual -> Y (fp32) and its 16-bit copy
+      if (ok) ok = mbar_wait(&bars[BAR_T_ACC_FULL], static_cast<uint32_t>(mt) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;  // keep arriving: the other threads' barriers stay consistent
+      tc_fence_after();
+      const int r = q4 * 32 + lane;
+      const bool row_ok = base + r < n_q;
+      const int64_t row = q_start + base + r;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        const int col = cg * 128 + ch * 32;
+        if (col >= t.N) break;  // warp-uniform
+        float4 xr[8];
+        if (row_ok) {
+          if (t.x_res != nullptr) {
+            const float4* xp = reinterpret_cast<const float4*>(t.x_res + row * t.ld_x + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xr[q] = xp[q];
+          } else {
+            const uint4* xp = reinterpret_cast<const uint4*>(t.x_lp + row * t.ld_x + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 xx = xp[q];
+              const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xx);
+              const float2 f0 = __bfloat1622float2(x2[0]), f1 = __bfloat1622float2(x2[1]);
+              const float2 f2 = __bfloat1622float2(x2[2]), f3 = __bfloat1622float2(x2[3]);
+              xr[2 * q] = make_float4(f0.x, f0.y, f1.x, f1.y);
+              xr[2 * q + 1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+            }
+          }
+        }
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(col), v);
+        tmem_ld_wait(v);
+        if (!row_ok) continue;
+        // accumulator + b2 + residual, in the order of the unfused f2 epilogue
+        float y[32];
+        const float4* b4 = reinterpret_cast<const float4*>(t.b2 + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = __ldg(b4 + q);
+          y[4 * q + 0] = __uint_as_float(v[4 * q + 0]) + bb.x + xr[q].x;
+          y[4 * q + 1] = __uint_as_float(v[4 * q + 1]) + bb.y + xr[q].y;
+          y[4 * q + 2] = __uint_as_float(v[4 * q + 2]) + bb.z + xr[q].z;
+          y[4 * q + 3] = __uint_as_float(v[4 * q + 3]) + bb.w + xr[q].w;
+        }
+        float4* yo = reinterpret_cast<float4*>(t.y + row * t.ld_y + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) yo[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+        if (t.y_lp != nullptr) {
+          uint4* lo = reinterpret_cast<uint4*>(static_cast<uint16_t*>(t.y_lp) + row * t.ld_y + col);
+          const bool h16 = t.ylp_f16 != 0;
+          auto pk2 = [h16](float a, float b) { return h16 ? pack_h2(a, b) : pack_bf16x2(a, b); };
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            lo[q] = make_uint4(pk2(y[8 * q], y[8 * q + 1]), pk2(y[8 * q + 2], y[8 * q + 3]),
+                               pk2(y[8 * q + 4], y[8 * q + 5]), pk2(y[8 * q + 6], y[8 * q + 7]));
+        }
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- kernel
 
 // F16: Q, K, V (and so P) are fp16 instead of bf16.  The causal element math
 // is fp32 either way; candidate mode with fp16 operands runs it on packed fp16
 // pairs (its per-key bias is precomputed, so the chain is short).
-template <bool CAND, int PHI, bool PAIRS, bool F16>
+// FUSED (causal mode only): the last head CTA of each query tile pair runs
+// the layer's f2 for the pair's rows (attn_f2_tail; tm_w2 maps the fp16 W2).
+template <bool CAND, int PHI, bool PAIRS, bool F16, bool FUSED>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w2,
                  const __grid_constant__ AttnParams p) {
+  static_assert(!(CAND && FUSED), "the fused f2 tail is for the causal layer path");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -535,6 +820,18 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bars[BAR_O_FULL + g], 1);
       mbar_init(&bars[BAR_DONE + g], 1);
+    }
+    if constexpr (FUSED) {
+      for (int st = 0; st < AttnSmem::kTailAStages; ++st) {
+        mbar_init(&bars[BAR_T_A_FULL + st], 16 * 32);  // every element thread
+        mbar_init(&bars[BAR_T_A_EMPTY + st], 1);
+      }
+      for (int st = 0; st < AttnSmem::kTailWStages; ++st) {
+        mbar_init(&bars[BAR_T_W_FULL + st], 1);
+        mbar_init(&bars[BAR_T_W_EMPTY + st], 1);
+      }
+      mbar_init(&bars[BAR_T_ACC_FULL], 1);
+      mbar_init(&bars[BAR_T_DONE], 1);
     }
     *sAbort = 0;
     fence_mbar_init();
@@ -1137,6 +1434,26 @@ hstu_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float dm = (hsum - other.x) * (1.0f / HC);
       float2* lp = reinterpret_cast<float2*>(p.ln_part + (row * p.H + h) * 2);
       *lp = make_float2(hsum + other.x, hm2 + other.y + dm * dm * (HC * HC / (2.0f * HC)));
+    }
+  }
+
+  if constexpr (FUSED) {
+    // The pair's AV rows and LayerNorm partial sums of this head are written;
+    // the CTA that completes the pair's H arrivals runs f2 for its rows.
+    __threadfence();
+    tc_fence_before();
+    __syncthreads();
+    volatile int* sLast = reinterpret_cast<volatile int*>(smem + AttnSmem::kMisc + 8);
+    if (tid == 0) {
+      // one counter per query tile pair, indexed by the pair's first row (< T)
+      const int old = atomicAdd(&p.tail.count[q_start + q0], 1);
+      *sLast = (old == p.H - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (*sLast) {
+      __threadfence();
+      tc_fence_after();
+      attn_f2_tail(&tm_w2, p, smem, bars, tmem, q_start, q0, n_q, ctl);
     }
   }
 

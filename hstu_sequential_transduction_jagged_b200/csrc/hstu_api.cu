@@ -102,12 +102,13 @@ const int64_t* thresholds_for(int Tb) {
 
 enum KernelKind : int {
   K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT,
-  K_SL, K_SL_GATHER, K_COUNT
+  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
                                            "fp32_attention",    "fp32_ln_gate", "weight_cvt",
-                                           "sl_select",         "sl_gather"};
+                                           "sl_select",         "sl_gather",
+                                           "attention_f2_fused"};
 
 struct Profiler {
   std::mutex mu;
@@ -160,26 +161,33 @@ class ProfScope {
 // ------------------------------------------------------------------ device info
 
 using AttnKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                             const AttnParams);
+                             const CUtensorMap, const AttnParams);
 
-template <bool CAND, bool PAIRS, bool F16>
+template <bool CAND, bool PAIRS, bool F16, bool FUSED>
 AttnKernelFn attn_kernel_for(int phi) {
   switch (phi) {
-    case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS, F16>;
-    case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS, F16>;
-    case HSTU_ACT_SOFTMAX: return hstu_attn_kernel<CAND, HSTU_ACT_SOFTMAX, PAIRS, F16>;
-    default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS, F16>;
+    case HSTU_ACT_SILU: return hstu_attn_kernel<CAND, HSTU_ACT_SILU, PAIRS, F16, FUSED>;
+    case HSTU_ACT_RELU: return hstu_attn_kernel<CAND, HSTU_ACT_RELU, PAIRS, F16, FUSED>;
+    case HSTU_ACT_SOFTMAX: return hstu_attn_kernel<CAND, HSTU_ACT_SOFTMAX, PAIRS, F16, FUSED>;
+    default: return hstu_attn_kernel<CAND, HSTU_ACT_IDENTITY, PAIRS, F16, FUSED>;
   }
 }
 
 template <bool F16>
 AttnKernelFn attn_kernel_ptr_t(bool cand, int phi, bool pairs) {
   if (cand)
-    return pairs ? attn_kernel_for<true, true, F16>(phi) : attn_kernel_for<true, false, F16>(phi);
-  return pairs ? attn_kernel_for<false, true, F16>(phi) : attn_kernel_for<false, false, F16>(phi);
+    return pairs ? attn_kernel_for<true, true, F16, false>(phi)
+                 : attn_kernel_for<true, false, F16, false>(phi);
+  return pairs ? attn_kernel_for<false, true, F16, false>(phi)
+               : attn_kernel_for<false, false, F16, false>(phi);
 }
 
-AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16) {
+// The layer-fused form exists for the causal kernel with fp16 operands (the
+// bf16 layer path).
+AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16, bool fused = false) {
+  if (fused)
+    return pairs ? attn_kernel_for<false, true, true, true>(phi)
+                 : attn_kernel_for<false, false, true, true>(phi);
   return f16 ? attn_kernel_ptr_t<true>(cand, phi, pairs) : attn_kernel_ptr_t<false>(cand, phi, pairs);
 }
 
@@ -208,6 +216,10 @@ hstu_status_t device_info(DeviceInfo** out) {
             HSTU_CHECK_CUDA(cudaFuncSetAttribute(
                 attn_kernel_ptr(cand != 0, phi, pairs != 0, f16 != 0),
                 cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    for (int phi = 0; phi < 4; ++phi)
+      for (int pairs = 0; pairs < 2; ++pairs)
+        HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(false, phi, pairs != 0, true, true),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
     const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
@@ -303,6 +315,7 @@ hstu_status_t check_cfg(const hstu_layer_cfg_t* c) {
   if (c->dtype != HSTU_BF16 && c->dtype != HSTU_FP32 && c->dtype != HSTU_FP16)
     return HSTU_ERR_INVALID_ARGUMENT;
   if (!(c->ln_eps >= 0.0f)) return HSTU_ERR_INVALID_ARGUMENT;
+  if ((c->flags & ~HSTU_FLAG_FUSED_F2) != 0) return HSTU_ERR_INVALID_ARGUMENT;
   if (c->dqk != ATT_HD || c->dv != ATT_HD) return HSTU_ERR_UNSUPPORTED;
   if (c->d_model % 64 != 0) return HSTU_ERR_UNSUPPORTED;
   if (c->num_pos_buckets > kMaxPos || c->num_time_buckets > MAX_TIME_BUCKETS)
@@ -353,6 +366,7 @@ struct LayerWs {
   __half* w1h;  // bf16 path: fp16 W1
   __half* w2h;  // bf16 path: fp16 W2
   __half* x16;  // bf16 path: fp16 copy of the fp32 layer input (x_in = NULL)
+  int32_t* count;  // bf16 path: [T] arrivals per query tile pair of the fused f2 tail
 };
 
 size_t weights_f16_bytes(const hstu_layer_cfg_t* c) {
@@ -367,7 +381,7 @@ size_t layer_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
   if (c->dtype == HSTU_BF16)
     return align_up(t * 3 * hv * 2, 256) + 2 * align_up(t * hv * 4, 256) +
            align_up(t * c->num_heads * 2 * sizeof(float), 256) + weights_f16_bytes(c) +
-           align_up(t * static_cast<size_t>(c->d_model) * 2, 256);
+           align_up(t * static_cast<size_t>(c->d_model) * 2, 256) + align_up(t * 4, 256);
   return align_up(t * n1_of(c) * 4, 256) + 2 * align_up(t * hv * 4, 256);
 }
 
@@ -389,6 +403,7 @@ LayerWs carve_layer(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
   p += align_up(t * hv * 4, 256);
   w.extra = p;
   w.w1h = w.w2h = w.x16 = nullptr;
+  w.count = nullptr;
   if (c->dtype == HSTU_BF16) {
     p += align_up(t * c->num_heads * 2 * sizeof(float), 256);
     w.w1h = reinterpret_cast<__half*>(p);
@@ -396,6 +411,8 @@ LayerWs carve_layer(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
     w.w2h = reinterpret_cast<__half*>(p);
     p += align_up(static_cast<size_t>(c->d_model) * hv * 2, 256);
     w.x16 = reinterpret_cast<__half*>(p);
+    p += align_up(t * static_cast<size_t>(c->d_model) * 2, 256);
+    w.count = reinterpret_cast<int32_t*>(p);
   }
   return w;
 }
@@ -453,6 +470,10 @@ struct AttnJob {
   float* ln_part;
   uint64_t timeout_ns;
   bool f16;                     // Q, K, V (and P) in fp16 instead of bf16
+  // layer-fused f2 (causal, f16): tail.count is [T_q] and zeroed here; w2h is
+  // the fp16 W2 [d, H*64]
+  const TailParams* tail = nullptr;
+  const void* w2h = nullptr;
 };
 
 // Tensor-core attention over 16-bit operands (bf16, or fp16 when j.f16).
@@ -463,7 +484,7 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   DeviceInfo* di = nullptr;
   hstu_status_t s = device_info(&di);
   if (s != HSTU_OK) return s;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mw;
   const int64_t hc = static_cast<int64_t>(c->num_heads) * ATT_HD;
   if ((s = make_map_16(&mq, j.q, j.T_q, hc, j.ldq, ATT_HD, ATT_ROWS, j.f16)) != HSTU_OK) return s;
   // with no key rows at all (every history empty) no K/V tile is ever loaded;
@@ -475,8 +496,20 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   if ((s = make_map_16(&mv, no_kv ? j.q : j.v, no_kv ? j.T_q : j.T_kv, hc,
                        no_kv ? j.ldq : j.ldv, ATT_HD, ATT_KEYS, j.f16)) != HSTU_OK)
     return s;
+  const bool fused = !CAND && j.tail != nullptr;
+  if (fused) {
+    if (!j.f16 || j.av_f32 == nullptr || j.ln_part == nullptr || j.w2h == nullptr ||
+        j.tail->N > 512 || j.tail->K != hc || hc > 512)
+      return HSTU_ERR_UNSUPPORTED;
+    if ((s = make_map_16(&mw, j.w2h, j.tail->N, hc, hc, 64, 256, true)) != HSTU_OK) return s;
+    // one arrival counter per query tile pair, indexed by the pair's first row
+    HSTU_CHECK_CUDA(cudaMemsetAsync(j.tail->count, 0, static_cast<size_t>(j.T_q) * sizeof(int32_t), st));
+  } else {
+    mw = mq;  // unused
+  }
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
+  if (fused) p.tail = *j.tail;
   p.kv_offsets = j.kv_offsets;
   p.q_offsets = j.q_offsets;
   p.timestamps = j.timestamps;
@@ -526,10 +559,12 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   if (!compute_octaves(c->num_time_buckets, p.thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
   dim3 grid(c->num_heads, j.batch, p.num_qpairs);
   const bool pairs = AttnSmem::bytes(p.pos_len, true, pos_elt) <= 227u * 1024u;
-  const size_t smem = AttnSmem::bytes(p.pos_len, pairs, pos_elt);
+  size_t smem = AttnSmem::bytes(p.pos_len, pairs, pos_elt);
+  if (fused) smem = std::max<size_t>(smem, AttnSmem::kTailBytes);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
-  ProfScope prof(CAND ? K_CAND_ATTN : K_ATTN, st);
-  attn_kernel_ptr(CAND, c->phi2, pairs, j.f16)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv, p);
+  ProfScope prof(CAND ? K_CAND_ATTN : (fused ? K_ATTN_FUSED : K_ATTN), st);
+  attn_kernel_ptr(CAND, c->phi2, pairs, j.f16, fused)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv,
+                                                                                       mw, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
   return HSTU_OK;
 }
@@ -809,6 +844,33 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
   j.ld_av = hv;
   j.ln_part = static_cast<float*>(ws.extra);
   j.f16 = true;
+  // on request, causal layers with d <= 512 and H * 64 <= 512 run f2 inside
+  // the attention kernel (the tail of the last head CTA of each query tile pair)
+  const bool fused = !cand && (c->flags & HSTU_FLAG_FUSED_F2) != 0 && c->d_model <= 512 &&
+                     hv <= 512;
+  if (fused) {
+    TailParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.count = ws.count;
+    tp.u = ws.u;
+    tp.ld_u = hv;
+    tp.x_res = x_res;
+    tp.x_lp = static_cast<const __nv_bfloat16*>(x_in);
+    tp.ld_x = d;
+    tp.b2 = w->b2;
+    tp.gamma = w->ln_gamma;
+    tp.beta = w->ln_beta;
+    tp.eps = c->ln_eps;
+    tp.y = y_out;
+    tp.y_lp = y_lp;
+    tp.ylp_f16 = ylp_f16 ? 1 : 0;
+    tp.ld_y = d;
+    tp.N = c->d_model;
+    tp.K = static_cast<int32_t>(hv);
+    j.tail = &tp;
+    j.w2h = ws.w2h;
+    return launch_attn_tc<false>(j, st);
+  }
   s = cand ? launch_attn_tc<true>(j, st) : launch_attn_tc<false>(j, st);
   if (s != HSTU_OK) return s;
   return launch_f2_bf16(c, w, ws.w2h, true, static_cast<const float*>(ws.av), hv, ws.u, hv,

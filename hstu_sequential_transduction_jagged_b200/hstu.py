@@ -40,12 +40,15 @@ class JaggedT(ctypes.Structure):
                 ("max_static", ctypes.c_int32)]
 
 
+FLAG_FUSED_F2 = 1
+
+
 class LayerCfgT(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int32), ("num_heads", ctypes.c_int32),
                 ("dqk", ctypes.c_int32), ("dv", ctypes.c_int32),
                 ("num_pos_buckets", ctypes.c_int32), ("num_time_buckets", ctypes.c_int32),
                 ("phi1", ctypes.c_int32), ("phi2", ctypes.c_int32), ("ln_eps", ctypes.c_float),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 class KernelTimeT(ctypes.Structure):
@@ -137,11 +140,12 @@ class LayerConfig:
     phi2: str = "silu"
     ln_eps: float = 1e-5
     dtype: str = "bf16"
+    fused_f2: bool = False  # True sets HSTU_FLAG_FUSED_F2
 
     def c(self) -> LayerCfgT:
         return LayerCfgT(self.d_model, self.num_heads, self.dqk, self.dv, self.num_pos_buckets,
                          self.num_time_buckets, ACT[self.phi1], ACT[self.phi2], self.ln_eps,
-                         DTYPE[self.dtype])
+                         DTYPE[self.dtype], FLAG_FUSED_F2 if self.fused_f2 else 0)
 
     @property
     def torch_dtype(self):

@@ -125,7 +125,20 @@ typedef struct {
   int32_t phi2;               /* hstu_act_t, SiLU by default (or SOFTMAX) */
   float ln_eps;               /* LayerNorm epsilon (1e-5) */
   int32_t dtype;              /* hstu_dtype_t of X, W1, W2 and all bf16 intermediates */
+  int32_t flags;              /* HSTU_FLAG_* bits, 0 by default */
 } hstu_layer_cfg_t;
+
+/* cfg.flags.  HSTU_FLAG_FUSED_F2: the causal bf16 layer (hstu_layer_fwd,
+ * hstu_forward, hstu_layer_fwd_static) runs f2 inside the attention kernel
+ * when d_model <= 512 and num_heads * dv <= 512: the last of a query tile
+ * pair's H head CTAs to finish builds Norm(AV) (.) U for the pair's 256 rows
+ * and computes their Y = X + f2(...), reading AV and U back through L2.  The
+ * results are bit-identical to the default form, which runs f2 as its own
+ * kernel after the attention kernel; on B200 at d_model 512 the default form
+ * is the faster one (the fused tail runs on one SM per tile pair and is bound
+ * by that SM's memory latency).  M-FALCON candidate layers always run f2 as
+ * its own kernel. */
+#define HSTU_FLAG_FUSED_F2 1
 
 /* Weights of one layer (all device pointers). */
 typedef struct {
