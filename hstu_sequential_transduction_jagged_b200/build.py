@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhstu.so")
 SOURCES = ["hstu_api.cu"]
-HEADERS = ["ptx.cuh", "status.cuh", "attn.cuh", "gemm.cuh", "fp32_path.cuh", "sl.cuh"]
+HEADERS = ["ptx.cuh", "status.cuh", "attn.cuh", "attn_bwd.cuh", "gemm.cuh", "fp32_path.cuh",
+           "sl.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,0 +1,427 @@
+// Backward of the causal pointwise attention (Eq. 2 of the review of "Actions
+// Speak Louder than Words", section 三 核心公式, differentiated):
+//   S = Q K^T + rab,  A = phi2(S) / N (visible pairs j <= i),  O = A V
+//   dV = A^T dO,  dS = (dO V^T) (.) phi2'(S) / N,  dQ = dS K,  dK = dS^T Q,
+//   drab_pos[h, min(i-j, P-1)] += dS_ij,  drab_time[h, bt(t_i - t_j)] += dS_ij.
+//
+// Two tcgen05 kernels over fp16 Q, K, V, dO (fp32 accumulation in tensor
+// memory, fp32 outputs):
+//   hstu_attn_bwd_kv_kernel: one CTA per (head, user, 128-key tile) walks the
+//     query tiles at and after its keys: S^T = K Q^T and dP^T = V dO^T into
+//     tensor memory, the element warps turn them into P^T and dS^T (fp16,
+//     over the columns they read), then dV += P^T dO and dK += dS^T Q
+//     accumulate in tensor memory.  The table gradients collect in shared
+//     memory (position: one shared atomic per pair; time: a running sum per
+//     row, flushed when the bucket changes) and go to global memory with one
+//     atomic per touched entry at the end.
+//   hstu_attn_bwd_q_kernel: one CTA per (head, user, 128-query tile) walks the
+//     key tiles up to its diagonal: S = Q K^T and dP = dO V^T, dS by the
+//     element warps, dQ += dS K.
+// Warp roles (320 threads): warps 0-7 element work (thread = one row of the
+// tile: lane quarter warp & 3, 64-column half warp >> 2), warp 8 TMA
+// producer, warp 9 MMA issue (one elected lane).  Every wait is bounded.
+#pragma once
+
+#include "attn.cuh"
+
+namespace hstu {
+
+constexpr int BW_ROWS = 128;          // rows of the tile the CTA owns
+constexpr int BW_COLS = 128;          // rows of each streamed tile
+constexpr int BW_THREADS = 320;
+constexpr int BW_PRODUCER_WARP = 8;
+constexpr int BW_MMA_WARP = 9;
+constexpr uint32_t BW_TILE_BYTES = 128 * ATT_HD * 2;  // one 128 x 64 fp16 tile: 16 KB
+
+struct AttnBwdParams {
+  const int64_t* offsets;      // [B+1]
+  const int64_t* timestamps;   // [T]
+  const float* rab_pos;        // [H, P]
+  const float* rab_time;       // [H, Tb]
+  float* dq;                   // [T, ld_g] fp32 (head h at columns h*64)
+  float* dk;
+  float* dv;
+  int64_t ld_g;
+  float* drab_pos;             // [H, P] fp32, accumulated into (caller zeroes)
+  float* drab_time;            // [H, Tb]
+  int32_t B, H, P, Tb, max_len;
+  int32_t phi2;
+  int32_t hist_len;            // position-gradient entries kept in shared memory
+  uint64_t timeout_ns;
+  int4 oct[32];                // time-bucket octave table (see time_bucket_octave)
+};
+
+struct BwSmem {
+  static constexpr uint32_t kOwn0 = 0;                      // K (kv kernel) or Q (q kernel)
+  static constexpr uint32_t kOwn1 = kOwn0 + BW_TILE_BYTES;  // V or dO
+  static constexpr uint32_t kStg = kOwn1 + BW_TILE_BYTES;   // 2 stages x (2 tiles)
+  static constexpr uint32_t kStgBytes = 2 * BW_TILE_BYTES;
+  static constexpr uint32_t kTimes = kStg + 2 * kStgBytes;  // 2 x 128 int32 (streamed rows)
+  static constexpr uint32_t kOct = kTimes + 2 * 128 * 4;    // 32 x int4
+  static constexpr uint32_t kRt = kOct + 32 * 16;           // Tb floats (rab_time row)
+  static constexpr uint32_t kTg = kRt + MAX_TIME_BUCKETS * 4;   // Tb floats (time gradient)
+  static constexpr uint32_t kBars = kTg + MAX_TIME_BUCKETS * 4; // 16 barriers
+  static constexpr uint32_t kMisc = kBars + 16 * 8;
+  static constexpr uint32_t kPg = kMisc + 64;               // hist_len floats (position gradient)
+  static constexpr uint32_t bytes(int hist_len) {
+    return kPg + static_cast<uint32_t>(hist_len) * 4u + 1024u;
+  }
+};
+
+enum : int {
+  BWB_OWN = 0,          // the CTA's own two tiles landed
+  BWB_FULL = 1,         // + stage
+  BWB_EMPTY = 3,        // + stage
+  BWB_S = 5,            // S and dP of the current tile are in tensor memory
+  BWB_P = 6,            // the element warps wrote P / dS
+  BWB_DONE = 7,         // every MMA completed
+  BWB_COUNT = 8
+};
+
+// phi2 and its derivative at s (pointwise modes)
+template <int PHI>
+__device__ __forceinline__ void phi_and_grad(float s, float& p, float& g) {
+  if constexpr (PHI == HSTU_ACT_SILU) {
+    const float sg = fmaf(0.5f, tanh_approx(0.5f * s), 0.5f);  // sigmoid(s)
+    p = s * sg;
+    g = sg * fmaf(s, 1.0f - sg, 1.0f);
+  } else if constexpr (PHI == HSTU_ACT_RELU) {
+    p = fmaxf(s, 0.0f);
+    g = s > 0.0f ? 1.0f : 0.0f;
+  } else {
+    p = s;
+    g = 1.0f;
+  }
+}
+
+// Seconds since the user's first event (int32, clamped; the span check is
+// made once per CTA).
+__device__ __forceinline__ int32_t bw_rel_time(const int64_t* ts, int64_t row, int64_t t_first) {
+  const int64_t d = ts[row] - t_first;
+  return d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d);
+}
+
+// KV = true: the dK/dV kernel (own tile = keys, streamed = queries at and
+// after the keys).  KV = false: the dQ kernel (own tile = queries, streamed =
+// keys up to the diagonal).  F16: fp16 operands (else bf16); P and dS are
+// packed in the operand type.
+template <bool KV, int PHI, bool F16>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ AttnBwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int h = blockIdx.x, u = blockIdx.y;
+  // longest work first: key tile 0 meets every query tile, query tile z meets z + 1 key tiles
+  const int ot = KV ? static_cast<int>(blockIdx.z)
+                    : static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);
+  const int64_t start = p.offsets[u];
+  const int n = static_cast<int>(p.offsets[u + 1] - start);
+  if (n > p.max_len || n < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_status(HSTU_ERR_DEVICE_CHECK);
+    return;
+  }
+  const int o0 = ot * BW_ROWS;  // first row (within the user) of the own tile
+  if (o0 >= n) return;          // uniform, before any allocation
+  const int n_tiles = (n + BW_COLS - 1) / BW_COLS;
+  // streamed tiles: queries ot .. n_tiles-1 (KV) or keys 0 .. ot (Q)
+  const int st0 = KV ? ot : 0;
+  const int n_st = KV ? n_tiles - ot : ot + 1;
+
+  uint8_t* sOwn0 = smem + BwSmem::kOwn0;
+  uint8_t* sOwn1 = smem + BwSmem::kOwn1;
+  uint8_t* sStg = smem + BwSmem::kStg;
+  int32_t* sTimes = reinterpret_cast<int32_t*>(smem + BwSmem::kTimes);
+  int4* sOct = reinterpret_cast<int4*>(smem + BwSmem::kOct);
+  float* sRt = reinterpret_cast<float*>(smem + BwSmem::kRt);
+  float* sTg = reinterpret_cast<float*>(smem + BwSmem::kTg);
+  float* sPg = reinterpret_cast<float*>(smem + BwSmem::kPg);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BwSmem::kBars);
+  uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + BwSmem::kMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + BwSmem::kMisc + 4);
+  const int warp = warp_id(), lane = lane_id(), tid = threadIdx.x;
+  const int64_t t_first = p.timestamps[start];
+  if (tid == 0 && p.timestamps[start + n - 1] - t_first >= static_cast<int64_t>(INT32_MAX) - 1)
+    record_status(HSTU_ERR_DEVICE_CHECK);
+
+  if (tid == 0) {
+    mbar_init(&bars[BWB_OWN], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[BWB_FULL + s], 1);
+      mbar_init(&bars[BWB_EMPTY + s], 1);
+    }
+    mbar_init(&bars[BWB_S], 1);
+    mbar_init(&bars[BWB_P], 8 * 32);
+    mbar_init(&bars[BWB_DONE], 1);
+    *sAbort = 0;
+    fence_mbar_init();
+  }
+  if (warp == BW_MMA_WARP) {
+    tmem_alloc(sTmemBase, 512);
+    tmem_relinquish();
+  }
+  if (tid < 32) sOct[tid] = p.oct[tid];
+  for (int k = tid; k < p.Tb; k += BW_THREADS) {
+    sRt[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
+    if (KV) sTg[k] = 0.0f;
+  }
+  if (KV)
+    for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmemBase;
+  const WaitCtl ctl{sAbort, p.timeout_ns};
+  // tensor memory: X = S^T or S (columns 0-127, later the packed P^T / dS
+  // over them), Y = dP^T or dP (128-255), acc0 (256-319), acc1 (320-383)
+  constexpr uint32_t kX = 0, kY = 128, kAcc0 = 256, kAcc1 = 320;
+
+  if (warp == BW_PRODUCER_WARP) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const int32_t orow = static_cast<int32_t>(start + o0);
+      mbar_arrive_expect_tx(&bars[BWB_OWN], 2 * BW_TILE_BYTES);
+      if (KV) {
+        tma_load_2d(sOwn0, &tm_k, &bars[BWB_OWN], h * ATT_HD, orow);
+        tma_load_2d(sOwn1, &tm_v, &bars[BWB_OWN], h * ATT_HD, orow);
+      } else {
+        tma_load_2d(sOwn0, &tm_q, &bars[BWB_OWN], h * ATT_HD, orow);
+        tma_load_2d(sOwn1, &tm_do, &bars[BWB_OWN], h * ATT_HD, orow);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_st; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&bars[BWB_EMPTY + s], ((it >> 1) & 1) ^ 1u, ctl)) break;
+        const int32_t row = static_cast<int32_t>(start + (st0 + it) * BW_COLS);
+        uint8_t* dst = sStg + s * BwSmem::kStgBytes;
+        mbar_arrive_expect_tx(&bars[BWB_FULL + s], 2 * BW_TILE_BYTES);
+        if (KV) {
+          tma_load_2d(dst, &tm_q, &bars[BWB_FULL + s], h * ATT_HD, row);
+          tma_load_2d(dst + BW_TILE_BYTES, &tm_do, &bars[BWB_FULL + s], h * ATT_HD, row);
+        } else {
+          tma_load_2d(dst, &tm_k, &bars[BWB_FULL + s], h * ATT_HD, row);
+          tma_load_2d(dst + BW_TILE_BYTES, &tm_v, &bars[BWB_FULL + s], h * ATT_HD, row);
+        }
+        ++issued;
+      }
+      // every load lands before shared memory is released
+      mbar_wait_drain(&bars[BWB_OWN], 0, p.timeout_ns);
+      for (int it = max(0, issued - 2); it < issued; ++it)
+        mbar_wait_drain(&bars[BWB_FULL + (it & 1)], static_cast<uint32_t>(it >> 1) & 1u, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == BW_MMA_WARP) {
+    const bool leader = elect_one();
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
+    };
+    constexpr uint32_t idesc_ss = idesc_16_f32(BW_ROWS, BW_COLS, false, false, F16);
+    constexpr uint32_t idesc_ts = idesc_16_f32(BW_ROWS, ATT_HD, false, true, F16);
+    const uint64_t dOwn0 = smem_desc_sw128(smem_u32(sOwn0), 16, 1024);
+    const uint64_t dOwn1 = smem_desc_sw128(smem_u32(sOwn1), 16, 1024);
+    bool ok = wait_all(&bars[BWB_OWN], 0);
+    tc_fence_after();
+    for (int it = 0; ok && it < n_st; ++it) {
+      const int s = it & 1;
+      ok = wait_all(&bars[BWB_FULL + s], (it >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(sStg + s * BwSmem::kStgBytes);
+      const uint64_t dS0k = smem_desc_sw128(sa, 16, 1024);                  // streamed tile 0, K-major
+      const uint64_t dS1k = smem_desc_sw128(sa + BW_TILE_BYTES, 16, 1024);  // streamed tile 1, K-major
+      if (leader) {
+        // X = own0 streamed0^T, Y = own1 streamed1^T (K = 64: four steps)
+#pragma unroll
+        for (int kk = 0; kk < ATT_HD / 16; ++kk)
+          mma_bf16_ss(tmem + kX, dOwn0 + 2 * kk, dS0k + 2 * kk, idesc_ss, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < ATT_HD / 16; ++kk)
+          mma_bf16_ss(tmem + kY, dOwn1 + 2 * kk, dS1k + 2 * kk, idesc_ss, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[BWB_S]);
+      }
+      __syncwarp();
+      ok = wait_all(&bars[BWB_P], static_cast<uint32_t>(it) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      // accumulate over the 128 streamed rows (K = 128: eight steps); the
+      // packed 16-bit operand of rows 0-63 sits at columns 0-31 of its
+      // region, rows 64-127 at columns 64-95
+      const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                // MN-major B
+      const uint64_t dS1m = smem_desc_sw128(sa + BW_TILE_BYTES, 8192, 1024);
+      if (leader) {
+        if (KV) {
+          // dV += P^T dO ; dK += dS^T Q
+#pragma unroll
+          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
+            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            mma_bf16_ts(tmem + kAcc0, tmem + kX + ac, dS1m + 128 * kk, idesc_ts,
+                        (it > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
+            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            mma_bf16_ts(tmem + kAcc1, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
+                        (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          // dQ += dS K
+#pragma unroll
+          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
+            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            mma_bf16_ts(tmem + kAcc0, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
+                        (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&bars[BWB_EMPTY + s]);
+      }
+      __syncwarp();
+    }
+    if (leader) mma_commit(&bars[BWB_DONE]);
+    __syncwarp();
+    mbar_wait_drain(&bars[BWB_DONE], 0, p.timeout_ns);
+  } else {
+    // ---------------- element warps
+    const int q4 = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const int r = q4 * 32 + lane;        // row of the own tile
+    const int orow = o0 + r;             // its index within the user
+    const bool own_ok = orow < n;
+    const int32_t t_own = own_ok ? bw_rel_time(p.timestamps, start + orow, t_first) : 0;
+    const float inv_n = 1.0f / static_cast<float>(n);
+    const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
+    // time-gradient running sum (KV): current bucket and its partial sum
+    int tb_cur = -1;
+    float tg_acc = 0.0f;
+    auto flush_tg = [&]() {
+      if (tb_cur >= 0 && tg_acc != 0.0f) atomicAdd(&sTg[tb_cur], tg_acc);
+      tg_acc = 0.0f;
+    };
+    float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1 (KV)
+    bool ok = true;
+    for (int it = 0; it < n_st; ++it) {
+      const int sbase = (st0 + it) * BW_COLS;  // first streamed row
+      // this tile's 128 streamed times (all element threads, then a barrier)
+      int32_t* tt = sTimes + (it & 1) * 128;
+      if (tid < 128 && tid >= 0) {
+        const int row = sbase + tid;
+        if (warp < 4) tt[tid] = row < n ? bw_rel_time(p.timestamps, start + row, t_first) : 0;
+      }
+      named_barrier_sync(1, 8 * 32);
+      if (ok) ok = mbar_wait(&bars[BWB_S], static_cast<uint32_t>(it) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          const int c0 = half * 64 + ch * 32;  // first column of this chunk
+          uint32_t xs[32], ys[32];
+          tmem_ld32(tmem + lane_off + kX + static_cast<uint32_t>(c0), xs);
+          tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
+          tmem_ld_wait(xs);
+          tmem_ld_wait(ys);
+          uint32_t px[16], py[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dsv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int srow = sbase + c0 + c + e;  // streamed row index within the user
+              // KV: own = key j, streamed = query i; Q: own = query i, streamed = key j
+              const int qi = KV ? srow : orow;
+              const int kj = KV ? orow : srow;
+              const bool vis = own_ok && srow < n && kj <= qi;
+              float pp = 0.0f, ds = 0.0f;
+              if (vis) {
+                const int dpos = qi - kj;
+                const int bp = min(dpos, p.P - 1);
+                const int32_t ti = KV ? tt[c0 + c + e] : t_own;
+                const int32_t tj = KV ? t_own : tt[c0 + c + e];
+                const int bt = min(time_bucket_octave(ti - tj, sOct), p.Tb - 1);
+                const float sv = __uint_as_float(xs[c + e]) + __ldg(rp + bp) + sRt[bt];
+                float ph, pg;
+                phi_and_grad<PHI>(sv, ph, pg);
+                pp = ph * inv_n;
+                ds = __uint_as_float(ys[c + e]) * pg * inv_n;
+                if (KV) {
+                  if (bp == p.P - 1) pg_clamp += ds;
+                  else if (bp < p.hist_len) atomicAdd(&sPg[bp], ds);
+                  if (bt != tb_cur) {
+                    flush_tg();
+                    tb_cur = bt;
+                  }
+                  tg_acc += ds;
+                }
+              }
+              pv[e] = pp;
+              dsv[e] = ds;
+            }
+            if constexpr (F16) {
+              px[c >> 1] = pack_h2(pv[0], pv[1]);
+              py[c >> 1] = pack_h2(dsv[0], dsv[1]);
+            } else {
+              px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+              py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            }
+          }
+          // the packed operands go over columns this warp has read:
+          // rows 0-63 of the streamed tile at columns 0-31, 64-127 at 64-95
+          const uint32_t pc = static_cast<uint32_t>(half * 64 + ch * 16);
+          __syncwarp();
+          if (KV) tmem_st16(tmem + lane_off + kX + pc, px);
+          tmem_st16(tmem + lane_off + kY + pc, py);
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[BWB_P]);
+    }
+    if (KV) flush_tg();
+    // ---------------- epilogue: the accumulators (rows of the own tile)
+    if (ok) ok = mbar_wait(&bars[BWB_DONE], 0, ctl);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const int64_t grow = start + orow;
+      for (int a = 0; a < (KV ? 2 : 1); ++a) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + (a == 0 ? kAcc0 : kAcc1) + static_cast<uint32_t>(half * 32), v);
+        tmem_ld_wait(v);
+        float* dst = KV ? (a == 0 ? p.dv : p.dk) : p.dq;
+        if (own_ok) {
+          float4* d4 = reinterpret_cast<float4*>(dst + grow * p.ld_g + h * ATT_HD + half * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            d4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        }
+      }
+    }
+    if (KV && pg_clamp != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + p.P - 1], pg_clamp);
+  }
+
+  // ---------------- table gradients (KV) and teardown
+  tc_fence_before();
+  __syncthreads();
+  if (KV) {
+    const int lim = min(p.hist_len, p.P - 1);
+    for (int k = tid; k < lim; k += BW_THREADS) {
+      const float g = sPg[k];
+      if (g != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + k], g);
+    }
+    for (int k = tid; k < p.Tb; k += BW_THREADS) {
+      const float g = sTg[k];
+      if (g != 0.0f) atomicAdd(&p.drab_time[static_cast<int64_t>(h) * p.Tb + k], g);
+    }
+  }
+  if (warp == BW_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace hstu

@@ -15,6 +15,7 @@
 
 #include "../../include/hstu.h"
 #include "attn.cuh"
+#include "attn_bwd.cuh"
 #include "fp32_path.cuh"
 #include "gemm.cuh"
 #include "sl.cuh"
@@ -102,13 +103,13 @@ const int64_t* thresholds_for(int Tb) {
 
 enum KernelKind : int {
   K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT,
-  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_COUNT
+  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_ATTN_BWD_KV, K_ATTN_BWD_Q, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
                                            "fp32_attention",    "fp32_ln_gate", "weight_cvt",
                                            "sl_select",         "sl_gather",
-                                           "attention_f2_fused"};
+                                           "attention_f2_fused", "attn_bwd_kv", "attn_bwd_q"};
 
 struct Profiler {
   std::mutex mu;
@@ -191,6 +192,23 @@ AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16, bool fuse
   return f16 ? attn_kernel_ptr_t<true>(cand, phi, pairs) : attn_kernel_ptr_t<false>(cand, phi, pairs);
 }
 
+using AttnBwdFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const AttnBwdParams);
+
+template <bool KV, bool F16>
+AttnBwdFn attn_bwd_kernel_for(int phi) {
+  switch (phi) {
+    case HSTU_ACT_SILU: return hstu_attn_bwd_kernel<KV, HSTU_ACT_SILU, F16>;
+    case HSTU_ACT_RELU: return hstu_attn_bwd_kernel<KV, HSTU_ACT_RELU, F16>;
+    default: return hstu_attn_bwd_kernel<KV, HSTU_ACT_IDENTITY, F16>;
+  }
+}
+
+AttnBwdFn attn_bwd_kernel_ptr(bool kv, int phi, bool f16) {
+  if (kv) return f16 ? attn_bwd_kernel_for<true, true>(phi) : attn_bwd_kernel_for<true, false>(phi);
+  return f16 ? attn_bwd_kernel_for<false, true>(phi) : attn_bwd_kernel_for<false, false>(phi);
+}
+
 struct DeviceInfo {
   int sm_count = 0;
   bool smem_set = false;
@@ -220,6 +238,11 @@ hstu_status_t device_info(DeviceInfo** out) {
       for (int pairs = 0; pairs < 2; ++pairs)
         HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(false, phi, pairs != 0, true, true),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    for (int kv = 0; kv < 2; ++kv)
+      for (int phi = 0; phi < 3; ++phi)
+        for (int f16 = 0; f16 < 2; ++f16)
+          HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_bwd_kernel_ptr(kv != 0, phi, f16 != 0),
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
     const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
@@ -566,6 +589,64 @@ hstu_status_t launch_attn_tc(const AttnJob& j, cudaStream_t st) {
   attn_kernel_ptr(CAND, c->phi2, pairs, j.f16, fused)<<<grid, ATT_THREADS, smem, st>>>(mq, mk, mv,
                                                                                        mw, p);
   HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+// Backward of the causal pointwise attention: dQ, dK, dV (fp32, [T, ld_g]) and
+// the table gradients (overwritten).  q, k, v, d_o are 16-bit [T, H*64] with
+// row strides ldq, ldk, ldv, ld_do.
+hstu_status_t launch_attn_bwd(const hstu_layer_cfg_t* c, const hstu_jagged_t* jag, const void* q,
+                              int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                              const void* d_o, int64_t ld_do, const float* rab_pos,
+                              const float* rab_time, float* dq, float* dk, float* dv, int64_t ld_g,
+                              float* drab_pos, float* drab_time, bool f16, cudaStream_t st) {
+  const int H = c->num_heads, P = c->num_pos_buckets, Tb = c->num_time_buckets;
+  HSTU_CHECK_CUDA(cudaMemsetAsync(drab_pos, 0, sizeof(float) * H * P, st));
+  HSTU_CHECK_CUDA(cudaMemsetAsync(drab_time, 0, sizeof(float) * H * Tb, st));
+  if (jag->batch == 0 || jag->total_tokens == 0 || jag->max_len == 0) return HSTU_OK;
+  DeviceInfo* di = nullptr;
+  hstu_status_t s = device_info(&di);
+  if (s != HSTU_OK) return s;
+  const int64_t T = jag->total_tokens, hv = static_cast<int64_t>(H) * ATT_HD;
+  CUtensorMap mq, mk, mv, mo;
+  if ((s = make_map_16(&mq, q, T, hv, ldq, ATT_HD, BW_COLS, f16)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mk, k, T, hv, ldk, ATT_HD, BW_COLS, f16)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mv, v, T, hv, ldv, ATT_HD, BW_COLS, f16)) != HSTU_OK) return s;
+  if ((s = make_map_16(&mo, d_o, T, hv, ld_do, ATT_HD, BW_COLS, f16)) != HSTU_OK) return s;
+  AttnBwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.offsets = jag->offsets;
+  p.timestamps = jag->timestamps;
+  p.rab_pos = rab_pos;
+  p.rab_time = rab_time;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.ld_g = ld_g;
+  p.drab_pos = drab_pos;
+  p.drab_time = drab_time;
+  p.B = jag->batch;
+  p.H = H;
+  p.P = P;
+  p.Tb = Tb;
+  p.max_len = jag->max_len;
+  p.phi2 = c->phi2;
+  p.hist_len = std::min(P, jag->max_len);
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (!compute_octaves(Tb, thresholds_for(Tb), p.oct)) return HSTU_ERR_UNSUPPORTED;
+  const size_t smem = BwSmem::bytes(p.hist_len);
+  if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
+  dim3 grid(H, jag->batch, (jag->max_len + BW_ROWS - 1) / BW_ROWS);
+  {
+    ProfScope prof(K_ATTN_BWD_KV, st);
+    attn_bwd_kernel_ptr(true, c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
+    HSTU_CHECK_CUDA(cudaGetLastError());
+  }
+  {
+    ProfScope prof(K_ATTN_BWD_Q, st);
+    attn_bwd_kernel_ptr(false, c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
+    HSTU_CHECK_CUDA(cudaGetLastError());
+  }
   return HSTU_OK;
 }
 
@@ -993,6 +1074,30 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
   if (cfg->dtype == HSTU_FP32) return launch_f32_attn(j, st);
   j.f16 = cfg->dtype == HSTU_FP16;
   return launch_attn_tc<false>(j, st);
+}
+
+hstu_status_t hstu_attn_bwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag, const void* q,
+                            const void* k, const void* v, const void* d_o, const float* rab_pos,
+                            const float* rab_time, float* dq, float* dk, float* dv,
+                            float* drab_pos, float* drab_time, void* stream) {
+  hstu_status_t s;
+  if ((s = check_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if (cfg->dtype == HSTU_FP32 || cfg->phi2 == HSTU_ACT_SOFTMAX || jag->segments != nullptr)
+    return HSTU_ERR_UNSUPPORTED;
+  if (rab_pos == nullptr || rab_time == nullptr || drab_pos == nullptr || drab_time == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (jag->total_tokens > 0 &&
+      (q == nullptr || k == nullptr || v == nullptr || d_o == nullptr || dq == nullptr ||
+       dk == nullptr || dv == nullptr))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  const int64_t hv = static_cast<int64_t>(cfg->num_heads) * ATT_HD;
+  return launch_attn_bwd(cfg, jag, q, hv, k, hv, v, hv, d_o, hv, rab_pos, rab_time, dq, dk, dv,
+                         hv, drab_pos, drab_time, cfg->dtype == HSTU_FP16,
+                         static_cast<cudaStream_t>(stream));
 }
 
 hstu_status_t hstu_attn_fwd_f32(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,

@@ -70,6 +70,7 @@ EXPORTS = {
     "hstu_mfalcon_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int64]),
     "hstu_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hstu_attn_fwd_f32": (ctypes.c_int, [ctypes.c_void_p] * 9),
+    "hstu_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 14),
     "mfalcon_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64, ctypes.c_int32]
                          + [ctypes.c_void_p] * 8),
     "hstu_layer_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
@@ -249,6 +250,21 @@ def attn_fwd_f32(cfg: LayerConfig, jag: Jagged, q, k, v, rab_pos, rab_time, av_o
                                    _p(rab_pos), _p(rab_time), _p(av_out), _stream(stream)),
            "hstu_attn_fwd_f32")
     return av_out
+
+
+def attn_bwd(cfg: LayerConfig, jag: Jagged, q, k, v, d_o, rab_pos, rab_time, stream=None):
+    """Backward of the causal attention: returns dq, dk, dv ([T, H*64] fp32) and
+    drab_pos [H, P], drab_time [H, Tb] (fp32) for dO = d_o."""
+    dev = rab_pos.device
+    T, hv = jag.total_tokens, cfg.num_heads * cfg.dv
+    dq, dk, dv = (torch.empty((max(T, 1), hv), dtype=torch.float32, device=dev) for _ in range(3))
+    drp = torch.empty((cfg.num_heads, cfg.num_pos_buckets), dtype=torch.float32, device=dev)
+    drt = torch.empty((cfg.num_heads, cfg.num_time_buckets), dtype=torch.float32, device=dev)
+    c, j = cfg.c(), jag.c()
+    _check(lib().hstu_attn_bwd(ctypes.byref(c), ctypes.byref(j), _p(q), _p(k), _p(v), _p(d_o),
+                               _p(rab_pos), _p(rab_time), _p(dq), _p(dk), _p(dv), _p(drp),
+                               _p(drt), _stream(stream)), "hstu_attn_bwd")
+    return dq[:T], dk[:T], dv[:T], drp, drt
 
 
 def mfalcon_attn_fwd(cfg: LayerConfig, history: Jagged, k_hist, v_hist, cand_offsets,

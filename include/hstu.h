@@ -180,6 +180,28 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
                             const float* rab_pos, const float* rab_time, void* av_out,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of the causal attention step (the derivative of hstu_attn_fwd's
+ * Eq. 2 of the review, section 三 核心公式; the pages print no backward):
+ * given dO = dL/dAV,
+ *   dV = A^T dO,  dS = (dO V^T) (.) phi2'(Q K^T + rab) / N on visible pairs,
+ *   dQ = dS K,  dK = dS^T Q,
+ *   drab_pos[h, min(i-j, P-1)] and drab_time[h, bt(t_i - t_j)] += dS_ij.
+ *   cfg         dtype HSTU_FP16 or HSTU_BF16 (operand type of q, k, v, d_o),
+ *               phi2 SiLU (SiLU'(s) = sigmoid(s)(1 + s(1 - sigmoid(s)))),
+ *               ReLU (ReLU'(0) = 0) or identity; HSTU_ACT_SOFTMAX and
+ *               HSTU_FP32 return HSTU_ERR_UNSUPPORTED
+ *   jag         causal only (segments must be NULL)
+ *   q, k, v, d_o device [T, H*64] in the operand type, 16-byte aligned
+ *   dq, dk, dv  device [T, H*64] fp32, written
+ *   drab_pos    device [H, P] fp32, drab_time device [H, Tb] fp32: overwritten
+ *               (zeroed, then accumulated with atomics: the summation order,
+ *               and so the last bits, vary from run to run)
+ * Runs two tcgen05 kernels (dK/dV with the table gradients, then dQ). */
+hstu_status_t hstu_attn_bwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
+                            const void* q, const void* k, const void* v, const void* d_o,
+                            const float* rab_pos, const float* rab_time, float* dq, float* dk,
+                            float* dv, float* drab_pos, float* drab_time, void* stream);
+
 /*
  * Eq. 2 alone with an fp32 result: the same computation as hstu_attn_fwd, with
  * AV written in fp32 (the precision the layer path hands to Norm(.) of Eq. 3)
