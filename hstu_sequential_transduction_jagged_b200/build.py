@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhstu.so")
 SOURCES = ["hstu_api.cu"]
 HEADERS = ["ptx.cuh", "status.cuh", "attn.cuh", "attn_bwd.cuh", "gemm.cuh", "fp32_path.cuh",
-           "sl.cuh"]
+           "sl.cuh", "layer_bwd.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -45,9 +45,12 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + ".tmp"
+    # the layer backward's weight-gradient GEMMs are plain cuBLAS GEMMs
+    cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc())), "lib64")
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
            "-I", os.path.join(ROOT, "include"), "-o", tmp,
-           *[os.path.join(CSRC, s) for s in SOURCES]]
+           *[os.path.join(CSRC, s) for s in SOURCES],
+           "-L", cuda_lib, "-lcublas", "-Xlinker", "-rpath," + cuda_lib]
     if extra:
         cmd[1:1] = list(extra)
     if verbose:

@@ -4,6 +4,7 @@
 // workspace carving, TMA tensor-map encoding and kernel launches on the
 // caller's stream.  The library is one translation unit so the device status
 // word in status.cuh is shared by all kernels.
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,6 +19,7 @@
 #include "attn_bwd.cuh"
 #include "fp32_path.cuh"
 #include "gemm.cuh"
+#include "layer_bwd.cuh"
 #include "sl.cuh"
 
 using namespace hstu;
@@ -103,13 +105,15 @@ const int64_t* thresholds_for(int Tb) {
 
 enum KernelKind : int {
   K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT,
-  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_ATTN_BWD_KV, K_ATTN_BWD_Q, K_COUNT
+  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_ATTN_BWD_KV, K_ATTN_BWD_Q, K_BWD_GEMM, K_GATE_BWD,
+  K_BWD_ELT, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
                                            "fp32_attention",    "fp32_ln_gate", "weight_cvt",
                                            "sl_select",         "sl_gather",
-                                           "attention_f2_fused", "attn_bwd_kv", "attn_bwd_q"};
+                                           "attention_f2_fused", "attn_bwd_kv", "attn_bwd_q",
+                                           "bwd_gemm_cublas", "gate_bwd", "bwd_elementwise"};
 
 struct Profiler {
   std::mutex mu;
@@ -959,6 +963,238 @@ hstu_status_t layer_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* 
                         ylp_f16, d, T, st);
 }
 
+// ------------------------------------------------------------------ layer backward
+
+// Workspace of hstu_layer_bwd: the forward's (recomputed intermediates), then
+// dG, G [T, H*64] fp32, dZ [T, n1] fp32, dAV [T, H*64] 16-bit, X [T, d] fp32,
+// fp32 copies of W1 and W2, and the cuBLAS workspace.
+constexpr size_t kCublasWsBytes = size_t(32) << 20;
+
+struct BwdWs {
+  LayerWs fwd;
+  float* dg;
+  float* g;
+  float* dz;
+  void* dav16;
+  float* x32;
+  float* w1f;
+  float* w2f;
+  void* cublas_ws;
+};
+
+size_t layer_bwd_ws_bytes(const hstu_layer_cfg_t* c, int64_t T) {
+  const size_t t = static_cast<size_t>(T);
+  const size_t hv = static_cast<size_t>(c->num_heads) * ATT_HD;
+  const size_t d = static_cast<size_t>(c->d_model), n1 = static_cast<size_t>(n1_of(c));
+  return layer_ws_bytes(c, T) + 2 * align_up(t * hv * 4, 256) + align_up(t * n1 * 4, 256) +
+         align_up(t * hv * 2, 256) + align_up(t * d * 4, 256) + align_up(n1 * d * 4, 256) +
+         align_up(d * hv * 4, 256) + kCublasWsBytes;
+}
+
+BwdWs carve_bwd(const hstu_layer_cfg_t* c, int64_t T, void* ws) {
+  const size_t t = static_cast<size_t>(T);
+  const size_t hv = static_cast<size_t>(c->num_heads) * ATT_HD;
+  const size_t d = static_cast<size_t>(c->d_model), n1 = static_cast<size_t>(n1_of(c));
+  BwdWs b;
+  b.fwd = carve_layer(c, T, ws);
+  uint8_t* p = static_cast<uint8_t*>(ws) + layer_ws_bytes(c, T);
+  auto take = [&](size_t bytes) { uint8_t* q = p; p += align_up(bytes, 256); return q; };
+  b.dg = reinterpret_cast<float*>(take(t * hv * 4));
+  b.g = reinterpret_cast<float*>(take(t * hv * 4));
+  b.dz = reinterpret_cast<float*>(take(t * n1 * 4));
+  b.dav16 = take(t * hv * 2);
+  b.x32 = reinterpret_cast<float*>(take(t * d * 4));
+  b.w1f = reinterpret_cast<float*>(take(n1 * d * 4));
+  b.w2f = reinterpret_cast<float*>(take(d * hv * 4));
+  b.cublas_ws = take(kCublasWsBytes);
+  return b;
+}
+
+// One cuBLAS handle per device, created on first use; calls on it are
+// serialised by the mutex (the stream and workspace are set per call).
+struct CublasSlot {
+  std::mutex mu;
+  cublasHandle_t h = nullptr;
+};
+
+CublasSlot* cublas_slot() {
+  static CublasSlot slots[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return &slots[dev];
+}
+
+// Row-major C[M, N] = op(A) op(B) + beta C in fp32 storage with TF32 tensor
+// cores (op(A) is [M, K]: A is [M, K] or, transposed, [K, M]).  Through the
+// column-major library: C^T = op(B)^T op(A)^T.
+hstu_status_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int64_t M, int64_t N, int64_t K,
+                      const float* A, int64_t lda, const float* B, int64_t ldb, float* C,
+                      int64_t ldc, float beta) {
+  if (M == 0 || N == 0) return HSTU_OK;
+  const float alpha = 1.0f;
+  const cublasStatus_t r = cublasGemmEx(
+      h, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, static_cast<int>(N),
+      static_cast<int>(M), static_cast<int>(K), &alpha, B, CUDA_R_32F, static_cast<int>(ldb), A,
+      CUDA_R_32F, static_cast<int>(lda), &beta, C, CUDA_R_32F, static_cast<int>(ldc),
+      CUBLAS_COMPUTE_32F_FAST_TF32, CUBLAS_GEMM_DEFAULT);
+  return r == CUBLAS_STATUS_SUCCESS ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t convert_bf16_to_f32(const void* src, float* dst, int64_t n, cudaStream_t st) {
+  if (n == 0) return HSTU_OK;
+  ProfScope prof(K_BWD_ELT, st);
+  hstu_bf16_to_f32_kernel<<<std::min<int64_t>((n + 255) / 256, 148 * 16), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(src), dst, n);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+hstu_status_t colsum(const float* a, int64_t lda, int64_t M, int N, float* out, cudaStream_t st) {
+  HSTU_CHECK_CUDA(cudaMemsetAsync(out, 0, sizeof(float) * N, st));
+  if (M == 0) return HSTU_OK;
+  const int rows = 512;
+  dim3 grid((N + 255) / 256, static_cast<unsigned>((M + rows - 1) / rows));
+  ProfScope prof(K_BWD_ELT, st);
+  hstu_colsum_kernel<<<grid, 256, 0, st>>>(a, lda, M, N, rows, out);
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+template <int KPL>
+void launch_gate_bwd_k(const float* av, const float* ln_part, const float* u, const float* dg,
+                       const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w, int64_t T,
+                       void* dav16, float* dz, int64_t ld_dz, float* g, float* dgamma,
+                       float* dbeta, cudaStream_t st) {
+  const int64_t blocks = std::min<int64_t>((T + 7) / 8, 148 * 8);
+  hstu_gate_bwd_kernel<KPL><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      av, ln_part, u, dg, w->ln_gamma, w->ln_beta, c->ln_eps, c->num_heads, T, dav16, 1, dz,
+      ld_dz, g, dgamma, dbeta, c->phi1 == HSTU_ACT_RELU ? 1 : 0);
+}
+
+hstu_status_t launch_gate_bwd(const float* av, const float* ln_part, const float* u,
+                              const float* dg, const hstu_layer_cfg_t* c,
+                              const hstu_layer_weights_t* w, int64_t T, void* dav16, float* dz,
+                              int64_t ld_dz, float* g, float* dgamma, float* dbeta,
+                              cudaStream_t st) {
+  ProfScope prof(K_GATE_BWD, st);
+  switch (c->num_heads) {
+#define HSTU_GATE_CASE(HH) \
+    case HH: launch_gate_bwd_k<2 * HH>(av, ln_part, u, dg, c, w, T, dav16, dz, ld_dz, g, dgamma, dbeta, st); break;
+    HSTU_GATE_CASE(1) HSTU_GATE_CASE(2) HSTU_GATE_CASE(3) HSTU_GATE_CASE(4)
+    HSTU_GATE_CASE(5) HSTU_GATE_CASE(6) HSTU_GATE_CASE(7) HSTU_GATE_CASE(8)
+    HSTU_GATE_CASE(10) HSTU_GATE_CASE(12) HSTU_GATE_CASE(16)
+#undef HSTU_GATE_CASE
+    default: return HSTU_ERR_UNSUPPORTED;
+  }
+  HSTU_CHECK_CUDA(cudaGetLastError());
+  return HSTU_OK;
+}
+
+// The backward of one bf16 layer: recompute f1 and the attention (the same
+// kernels as the forward), then the chain rule through Eq. 3, the attention
+// and Eq. 1.
+hstu_status_t layer_bwd_bf16(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w,
+                             const hstu_jagged_t* jag, const void* x_in, const float* x_res,
+                             const float* dy, float* dx, const hstu_layer_grads_t* gr,
+                             const BwdWs& b, cudaStream_t st) {
+  const int64_t T = jag->total_tokens;
+  const int hv = c->num_heads * ATT_HD, d = c->d_model, n1 = n1_of(c);
+  const LayerWs& ws = b.fwd;
+  hstu_status_t s;
+  // ---- forward recompute: f1 (U fp32; V, Q, K fp16) and the attention (AV, LN partials)
+  const bool x_f16 = x_in == nullptr;
+  if (x_f16 && (s = convert_f32_to_f16(x_res, ws.x16, T * d, st)) != HSTU_OK) return s;
+  if (x_f16 && (s = convert_bf16_to_f16(w->w1, ws.w1h, static_cast<int64_t>(n1) * d, st)) != HSTU_OK)
+    return s;
+  __half* vqk = static_cast<__half*>(ws.z);
+  void* dst[4] = {ws.u, vqk, vqk + hv, vqk + 2 * hv};
+  int64_t ldd[4] = {hv, 3 * hv, 3 * hv, 3 * hv};
+  s = launch_f1_bf16(c, x_f16 ? static_cast<const void*>(ws.x16) : x_in, d, T,
+                     x_f16 ? static_cast<const void*>(ws.w1h) : w->w1, w->b1, dst, ldd, 1u, 0xEu,
+                     x_f16, st);
+  if (s != HSTU_OK) return s;
+  AttnJob j;
+  std::memset(&j, 0, sizeof(j));
+  j.cfg = c;
+  j.kv_offsets = jag->offsets;
+  j.timestamps = jag->timestamps;
+  j.batch = jag->batch;
+  j.max_q_len = j.max_kv_len = jag->max_len;
+  j.T_q = j.T_kv = T;
+  j.q = vqk + hv; j.ldq = 3 * hv;
+  j.k = vqk + 2 * hv; j.ldk = 3 * hv;
+  j.v = vqk; j.ldv = 3 * hv;
+  j.rab_pos = w->rab_pos;
+  j.rab_time = w->rab_time;
+  j.av_f32 = static_cast<float*>(ws.av);
+  j.ld_av = hv;
+  j.ln_part = static_cast<float*>(ws.extra);
+  j.timeout_ns = kDefaultTimeoutNs;
+  j.f16 = true;
+  if ((s = launch_attn_tc<false>(j, st)) != HSTU_OK) return s;
+  // ---- fp32 operands of the library GEMMs
+  if ((s = convert_bf16_to_f32(w->w1, b.w1f, static_cast<int64_t>(n1) * d, st)) != HSTU_OK) return s;
+  if ((s = convert_bf16_to_f32(w->w2, b.w2f, static_cast<int64_t>(d) * hv, st)) != HSTU_OK) return s;
+  const float* x32 = x_res;
+  if (!x_f16) {
+    if ((s = convert_bf16_to_f32(x_in, b.x32, T * d, st)) != HSTU_OK) return s;
+    x32 = b.x32;
+  }
+  CublasSlot* cs = cublas_slot();
+  if (cs == nullptr) return HSTU_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(cs->mu);
+  if (cs->h == nullptr && cublasCreate(&cs->h) != CUBLAS_STATUS_SUCCESS) {
+    cs->h = nullptr;
+    return HSTU_ERR_CUDA;
+  }
+  if (cublasSetStream(cs->h, st) != CUBLAS_STATUS_SUCCESS ||
+      cublasSetWorkspace(cs->h, b.cublas_ws, kCublasWsBytes) != CUBLAS_STATUS_SUCCESS)
+    return HSTU_ERR_CUDA;
+  // ---- Y = X + G W2^T + b2:  dG = dY W2,  dW2 = dY^T G,  db2 = colsum(dY)
+  {
+    ProfScope prof(K_BWD_GEMM, st);
+    if ((s = gemm_rm(cs->h, false, false, T, hv, d, dy, d, b.w2f, hv, b.dg, hv, 0.0f)) != HSTU_OK)
+      return s;
+  }
+  // ---- G = Ln(AV) (.) U: dU (masked), G, dAV (fp16), dgamma / dbeta
+  if (gr->dgamma != nullptr) HSTU_CHECK_CUDA(cudaMemsetAsync(gr->dgamma, 0, sizeof(float) * hv, st));
+  if (gr->dbeta != nullptr) HSTU_CHECK_CUDA(cudaMemsetAsync(gr->dbeta, 0, sizeof(float) * hv, st));
+  if ((s = launch_gate_bwd(static_cast<const float*>(ws.av), static_cast<const float*>(ws.extra),
+                           ws.u, b.dg, c, w, T, b.dav16, b.dz, n1, b.g,
+                           w->ln_gamma != nullptr ? gr->dgamma : nullptr,
+                           w->ln_beta != nullptr ? gr->dbeta : nullptr, st)) != HSTU_OK)
+    return s;
+  {
+    ProfScope prof(K_BWD_GEMM, st);
+    if ((s = gemm_rm(cs->h, true, false, d, hv, T, dy, d, b.g, hv, gr->dw2, hv, 0.0f)) != HSTU_OK)
+      return s;
+  }
+  if ((s = colsum(dy, d, T, d, gr->db2, st)) != HSTU_OK) return s;
+  // ---- attention: dV, dQ, dK straight into their dZ column blocks, table gradients
+  if ((s = launch_attn_bwd(c, jag, vqk + hv, 3 * hv, vqk + 2 * hv, 3 * hv, vqk, 3 * hv, b.dav16, hv,
+                           w->rab_pos, w->rab_time, b.dz + 2 * hv, b.dz + 3 * hv, b.dz + hv, n1,
+                           gr->drab_pos, gr->drab_time, true, st)) != HSTU_OK)
+    return s;
+  // ---- Z = phi1(X W1^T + b1): mask, db1, dW1 = dZ^T X, dX = dY + dZ W1
+  if (c->phi1 == HSTU_ACT_RELU) {
+    ProfScope prof(K_BWD_ELT, st);
+    const int64_t total = T * 3 * hv;
+    hstu_relu_mask_kernel<<<std::min<int64_t>((total + 255) / 256, 148 * 16), 256, 0, st>>>(
+        b.dz, n1, hv, vqk, 3 * hv, 3 * hv, T);
+    HSTU_CHECK_CUDA(cudaGetLastError());
+  }
+  if ((s = colsum(b.dz, n1, T, n1, gr->db1, st)) != HSTU_OK) return s;
+  {
+    ProfScope prof(K_BWD_GEMM, st);
+    if ((s = gemm_rm(cs->h, true, false, n1, d, T, b.dz, n1, x32, d, gr->dw1, d, 0.0f)) != HSTU_OK)
+      return s;
+    HSTU_CHECK_CUDA(cudaMemcpyAsync(dx, dy, sizeof(float) * T * d, cudaMemcpyDeviceToDevice, st));
+    if ((s = gemm_rm(cs->h, false, false, T, d, n1, b.dz, n1, b.w1f, d, dx, d, 1.0f)) != HSTU_OK)
+      return s;
+  }
+  return HSTU_OK;
+}
+
 hstu_status_t check_weights(const hstu_layer_cfg_t* c, const hstu_layer_weights_t* w) {
   if (w == nullptr || w->w1 == nullptr || w->b1 == nullptr || w->w2 == nullptr ||
       w->b2 == nullptr || w->rab_pos == nullptr || w->rab_time == nullptr)
@@ -1074,6 +1310,49 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
   if (cfg->dtype == HSTU_FP32) return launch_f32_attn(j, st);
   j.f16 = cfg->dtype == HSTU_FP16;
   return launch_attn_tc<false>(j, st);
+}
+
+size_t hstu_layer_bwd_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total_tokens) {
+  if (check_layer_cfg(cfg) != HSTU_OK || total_tokens < 0 || cfg->dtype != HSTU_BF16) return 0;
+  return layer_bwd_ws_bytes(cfg, total_tokens);
+}
+
+hstu_status_t hstu_layer_bwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                             const hstu_jagged_t* jag, const void* x_in, const float* x_res,
+                             const float* dy, float* dx, const hstu_layer_grads_t* grads,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  hstu_status_t s;
+  if ((s = check_layer_cfg(cfg)) != HSTU_OK) return s;
+  if ((s = check_jag(jag)) != HSTU_OK) return s;
+  if ((s = check_weights(cfg, w)) != HSTU_OK) return s;
+  if (cfg->dtype != HSTU_BF16 || jag->segments != nullptr || cfg->phi2 == HSTU_ACT_SOFTMAX ||
+      (cfg->phi1 != HSTU_ACT_RELU && cfg->phi1 != HSTU_ACT_IDENTITY) || cfg->num_heads > 16)
+    return HSTU_ERR_UNSUPPORTED;
+  if (grads == nullptr || grads->dw1 == nullptr || grads->db1 == nullptr || grads->dw2 == nullptr ||
+      grads->db2 == nullptr || grads->drab_pos == nullptr || grads->drab_time == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  const int64_t T = jag->total_tokens;
+  const int hv = cfg->num_heads * ATT_HD, d = cfg->d_model, n1 = n1_of(cfg);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0 || jag->batch == 0) {
+    // no tokens: every gradient is zero
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->dw1, 0, sizeof(float) * n1 * d, st));
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->db1, 0, sizeof(float) * n1, st));
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->dw2, 0, sizeof(float) * d * hv, st));
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->db2, 0, sizeof(float) * d, st));
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->drab_pos, 0, sizeof(float) * cfg->num_heads * cfg->num_pos_buckets, st));
+    HSTU_CHECK_CUDA(cudaMemsetAsync(grads->drab_time, 0, sizeof(float) * cfg->num_heads * cfg->num_time_buckets, st));
+    if (grads->dgamma != nullptr) HSTU_CHECK_CUDA(cudaMemsetAsync(grads->dgamma, 0, sizeof(float) * hv, st));
+    if (grads->dbeta != nullptr) HSTU_CHECK_CUDA(cudaMemsetAsync(grads->dbeta, 0, sizeof(float) * hv, st));
+    return HSTU_OK;
+  }
+  if ((x_in == nullptr && x_res == nullptr) || dy == nullptr || dx == nullptr)
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(x_res) || !aligned16(dy) || !aligned16(dx) ||
+      !aligned16(workspace))
+    return HSTU_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || ws_bytes < layer_bwd_ws_bytes(cfg, T)) return HSTU_ERR_WORKSPACE_TOO_SMALL;
+  return layer_bwd_bf16(cfg, w, jag, x_in, x_res, dy, dx, grads, carve_bwd(cfg, T, workspace), st);
 }
 
 hstu_status_t hstu_attn_bwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag, const void* q,

@@ -71,6 +71,9 @@ EXPORTS = {
     "hstu_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hstu_attn_fwd_f32": (ctypes.c_int, [ctypes.c_void_p] * 9),
     "hstu_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 14),
+    "hstu_layer_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_void_p, ctypes.c_int64]),
+    "hstu_layer_bwd": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                              ctypes.c_void_p]),
     "mfalcon_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int64, ctypes.c_int32]
                          + [ctypes.c_void_p] * 8),
     "hstu_layer_fwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_size_t, ctypes.c_void_p]),
@@ -265,6 +268,42 @@ def attn_bwd(cfg: LayerConfig, jag: Jagged, q, k, v, d_o, rab_pos, rab_time, str
                                _p(rab_pos), _p(rab_time), _p(dq), _p(dk), _p(dv), _p(drp),
                                _p(drt), _stream(stream)), "hstu_attn_bwd")
     return dq[:T], dk[:T], dv[:T], drp, drt
+
+
+class LayerGradsT(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dw1", "db1", "dw2", "db2", "drab_pos", "drab_time", "dgamma", "dbeta")]
+
+
+def layer_bwd_workspace_bytes(cfg: LayerConfig, total_tokens: int) -> int:
+    c = cfg.c()
+    return int(lib().hstu_layer_bwd_workspace_bytes(ctypes.byref(c), total_tokens))
+
+
+def layer_bwd(cfg: LayerConfig, w: "LayerWeights", jag: Jagged, x_in, dy, x_res=None,
+              workspace=None, stream=None) -> dict:
+    """Backward of one bf16 layer for dY = dy ([T, d] fp32): returns a dict with
+    dx [T, d] and the parameter gradients (fp32): dw1, db1, dw2, db2, drab_pos,
+    drab_time and, when the layer has them, dgamma / dbeta."""
+    dev = dy.device
+    T, d, hv, n1 = jag.total_tokens, cfg.d_model, cfg.num_heads * cfg.dv, cfg.n1
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty((max(T, 1), d), **f32), "dw1": torch.empty((n1, d), **f32),
+           "db1": torch.empty(n1, **f32), "dw2": torch.empty((d, hv), **f32),
+           "db2": torch.empty(d, **f32),
+           "drab_pos": torch.empty((cfg.num_heads, cfg.num_pos_buckets), **f32),
+           "drab_time": torch.empty((cfg.num_heads, cfg.num_time_buckets), **f32),
+           "dgamma": torch.empty(hv, **f32) if w.ln_gamma is not None else None,
+           "dbeta": torch.empty(hv, **f32) if w.ln_beta is not None else None}
+    g = LayerGradsT(*[None if out[n] is None else out[n].data_ptr() for n in
+                      ("dw1", "db1", "dw2", "db2", "drab_pos", "drab_time", "dgamma", "dbeta")])
+    ws = _workspace(layer_bwd_workspace_bytes(cfg, T), dev, workspace)
+    c, j, wc = cfg.c(), jag.c(), w.c()
+    _check(lib().hstu_layer_bwd(ctypes.byref(c), ctypes.byref(wc), ctypes.byref(j), _p(x_in),
+                                _p(x_res), _p(dy), _p(out["dx"]), ctypes.byref(g), _p(ws),
+                                ws.numel(), _stream(stream)), "hstu_layer_bwd")
+    out["dx"] = out["dx"][:T]
+    return out
 
 
 def mfalcon_attn_fwd(cfg: LayerConfig, history: Jagged, k_hist, v_hist, cand_offsets,

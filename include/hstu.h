@@ -180,6 +180,18 @@ hstu_status_t hstu_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* ja
                             const float* rab_pos, const float* rab_time, void* av_out,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Gradients of one layer's parameters (all device fp32, overwritten). */
+typedef struct {
+  float* dw1;        /* [2H(dqk+dv), d] */
+  float* db1;        /* [2H(dqk+dv)] */
+  float* dw2;        /* [d, H*dv] */
+  float* db2;        /* [d] */
+  float* drab_pos;   /* [H, P] */
+  float* drab_time;  /* [H, Tb] */
+  float* dgamma;     /* [H*dv], or NULL (written when the layer has ln_gamma) */
+  float* dbeta;      /* [H*dv], or NULL (written when the layer has ln_beta) */
+} hstu_layer_grads_t;
+
 /* Backward of the causal attention step (the derivative of hstu_attn_fwd's
  * Eq. 2 of the review, section 三 核心公式; the pages print no backward):
  * given dO = dL/dAV,
@@ -262,6 +274,36 @@ hstu_status_t mfalcon_attn_fwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t*
 hstu_status_t hstu_layer_fwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
                              const hstu_jagged_t* jag, const void* x_in, const float* x_res,
                              float* y_out, void* y_out_lp, void* kv_cache_out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of hstu_layer_bwd for T tokens. */
+size_t hstu_layer_bwd_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total_tokens);
+
+/* Backward of one bf16 layer (the derivative of hstu_layer_fwd; the pages
+ * print no backward, so this is the chain rule through Eq. 1-3 of the review
+ * and the residual): given dY = dL/dY, writes dX = dL/dX and the parameter
+ * gradients.  The forward intermediates are recomputed from X with the
+ * forward's own kernels (f1, attention), so only X is kept between the
+ * passes.  Then:
+ *   dG = dY W2, dW2 = dY^T G, db2 = sum dY                  (GEMMs: cuBLAS, TF32)
+ *   dU, dAV, dgamma, dbeta through G = LayerNorm(AV) (.) U  (one warp per row)
+ *   dQ, dK, dV, drab_pos, drab_time                         (hstu_attn_bwd's kernels)
+ *   dZ = [dU | dV | dQ | dK] (.) phi1', db1 = sum dZ,
+ *   dW1 = dZ^T X, dX = dY + dZ W1                           (GEMMs: cuBLAS, TF32)
+ *   cfg       dtype HSTU_BF16; phi1 ReLU (ReLU'(0) = 0) or identity; phi2
+ *             SiLU, ReLU or identity; HSTU_ERR_UNSUPPORTED otherwise
+ *   jag       causal (segments NULL)
+ *   x_in      device [T, d] bf16 layer input, or NULL with x_res (as in
+ *             hstu_layer_fwd: f1 then read x_res rounded to fp16)
+ *   x_res     device [T, d] fp32 or NULL
+ *   dy        device [T, d] fp32
+ *   dx        device [T, d] fp32, written
+ *   grads     parameter gradients, overwritten
+ * The first call on a device creates that device's cuBLAS handle; its
+ * workspace is carved from `workspace`. */
+hstu_status_t hstu_layer_bwd(const hstu_layer_cfg_t* cfg, const hstu_layer_weights_t* w,
+                             const hstu_jagged_t* jag, const void* x_in, const float* x_res,
+                             const float* dy, float* dx, const hstu_layer_grads_t* grads,
                              void* workspace, size_t ws_bytes, void* stream);
 
 /*

@@ -109,8 +109,13 @@ def attention_bwd_user(q, k, v, ts, rab_pos, rab_time, n_norm, H, dqk, dv, phi2,
     return dq, dk, dvv, drp, drt
 
 
-def layer_bwd(x, offsets, timestamps, layer, cfg, dy, segments=None) -> dict:
+def layer_bwd(x, offsets, timestamps, layer, cfg, dy, segments=None, x_f1=None) -> dict:
     """Gradients of sum(dY (.) Y) for one HSTU layer Y = layer_fwd(X).
+
+    `x_f1` is the input f1 reads when it differs from the residual input x (a
+    layer handed its input in two precisions, e.g. an fp32 residual stream of
+    which f1 reads a 16-bit copy); the rounding between them passes the
+    gradient unchanged, so dX = dY + dZpre W1 either way and dW1 = dZpre^T x_f1.
 
     Returns dx [T, d], dw1 [n1, d], db1 [n1], dw2 [d, H*dv], db2 [d],
     drab_pos [H, P], drab_time [H, Tb], dgamma / dbeta ([H*dv], or None when
@@ -118,6 +123,7 @@ def layer_bwd(x, offsets, timestamps, layer, cfg, dy, segments=None) -> dict:
     dv, du [T, H*64] and dav [T, H*dv].
     """
     x = np.asarray(x, dtype=np.float64)
+    xf = x if x_f1 is None else np.asarray(x_f1, dtype=np.float64)
     dy = np.asarray(dy, dtype=np.float64)
     H, dqk, dvw = cfg.num_heads, cfg.dqk, cfg.dv
     hv, hq = H * dvw, H * dqk
@@ -139,7 +145,7 @@ def layer_bwd(x, offsets, timestamps, layer, cfg, dy, segments=None) -> dict:
         n = e0 - s0
         if n == 0:
             continue
-        xu, dyu = x[s0:e0], dy[s0:e0]
+        xu, dyu = xf[s0:e0], dy[s0:e0]
         pre = xu @ w1.T + b1
         z = F.phi(pre, cfg.phi1)
         uu, vv = z[:, 0:hv], z[:, hv:2 * hv]

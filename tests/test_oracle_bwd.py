@@ -144,3 +144,15 @@ def test_planted_mistakes_fail_the_pins(monkeypatch, plant):
     got = B.layer_bwd(x, offsets, ts, layer, cfg, dy)
     with pytest.raises(AssertionError):
         _fd_check(cfg, layer, offsets, ts, x, dy, got)
+
+
+def test_separate_f1_input_reduces_to_the_pinned_gradient():
+    """x_f1 (the input f1 reads) differing from the residual input: every
+    gradient equals that of the layer fed x_f1 alone, because the residual
+    term sum(dY (.) X) has gradient dY whichever X it is."""
+    cfg, layer, offsets, ts, x, dy = _case("silu", seed=9, lengths=(4, 3))
+    xr = np.round(x * 64.0) / 64.0  # a coarser copy, as a 16-bit f1 input would be
+    split = B.layer_bwd(x, offsets, ts, layer, cfg, dy, x_f1=xr)
+    alone = B.layer_bwd(xr, offsets, ts, layer, cfg, dy)
+    for name in ("dx", "dw1", "db1", "dw2", "db2", "drab_pos", "drab_time", "dgamma", "dbeta"):
+        assert np.allclose(split[name], alone[name], rtol=0, atol=1e-12), name
