@@ -47,6 +47,8 @@ WORKLOAD_TEXT = {
                       "1024 U+S tokens, 6144 R tokens, 1024 candidates timed across R",
     "sl-sampler": "GPU Stochastic Length sampler on 64 users x 4096 events (alpha 1.6), d_model "
                   "512 bf16 rows gathered",
+    "long-bf16-train": "training step on the long-sequence workload: forward and backward of "
+                       "both layers (hstu_layer_fwd, hstu_layer_bwd), synthetic dL/dY",
     "long-bf16-fused": "the long-sequence workload with f2 inside the attention kernel "
                        "(HSTU_FLAG_FUSED_F2: the last head CTA of each query tile pair runs it)",
 }
@@ -605,6 +607,79 @@ def measure_sl_sampler(ctx, steps, warmup):
                 "ms_per_launch": ms_g / n_g}}
 
 
+TRAIN_METRIC = "HSTU training step (forward + backward of every layer) tokens/sec at 1 B200"
+
+
+def measure_train(ctx, steps, warmup, sample_clocks=False, batch=None):
+    """Forward and backward of both layers of the long-sequence workload: layer
+    0 from the bf16 input, layer 1 from layer 0's fp32 output; backward with a
+    fixed synthetic dL/dY through layer 1, then layer 0 (all parameter
+    gradients and dX).  No optimizer."""
+    torch, H = ctx.torch, ctx.H
+    from gen.device import case_tensors
+    case = make_workload("long-bf16", batch=batch)
+    c = case.cfg
+    T, L = case.total_tokens, c.num_layers
+    t = case_tensors(case, ctx.dev)
+    jag = H.Jagged(t["offsets"], t["timestamps"], case.max_len, T)
+    weights = [H.LayerWeights(**lw) for lw in t["layers"]]
+    cfg = H.LayerConfig(c.d_model, c.num_heads, c.num_pos_buckets, c.num_time_buckets,
+                        dqk=c.dqk, dv=c.dv, phi1=c.phi1, phi2=c.phi2, ln_eps=c.ln_eps,
+                        dtype=c.dtype)
+    fws = torch.empty(H.layer_workspace_bytes(cfg, T), dtype=torch.uint8, device=ctx.dev)
+    bws = torch.empty(H.layer_bwd_workspace_bytes(cfg, T), dtype=torch.uint8, device=ctx.dev)
+    ys = [torch.empty((T, c.d_model), dtype=torch.float32, device=ctx.dev) for _ in range(L)]
+    g = torch.Generator(device=ctx.dev).manual_seed(0)
+    dy_top = torch.randn((T, c.d_model), generator=g, device=ctx.dev, dtype=torch.float32)
+
+    def step():
+        for l in range(L):
+            if l == 0:
+                H.layer_fwd(cfg, weights[0], jag, t["x"], y_out=ys[0], workspace=fws)
+            else:
+                H.layer_fwd(cfg, weights[l], jag, None, x_res=ys[l - 1], y_out=ys[l], workspace=fws)
+        dy = dy_top
+        for l in reversed(range(L)):
+            if l == 0:
+                r = H.layer_bwd(cfg, weights[0], jag, t["x"], dy, workspace=bws)
+            else:
+                r = H.layer_bwd(cfg, weights[l], jag, None, dy, x_res=ys[l - 1], workspace=bws)
+            dy = r["dx"]
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    step_ms, kernels, clocks = ctx.timed_steps(step, steps, sample_clocks)
+    total = ctx.max_over_ranks(sum(step_ms))
+    ms = total / steps
+    value = ctx.world * T / (ms / 1000.0)
+    pairs = visible_pairs(case)
+    # attention backward, FlashAttention convention: five 2*64-flop products
+    # per visible (i, j, head): S (recomputed), dP, dV, dQ, dK
+    bwd_flop = pairs * c.num_heads * 5 * 2 * 64
+    n_kv, ms_kv = kernels.get("attn_bwd_kv", (0, 0.0))
+    n_q, ms_q = kernels.get("attn_bwd_q", (0, 0.0))
+    roof = None
+    if n_kv and n_q:
+        per = ms_kv / n_kv + ms_q / n_q
+        ach = bwd_flop / (per / 1000.0) / 1e12
+        roof = {"kernel": "hstu_attn_bwd_kernel (dK/dV + dQ, per layer)", "bound": "tensor",
+                "achieved": ach, "peak": ctx.peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / ctx.peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{ctx.peak_src} bf16 dense, burst ({PEAK_RULE})",
+                "algorithmic_flop_per_launch": bwd_flop,
+                "flop_rule": "5 x 2 x 64 flop per visible (i, j, head): S, dP, dV, dQ, dK",
+                "ms_per_launch": per}
+    return {"metric": TRAIN_METRIC, "value": value, "unit": "tokens/s",
+            "workload": "training step on the long-sequence workload (2 layers bf16, d_model "
+                        "512, 8 heads, 8 users x 8192): forward and backward of both layers, "
+                        "synthetic dL/dY, no optimizer",
+            "ms_per_step": ms, "ms_per_step_median": _median(step_ms), "tokens_per_step": T,
+            "layers": L, "roofline": roof, "kernels": _kernel_table(kernels),
+            "gpu_launches": sum(n for n, _ in kernels.values()), "clocks": clocks}
+
+
 def measure_mfalcon(ctx, steps, warmup, with_e2e, sample_clocks=True, batch=None):
     """Time mfalcon_score over every candidate of the M-FALCON workload (the
     history is encoded once beforehand, with its K/V kept per layer)."""
@@ -725,6 +800,11 @@ def main():
         if rank == 0:
             print(json.dumps({**r, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                               "higher_is_better": True, "data": "synthetic"}), flush=True)
+    elif args.workload == "long-bf16-train":
+        r = measure_train(ctx, args.steps, args.warmup, batch=args.batch)
+        if rank == 0:
+            print(json.dumps({**r, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "higher_is_better": True, "data": "synthetic"}), flush=True)
     elif args.workload == "mfalcon":
         r = measure_mfalcon(ctx, args.steps, args.warmup, not args.no_e2e, batch=args.batch)
         line = {"metric": MFALCON_METRIC, "value": r["value"], "unit": "candidates/s",
@@ -772,6 +852,7 @@ def main():
                                                      False, sample_clocks=(name == "sl-bf16")))
             subs["mfalcon"] = measure_mfalcon(ctx, min(args.steps, 20), args.warmup, True)
             subs["sl-sampler"] = measure_sl_sampler(ctx, min(args.steps, 20), args.warmup)
+            subs["long-bf16-train"] = measure_train(ctx, min(args.steps, 10), args.warmup)
             line["workloads"] = subs
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_extrapolated(case)
