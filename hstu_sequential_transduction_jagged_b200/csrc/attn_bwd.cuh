@@ -17,9 +17,13 @@
 //   hstu_attn_bwd_q_kernel: one CTA per (head, user, 128-query tile) walks the
 //     key tiles up to its diagonal: S = Q K^T and dP = dO V^T, dS by the
 //     element warps, dQ += dS K.
-// Warp roles (320 threads): warps 0-7 element work (thread = one row of the
-// tile: lane quarter warp & 3, 64-column half warp >> 2), warp 8 TMA
-// producer, warp 9 MMA issue (one elected lane).  Every wait is bounded.
+// Warp roles (576 threads): warps 0-15 element work (thread = one row of the
+// own tile: lane quarter warp & 3; 32 of the streamed tile's 128 rows:
+// column group warp >> 2), warp 16 TMA producer, warp 17 MMA issue (one
+// elected lane).  Per element the time bucket comes from an exact
+// incremental walk over the thread's monotone time differences, and the
+// position bias from the tile pair's 255-entry band staged in shared memory.
+// Every wait is bounded.
 #pragma once
 
 #include "attn.cuh"
@@ -28,9 +32,10 @@ namespace hstu {
 
 constexpr int BW_ROWS = 128;          // rows of the tile the CTA owns
 constexpr int BW_COLS = 128;          // rows of each streamed tile
-constexpr int BW_THREADS = 320;
-constexpr int BW_PRODUCER_WARP = 8;
-constexpr int BW_MMA_WARP = 9;
+constexpr int BW_ELEM_WARPS = 16;
+constexpr int BW_THREADS = (BW_ELEM_WARPS + 2) * 32;
+constexpr int BW_PRODUCER_WARP = BW_ELEM_WARPS;
+constexpr int BW_MMA_WARP = BW_ELEM_WARPS + 1;
 constexpr uint32_t BW_TILE_BYTES = 128 * ATT_HD * 2;  // one 128 x 64 fp16 tile: 16 KB
 
 struct AttnBwdParams {
@@ -48,7 +53,7 @@ struct AttnBwdParams {
   int32_t phi2;
   int32_t hist_len;            // position-gradient entries kept in shared memory
   uint64_t timeout_ns;
-  int4 oct[32];                // time-bucket octave table (see time_bucket_octave)
+  int32_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0), clamped to int32
 };
 
 struct BwSmem {
@@ -57,8 +62,9 @@ struct BwSmem {
   static constexpr uint32_t kStg = kOwn1 + BW_TILE_BYTES;   // 2 stages x (2 tiles)
   static constexpr uint32_t kStgBytes = 2 * BW_TILE_BYTES;
   static constexpr uint32_t kTimes = kStg + 2 * kStgBytes;  // 2 x 128 int32 (streamed rows)
-  static constexpr uint32_t kOct = kTimes + 2 * 128 * 4;    // 32 x int4
-  static constexpr uint32_t kRt = kOct + 32 * 16;           // Tb floats (rab_time row)
+  static constexpr uint32_t kBand = kTimes + 2 * 128 * 4;   // 2 x 256 floats: rab_pos band
+  static constexpr uint32_t kThr = kBand + 2 * 256 * 4;     // Tb int32 thresholds
+  static constexpr uint32_t kRt = kThr + MAX_TIME_BUCKETS * 4;  // Tb floats (rab_time row)
   static constexpr uint32_t kTg = kRt + MAX_TIME_BUCKETS * 4;   // Tb floats (time gradient)
   static constexpr uint32_t kBars = kTg + MAX_TIME_BUCKETS * 4; // 16 barriers
   static constexpr uint32_t kMisc = kBars + 16 * 8;
@@ -134,7 +140,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint8_t* sOwn1 = smem + BwSmem::kOwn1;
   uint8_t* sStg = smem + BwSmem::kStg;
   int32_t* sTimes = reinterpret_cast<int32_t*>(smem + BwSmem::kTimes);
-  int4* sOct = reinterpret_cast<int4*>(smem + BwSmem::kOct);
+  float* sBand = reinterpret_cast<float*>(smem + BwSmem::kBand);
+  int32_t* sThr = reinterpret_cast<int32_t*>(smem + BwSmem::kThr);
   float* sRt = reinterpret_cast<float*>(smem + BwSmem::kRt);
   float* sTg = reinterpret_cast<float*>(smem + BwSmem::kTg);
   float* sPg = reinterpret_cast<float*>(smem + BwSmem::kPg);
@@ -153,7 +160,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&bars[BWB_EMPTY + s], 1);
     }
     mbar_init(&bars[BWB_S], 1);
-    mbar_init(&bars[BWB_P], 8 * 32);
+    mbar_init(&bars[BWB_P], BW_ELEM_WARPS * 32);
     mbar_init(&bars[BWB_DONE], 1);
     *sAbort = 0;
     fence_mbar_init();
@@ -162,8 +169,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tmem_alloc(sTmemBase, 512);
     tmem_relinquish();
   }
-  if (tid < 32) sOct[tid] = p.oct[tid];
   for (int k = tid; k < p.Tb; k += BW_THREADS) {
+    sThr[k] = p.thr[k];
     sRt[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     if (KV) sTg[k] = 0.0f;
   }
@@ -249,8 +256,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!ok) break;
       tc_fence_after();
       // accumulate over the 128 streamed rows (K = 128: eight steps); the
-      // packed 16-bit operand of rows 0-63 sits at columns 0-31 of its
-      // region, rows 64-127 at columns 64-95
+      // packed 16-bit operand of rows 32g .. 32g + 31 sits at columns
+      // 32g .. 32g + 15 of its region
       const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                // MN-major B
       const uint64_t dS1m = smem_desc_sw128(sa + BW_TILE_BYTES, 8192, 1024);
       if (leader) {
@@ -258,13 +265,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           // dV += P^T dO ; dK += dS^T Q
 #pragma unroll
           for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
             mma_bf16_ts(tmem + kAcc0, tmem + kX + ac, dS1m + 128 * kk, idesc_ts,
                         (it > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
             mma_bf16_ts(tmem + kAcc1, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
                         (it > 0 || kk > 0) ? 1u : 0u);
           }
@@ -272,7 +279,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           // dQ += dS K
 #pragma unroll
           for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
             mma_bf16_ts(tmem + kAcc0, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
                         (it > 0 || kk > 0) ? 1u : 0u);
           }
@@ -286,7 +293,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_wait_drain(&bars[BWB_DONE], 0, p.timeout_ns);
   } else {
     // ---------------- element warps
-    const int q4 = warp & 3, half = warp >> 2;
+    const int q4 = warp & 3, cg = warp >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const int r = q4 * 32 + lane;        // row of the own tile
     const int orow = o0 + r;             // its index within the user
@@ -294,108 +301,124 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int32_t t_own = own_ok ? bw_rel_time(p.timestamps, start + orow, t_first) : 0;
     const float inv_n = 1.0f / static_cast<float>(n);
     const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
-    // time-gradient running sum (KV): current bucket and its partial sum
-    int tb_cur = -1;
+    const int c0 = cg * 32;              // this warp's 32 streamed rows of each tile
+    // Time-bucket walk over this thread's visible pairs in the order visited:
+    // KV: dt = t_i - t_own grows with the query i (bucket goes up from 0);
+    // Q:  dt = t_own - t_j shrinks with the key j (bucket goes down from Tb-1).
+    // The bucket of dt is the largest b with thr[b] <= dt (thr[0] = 0).
+    int tb = KV ? 0 : p.Tb - 1;
+    float rt_cur = sRt[tb];
+    // time-gradient running sum (KV): partial sum of the current bucket
     float tg_acc = 0.0f;
-    auto flush_tg = [&]() {
-      if (tb_cur >= 0 && tg_acc != 0.0f) atomicAdd(&sTg[tb_cur], tg_acc);
-      tg_acc = 0.0f;
-    };
     float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1 (KV)
     bool ok = true;
     for (int it = 0; it < n_st; ++it) {
       const int sbase = (st0 + it) * BW_COLS;  // first streamed row
-      // this tile's 128 streamed times (all element threads, then a barrier)
+      // this tile's 128 streamed times and the 255-entry position-bias band:
+      // entry e holds rab_pos[min(|D|, P - 1)] for D = i - j = dbase + e - 127
       int32_t* tt = sTimes + (it & 1) * 128;
-      if (tid < 128 && tid >= 0) {
+      float* band = sBand + (it & 1) * 256;
+      const int dbase = KV ? sbase - o0 : o0 - sbase;
+      if (tid < 128) {
         const int row = sbase + tid;
-        if (warp < 4) tt[tid] = row < n ? bw_rel_time(p.timestamps, start + row, t_first) : 0;
+        tt[tid] = row < n ? bw_rel_time(p.timestamps, start + row, t_first) : 0;
+      } else if (tid < 128 + 255) {
+        const int e = tid - 128;
+        const int dd = dbase + e - 127;
+        band[e] = dd >= 0 ? __ldg(rp + min(dd, p.P - 1)) : 0.0f;
       }
-      named_barrier_sync(1, 8 * 32);
+      named_barrier_sync(1, BW_ELEM_WARPS * 32);
       if (ok) ok = mbar_wait(&bars[BWB_S], static_cast<uint32_t>(it) & 1u, ctl);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          const int c0 = half * 64 + ch * 32;  // first column of this chunk
-          uint32_t xs[32], ys[32];
-          tmem_ld32(tmem + lane_off + kX + static_cast<uint32_t>(c0), xs);
-          tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
-          tmem_ld_wait(xs);
-          tmem_ld_wait(ys);
-          uint32_t px[16], py[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float pv[2], dsv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int srow = sbase + c0 + c + e;  // streamed row index within the user
-              // KV: own = key j, streamed = query i; Q: own = query i, streamed = key j
-              const int qi = KV ? srow : orow;
-              const int kj = KV ? orow : srow;
-              const bool vis = own_ok && srow < n && kj <= qi;
-              float pp = 0.0f, ds = 0.0f;
-              if (vis) {
-                const int dpos = qi - kj;
-                const int bp = min(dpos, p.P - 1);
-                const int32_t ti = KV ? tt[c0 + c + e] : t_own;
-                const int32_t tj = KV ? t_own : tt[c0 + c + e];
-                const int bt = min(time_bucket_octave(ti - tj, sOct), p.Tb - 1);
-                const float sv = __uint_as_float(xs[c + e]) + __ldg(rp + bp) + sRt[bt];
-                float ph, pg;
-                phi_and_grad<PHI>(sv, ph, pg);
-                pp = ph * inv_n;
-                ds = __uint_as_float(ys[c + e]) * pg * inv_n;
-                if (KV) {
-                  if (bp == p.P - 1) pg_clamp += ds;
-                  else if (bp < p.hist_len) atomicAdd(&sPg[bp], ds);
-                  if (bt != tb_cur) {
-                    flush_tg();
-                    tb_cur = bt;
-                  }
-                  tg_acc += ds;
-                }
-              }
-              pv[e] = pp;
-              dsv[e] = ds;
-            }
-            if constexpr (F16) {
-              px[c >> 1] = pack_h2(pv[0], pv[1]);
-              py[c >> 1] = pack_h2(dsv[0], dsv[1]);
-            } else {
-              px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-              py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-            }
-          }
-          // the packed operands go over columns this warp has read:
-          // rows 0-63 of the streamed tile at columns 0-31, 64-127 at 64-95
-          const uint32_t pc = static_cast<uint32_t>(half * 64 + ch * 16);
-          __syncwarp();
-          if (KV) tmem_st16(tmem + lane_off + kX + pc, px);
-          tmem_st16(tmem + lane_off + kY + pc, py);
-          tmem_st_wait();
+        uint32_t xs[32], ys[32];
+        tmem_ld32(tmem + lane_off + kX + static_cast<uint32_t>(c0), xs);
+        tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
+        tmem_ld_wait(xs);
+        tmem_ld_wait(ys);
+        // visible streamed columns of this thread: KV: i >= j and i < n;
+        // Q: j <= i (and j < n, implied)
+        int c_lo = 0, c_hi = 31;
+        if (!own_ok) {
+          c_lo = 32;
+        } else if (KV) {
+          c_lo = max(0, orow - (sbase + c0));
+          c_hi = min(31, n - 1 - (sbase + c0));
+        } else {
+          c_hi = min(31, orow - (sbase + c0));
         }
+        uint32_t px[16], py[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int cc = c + e;
+            float pp = 0.0f, ds = 0.0f;
+            if (cc >= c_lo && cc <= c_hi) {
+              const int32_t dt = KV ? tt[c0 + cc] - t_own : t_own - tt[c0 + cc];
+              if (KV) {
+                if (tb + 1 < p.Tb && dt >= sThr[tb + 1]) {
+                  if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+                  tg_acc = 0.0f;
+                  do { ++tb; } while (tb + 1 < p.Tb && dt >= sThr[tb + 1]);
+                  rt_cur = sRt[tb];
+                }
+              } else if (tb > 0 && dt < sThr[tb]) {
+                do { --tb; } while (tb > 0 && dt < sThr[tb]);
+                rt_cur = sRt[tb];
+              }
+              // D = i - j; band index D - dbase + 127
+              const int dpos = KV ? (sbase + c0 + cc) - orow : orow - (sbase + c0 + cc);
+              const float sv = __uint_as_float(xs[cc]) + band[dpos - dbase + 127] + rt_cur;
+              float ph, pg;
+              phi_and_grad<PHI>(sv, ph, pg);
+              pp = ph * inv_n;
+              ds = __uint_as_float(ys[cc]) * pg * inv_n;
+              if (KV) {
+                if (dpos >= p.P - 1) pg_clamp += ds;
+                else atomicAdd(&sPg[dpos], ds);  // dpos < min(P - 1, max_len) <= hist_len
+                tg_acc += ds;
+              }
+            }
+            pv[e] = pp;
+            dsv[e] = ds;
+          }
+          if constexpr (F16) {
+            px[c >> 1] = pack_h2(pv[0], pv[1]);
+            py[c >> 1] = pack_h2(dsv[0], dsv[1]);
+          } else {
+            px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+            py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+          }
+        }
+        // the packed operands go over the first 16 of the 32 columns this warp read
+        __syncwarp();
+        if (KV) tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
+        tmem_st16(tmem + lane_off + kY + static_cast<uint32_t>(c0), py);
+        tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&bars[BWB_P]);
     }
-    if (KV) flush_tg();
-    // ---------------- epilogue: the accumulators (rows of the own tile)
+    if (KV && tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+    // ---------------- epilogue: the accumulators (rows of the own tile); the
+    // four column groups take 16 of the 64 accumulator columns each
     if (ok) ok = mbar_wait(&bars[BWB_DONE], 0, ctl);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const int64_t grow = start + orow;
       for (int a = 0; a < (KV ? 2 : 1); ++a) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + (a == 0 ? kAcc0 : kAcc1) + static_cast<uint32_t>(half * 32), v);
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_off + (a == 0 ? kAcc0 : kAcc1) + static_cast<uint32_t>(cg * 16), v);
         tmem_ld_wait(v);
         float* dst = KV ? (a == 0 ? p.dv : p.dk) : p.dq;
         if (own_ok) {
-          float4* d4 = reinterpret_cast<float4*>(dst + grow * p.ld_g + h * ATT_HD + half * 32);
+          float4* d4 = reinterpret_cast<float4*>(dst + grow * p.ld_g + h * ATT_HD + cg * 16);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
+          for (int q = 0; q < 4; ++q)
             d4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
         }

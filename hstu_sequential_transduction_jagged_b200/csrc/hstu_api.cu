@@ -637,7 +637,9 @@ hstu_status_t launch_attn_bwd(const hstu_layer_cfg_t* c, const hstu_jagged_t* ja
   p.phi2 = c->phi2;
   p.hist_len = std::min(P, jag->max_len);
   p.timeout_ns = kDefaultTimeoutNs;
-  if (!compute_octaves(Tb, thresholds_for(Tb), p.oct)) return HSTU_ERR_UNSUPPORTED;
+  const int64_t* thr = thresholds_for(Tb);
+  for (int b = 0; b < Tb; ++b)
+    p.thr[b] = thr[b] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(thr[b]) : INT32_MAX;
   const size_t smem = BwSmem::bytes(p.hist_len);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   dim3 grid(H, jag->batch, (jag->max_len + BW_ROWS - 1) / BW_ROWS);
