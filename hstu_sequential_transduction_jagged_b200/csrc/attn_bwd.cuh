@@ -68,7 +68,8 @@ struct BwSmem {
   static constexpr uint32_t kTg = kRt + MAX_TIME_BUCKETS * 4;   // Tb floats (time gradient)
   static constexpr uint32_t kBars = kTg + MAX_TIME_BUCKETS * 4; // 16 barriers
   static constexpr uint32_t kMisc = kBars + 16 * 8;
-  static constexpr uint32_t kPg = kMisc + 64;               // hist_len floats (position gradient)
+  static constexpr uint32_t kDiag = kMisc + 64;             // per element warp 64 floats
+  static constexpr uint32_t kPg = kDiag + BW_ELEM_WARPS * 64 * 4;  // hist_len floats (position gradient)
   static constexpr uint32_t bytes(int hist_len) {
     return kPg + static_cast<uint32_t>(hist_len) * 4u + 1024u;
   }
@@ -145,6 +146,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   float* sRt = reinterpret_cast<float*>(smem + BwSmem::kRt);
   float* sTg = reinterpret_cast<float*>(smem + BwSmem::kTg);
   float* sPg = reinterpret_cast<float*>(smem + BwSmem::kPg);
+  float* sDiag = reinterpret_cast<float*>(smem + BwSmem::kDiag);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BwSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + BwSmem::kMisc);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + BwSmem::kMisc + 4);
@@ -176,6 +178,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   }
   if (KV)
     for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
+  if (KV)
+    for (int k = tid; k < BW_ELEM_WARPS * 64; k += BW_THREADS) sDiag[k] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -308,6 +312,15 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // The bucket of dt is the largest b with thr[b] <= dt (thr[0] = 0).
     int tb = KV ? 0 : p.Tb - 1;
     float rt_cur = sRt[tb];
+    // the edge the walk compares against: thr[tb + 1] (KV, INT32_MAX past the
+    // last bucket) or thr[tb] (Q)
+    int32_t edge = KV ? (p.Tb > 1 ? sThr[1] : INT32_MAX) : sThr[tb];
+    // position-table gradient (KV): this warp's 32 x 32 block adds dS to its
+    // 63 diagonals D = i - j = dg0 + cc - lane in `diag` (index cc - lane + 31).
+    // The 32 lanes of one column touch 32 different diagonals, so the adds are
+    // plain read-modify-writes (a __syncwarp before each keeps the lanes in
+    // step); the block's diagonals go to the CTA histogram afterwards.
+    float* diag = sDiag + warp * 64;
     // time-gradient running sum (KV): partial sum of the current bucket
     float tg_acc = 0.0f;
     float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1 (KV)
@@ -355,18 +368,22 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int cc = c + e;
-            float pp = 0.0f, ds = 0.0f;
+            float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
             if (cc >= c_lo && cc <= c_hi) {
               const int32_t dt = KV ? tt[c0 + cc] - t_own : t_own - tt[c0 + cc];
               if (KV) {
-                if (tb + 1 < p.Tb && dt >= sThr[tb + 1]) {
+                if (dt >= edge) {
                   if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
                   tg_acc = 0.0f;
-                  do { ++tb; } while (tb + 1 < p.Tb && dt >= sThr[tb + 1]);
+                  do {
+                    ++tb;
+                    edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
+                  } while (dt >= edge);
                   rt_cur = sRt[tb];
                 }
-              } else if (tb > 0 && dt < sThr[tb]) {
+              } else if (dt < edge) {
                 do { --tb; } while (tb > 0 && dt < sThr[tb]);
+                edge = sThr[tb];
                 rt_cur = sRt[tb];
               }
               // D = i - j; band index D - dbase + 127
@@ -378,9 +395,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               ds = __uint_as_float(ys[cc]) * pg * inv_n;
               if (KV) {
                 if (dpos >= p.P - 1) pg_clamp += ds;
-                else atomicAdd(&sPg[dpos], ds);  // dpos < min(P - 1, max_len) <= hist_len
+                else dsp = ds;
                 tg_acc += ds;
               }
+            }
+            if (KV) {
+              __syncwarp();
+              diag[cc - lane + 31] += dsp;
             }
             pv[e] = pp;
             dsv[e] = ds;
@@ -391,6 +412,19 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           } else {
             px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
             py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+          }
+        }
+        if (KV) {
+          // this block's diagonals into the CTA histogram (dpos < P - 1 <= hist_len
+          // there; clamped pairs went to pg_clamp), and the buffer cleared
+          __syncwarp();
+          const int dg0 = (sbase + c0) - (o0 + q4 * 32);
+#pragma unroll
+          for (int k = lane; k < 63; k += 32) {
+            const float v = diag[k];
+            const int dd = dg0 + k - 31;
+            if (v != 0.0f && dd >= 0 && dd < p.P - 1) atomicAdd(&sPg[dd], v);
+            diag[k] = 0.0f;
           }
         }
         // the packed operands go over the first 16 of the 32 columns this warp read
