@@ -291,7 +291,11 @@ struct AttnSmem {
   static constexpr uint32_t kTailABlock = ATT_ROWS * 128;
   static constexpr int kTailAStages = 3;
   static constexpr uint32_t kTailA = (kPos + 1023u) & ~1023u;
-  static constexpr uint32_t kTailBytes = kTailA + kTailAStages * kTailABlock + 1024u;  // + align slack
+  // epilogue staging, per element warp 32 rows x 32 fp32 (4 KB), over the A
+  // ring (idle between a tile's last MMA and the next tile's A build)
+  static constexpr uint32_t kTailStage = kTailA;
+  static constexpr uint32_t kTailBytes = kTailA + 16 * 4096 + 1024u;  // + align slack
+  static_assert(16 * 4096 >= kTailAStages * kTailABlock, "staging covers the A ring");
   static_assert(kTailW + kTailWStages * kTailBox <= kKeyInfo, "tail W2 ring overlaps the side data");
   static constexpr uint32_t bytes(int pos_len, bool pairs, uint32_t elt = 4u) {
     return kPos + static_cast<uint32_t>(pos_len) * elt * (pairs ? 2u : 1u) + 1024u;  // + align slack
@@ -613,59 +617,58 @@ __device__ __forceinline__ void attn_f2_tail(const CUtensorMap* tm_w2, const Att
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;  // keep arriving: the other threads' barriers stay consistent
       tc_fence_after();
-      const int r = q4 * 32 + lane;
-      const bool row_ok = base + r < n_q;
-      const int64_t row = q_start + base + r;
+      // Each warp owns rows base + 32 q4 .. + 31 (its tensor-memory lane
+      // quarter) and 128 columns.  Per 32-column chunk the accumulators go
+      // through a 128B-swizzled 32 x 32 staging block, so that the residual
+      // loads and the Y stores run along rows: lane l takes row 4k + l / 8 and
+      // columns 4 (l % 8) .. + 3 of the chunk, one 128-byte row segment per 8
+      // lanes.  Y = (accumulator + b2) + residual, the unfused epilogue's order.
+      uint8_t* stg = smem + AttnSmem::kTailStage + warp * 4096;
+      const int r0 = base + q4 * 32;          // first row of this warp (within the user)
+      const int rsub = lane >> 3, j4 = lane & 7;
+      const bool h16 = t.ylp_f16 != 0;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         const int col = cg * 128 + ch * 32;
         if (col >= t.N) break;  // warp-uniform
-        float4 xr[8];
-        if (row_ok) {
-          if (t.x_res != nullptr) {
-            const float4* xp = reinterpret_cast<const float4*>(t.x_res + row * t.ld_x + col);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) xr[q] = xp[q];
-          } else {
-            const uint4* xp = reinterpret_cast<const uint4*>(t.x_lp + row * t.ld_x + col);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 xx = xp[q];
-              const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xx);
-              const float2 f0 = __bfloat1622float2(x2[0]), f1 = __bfloat1622float2(x2[1]);
-              const float2 f2 = __bfloat1622float2(x2[2]), f3 = __bfloat1622float2(x2[3]);
-              xr[2 * q] = make_float4(f0.x, f0.y, f1.x, f1.y);
-              xr[2 * q + 1] = make_float4(f2.x, f2.y, f3.x, f3.y);
-            }
-          }
-        }
         uint32_t v[32];
         __syncwarp();
         tmem_ld32(tmem + lane_off + static_cast<uint32_t>(col), v);
         tmem_ld_wait(v);
-        if (!row_ok) continue;
-        // accumulator + b2 + residual, in the order of the unfused f2 epilogue
-        float y[32];
-        const float4* b4 = reinterpret_cast<const float4*>(t.b2 + col);
+        // row `lane` of the block: 16-byte chunk q at (q ^ (lane & 7))
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 bb = __ldg(b4 + q);
-          y[4 * q + 0] = __uint_as_float(v[4 * q + 0]) + bb.x + xr[q].x;
-          y[4 * q + 1] = __uint_as_float(v[4 * q + 1]) + bb.y + xr[q].y;
-          y[4 * q + 2] = __uint_as_float(v[4 * q + 2]) + bb.z + xr[q].z;
-          y[4 * q + 3] = __uint_as_float(v[4 * q + 3]) + bb.w + xr[q].w;
-        }
-        float4* yo = reinterpret_cast<float4*>(t.y + row * t.ld_y + col);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) yo[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-        if (t.y_lp != nullptr) {
-          uint4* lo = reinterpret_cast<uint4*>(static_cast<uint16_t*>(t.y_lp) + row * t.ld_y + col);
-          const bool h16 = t.ylp_f16 != 0;
-          auto pk2 = [h16](float a, float b) { return h16 ? pack_h2(a, b) : pack_bf16x2(a, b); };
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            lo[q] = make_uint4(pk2(y[8 * q], y[8 * q + 1]), pk2(y[8 * q + 2], y[8 * q + 3]),
-                               pk2(y[8 * q + 4], y[8 * q + 5]), pk2(y[8 * q + 6], y[8 * q + 7]));
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+              make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        __syncwarp();
+        const float4 bb = __ldg(reinterpret_cast<const float4*>(t.b2 + col) + j4);
+#pragma unroll 2
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + rsub;
+          if (r0 + rr < n_q) {
+            const int64_t grow = q_start + r0 + rr;
+            const float4 a = *reinterpret_cast<const float4*>(stg + rr * 128 + ((j4 ^ (rr & 7)) << 4));
+            float4 xx;
+            if (t.x_res != nullptr) {
+              xx = *reinterpret_cast<const float4*>(t.x_res + grow * t.ld_x + col + 4 * j4);
+            } else {
+              const uint2 xb = *reinterpret_cast<const uint2*>(t.x_lp + grow * t.ld_x + col + 4 * j4);
+              const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.x));
+              const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb.y));
+              xx = make_float4(f0.x, f0.y, f1.x, f1.y);
+            }
+            float4 y;
+            y.x = a.x + bb.x + xx.x;
+            y.y = a.y + bb.y + xx.y;
+            y.z = a.z + bb.z + xx.z;
+            y.w = a.w + bb.w + xx.w;
+            *reinterpret_cast<float4*>(t.y + grow * t.ld_y + col + 4 * j4) = y;
+            if (t.y_lp != nullptr) {
+              auto pk2 = [h16](float a0, float a1) { return h16 ? pack_h2(a0, a1) : pack_bf16x2(a0, a1); };
+              *reinterpret_cast<uint2*>(static_cast<uint16_t*>(t.y_lp) + grow * t.ld_y + col + 4 * j4) =
+                  make_uint2(pk2(y.x, y.y), pk2(y.z, y.w));
+            }
+          }
         }
       }
     }
