@@ -559,21 +559,24 @@ __device__ __forceinline__ void attn_f2_tail(const CUtensorMap* tm_w2, const Att
       named_barrier_sync(3, 16 * 32);
       // A blocks: 128 rows x 8 chunks of 8 columns; this thread's two chunks
       // (rows tid/8 and tid/8 + 64, chunk tid%8) of every block
+      // lane j of each group of 8 takes columns 4j .. 4j + 3 and 32 + 4j .. + 3
+      // of the block: each load instruction reads whole 128-byte rows; the
+      // results go to the two 8-byte halves of their swizzled 16-byte chunks
       const int j = tid & 7;
       for (int kb = 0; kb < k_blocks; ++kb) {
-        const int col = kb * 64 + j * 8;
+        const int colA = kb * 64 + 4 * j, colB = colA + 32;
         float4 av[2][2], uv[2][2];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int r = (tid >> 3) + h2 * 64;
           if (base + r < n_q) {
             const int64_t row = q_start + base + r;
-            const float4* ap = reinterpret_cast<const float4*>(p.av_f32 + row * p.ld_av + col);
-            const float4* up = reinterpret_cast<const float4*>(t.u + row * t.ld_u + col);
-            av[h2][0] = __ldcg(ap);
-            av[h2][1] = __ldcg(ap + 1);
-            uv[h2][0] = up[0];
-            uv[h2][1] = up[1];
+            const float* ap = p.av_f32 + row * p.ld_av;
+            const float* up = t.u + row * t.ld_u;
+            av[h2][0] = __ldcg(reinterpret_cast<const float4*>(ap + colA));
+            av[h2][1] = __ldcg(reinterpret_cast<const float4*>(ap + colB));
+            uv[h2][0] = *reinterpret_cast<const float4*>(up + colA);
+            uv[h2][1] = *reinterpret_cast<const float4*>(up + colB);
           } else {
             av[h2][0] = av[h2][1] = uv[h2][0] = uv[h2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
@@ -581,8 +584,9 @@ __device__ __forceinline__ void attn_f2_tail(const CUtensorMap* tm_w2, const Att
         float gm[8], bt[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          gm[e] = t.gamma != nullptr ? __ldg(t.gamma + col + e) : 1.0f;
-          bt[e] = t.beta != nullptr ? __ldg(t.beta + col + e) : 0.0f;
+          const int c = (e < 4 ? colA : colB - 4) + e;
+          gm[e] = t.gamma != nullptr ? __ldg(t.gamma + c) : 1.0f;
+          bt[e] = t.beta != nullptr ? __ldg(t.beta + c) : 0.0f;
         }
         if (ok) ok = mbar_wait(&bars[BAR_T_A_EMPTY + as], aph ^ 1u, ctl);
         uint8_t* blk = sA + as * kABlk;
@@ -602,10 +606,15 @@ __device__ __forceinline__ void attn_f2_tail(const CUtensorMap* tm_w2, const Att
                 fmaf((af[2 * e + 1] - sr.x) * sr.y, gm[2 * e + 1], bt[2 * e + 1]) * uf[2 * e + 1];
             w[e] = pack_h2(g0, g1);
           }
-          // rows past the end carry zeros (their statistics and data are zero)
-          if (ok)
-            *reinterpret_cast<uint4*>(blk + r * 128 + ((j ^ (r & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+          // rows past the end carry zeros (their statistics and data are zero);
+          // columns 4j.. sit in chunk j / 2, 32 + 4j.. in chunk 4 + j / 2
+          if (ok) {
+            const int half8 = (j & 1) * 8;
+            *reinterpret_cast<uint2*>(blk + r * 128 + (((j >> 1) ^ (r & 7)) << 4) + half8) =
+                make_uint2(w[0], w[1]);
+            *reinterpret_cast<uint2*>(blk + r * 128 + (((4 + (j >> 1)) ^ (r & 7)) << 4) + half8) =
+                make_uint2(w[2], w[3]);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();  // the previous tile's tensor-memory reads, before the MMAs reuse it
