@@ -108,3 +108,37 @@ def test_status_strings(H):
     for code in range(7):
         assert L.hstu_status_string(code)
     assert b"unknown" in L.hstu_status_string(99)
+
+
+def test_backward_and_flag_validation_without_device(H):
+    """hstu_attn_bwd / hstu_layer_bwd / cfg.flags reject bad arguments on the
+    host (before any device work)."""
+    L = H.lib()
+    ok_jag = H.JaggedT(0, 0, 0, None, None)
+    # unknown flag bits
+    bad_flags = _cfg(H).c()
+    bad_flags.flags = 6
+    st = L.hstu_attn_fwd(ctypes.byref(bad_flags), ctypes.byref(ok_jag), None, None, None, None,
+                         None, None, None, 0, None)
+    assert st == 1
+    # the backward has no softmax, fp32 or generalised-mask form
+    soft = _cfg(H, phi2="softmax", dtype="fp16").c()
+    st = L.hstu_attn_bwd(ctypes.byref(soft), ctypes.byref(ok_jag), *([None] * 12))
+    assert st == 2
+    f32 = _cfg(H, dtype="fp32").c()
+    st = L.hstu_attn_bwd(ctypes.byref(f32), ctypes.byref(ok_jag), *([None] * 12))
+    assert st == 2
+    seg_jag = H.JaggedT(0, 0, 0, None, None, 16, 0)  # segments given
+    good16 = _cfg(H, dtype="fp16").c()
+    st = L.hstu_attn_bwd(ctypes.byref(good16), ctypes.byref(seg_jag), *([None] * 12))
+    assert st == 2
+    # NULL tables
+    st = L.hstu_attn_bwd(ctypes.byref(good16), ctypes.byref(ok_jag), *([None] * 12))
+    assert st == 1
+    # layer backward: bf16 only, NULL weights / gradients rejected
+    bf = _cfg(H).c()
+    st = L.hstu_layer_bwd(ctypes.byref(bf), None, ctypes.byref(ok_jag), *([None] * 6), 0, None)
+    assert st == 1
+    assert L.hstu_layer_bwd_workspace_bytes(ctypes.byref(f32), 100) == 0
+    assert L.hstu_layer_bwd_workspace_bytes(ctypes.byref(bf), 1000) > H.layer_workspace_bytes(
+        _cfg(H), 1000)
