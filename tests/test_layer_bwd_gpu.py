@@ -100,3 +100,34 @@ def test_layer_backward_rejects_unsupported(H):
     dy = torch.zeros((case.total_tokens, case.cfg.d_model), dtype=torch.float32, device="cuda")
     with pytest.raises(H.HSTUError):
         H.layer_bwd(config_of(H, case.cfg), weights[0], jag, t["x"], dy)
+
+
+def test_two_layer_chain(H):
+    """The training step's chain: backward through layer 1, then through layer 0
+    with the dX of one as the dY of the other; every gradient of both layers
+    and the input gradient against the oracle chained the same way.  Layer 1
+    takes the oracle's layer-0 output (fp32) on both sides: f1 reads it rounded
+    to fp16, and an input that differed by the forward's own rounding would
+    flip ReLU' on near-zero pre-activations (whole gradient entries), which a
+    chained forward on each side would compare rather than the backward."""
+    case = make_case("sl-bf16", seed=97, lengths=[600, 129, 1], num_layers=2)
+    t, jag, weights = upload(H, case)
+    cfg = config_of(H, case.cfg)
+    rng = np.random.default_rng(98)
+    dy = rng.standard_normal((case.total_tokens, case.cfg.d_model)).astype(np.float32)
+    y0_ref = O.layer_fwd(case.x, case.offsets, case.timestamps, case.layers[0], case.cfg,
+                         keep_stages=False)["y"].astype(np.float32)
+    g1 = H.layer_bwd(cfg, weights[1], jag, None, tensor(dy, torch.float32, "cuda"),
+                     x_res=tensor(y0_ref, torch.float32, "cuda"))
+    g0 = H.layer_bwd(cfg, weights[0], jag, t["x"], g1["dx"])
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    w1 = OB.layer_bwd(y0_ref.astype(np.float64), case.offsets, case.timestamps, case.layers[1],
+                      case.cfg, dy.astype(np.float64),
+                      x_f1=round_fp16(y0_ref).astype(np.float64))
+    w0 = OB.layer_bwd(case.x, case.offsets, case.timestamps, case.layers[0], case.cfg, w1["dx"])
+    for tag, got, want in (("layer 1", g1, w1), ("layer 0", g0, w0)):
+        for name in NAMES:
+            if want[name] is None:
+                continue
+            _check(got[name].cpu().numpy(), want[name], f"two-layer chain {tag} {name}")
