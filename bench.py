@@ -246,9 +246,11 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     case = make_workload(args.workload)
+    # each step a bounded sample: the whole run stays near 2.5 minutes of host time
+    per_step = max(0.5, min(args.ref_seconds, 150.0 / max(1, args.steps)))
     for _ in range(args.warmup):
-        oracle_extrapolated(case, target_s=1.0)
-    samples = [oracle_extrapolated(case, target_s=args.ref_seconds) for _ in range(args.steps)]
+        oracle_extrapolated(case, target_s=0.5)
+    samples = [oracle_extrapolated(case, target_s=per_step) for _ in range(args.steps)]
     vals = sorted(s["value"] for s in samples)
     v = vals[len(vals) // 2]
     last = samples[-1]
