@@ -660,13 +660,13 @@ def measure_train(ctx, steps, warmup, sample_clocks=False, batch=None):
     # attention backward, FlashAttention convention: five 2*64-flop products
     # per visible (i, j, head): S (recomputed), dP, dV, dQ, dK
     bwd_flop = pairs * c.num_heads * 5 * 2 * 64
-    n_kv, ms_kv = kernels.get("attn_bwd_kv", (0, 0.0))
-    n_q, ms_q = kernels.get("attn_bwd_q", (0, 0.0))
+    n_b, ms_b = kernels.get("attention_bwd", (0, 0.0))
     roof = None
-    if n_kv and n_q:
-        per = ms_kv / n_kv + ms_q / n_q
+    if n_b:
+        per = ms_b / n_b
         ach = bwd_flop / (per / 1000.0) / 1e12
-        roof = {"kernel": "hstu_attn_bwd_kernel (dK/dV + dQ, per layer)", "bound": "tensor",
+        roof = {"kernel": "hstu_attn_bwd_kernel (dK, dV and dQ, one launch per layer)",
+                "bound": "tensor",
                 "achieved": ach, "peak": ctx.peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": ach / ctx.peaks["bf16_tflops"], "traffic": None,
                 "peak_source": f"{ctx.peak_src} bf16 dense, burst ({PEAK_RULE})",

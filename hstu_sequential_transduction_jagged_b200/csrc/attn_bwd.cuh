@@ -4,26 +4,27 @@
 //   dV = A^T dO,  dS = (dO V^T) (.) phi2'(S) / N,  dQ = dS K,  dK = dS^T Q,
 //   drab_pos[h, min(i-j, P-1)] += dS_ij,  drab_time[h, bt(t_i - t_j)] += dS_ij.
 //
-// Two tcgen05 kernels over fp16 Q, K, V, dO (fp32 accumulation in tensor
-// memory, fp32 outputs):
-//   hstu_attn_bwd_kv_kernel: one CTA per (head, user, 128-key tile) walks the
-//     query tiles at and after its keys: S^T = K Q^T and dP^T = V dO^T into
-//     tensor memory, the element warps turn them into P^T and dS^T (fp16,
-//     over the columns they read), then dV += P^T dO and dK += dS^T Q
-//     accumulate in tensor memory.  The table gradients collect in shared
-//     memory (position: one shared atomic per pair; time: a running sum per
-//     row, flushed when the bucket changes) and go to global memory with one
-//     atomic per touched entry at the end.
-//   hstu_attn_bwd_q_kernel: one CTA per (head, user, 128-query tile) walks the
-//     key tiles up to its diagonal: S = Q K^T and dP = dO V^T, dS by the
-//     element warps, dQ += dS K.
-// Warp roles (576 threads): warps 0-15 element work (thread = one row of the
-// own tile: lane quarter warp & 3; 32 of the streamed tile's 128 rows:
-// column group warp >> 2), warp 16 TMA producer, warp 17 MMA issue (one
-// elected lane).  Per element the time bucket comes from an exact
-// incremental walk over the thread's monotone time differences, and the
-// position bias from the tile pair's 255-entry band staged in shared memory.
-// Every wait is bounded.
+// One tcgen05 kernel over fp16 (or bf16) Q, K, V, dO with fp32 accumulation
+// in tensor memory and fp32 outputs.  A CTA owns one (head, user, 128-key
+// tile) and walks the query tiles at and after its keys.  For each tile pair:
+//   S^T = K Q^T and dP^T = V dO^T go to tensor memory; the element warps turn
+//   them into P^T and dS^T (16-bit, over the columns they read) and also write
+//   dS^T to shared memory; then
+//   dQ_part = dS K (A = dS^T read transposed from shared memory) goes to one of
+//   two tensor-memory buffers, and dV += P^T dO, dK += dS^T Q accumulate.
+// While the tensor core runs the next tile pair's MMAs the element warps add
+// the previous dQ_part into dQ in global memory (fp32 vector atomics: the
+// caller's dQ is zeroed first, and the order of the additions is not fixed).
+// dK and dV rows belong to one CTA and are stored once at the end.  The table
+// gradients collect in shared memory (position: a per-warp diagonal buffer
+// flushed per tile pair; time: a running sum per row, flushed when the bucket
+// changes) and go to global memory with one atomic per touched entry at the end.
+// Warp roles (576 threads): warps 0-15 element work (thread = one key row:
+// lane quarter warp & 3; 32 of the query tile's 128 rows: column group
+// warp >> 2), warp 16 TMA producer, warp 17 MMA issue (one elected lane).  Per
+// element the time bucket comes from an exact incremental walk over the
+// thread's increasing time differences, and the position bias from the tile
+// pair's 255-entry band staged in shared memory.  Every wait is bounded.
 #pragma once
 
 #include "attn.cuh"
@@ -43,7 +44,7 @@ struct AttnBwdParams {
   const int64_t* timestamps;   // [T]
   const float* rab_pos;        // [H, P]
   const float* rab_time;       // [H, Tb]
-  float* dq;                   // [T, ld_g] fp32 (head h at columns h*64)
+  float* dq;                   // [T, ld_g] fp32 (head h at columns h*64), accumulated into (caller zeroes)
   float* dk;
   float* dv;
   int64_t ld_g;
@@ -57,11 +58,14 @@ struct AttnBwdParams {
 };
 
 struct BwSmem {
-  static constexpr uint32_t kOwn0 = 0;                      // K (kv kernel) or Q (q kernel)
-  static constexpr uint32_t kOwn1 = kOwn0 + BW_TILE_BYTES;  // V or dO
-  static constexpr uint32_t kStg = kOwn1 + BW_TILE_BYTES;   // 2 stages x (2 tiles)
+  static constexpr uint32_t kOwn0 = 0;                      // K tile
+  static constexpr uint32_t kOwn1 = kOwn0 + BW_TILE_BYTES;  // V tile
+  static constexpr uint32_t kStg = kOwn1 + BW_TILE_BYTES;   // 2 stages x (Q, dO tiles)
   static constexpr uint32_t kStgBytes = 2 * BW_TILE_BYTES;
-  static constexpr uint32_t kTimes = kStg + 2 * kStgBytes;  // 2 x 128 int32 (streamed rows)
+  // dS^T of the current tile pair, 16-bit, 128B-swizzled rows of 64 queries:
+  // queries 0-63 at kDs, 64-127 at kDs + BW_TILE_BYTES (row = key, 128 B)
+  static constexpr uint32_t kDs = kStg + 2 * kStgBytes;
+  static constexpr uint32_t kTimes = kDs + 2 * BW_TILE_BYTES;  // 2 x 128 int32 (query rows)
   static constexpr uint32_t kBand = kTimes + 2 * 128 * 4;   // 2 x 256 floats: rab_pos band
   static constexpr uint32_t kThr = kBand + 2 * 256 * 4;     // Tb int32 thresholds
   static constexpr uint32_t kRt = kThr + MAX_TIME_BUCKETS * 4;  // Tb floats (rab_time row)
@@ -79,10 +83,11 @@ enum : int {
   BWB_OWN = 0,          // the CTA's own two tiles landed
   BWB_FULL = 1,         // + stage
   BWB_EMPTY = 3,        // + stage
-  BWB_S = 5,            // S and dP of the current tile are in tensor memory
-  BWB_P = 6,            // the element warps wrote P / dS
+  BWB_S = 5,            // S^T and dP^T of the current tile pair are in tensor memory
+  BWB_P = 6,            // the element warps wrote P^T / dS^T
   BWB_DONE = 7,         // every MMA completed
-  BWB_COUNT = 8
+  BWB_DQ = 8,           // the tile pair's dQ_part is in tensor memory (dS^T read)
+  BWB_COUNT = 9
 };
 
 // phi2 and its derivative at s (pointwise modes)
@@ -108,11 +113,8 @@ __device__ __forceinline__ int32_t bw_rel_time(const int64_t* ts, int64_t row, i
   return d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d);
 }
 
-// KV = true: the dK/dV kernel (own tile = keys, streamed = queries at and
-// after the keys).  KV = false: the dQ kernel (own tile = queries, streamed =
-// keys up to the diagonal).  F16: fp16 operands (else bf16); P and dS are
-// packed in the operand type.
-template <bool KV, int PHI, bool F16>
+// F16: fp16 operands (else bf16); P and dS are packed in the operand type.
+template <int PHI, bool F16>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -121,25 +123,23 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int h = blockIdx.x, u = blockIdx.y;
-  // longest work first: key tile 0 meets every query tile, query tile z meets z + 1 key tiles
-  const int ot = KV ? static_cast<int>(blockIdx.z)
-                    : static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);
+  // longest work first: key tile 0 meets every query tile
+  const int ot = static_cast<int>(blockIdx.z);
   const int64_t start = p.offsets[u];
   const int n = static_cast<int>(p.offsets[u + 1] - start);
   if (n > p.max_len || n < 0) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_status(HSTU_ERR_DEVICE_CHECK);
     return;
   }
-  const int o0 = ot * BW_ROWS;  // first row (within the user) of the own tile
+  const int o0 = ot * BW_ROWS;  // first key (within the user) of the own tile
   if (o0 >= n) return;          // uniform, before any allocation
   const int n_tiles = (n + BW_COLS - 1) / BW_COLS;
-  // streamed tiles: queries ot .. n_tiles-1 (KV) or keys 0 .. ot (Q)
-  const int st0 = KV ? ot : 0;
-  const int n_st = KV ? n_tiles - ot : ot + 1;
+  const int n_st = n_tiles - ot;  // query tiles ot .. n_tiles - 1
 
   uint8_t* sOwn0 = smem + BwSmem::kOwn0;
   uint8_t* sOwn1 = smem + BwSmem::kOwn1;
   uint8_t* sStg = smem + BwSmem::kStg;
+  uint8_t* sDs = smem + BwSmem::kDs;
   int32_t* sTimes = reinterpret_cast<int32_t*>(smem + BwSmem::kTimes);
   float* sBand = reinterpret_cast<float*>(smem + BwSmem::kBand);
   int32_t* sThr = reinterpret_cast<int32_t*>(smem + BwSmem::kThr);
@@ -164,6 +164,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars[BWB_S], 1);
     mbar_init(&bars[BWB_P], BW_ELEM_WARPS * 32);
     mbar_init(&bars[BWB_DONE], 1);
+    mbar_init(&bars[BWB_DQ], 1);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -174,20 +175,19 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   for (int k = tid; k < p.Tb; k += BW_THREADS) {
     sThr[k] = p.thr[k];
     sRt[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
-    if (KV) sTg[k] = 0.0f;
+    sTg[k] = 0.0f;
   }
-  if (KV)
-    for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
-  if (KV)
-    for (int k = tid; k < BW_ELEM_WARPS * 64; k += BW_THREADS) sDiag[k] = 0.0f;
+  for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
+  for (int k = tid; k < BW_ELEM_WARPS * 64; k += BW_THREADS) sDiag[k] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmemBase;
   const WaitCtl ctl{sAbort, p.timeout_ns};
-  // tensor memory: X = S^T or S (columns 0-127, later the packed P^T / dS
-  // over them), Y = dP^T or dP (128-255), acc0 (256-319), acc1 (320-383)
-  constexpr uint32_t kX = 0, kY = 128, kAcc0 = 256, kAcc1 = 320;
+  // tensor memory: X = S^T (columns 0-127, later the packed P^T over them),
+  // Y = dP^T (128-255, later the packed dS^T), dV (256-319), dK (320-383),
+  // dQ_part of even / odd tile pairs (384-447 / 448-511)
+  constexpr uint32_t kX = 0, kY = 128, kAcc0 = 256, kAcc1 = 320, kDq = 384;
 
   if (warp == BW_PRODUCER_WARP) {
     if (lane == 0) {
@@ -197,27 +197,17 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tma_prefetch_desc(&tm_do);
       const int32_t orow = static_cast<int32_t>(start + o0);
       mbar_arrive_expect_tx(&bars[BWB_OWN], 2 * BW_TILE_BYTES);
-      if (KV) {
-        tma_load_2d(sOwn0, &tm_k, &bars[BWB_OWN], h * ATT_HD, orow);
-        tma_load_2d(sOwn1, &tm_v, &bars[BWB_OWN], h * ATT_HD, orow);
-      } else {
-        tma_load_2d(sOwn0, &tm_q, &bars[BWB_OWN], h * ATT_HD, orow);
-        tma_load_2d(sOwn1, &tm_do, &bars[BWB_OWN], h * ATT_HD, orow);
-      }
+      tma_load_2d(sOwn0, &tm_k, &bars[BWB_OWN], h * ATT_HD, orow);
+      tma_load_2d(sOwn1, &tm_v, &bars[BWB_OWN], h * ATT_HD, orow);
       int issued = 0;
       for (int it = 0; it < n_st; ++it) {
         const int s = it & 1;
         if (!mbar_wait(&bars[BWB_EMPTY + s], ((it >> 1) & 1) ^ 1u, ctl)) break;
-        const int32_t row = static_cast<int32_t>(start + (st0 + it) * BW_COLS);
+        const int32_t row = static_cast<int32_t>(start + (ot + it) * BW_COLS);
         uint8_t* dst = sStg + s * BwSmem::kStgBytes;
         mbar_arrive_expect_tx(&bars[BWB_FULL + s], 2 * BW_TILE_BYTES);
-        if (KV) {
-          tma_load_2d(dst, &tm_q, &bars[BWB_FULL + s], h * ATT_HD, row);
-          tma_load_2d(dst + BW_TILE_BYTES, &tm_do, &bars[BWB_FULL + s], h * ATT_HD, row);
-        } else {
-          tma_load_2d(dst, &tm_k, &bars[BWB_FULL + s], h * ATT_HD, row);
-          tma_load_2d(dst + BW_TILE_BYTES, &tm_v, &bars[BWB_FULL + s], h * ATT_HD, row);
-        }
+        tma_load_2d(dst, &tm_q, &bars[BWB_FULL + s], h * ATT_HD, row);
+        tma_load_2d(dst + BW_TILE_BYTES, &tm_do, &bars[BWB_FULL + s], h * ATT_HD, row);
         ++issued;
       }
       // every load lands before shared memory is released
@@ -233,8 +223,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     };
     constexpr uint32_t idesc_ss = idesc_16_f32(BW_ROWS, BW_COLS, false, false, F16);
     constexpr uint32_t idesc_ts = idesc_16_f32(BW_ROWS, ATT_HD, false, true, F16);
-    const uint64_t dOwn0 = smem_desc_sw128(smem_u32(sOwn0), 16, 1024);
-    const uint64_t dOwn1 = smem_desc_sw128(smem_u32(sOwn1), 16, 1024);
+    constexpr uint32_t idesc_dq = idesc_16_f32(BW_COLS, ATT_HD, true, true, F16);
+    const uint64_t dOwn0 = smem_desc_sw128(smem_u32(sOwn0), 16, 1024);   // K, K-major A
+    const uint64_t dOwn1 = smem_desc_sw128(smem_u32(sOwn1), 16, 1024);   // V, K-major A
+    const uint64_t dOwn0m = smem_desc_sw128(smem_u32(sOwn0), 8192, 1024);  // K, MN-major B
+    // dS as an MN-major A (M = 128 queries: two 64-query halves BW_TILE_BYTES
+    // apart; K = keys: 8-row groups 1024 bytes apart)
+    const uint64_t dDsm = smem_desc_sw128(smem_u32(sDs), BW_TILE_BYTES, 1024);
     bool ok = wait_all(&bars[BWB_OWN], 0);
     tc_fence_after();
     for (int it = 0; ok && it < n_st; ++it) {
@@ -243,10 +238,10 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!ok) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(sStg + s * BwSmem::kStgBytes);
-      const uint64_t dS0k = smem_desc_sw128(sa, 16, 1024);                  // streamed tile 0, K-major
-      const uint64_t dS1k = smem_desc_sw128(sa + BW_TILE_BYTES, 16, 1024);  // streamed tile 1, K-major
+      const uint64_t dS0k = smem_desc_sw128(sa, 16, 1024);                  // Q, K-major
+      const uint64_t dS1k = smem_desc_sw128(sa + BW_TILE_BYTES, 16, 1024);  // dO, K-major
       if (leader) {
-        // X = own0 streamed0^T, Y = own1 streamed1^T (K = 64: four steps)
+        // S^T = K Q^T, dP^T = V dO^T (K = 64: four steps)
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk)
           mma_bf16_ss(tmem + kX, dOwn0 + 2 * kk, dS0k + 2 * kk, idesc_ss, kk > 0 ? 1u : 0u);
@@ -259,34 +254,29 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = wait_all(&bars[BWB_P], static_cast<uint32_t>(it) & 1u);
       if (!ok) break;
       tc_fence_after();
-      // accumulate over the 128 streamed rows (K = 128: eight steps); the
-      // packed 16-bit operand of rows 32g .. 32g + 31 sits at columns
-      // 32g .. 32g + 15 of its region
-      const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                // MN-major B
-      const uint64_t dS1m = smem_desc_sw128(sa + BW_TILE_BYTES, 8192, 1024);
+      const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                // Q, MN-major B
+      const uint64_t dS1m = smem_desc_sw128(sa + BW_TILE_BYTES, 8192, 1024);  // dO, MN-major B
       if (leader) {
-        if (KV) {
-          // dV += P^T dO ; dK += dS^T Q
+        // dQ_part = dS K over the 128 keys (eight steps of 16 keys, 2 KB each)
+        const uint32_t dq_acc = tmem + kDq + 64u * static_cast<uint32_t>(it & 1);
 #pragma unroll
-          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
-            mma_bf16_ts(tmem + kAcc0, tmem + kX + ac, dS1m + 128 * kk, idesc_ts,
-                        (it > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < BW_ROWS / 16; ++kk)
+          mma_bf16_ss(dq_acc, dDsm + 128 * kk, dOwn0m + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[BWB_DQ]);
+        // dV += P^T dO ; dK += dS^T Q over the 128 queries (eight steps); the
+        // packed 16-bit operand of queries 32g .. 32g + 31 sits at columns
+        // 32g .. 32g + 15 of its region
 #pragma unroll
-          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
-            mma_bf16_ts(tmem + kAcc1, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
-                        (it > 0 || kk > 0) ? 1u : 0u);
-          }
-        } else {
-          // dQ += dS K
+        for (int kk = 0; kk < BW_COLS / 16; ++kk) {
+          const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
+          mma_bf16_ts(tmem + kAcc0, tmem + kX + ac, dS1m + 128 * kk, idesc_ts,
+                      (it > 0 || kk > 0) ? 1u : 0u);
+        }
 #pragma unroll
-          for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-            const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
-            mma_bf16_ts(tmem + kAcc0, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
-                        (it > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < BW_COLS / 16; ++kk) {
+          const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
+          mma_bf16_ts(tmem + kAcc1, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
+                      (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars[BWB_EMPTY + s]);
       }
@@ -299,39 +289,55 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ---------------- element warps
     const int q4 = warp & 3, cg = warp >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const int r = q4 * 32 + lane;        // row of the own tile
+    const int r = q4 * 32 + lane;        // key row of the own tile
     const int orow = o0 + r;             // its index within the user
     const bool own_ok = orow < n;
     const int32_t t_own = own_ok ? bw_rel_time(p.timestamps, start + orow, t_first) : 0;
     const float inv_n = 1.0f / static_cast<float>(n);
     const float* rp = p.rab_pos + static_cast<int64_t>(h) * p.P;
-    const int c0 = cg * 32;              // this warp's 32 streamed rows of each tile
+    const int c0 = cg * 32;              // this warp's 32 queries of each tile
+    // this thread's 64-byte slice of the dS^T rows in shared memory (four
+    // 16-byte chunks of 8 queries, 128B swizzle: chunk index ^ (row & 7))
+    uint8_t* ds_row = sDs + (cg >> 1) * BW_TILE_BYTES + r * 128;
+    const int ds_chunk0 = (cg & 1) * 4;
+    // the previous tile pair's dQ_part (rows = its queries) into global dQ
+    auto drain_dq = [&](int j) {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_off + kDq + 64u * static_cast<uint32_t>(j & 1) +
+                    static_cast<uint32_t>(cg * 16), v);
+      tmem_ld_wait(v);
+      const int qrow = (ot + j) * BW_COLS + r;
+      if (qrow < n) {
+        float4* d4 = reinterpret_cast<float4*>(p.dq + (start + qrow) * p.ld_g + h * ATT_HD + cg * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          atomicAdd(d4 + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      }
+    };
     // Time-bucket walk over this thread's visible pairs in the order visited:
-    // KV: dt = t_i - t_own grows with the query i (bucket goes up from 0);
-    // Q:  dt = t_own - t_j shrinks with the key j (bucket goes down from Tb-1).
+    // dt = t_i - t_own grows with the query i, so the bucket goes up from 0.
     // The bucket of dt is the largest b with thr[b] <= dt (thr[0] = 0).
-    int tb = KV ? 0 : p.Tb - 1;
-    float rt_cur = sRt[tb];
-    // the edge the walk compares against: thr[tb + 1] (KV, INT32_MAX past the
-    // last bucket) or thr[tb] (Q)
-    int32_t edge = KV ? (p.Tb > 1 ? sThr[1] : INT32_MAX) : sThr[tb];
-    // position-table gradient (KV): this warp's 32 x 32 block adds dS to its
-    // 63 diagonals D = i - j = dg0 + cc - lane in `diag` (index cc - lane + 31).
+    int tb = 0;
+    float rt_cur = sRt[0];
+    // the edge the walk compares against: thr[tb + 1] (INT32_MAX past the last bucket)
+    int32_t edge = p.Tb > 1 ? sThr[1] : INT32_MAX;
+    // position-table gradient: this warp's 32 x 32 block adds dS to its 63
+    // diagonals D = i - j = dg0 + cc - lane in `diag` (index cc - lane + 31).
     // The 32 lanes of one column touch 32 different diagonals, so the adds are
     // plain read-modify-writes (a __syncwarp before each keeps the lanes in
     // step); the block's diagonals go to the CTA histogram afterwards.
     float* diag = sDiag + warp * 64;
-    // time-gradient running sum (KV): partial sum of the current bucket
-    float tg_acc = 0.0f;
-    float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1 (KV)
+    float tg_acc = 0.0f;    // time-gradient running sum of the current bucket
+    float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1
     bool ok = true;
     for (int it = 0; it < n_st; ++it) {
-      const int sbase = (st0 + it) * BW_COLS;  // first streamed row
-      // this tile's 128 streamed times and the 255-entry position-bias band:
-      // entry e holds rab_pos[min(|D|, P - 1)] for D = i - j = dbase + e - 127
+      const int sbase = (ot + it) * BW_COLS;  // first query of the tile
+      // this tile's 128 query times and the 255-entry position-bias band:
+      // entry e holds rab_pos[min(D, P - 1)] for D = i - j = dbase + e - 127
       int32_t* tt = sTimes + (it & 1) * 128;
       float* band = sBand + (it & 1) * 256;
-      const int dbase = KV ? sbase - o0 : o0 - sbase;
+      const int dbase = sbase - o0;
       if (tid < 128) {
         const int row = sbase + tid;
         tt[tid] = row < n ? bw_rel_time(p.timestamps, start + row, t_first) : 0;
@@ -350,16 +356,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
         tmem_ld_wait(xs);
         tmem_ld_wait(ys);
-        // visible streamed columns of this thread: KV: i >= j and i < n;
-        // Q: j <= i (and j < n, implied)
+        // visible queries of this thread: i >= j and i < n
         int c_lo = 0, c_hi = 31;
         if (!own_ok) {
           c_lo = 32;
-        } else if (KV) {
+        } else {
           c_lo = max(0, orow - (sbase + c0));
           c_hi = min(31, n - 1 - (sbase + c0));
-        } else {
-          c_hi = min(31, orow - (sbase + c0));
         }
         uint32_t px[16], py[16];
 #pragma unroll
@@ -370,39 +373,29 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int cc = c + e;
             float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
             if (cc >= c_lo && cc <= c_hi) {
-              const int32_t dt = KV ? tt[c0 + cc] - t_own : t_own - tt[c0 + cc];
-              if (KV) {
-                if (dt >= edge) {
-                  if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
-                  tg_acc = 0.0f;
-                  do {
-                    ++tb;
-                    edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
-                  } while (dt >= edge);
-                  rt_cur = sRt[tb];
-                }
-              } else if (dt < edge) {
-                do { --tb; } while (tb > 0 && dt < sThr[tb]);
-                edge = sThr[tb];
+              const int32_t dt = tt[c0 + cc] - t_own;
+              if (dt >= edge) {
+                if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+                tg_acc = 0.0f;
+                do {
+                  ++tb;
+                  edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
+                } while (dt >= edge);
                 rt_cur = sRt[tb];
               }
               // D = i - j; band index D - dbase + 127
-              const int dpos = KV ? (sbase + c0 + cc) - orow : orow - (sbase + c0 + cc);
+              const int dpos = (sbase + c0 + cc) - orow;
               const float sv = __uint_as_float(xs[cc]) + band[dpos - dbase + 127] + rt_cur;
               float ph, pg;
               phi_and_grad<PHI>(sv, ph, pg);
               pp = ph * inv_n;
               ds = __uint_as_float(ys[cc]) * pg * inv_n;
-              if (KV) {
-                if (dpos >= p.P - 1) pg_clamp += ds;
-                else dsp = ds;
-                tg_acc += ds;
-              }
+              if (dpos >= p.P - 1) pg_clamp += ds;
+              else dsp = ds;
+              tg_acc += ds;
             }
-            if (KV) {
-              __syncwarp();
-              diag[cc - lane + 31] += dsp;
-            }
+            __syncwarp();
+            diag[cc - lane + 31] += dsp;
             pv[e] = pp;
             dsv[e] = ds;
           }
@@ -414,29 +407,51 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
           }
         }
-        if (KV) {
-          // this block's diagonals into the CTA histogram (dpos < P - 1 <= hist_len
-          // there; clamped pairs went to pg_clamp), and the buffer cleared
-          __syncwarp();
-          const int dg0 = (sbase + c0) - (o0 + q4 * 32);
+        // this block's diagonals into the CTA histogram (0 <= D < P - 1 there:
+        // clamped pairs went to pg_clamp; entries past the shared histogram go
+        // to global memory), and the buffer cleared
+        __syncwarp();
+        const int dg0 = (sbase + c0) - (o0 + q4 * 32);
 #pragma unroll
-          for (int k = lane; k < 63; k += 32) {
-            const float v = diag[k];
-            const int dd = dg0 + k - 31;
-            if (v != 0.0f && dd >= 0 && dd < p.P - 1) atomicAdd(&sPg[dd], v);
-            diag[k] = 0.0f;
+        for (int k = lane; k < 63; k += 32) {
+          const float v = diag[k];
+          const int dd = dg0 + k - 31;
+          if (v != 0.0f && dd >= 0 && dd < p.P - 1) {
+            if (dd < p.hist_len) atomicAdd(&sPg[dd], v);
+            else atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + dd], v);
           }
+          diag[k] = 0.0f;
+        }
+        // dS^T rows to shared memory for the dQ MMA, once the previous tile
+        // pair's dQ MMAs have read them
+        if (it > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
+          tc_fence_after();
+        }
+        if (ok) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + k) ^ (r & 7)) << 4)) =
+                make_uint4(py[4 * k], py[4 * k + 1], py[4 * k + 2], py[4 * k + 3]);
+          fence_proxy_async_smem();
         }
         // the packed operands go over the first 16 of the 32 columns this warp read
         __syncwarp();
-        if (KV) tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
+        tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
         tmem_st16(tmem + lane_off + kY + static_cast<uint32_t>(c0), py);
         tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&bars[BWB_P]);
+      // the previous tile pair's dQ_part, while this pair's MMAs run
+      if (ok && it > 0) drain_dq(it - 1);
     }
-    if (KV && tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+    if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+    if (ok && n_st > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(n_st - 1) & 1u, ctl));
+      tc_fence_after();
+      if (ok) drain_dq(n_st - 1);
+    }
     // ---------------- epilogue: the accumulators (rows of the own tile); the
     // four column groups take 16 of the 64 accumulator columns each
     if (ok) ok = mbar_wait(&bars[BWB_DONE], 0, ctl);
@@ -444,11 +459,11 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (ok) {
       tc_fence_after();
       const int64_t grow = start + orow;
-      for (int a = 0; a < (KV ? 2 : 1); ++a) {
+      for (int a = 0; a < 2; ++a) {
         uint32_t v[16];
         tmem_ld16(tmem + lane_off + (a == 0 ? kAcc0 : kAcc1) + static_cast<uint32_t>(cg * 16), v);
         tmem_ld_wait(v);
-        float* dst = KV ? (a == 0 ? p.dv : p.dk) : p.dq;
+        float* dst = a == 0 ? p.dv : p.dk;
         if (own_ok) {
           float4* d4 = reinterpret_cast<float4*>(dst + grow * p.ld_g + h * ATT_HD + cg * 16);
 #pragma unroll
@@ -458,22 +473,20 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
       }
     }
-    if (KV && pg_clamp != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + p.P - 1], pg_clamp);
+    if (pg_clamp != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + p.P - 1], pg_clamp);
   }
 
-  // ---------------- table gradients (KV) and teardown
+  // ---------------- table gradients and teardown
   tc_fence_before();
   __syncthreads();
-  if (KV) {
-    const int lim = min(p.hist_len, p.P - 1);
-    for (int k = tid; k < lim; k += BW_THREADS) {
-      const float g = sPg[k];
-      if (g != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + k], g);
-    }
-    for (int k = tid; k < p.Tb; k += BW_THREADS) {
-      const float g = sTg[k];
-      if (g != 0.0f) atomicAdd(&p.drab_time[static_cast<int64_t>(h) * p.Tb + k], g);
-    }
+  const int lim = min(p.hist_len, p.P - 1);
+  for (int k = tid; k < lim; k += BW_THREADS) {
+    const float g = sPg[k];
+    if (g != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + k], g);
+  }
+  for (int k = tid; k < p.Tb; k += BW_THREADS) {
+    const float g = sTg[k];
+    if (g != 0.0f) atomicAdd(&p.drab_time[static_cast<int64_t>(h) * p.Tb + k], g);
   }
   if (warp == BW_MMA_WARP) {
     tc_fence_after();

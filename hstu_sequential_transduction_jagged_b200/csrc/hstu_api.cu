@@ -105,14 +105,14 @@ const int64_t* thresholds_for(int Tb) {
 
 enum KernelKind : int {
   K_F1 = 0, K_ATTN, K_F2, K_CAND_ATTN, K_SCORE, K_F32_LINEAR, K_F32_ATTN, K_F32_LN, K_CVT,
-  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_ATTN_BWD_KV, K_ATTN_BWD_Q, K_BWD_GEMM, K_GATE_BWD,
+  K_SL, K_SL_GATHER, K_ATTN_FUSED, K_ATTN_BWD, K_BWD_GEMM, K_GATE_BWD,
   K_BWD_ELT, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {"f1_gemm",     "attention",      "f2_gemm",
                                            "mfalcon_attention", "score",    "fp32_linear",
                                            "fp32_attention",    "fp32_ln_gate", "weight_cvt",
                                            "sl_select",         "sl_gather",
-                                           "attention_f2_fused", "attn_bwd_kv", "attn_bwd_q",
+                                           "attention_f2_fused", "attention_bwd",
                                            "bwd_gemm_cublas", "gate_bwd", "bwd_elementwise"};
 
 struct Profiler {
@@ -199,18 +199,17 @@ AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16, bool fuse
 using AttnBwdFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                           const CUtensorMap, const AttnBwdParams);
 
-template <bool KV, bool F16>
+template <bool F16>
 AttnBwdFn attn_bwd_kernel_for(int phi) {
   switch (phi) {
-    case HSTU_ACT_SILU: return hstu_attn_bwd_kernel<KV, HSTU_ACT_SILU, F16>;
-    case HSTU_ACT_RELU: return hstu_attn_bwd_kernel<KV, HSTU_ACT_RELU, F16>;
-    default: return hstu_attn_bwd_kernel<KV, HSTU_ACT_IDENTITY, F16>;
+    case HSTU_ACT_SILU: return hstu_attn_bwd_kernel<HSTU_ACT_SILU, F16>;
+    case HSTU_ACT_RELU: return hstu_attn_bwd_kernel<HSTU_ACT_RELU, F16>;
+    default: return hstu_attn_bwd_kernel<HSTU_ACT_IDENTITY, F16>;
   }
 }
 
-AttnBwdFn attn_bwd_kernel_ptr(bool kv, int phi, bool f16) {
-  if (kv) return f16 ? attn_bwd_kernel_for<true, true>(phi) : attn_bwd_kernel_for<true, false>(phi);
-  return f16 ? attn_bwd_kernel_for<false, true>(phi) : attn_bwd_kernel_for<false, false>(phi);
+AttnBwdFn attn_bwd_kernel_ptr(int phi, bool f16) {
+  return f16 ? attn_bwd_kernel_for<true>(phi) : attn_bwd_kernel_for<false>(phi);
 }
 
 struct DeviceInfo {
@@ -242,11 +241,10 @@ hstu_status_t device_info(DeviceInfo** out) {
       for (int pairs = 0; pairs < 2; ++pairs)
         HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_kernel_ptr(false, phi, pairs != 0, true, true),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
-    for (int kv = 0; kv < 2; ++kv)
-      for (int phi = 0; phi < 3; ++phi)
-        for (int f16 = 0; f16 < 2; ++f16)
-          HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_bwd_kernel_ptr(kv != 0, phi, f16 != 0),
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
+    for (int phi = 0; phi < 3; ++phi)
+      for (int f16 = 0; f16 < 2; ++f16)
+        HSTU_CHECK_CUDA(cudaFuncSetAttribute(attn_bwd_kernel_ptr(phi, f16 != 0),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, att_max));
     const int g1 = static_cast<int>(F1Smem::kBytes);
     HSTU_CHECK_CUDA(cudaFuncSetAttribute(hstu_f1_kernel<HSTU_ACT_RELU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, g1));
@@ -635,22 +633,22 @@ hstu_status_t launch_attn_bwd(const hstu_layer_cfg_t* c, const hstu_jagged_t* ja
   p.Tb = Tb;
   p.max_len = jag->max_len;
   p.phi2 = c->phi2;
-  p.hist_len = std::min(P, jag->max_len);
+  // position-gradient entries kept in shared memory (the rest go to global
+  // memory with one atomic per touched entry)
+  const int hist_cap = static_cast<int>((227u * 1024u - BwSmem::bytes(0)) / 4u);
+  p.hist_len = std::min(std::min(P, jag->max_len), hist_cap);
   p.timeout_ns = kDefaultTimeoutNs;
   const int64_t* thr = thresholds_for(Tb);
   for (int b = 0; b < Tb; ++b)
     p.thr[b] = thr[b] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(thr[b]) : INT32_MAX;
   const size_t smem = BwSmem::bytes(p.hist_len);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
+  // dQ is accumulated into (one vector atomic per element per key tile)
+  HSTU_CHECK_CUDA(cudaMemset2DAsync(dq, sizeof(float) * ld_g, 0, sizeof(float) * hv, T, st));
   dim3 grid(H, jag->batch, (jag->max_len + BW_ROWS - 1) / BW_ROWS);
   {
-    ProfScope prof(K_ATTN_BWD_KV, st);
-    attn_bwd_kernel_ptr(true, c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
-    HSTU_CHECK_CUDA(cudaGetLastError());
-  }
-  {
-    ProfScope prof(K_ATTN_BWD_Q, st);
-    attn_bwd_kernel_ptr(false, c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
+    ProfScope prof(K_ATTN_BWD, st);
+    attn_bwd_kernel_ptr(c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
     HSTU_CHECK_CUDA(cudaGetLastError());
   }
   return HSTU_OK;
