@@ -66,14 +66,16 @@ struct BwSmem {
   // queries 0-63 at kDs, 64-127 at kDs + BW_TILE_BYTES (row = key, 128 B)
   static constexpr uint32_t kDs = kStg + 2 * kStgBytes;
   static constexpr uint32_t kTimes = kDs + 2 * BW_TILE_BYTES;  // 2 x 128 int32 (query rows)
-  static constexpr uint32_t kBand = kTimes + 2 * 128 * 4;   // 2 x 256 floats: rab_pos band
-  static constexpr uint32_t kThr = kBand + 2 * 256 * 4;     // Tb int32 thresholds
+  // 2 x 256 float pairs: entry e of the rab_pos band with its successor
+  static constexpr uint32_t kBand = kTimes + 2 * 128 * 4;
+  static constexpr uint32_t kThr = kBand + 2 * 256 * 8;     // Tb int32 thresholds
   static constexpr uint32_t kRt = kThr + MAX_TIME_BUCKETS * 4;  // Tb floats (rab_time row)
   static constexpr uint32_t kTg = kRt + MAX_TIME_BUCKETS * 4;   // Tb floats (time gradient)
   static constexpr uint32_t kBars = kTg + MAX_TIME_BUCKETS * 4; // 16 barriers
   static constexpr uint32_t kMisc = kBars + 16 * 8;
-  static constexpr uint32_t kDiag = kMisc + 64;             // per element warp 64 floats
-  static constexpr uint32_t kPg = kDiag + BW_ELEM_WARPS * 64 * 4;  // hist_len floats (position gradient)
+  // per element warp two 64-float diagonal buffers (odd lanes, even lanes)
+  static constexpr uint32_t kDiag = kMisc + 64;
+  static constexpr uint32_t kPg = kDiag + BW_ELEM_WARPS * 128 * 4;  // hist_len floats (position gradient)
   static constexpr uint32_t bytes(int hist_len) {
     return kPg + static_cast<uint32_t>(hist_len) * 4u + 1024u;
   }
@@ -103,6 +105,32 @@ __device__ __forceinline__ void phi_and_grad(float s, float& p, float& g) {
   } else {
     p = s;
     g = 1.0f;
+  }
+}
+
+// phi2 / N and phi2' / N of a packed pair of pre-activations
+template <int PHI>
+__device__ __forceinline__ void phi_grad_pair(uint64_t s2, float inv_n, uint64_t& p2, uint64_t& g2) {
+  if constexpr (PHI == HSTU_ACT_SILU) {
+    // sigmoid(s) = 0.5 + 0.5 tanh(s / 2);  SiLU' = sigmoid(s) (1 + s (1 - sigmoid(s)))
+    float a, b;
+    f2_unpack(f2_mul(s2, f2_pack(0.5f, 0.5f)), a, b);
+    const uint64_t t = f2_pack(tanh_approx(a), tanh_approx(b));
+    const float hn = 0.5f * inv_n;
+    const uint64_t sgn = f2_fma(t, f2_pack(hn, hn), f2_pack(hn, hn));              // sigmoid / N
+    const uint64_t om = f2_fma(t, f2_pack(-0.5f, -0.5f), f2_pack(0.5f, 0.5f));     // 1 - sigmoid
+    p2 = f2_mul(s2, sgn);
+    g2 = f2_mul(sgn, f2_fma(s2, om, f2_pack(1.0f, 1.0f)));
+  } else {
+    float a, b;
+    f2_unpack(s2, a, b);
+    if constexpr (PHI == HSTU_ACT_RELU) {
+      p2 = f2_pack(fmaxf(a, 0.0f) * inv_n, fmaxf(b, 0.0f) * inv_n);
+      g2 = f2_pack(a > 0.0f ? inv_n : 0.0f, b > 0.0f ? inv_n : 0.0f);
+    } else {
+      p2 = f2_pack(a * inv_n, b * inv_n);
+      g2 = f2_pack(inv_n, inv_n);
+    }
   }
 }
 
@@ -178,7 +206,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     sTg[k] = 0.0f;
   }
   for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
-  for (int k = tid; k < BW_ELEM_WARPS * 64; k += BW_THREADS) sDiag[k] = 0.0f;
+  for (int k = tid; k < BW_ELEM_WARPS * 128; k += BW_THREADS) sDiag[k] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -322,21 +350,39 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     float rt_cur = sRt[0];
     // the edge the walk compares against: thr[tb + 1] (INT32_MAX past the last bucket)
     int32_t edge = p.Tb > 1 ? sThr[1] : INT32_MAX;
-    // position-table gradient: this warp's 32 x 32 block adds dS to its 63
-    // diagonals D = i - j = dg0 + cc - lane in `diag` (index cc - lane + 31).
-    // The 32 lanes of one column touch 32 different diagonals, so the adds are
-    // plain read-modify-writes (a __syncwarp before each keeps the lanes in
-    // step); the block's diagonals go to the CTA histogram afterwards.
-    float* diag = sDiag + warp * 64;
     float tg_acc = 0.0f;    // time-gradient running sum of the current bucket
     float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1
+    // moves the walk to the bucket of dt, flushing the running sum on a change
+    auto walk_to = [&](int32_t dt) {
+      if (dt >= edge) {
+        if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+        tg_acc = 0.0f;
+        do {
+          ++tb;
+          edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
+        } while (dt >= edge);
+        rt_cur = sRt[tb];
+      }
+    };
+    // position-table gradient: this warp's 32 x 32 block adds dS to its 63
+    // diagonals k = cc - lane + 31 (D = i - j = dg0 + k - 31).  Odd lanes add
+    // into diagB[k], even lanes into diagA[k + 1], so that the two diagonals of
+    // a column pair are one aligned 8-byte entry for every lane.  The 32 lanes
+    // of one column touch 32 different diagonals, so the adds are plain
+    // read-modify-writes (a __syncwarp before each keeps the lanes in step);
+    // the block's diagonals go to the CTA histogram afterwards.
+    float* diagB = sDiag + warp * 128;
+    float* diagA = diagB + 64;
+    float* dlp = ((lane & 1) ? diagB : diagA + 1) + 31 - lane;  // dlp[cc]: this lane's entry
+    const unsigned full = 0xffffffffu;
     bool ok = true;
     for (int it = 0; it < n_st; ++it) {
       const int sbase = (ot + it) * BW_COLS;  // first query of the tile
       // this tile's 128 query times and the 255-entry position-bias band:
       // entry e holds rab_pos[min(D, P - 1)] for D = i - j = dbase + e - 127
+      // (0 for D < 0), paired with entry e + 1
       int32_t* tt = sTimes + (it & 1) * 128;
-      float* band = sBand + (it & 1) * 256;
+      uint64_t* bandp = reinterpret_cast<uint64_t*>(sBand) + (it & 1) * 256;
       const int dbase = sbase - o0;
       if (tid < 128) {
         const int row = sbase + tid;
@@ -344,11 +390,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       } else if (tid < 128 + 255) {
         const int e = tid - 128;
         const int dd = dbase + e - 127;
-        band[e] = dd >= 0 ? __ldg(rp + min(dd, p.P - 1)) : 0.0f;
+        const float v0 = dd >= 0 ? __ldg(rp + min(dd, p.P - 1)) : 0.0f;
+        const float v1 = dd + 1 >= 0 ? __ldg(rp + min(dd + 1, p.P - 1)) : 0.0f;
+        bandp[e] = f2_pack(v0, v1);
       }
       named_barrier_sync(1, BW_ELEM_WARPS * 32);
       if (ok) ok = mbar_wait(&bars[BWB_S], static_cast<uint32_t>(it) & 1u, ctl);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(full, ok);
       if (ok) {
         tc_fence_after();
         uint32_t xs[32], ys[32];
@@ -356,76 +404,156 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
         tmem_ld_wait(xs);
         tmem_ld_wait(ys);
-        // visible queries of this thread: i >= j and i < n
-        int c_lo = 0, c_hi = 31;
-        if (!own_ok) {
-          c_lo = 32;
-        } else {
-          c_lo = max(0, orow - (sbase + c0));
-          c_hi = min(31, n - 1 - (sbase + c0));
-        }
         uint32_t px[16], py[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int cc = c + e;
-            float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
-            if (cc >= c_lo && cc <= c_hi) {
-              const int32_t dt = tt[c0 + cc] - t_own;
-              if (dt >= edge) {
-                if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
-                tg_acc = 0.0f;
-                do {
-                  ++tb;
-                  edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
-                } while (dt >= edge);
-                rt_cur = sRt[tb];
-              }
-              // D = i - j; band index D - dbase + 127
-              const int dpos = (sbase + c0 + cc) - orow;
-              const float sv = __uint_as_float(xs[cc]) + band[dpos - dbase + 127] + rt_cur;
-              float ph, pg;
-              phi_and_grad<PHI>(sv, ph, pg);
-              pp = ph * inv_n;
-              ds = __uint_as_float(ys[cc]) * pg * inv_n;
-              if (dpos >= p.P - 1) pg_clamp += ds;
-              else dsp = ds;
-              tg_acc += ds;
-            }
-            __syncwarp();
-            diag[cc - lane + 31] += dsp;
-            pv[e] = pp;
-            dsv[e] = ds;
-          }
-          if constexpr (F16) {
-            px[c >> 1] = pack_h2(pv[0], pv[1]);
-            py[c >> 1] = pack_h2(dsv[0], dsv[1]);
+        // band pair of column cc (even): bp[cc]
+        const uint64_t* bp = bandp + (c0 - r + 127);
+        // every column of the block visible (not the diagonal tile, not past
+        // the user's end) and no pair in the clamped position bucket
+        const bool interior = it > 0 && sbase + c0 + 32 <= n &&
+                              sbase + c0 + 31 - (o0 + q4 * 32) < p.P - 1;
+        // general path: per element visibility, walk and clamp
+        auto general = [&]() {
+          int c_lo = 0, c_hi = 31;
+          if (!own_ok) {
+            c_lo = 32;
           } else {
-            px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-            py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            c_lo = max(0, orow - (sbase + c0));
+            c_hi = min(31, n - 1 - (sbase + c0));
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dsv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int cc = c + e;
+              float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
+              if (cc >= c_lo && cc <= c_hi) {
+                walk_to(tt[c0 + cc] - t_own);
+                const int dpos = (sbase + c0 + cc) - orow;  // D = i - j
+                float b0, b1;
+                f2_unpack(bp[cc], b0, b1);
+                const float sv = __uint_as_float(xs[cc]) + b0 + rt_cur;
+                float ph, pg;
+                phi_and_grad<PHI>(sv, ph, pg);
+                pp = ph * inv_n;
+                ds = __uint_as_float(ys[cc]) * pg * inv_n;
+                if (dpos >= p.P - 1) pg_clamp += ds;
+                else dsp = ds;
+                tg_acc += ds;
+              }
+              __syncwarp();
+              dlp[cc] += dsp;
+              pv[e] = pp;
+              dsv[e] = ds;
+            }
+            if constexpr (F16) {
+              px[c >> 1] = pack_h2(pv[0], pv[1]);
+              py[c >> 1] = pack_h2(dsv[0], dsv[1]);
+            } else {
+              px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+              py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            }
+          }
+        };
+        // interior path over column pairs: rt_pair(c) gives the pair's time
+        // bias, ds_sink(c, ds2) sees its dS
+        auto interior_pairs = [&](auto rt_pair, auto ds_sink) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const uint64_t s2 = f2_add(f2_pack(__uint_as_float(xs[c]), __uint_as_float(xs[c + 1])),
+                                       f2_add(bp[c], rt_pair(c)));
+            uint64_t p2, g2;
+            phi_grad_pair<PHI>(s2, inv_n, p2, g2);
+            const uint64_t ds2 =
+                f2_mul(f2_pack(__uint_as_float(ys[c]), __uint_as_float(ys[c + 1])), g2);
+            ds_sink(c, ds2);
+            __syncwarp();
+            uint64_t* dd = reinterpret_cast<uint64_t*>(dlp + c);
+            *dd = f2_add(*dd, ds2);
+            if constexpr (F16) {
+              px[c >> 1] = f2_to_h2(p2);
+              py[c >> 1] = f2_to_h2(ds2);
+            } else {
+              px[c >> 1] = f2_to_bf16x2(p2);
+              py[c >> 1] = f2_to_bf16x2(ds2);
+            }
+          }
+        };
+        if (!interior) {
+          general();
+        } else {
+          const int32_t dt_first = tt[c0] - t_own;
+          const int32_t dt_last = tt[c0 + 31] - t_own;
+          if (__all_sync(full, dt_last < edge)) {
+            // every lane stays in its bucket: its bias is rt_cur
+            const uint64_t rt2 = f2_pack(rt_cur, rt_cur);
+            uint64_t tg2 = f2_pack(0.0f, 0.0f);
+            interior_pairs([&](int) { return rt2; },
+                           [&](int, uint64_t d) { tg2 = f2_add(tg2, d); });
+            float a0, a1;
+            f2_unpack(tg2, a0, a1);
+            tg_acc += a0 + a1;
+          } else {
+            walk_to(dt_first);
+            int bl = tb;  // bucket of the block's last column
+            int32_t el = edge;
+            while (dt_last >= el) {
+              ++bl;
+              el = bl + 1 < p.Tb ? sThr[bl + 1] : INT32_MAX;
+            }
+            const int B_lo = __reduce_min_sync(full, tb), B_hi = __reduce_max_sync(full, bl);
+            if (B_hi - B_lo <= 1) {
+              // two buckets in the warp: B_hi iff dt >= thr[B_hi]
+              const float rt_lo = sRt[B_lo], rt_hi = sRt[B_hi];
+              const int32_t thr_hi = B_hi > B_lo ? sThr[B_hi] : INT32_MAX;
+              uint64_t tg2 = f2_pack(0.0f, 0.0f), hi2 = f2_pack(0.0f, 0.0f);
+              interior_pairs(
+                  [&](int c) {
+                    const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
+                    return f2_pack(t2.x - t_own >= thr_hi ? rt_hi : rt_lo,
+                                   t2.y - t_own >= thr_hi ? rt_hi : rt_lo);
+                  },
+                  [&](int c, uint64_t d) {
+                    const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
+                    float d0, d1;
+                    f2_unpack(d, d0, d1);
+                    hi2 = f2_add(hi2, f2_pack(t2.x - t_own >= thr_hi ? d0 : 0.0f,
+                                              t2.y - t_own >= thr_hi ? d1 : 0.0f));
+                    tg2 = f2_add(tg2, d);
+                  });
+              float a0, a1, h0, h1;
+              f2_unpack(tg2, a0, a1);
+              f2_unpack(hi2, h0, h1);
+              const float hsum = h0 + h1;
+              // the lane's elements below thr_hi belong to its current bucket
+              tg_acc += (a0 + a1) - hsum;
+              walk_to(dt_last);
+              tg_acc += hsum;
+            } else {
+              general();
+            }
           }
         }
         // this block's diagonals into the CTA histogram (0 <= D < P - 1 there:
         // clamped pairs went to pg_clamp; entries past the shared histogram go
-        // to global memory), and the buffer cleared
+        // to global memory), and the buffers cleared
         __syncwarp();
         const int dg0 = (sbase + c0) - (o0 + q4 * 32);
 #pragma unroll
         for (int k = lane; k < 63; k += 32) {
-          const float v = diag[k];
+          const float v = diagB[k] + diagA[k + 1];
           const int dd = dg0 + k - 31;
           if (v != 0.0f && dd >= 0 && dd < p.P - 1) {
             if (dd < p.hist_len) atomicAdd(&sPg[dd], v);
             else atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + dd], v);
           }
-          diag[k] = 0.0f;
+          diagB[k] = 0.0f;
+          diagA[k + 1] = 0.0f;
         }
         // dS^T rows to shared memory for the dQ MMA, once the previous tile
         // pair's dQ MMAs have read them
         if (it > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
+          ok = __all_sync(full, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
           tc_fence_after();
         }
         if (ok) {
