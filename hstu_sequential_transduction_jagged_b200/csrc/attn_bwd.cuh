@@ -134,6 +134,24 @@ __device__ __forceinline__ void phi_grad_pair(uint64_t s2, float inv_n, uint64_t
   }
 }
 
+// sTg[b] += v for every lane with `act`, as one shared-memory atomic per
+// distinct b (a shared fp32 atomic is a compare-and-swap loop, so 32 lanes on
+// one address would retry one after the other).  Warp-converged callers only.
+__device__ __forceinline__ void warp_bucket_add(float* sTg, bool act, int b, float v) {
+  const unsigned full = 0xffffffffu;
+  unsigned m = __ballot_sync(full, act);
+  while (m != 0u) {
+    const int leader = __ffs(m) - 1;
+    const int bb = __shfl_sync(full, b, leader);
+    const bool mine = act && b == bb;
+    float sum = mine ? v : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(full, sum, o);
+    if (lane_id() == leader) atomicAdd(&sTg[bb], sum);
+    m &= ~__ballot_sync(full, mine);
+  }
+}
+
 // Seconds since the user's first event (int32, clamped; the span check is
 // made once per CTA).
 __device__ __forceinline__ int32_t bw_rel_time(const int64_t* ts, int64_t row, int64_t t_first) {
@@ -352,16 +370,32 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     int32_t edge = p.Tb > 1 ? sThr[1] : INT32_MAX;
     float tg_acc = 0.0f;    // time-gradient running sum of the current bucket
     float pg_clamp = 0.0f;  // position gradient of the clamped bucket P - 1
-    // moves the walk to the bucket of dt, flushing the running sum on a change
+    // moves every lane's walk to the bucket of its dt (dt < edge: no move),
+    // flushing the running sums that change bucket; warp-converged callers
+    const unsigned full = 0xffffffffu;
+    auto advance = [&](int32_t dt) {
+      tg_acc = 0.0f;
+      do {
+        ++tb;
+        edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
+      } while (dt >= edge);
+      rt_cur = sRt[tb];
+    };
     auto walk_to = [&](int32_t dt) {
+      const bool mv = dt >= edge;
+      if (__any_sync(full, mv)) {
+        warp_bucket_add(sTg, mv && tg_acc != 0.0f, tb, tg_acc);
+        if (mv) advance(dt);
+      }
+    };
+    // the same for one lane on its own (the general path, where lanes sit in
+    // many different buckets): the running sum goes to global memory with a
+    // reduction that does not return
+    float* drt = p.drab_time + static_cast<int64_t>(h) * p.Tb;
+    auto walk_lane = [&](int32_t dt) {
       if (dt >= edge) {
-        if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
-        tg_acc = 0.0f;
-        do {
-          ++tb;
-          edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
-        } while (dt >= edge);
-        rt_cur = sRt[tb];
+        if (tg_acc != 0.0f) atomicAdd(&drt[tb], tg_acc);
+        advance(dt);
       }
     };
     // position-table gradient: this warp's 32 x 32 block adds dS to its 63
@@ -374,7 +408,6 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     float* diagB = sDiag + warp * 128;
     float* diagA = diagB + 64;
     float* dlp = ((lane & 1) ? diagB : diagA + 1) + 31 - lane;  // dlp[cc]: this lane's entry
-    const unsigned full = 0xffffffffu;
     bool ok = true;
     for (int it = 0; it < n_st; ++it) {
       const int sbase = (ot + it) * BW_COLS;  // first query of the tile
@@ -399,19 +432,25 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = __all_sync(full, ok);
       if (ok) {
         tc_fence_after();
-        uint32_t xs[32], ys[32];
-        tmem_ld32(tmem + lane_off + kX + static_cast<uint32_t>(c0), xs);
-        tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
-        tmem_ld_wait(xs);
-        tmem_ld_wait(ys);
-        uint32_t px[16], py[16];
-        // band pair of column cc (even): bp[cc]
+        // dS^T goes to shared memory below, once the previous tile pair's dQ
+        // MMAs have read it (they were issued before this pair's S MMAs)
+        if (it > 0) {
+          ok = __all_sync(full, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
+          tc_fence_after();
+        }
+      }
+      if (ok) {
+        // band pair of column cc: bp[cc]
         const uint64_t* bp = bandp + (c0 - r + 127);
         // every column of the block visible (not the diagonal tile, not past
         // the user's end) and no pair in the clamped position bucket
         const bool interior = it > 0 && sbase + c0 + 32 <= n &&
                               sbase + c0 + 31 - (o0 + q4 * 32) < p.P - 1;
-        // general path: per element visibility, walk and clamp
+        // General path: per element visibility, walk and clamp.  A rolled loop
+        // over four 8-column groups (the rare blocks keep their code small): it
+        // reads S^T / dP^T from tensor memory and stores the packed P^T / dS^T
+        // of each group itself (group g over columns 4g .. 4g + 3, which held
+        // raw values the loop has already read).
         auto general = [&]() {
           int c_lo = 0, c_hi = 31;
           if (!own_ok) {
@@ -420,68 +459,89 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             c_lo = max(0, orow - (sbase + c0));
             c_hi = min(31, n - 1 - (sbase + c0));
           }
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g) {
+            uint32_t x8[8], y8[8];
+            tmem_ld8(tmem + lane_off + kX + static_cast<uint32_t>(c0 + 8 * g), x8);
+            tmem_ld8(tmem + lane_off + kY + static_cast<uint32_t>(c0 + 8 * g), y8);
+            tmem_ld_wait(x8, y8);
+            uint32_t pk[4], dk[4];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float pv[2], dsv[2];
+            for (int c = 0; c < 8; c += 2) {
+              float pv[2], dsv[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int cc = c + e;
-              float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
-              if (cc >= c_lo && cc <= c_hi) {
-                walk_to(tt[c0 + cc] - t_own);
-                const int dpos = (sbase + c0 + cc) - orow;  // D = i - j
-                float b0, b1;
-                f2_unpack(bp[cc], b0, b1);
-                const float sv = __uint_as_float(xs[cc]) + b0 + rt_cur;
-                float ph, pg;
-                phi_and_grad<PHI>(sv, ph, pg);
-                pp = ph * inv_n;
-                ds = __uint_as_float(ys[cc]) * pg * inv_n;
-                if (dpos >= p.P - 1) pg_clamp += ds;
-                else dsp = ds;
-                tg_acc += ds;
+              for (int e = 0; e < 2; ++e) {
+                const int cc = 8 * g + c + e;
+                float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
+                if (cc >= c_lo && cc <= c_hi) {
+                  walk_lane(tt[c0 + cc] - t_own);
+                  const int dpos = (sbase + c0 + cc) - orow;  // D = i - j
+                  float b0, b1;
+                  f2_unpack(bp[cc], b0, b1);
+                  const float sv = __uint_as_float(x8[c + e]) + b0 + rt_cur;
+                  float ph, pg;
+                  phi_and_grad<PHI>(sv, ph, pg);
+                  pp = ph * inv_n;
+                  ds = __uint_as_float(y8[c + e]) * pg * inv_n;
+                  if (dpos >= p.P - 1) pg_clamp += ds;
+                  else dsp = ds;
+                  tg_acc += ds;
+                }
+                __syncwarp();
+                dlp[cc] += dsp;
+                pv[e] = pp;
+                dsv[e] = ds;
               }
-              __syncwarp();
-              dlp[cc] += dsp;
-              pv[e] = pp;
-              dsv[e] = ds;
+              if constexpr (F16) {
+                pk[c >> 1] = pack_h2(pv[0], pv[1]);
+                dk[c >> 1] = pack_h2(dsv[0], dsv[1]);
+              } else {
+                pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+                dk[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+              }
             }
-            if constexpr (F16) {
-              px[c >> 1] = pack_h2(pv[0], pv[1]);
-              py[c >> 1] = pack_h2(dsv[0], dsv[1]);
-            } else {
-              px[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-              py[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-            }
-          }
-        };
-        // interior path over column pairs: rt_pair(c) gives the pair's time
-        // bias, ds_sink(c, ds2) sees its dS
-        auto interior_pairs = [&](auto rt_pair, auto ds_sink) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const uint64_t s2 = f2_add(f2_pack(__uint_as_float(xs[c]), __uint_as_float(xs[c + 1])),
-                                       f2_add(bp[c], rt_pair(c)));
-            uint64_t p2, g2;
-            phi_grad_pair<PHI>(s2, inv_n, p2, g2);
-            const uint64_t ds2 =
-                f2_mul(f2_pack(__uint_as_float(ys[c]), __uint_as_float(ys[c + 1])), g2);
-            ds_sink(c, ds2);
             __syncwarp();
-            uint64_t* dd = reinterpret_cast<uint64_t*>(dlp + c);
-            *dd = f2_add(*dd, ds2);
-            if constexpr (F16) {
-              px[c >> 1] = f2_to_h2(p2);
-              py[c >> 1] = f2_to_h2(ds2);
-            } else {
-              px[c >> 1] = f2_to_bf16x2(p2);
-              py[c >> 1] = f2_to_bf16x2(ds2);
-            }
+            tmem_st4(tmem + lane_off + kX + static_cast<uint32_t>(c0 + 4 * g), pk);
+            tmem_st4(tmem + lane_off + kY + static_cast<uint32_t>(c0 + 4 * g), dk);
+            *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + g) ^ (r & 7)) << 4)) =
+                make_uint4(dk[0], dk[1], dk[2], dk[3]);
           }
         };
         if (!interior) {
           general();
         } else {
+          uint32_t xs[32], ys[32];
+          tmem_ld32(tmem + lane_off + kX + static_cast<uint32_t>(c0), xs);
+          tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
+          tmem_ld_wait(xs);
+          tmem_ld_wait(ys);
+          uint32_t px[16], py[16];
+          // interior path over column pairs: rt_pair(c) gives the pair's time
+          // bias, ds_sink(c, ds2) sees its dS; returns false (nothing written)
+          // when the block falls back to the general path
+          auto interior_pairs = [&](auto rt_pair, auto ds_sink) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const uint64_t s2 = f2_add(f2_pack(__uint_as_float(xs[c]), __uint_as_float(xs[c + 1])),
+                                         f2_add(bp[c], rt_pair(c)));
+              uint64_t p2, g2;
+              phi_grad_pair<PHI>(s2, inv_n, p2, g2);
+              const uint64_t ds2 =
+                  f2_mul(f2_pack(__uint_as_float(ys[c]), __uint_as_float(ys[c + 1])), g2);
+              ds_sink(c, ds2);
+              __syncwarp();
+              uint64_t* dd = reinterpret_cast<uint64_t*>(dlp + c);
+              *dd = f2_add(*dd, ds2);
+              if constexpr (F16) {
+                px[c >> 1] = f2_to_h2(p2);
+                py[c >> 1] = f2_to_h2(ds2);
+              } else {
+                px[c >> 1] = f2_to_bf16x2(p2);
+                py[c >> 1] = f2_to_bf16x2(ds2);
+              }
+            }
+          };
+          bool packed = true;  // px / py hold the block's packed P^T / dS^T
           const int32_t dt_first = tt[c0] - t_own;
           const int32_t dt_last = tt[c0 + 31] - t_own;
           if (__all_sync(full, dt_last < edge)) {
@@ -530,10 +590,23 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               walk_to(dt_last);
               tg_acc += hsum;
             } else {
+              packed = false;
               general();
             }
           }
+          if (packed) {
+            // dS^T rows to shared memory for the dQ MMA; the packed operands
+            // over the first 16 of the 32 columns this warp read
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + k) ^ (r & 7)) << 4)) =
+                  make_uint4(py[4 * k], py[4 * k + 1], py[4 * k + 2], py[4 * k + 3]);
+            __syncwarp();
+            tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
+            tmem_st16(tmem + lane_off + kY + static_cast<uint32_t>(c0), py);
+          }
         }
+        fence_proxy_async_smem();
         // this block's diagonals into the CTA histogram (0 <= D < P - 1 there:
         // clamped pairs went to pg_clamp; entries past the shared histogram go
         // to global memory), and the buffers cleared
@@ -550,23 +623,6 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           diagB[k] = 0.0f;
           diagA[k + 1] = 0.0f;
         }
-        // dS^T rows to shared memory for the dQ MMA, once the previous tile
-        // pair's dQ MMAs have read them
-        if (it > 0) {
-          ok = __all_sync(full, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
-          tc_fence_after();
-        }
-        if (ok) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + k) ^ (r & 7)) << 4)) =
-                make_uint4(py[4 * k], py[4 * k + 1], py[4 * k + 2], py[4 * k + 3]);
-          fence_proxy_async_smem();
-        }
-        // the packed operands go over the first 16 of the 32 columns this warp read
-        __syncwarp();
-        tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
-        tmem_st16(tmem + lane_off + kY + static_cast<uint32_t>(c0), py);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -574,7 +630,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // the previous tile pair's dQ_part, while this pair's MMAs run
       if (ok && it > 0) drain_dq(it - 1);
     }
-    if (tg_acc != 0.0f) atomicAdd(&sTg[tb], tg_acc);
+    warp_bucket_add(sTg, tg_acc != 0.0f, tb, tg_acc);
     if (ok && n_st > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(n_st - 1) & 1u, ctl));
       tc_fence_after();
