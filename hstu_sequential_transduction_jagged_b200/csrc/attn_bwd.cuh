@@ -65,7 +65,8 @@ struct BwSmem {
   // dS^T of the current tile pair, 16-bit, 128B-swizzled rows of 64 queries:
   // queries 0-63 at kDs, 64-127 at kDs + BW_TILE_BYTES (row = key, 128 B)
   static constexpr uint32_t kDs = kStg + 2 * kStgBytes;
-  static constexpr uint32_t kTimes = kDs + 2 * BW_TILE_BYTES;  // 2 x 128 int32 (query rows)
+  static constexpr uint32_t kPt = kDs + 2 * BW_TILE_BYTES;     // P^T, the same layout
+  static constexpr uint32_t kTimes = kPt + 2 * BW_TILE_BYTES;  // 2 x 128 int32 (query rows)
   // 2 x 256 float pairs: entry e of the rab_pos band with its successor
   static constexpr uint32_t kBand = kTimes + 2 * 128 * 4;
   static constexpr uint32_t kThr = kBand + 2 * 256 * 8;     // Tb int32 thresholds
@@ -88,8 +89,9 @@ enum : int {
   BWB_S = 5,            // S^T and dP^T of the current tile pair are in tensor memory
   BWB_P = 6,            // the element warps wrote P^T / dS^T
   BWB_DONE = 7,         // every MMA completed
-  BWB_DQ = 8,           // the tile pair's dQ_part is in tensor memory (dS^T read)
-  BWB_COUNT = 9
+  BWB_S3 = 8,           // dQ_part, dV and dK MMAs of the tile pair done (P^T, dS^T read)
+  BWB_XYF = 9,          // the element warps read S^T / dP^T: tensor memory X / Y free
+  BWB_COUNT = 10
 };
 
 // phi2 and its derivative at s (pointwise modes)
@@ -186,6 +188,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint8_t* sOwn1 = smem + BwSmem::kOwn1;
   uint8_t* sStg = smem + BwSmem::kStg;
   uint8_t* sDs = smem + BwSmem::kDs;
+  uint8_t* sPt = smem + BwSmem::kPt;
   int32_t* sTimes = reinterpret_cast<int32_t*>(smem + BwSmem::kTimes);
   float* sBand = reinterpret_cast<float*>(smem + BwSmem::kBand);
   int32_t* sThr = reinterpret_cast<int32_t*>(smem + BwSmem::kThr);
@@ -210,7 +213,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars[BWB_S], 1);
     mbar_init(&bars[BWB_P], BW_ELEM_WARPS * 32);
     mbar_init(&bars[BWB_DONE], 1);
-    mbar_init(&bars[BWB_DQ], 1);
+    mbar_init(&bars[BWB_S3], 1);
+    mbar_init(&bars[BWB_XYF], BW_ELEM_WARPS * 32);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -230,9 +234,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   tc_fence_after();
   const uint32_t tmem = *sTmemBase;
   const WaitCtl ctl{sAbort, p.timeout_ns};
-  // tensor memory: X = S^T (columns 0-127, later the packed P^T over them),
-  // Y = dP^T (128-255, later the packed dS^T), dV (256-319), dK (320-383),
-  // dQ_part of even / odd tile pairs (384-447 / 448-511)
+  // tensor memory: X = S^T (columns 0-127), Y = dP^T (128-255), dV (256-319),
+  // dK (320-383), dQ_part of even / odd tile pairs (384-447 / 448-511)
   constexpr uint32_t kX = 0, kY = 128, kAcc0 = 256, kAcc1 = 320, kDq = 384;
 
   if (warp == BW_PRODUCER_WARP) {
@@ -268,7 +271,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       return __all_sync(0xffffffffu, mbar_wait(bar, par, ctl));
     };
     constexpr uint32_t idesc_ss = idesc_16_f32(BW_ROWS, BW_COLS, false, false, F16);
-    constexpr uint32_t idesc_ts = idesc_16_f32(BW_ROWS, ATT_HD, false, true, F16);
+    constexpr uint32_t idesc_acc = idesc_16_f32(BW_ROWS, ATT_HD, false, true, F16);
     constexpr uint32_t idesc_dq = idesc_16_f32(BW_COLS, ATT_HD, true, true, F16);
     const uint64_t dOwn0 = smem_desc_sw128(smem_u32(sOwn0), 16, 1024);   // K, K-major A
     const uint64_t dOwn1 = smem_desc_sw128(smem_u32(sOwn1), 16, 1024);   // V, K-major A
@@ -276,18 +279,19 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // dS as an MN-major A (M = 128 queries: two 64-query halves BW_TILE_BYTES
     // apart; K = keys: 8-row groups 1024 bytes apart)
     const uint64_t dDsm = smem_desc_sw128(smem_u32(sDs), BW_TILE_BYTES, 1024);
-    bool ok = wait_all(&bars[BWB_OWN], 0);
-    tc_fence_after();
-    for (int it = 0; ok && it < n_st; ++it) {
-      const int s = it & 1;
-      ok = wait_all(&bars[BWB_FULL + s], (it >> 1) & 1);
-      if (!ok) break;
+    // dS^T and P^T as K-major A (M = 128 keys, K = queries: 16-query steps of
+    // 32 bytes inside a 64-query half, the second half BW_TILE_BYTES further)
+    const uint64_t dDsk = smem_desc_sw128(smem_u32(sDs), 16, 1024);
+    const uint64_t dPtk = smem_desc_sw128(smem_u32(sPt), 16, 1024);
+    // S^T = K Q^T, dP^T = V dO^T of tile pair j (K = 64: four steps)
+    auto issue_sdp = [&](int j) -> bool {
+      const int s = j & 1;
+      if (!wait_all(&bars[BWB_FULL + s], (j >> 1) & 1)) return false;
       tc_fence_after();
       const uint32_t sa = smem_u32(sStg + s * BwSmem::kStgBytes);
       const uint64_t dS0k = smem_desc_sw128(sa, 16, 1024);                  // Q, K-major
       const uint64_t dS1k = smem_desc_sw128(sa + BW_TILE_BYTES, 16, 1024);  // dO, K-major
       if (leader) {
-        // S^T = K Q^T, dP^T = V dO^T (K = 64: four steps)
 #pragma unroll
         for (int kk = 0; kk < ATT_HD / 16; ++kk)
           mma_bf16_ss(tmem + kX, dOwn0 + 2 * kk, dS0k + 2 * kk, idesc_ss, kk > 0 ? 1u : 0u);
@@ -297,10 +301,27 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         mma_commit(&bars[BWB_S]);
       }
       __syncwarp();
+      return true;
+    };
+    bool ok = wait_all(&bars[BWB_OWN], 0);
+    tc_fence_after();
+    if (ok) ok = issue_sdp(0);
+    for (int it = 0; ok && it < n_st; ++it) {
+      // the next tile pair's S^T / dP^T as soon as this pair's are read, so
+      // they run while the element warps work on this pair
+      if (it + 1 < n_st) {
+        ok = wait_all(&bars[BWB_XYF], static_cast<uint32_t>(it) & 1u);
+        if (!ok) break;
+        tc_fence_after();
+        ok = issue_sdp(it + 1);
+        if (!ok) break;
+      }
       ok = wait_all(&bars[BWB_P], static_cast<uint32_t>(it) & 1u);
       if (!ok) break;
       tc_fence_after();
-      const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                // Q, MN-major B
+      const int s = it & 1;
+      const uint32_t sa = smem_u32(sStg + s * BwSmem::kStgBytes);
+      const uint64_t dS0m = smem_desc_sw128(sa, 8192, 1024);                  // Q, MN-major B
       const uint64_t dS1m = smem_desc_sw128(sa + BW_TILE_BYTES, 8192, 1024);  // dO, MN-major B
       if (leader) {
         // dQ_part = dS K over the 128 keys (eight steps of 16 keys, 2 KB each)
@@ -308,22 +329,20 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < BW_ROWS / 16; ++kk)
           mma_bf16_ss(dq_acc, dDsm + 128 * kk, dOwn0m + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
-        mma_commit(&bars[BWB_DQ]);
-        // dV += P^T dO ; dK += dS^T Q over the 128 queries (eight steps); the
-        // packed 16-bit operand of queries 32g .. 32g + 31 sits at columns
-        // 32g .. 32g + 15 of its region
+        // dV += P^T dO ; dK += dS^T Q over the 128 queries (eight steps)
 #pragma unroll
         for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-          const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
-          mma_bf16_ts(tmem + kAcc0, tmem + kX + ac, dS1m + 128 * kk, idesc_ts,
+          const uint64_t ak = static_cast<uint64_t>((kk >> 2) * (BW_TILE_BYTES >> 4) + (kk & 3) * 2);
+          mma_bf16_ss(tmem + kAcc0, dPtk + ak, dS1m + 128 * kk, idesc_acc,
                       (it > 0 || kk > 0) ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < BW_COLS / 16; ++kk) {
-          const uint32_t ac = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
-          mma_bf16_ts(tmem + kAcc1, tmem + kY + ac, dS0m + 128 * kk, idesc_ts,
+          const uint64_t ak = static_cast<uint64_t>((kk >> 2) * (BW_TILE_BYTES >> 4) + (kk & 3) * 2);
+          mma_bf16_ss(tmem + kAcc1, dDsk + ak, dS0m + 128 * kk, idesc_acc,
                       (it > 0 || kk > 0) ? 1u : 0u);
         }
+        mma_commit(&bars[BWB_S3]);
         mma_commit(&bars[BWB_EMPTY + s]);
       }
       __syncwarp();
@@ -345,6 +364,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // this thread's 64-byte slice of the dS^T rows in shared memory (four
     // 16-byte chunks of 8 queries, 128B swizzle: chunk index ^ (row & 7))
     uint8_t* ds_row = sDs + (cg >> 1) * BW_TILE_BYTES + r * 128;
+    uint8_t* pt_row = ds_row + (BwSmem::kPt - BwSmem::kDs);  // the same slice of P^T
     const int ds_chunk0 = (cg & 1) * 4;
     // the previous tile pair's dQ_part (rows = its queries) into global dQ
     auto drain_dq = [&](int j) {
@@ -408,38 +428,53 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     float* diagB = sDiag + warp * 128;
     float* diagA = diagB + 64;
     float* dlp = ((lane & 1) ? diagB : diagA + 1) + 31 - lane;  // dlp[cc]: this lane's entry
+    // Staging of tile pair j's 128 query times and 255-entry position-bias
+    // band (entry e: rab_pos[min(D, P - 1)] for D = i - j = (j's first query -
+    // o0) + e - 127, 0 for D < 0, paired with entry e + 1): the global loads of
+    // the next pair are issued before this pair's work and stored after it.
+    int64_t pf_t = 0;
+    float pf_b0 = 0.0f, pf_b1 = 0.0f;
+    auto stage_load = [&](int j) {
+      const int sb = (ot + j) * BW_COLS;
+      if (tid < 128) {
+        const int row = sb + tid;
+        pf_t = row < n ? p.timestamps[start + row] : t_first;
+      } else if (tid < 128 + 255) {
+        const int dd = sb - o0 + (tid - 128) - 127;
+        pf_b0 = dd >= 0 ? __ldg(rp + min(dd, p.P - 1)) : 0.0f;
+        pf_b1 = dd + 1 >= 0 ? __ldg(rp + min(dd + 1, p.P - 1)) : 0.0f;
+      }
+    };
+    auto stage_store = [&](int j) {
+      if (tid < 128) {
+        const int64_t d = pf_t - t_first;
+        sTimes[(j & 1) * 128 + tid] =
+            d >= static_cast<int64_t>(INT32_MAX) - 1 ? INT32_MAX - 1 : static_cast<int32_t>(d);
+      } else if (tid < 128 + 255) {
+        reinterpret_cast<uint64_t*>(sBand)[(j & 1) * 256 + tid - 128] = f2_pack(pf_b0, pf_b1);
+      }
+    };
+    stage_load(0);
+    stage_store(0);
     bool ok = true;
     for (int it = 0; it < n_st; ++it) {
       const int sbase = (ot + it) * BW_COLS;  // first query of the tile
-      // this tile's 128 query times and the 255-entry position-bias band:
-      // entry e holds rab_pos[min(D, P - 1)] for D = i - j = dbase + e - 127
-      // (0 for D < 0), paired with entry e + 1
-      int32_t* tt = sTimes + (it & 1) * 128;
-      uint64_t* bandp = reinterpret_cast<uint64_t*>(sBand) + (it & 1) * 256;
-      const int dbase = sbase - o0;
-      if (tid < 128) {
-        const int row = sbase + tid;
-        tt[tid] = row < n ? bw_rel_time(p.timestamps, start + row, t_first) : 0;
-      } else if (tid < 128 + 255) {
-        const int e = tid - 128;
-        const int dd = dbase + e - 127;
-        const float v0 = dd >= 0 ? __ldg(rp + min(dd, p.P - 1)) : 0.0f;
-        const float v1 = dd + 1 >= 0 ? __ldg(rp + min(dd + 1, p.P - 1)) : 0.0f;
-        bandp[e] = f2_pack(v0, v1);
-      }
+      const int32_t* tt = sTimes + (it & 1) * 128;
+      const uint64_t* bandp = reinterpret_cast<const uint64_t*>(sBand) + (it & 1) * 256;
       named_barrier_sync(1, BW_ELEM_WARPS * 32);
+      if (it + 1 < n_st) stage_load(it + 1);
       if (ok) ok = mbar_wait(&bars[BWB_S], static_cast<uint32_t>(it) & 1u, ctl);
       ok = __all_sync(full, ok);
-      if (ok) {
-        tc_fence_after();
-        // dS^T goes to shared memory below, once the previous tile pair's dQ
-        // MMAs have read it (they were issued before this pair's S MMAs)
+      bool xy_read = false;  // this thread arrived on BWB_XYF for the pair
+      // the previous pair's dQ / dV / dK MMAs read P^T and dS^T from shared memory
+      auto wait_s3 = [&]() {
         if (it > 0) {
-          ok = __all_sync(full, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(it - 1) & 1u, ctl));
+          ok = __all_sync(full, mbar_wait(&bars[BWB_S3], static_cast<uint32_t>(it - 1) & 1u, ctl));
           tc_fence_after();
         }
-      }
+      };
       if (ok) {
+        tc_fence_after();
         // band pair of column cc: bp[cc]
         const uint64_t* bp = bandp + (c0 - r + 127);
         // every column of the block visible (not the diagonal tile, not past
@@ -447,11 +482,11 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const bool interior = it > 0 && sbase + c0 + 32 <= n &&
                               sbase + c0 + 31 - (o0 + q4 * 32) < p.P - 1;
         // General path: per element visibility, walk and clamp.  A rolled loop
-        // over four 8-column groups (the rare blocks keep their code small): it
-        // reads S^T / dP^T from tensor memory and stores the packed P^T / dS^T
-        // of each group itself (group g over columns 4g .. 4g + 3, which held
-        // raw values the loop has already read).
+        // over four 8-column groups (the rare blocks keep their code small)
+        // that reads S^T / dP^T from tensor memory and writes each group's
+        // packed P^T / dS^T to shared memory.
         auto general = [&]() {
+          wait_s3();
           int c_lo = 0, c_hi = 31;
           if (!own_ok) {
             c_lo = 32;
@@ -500,14 +535,43 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 dk[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
               }
             }
-            __syncwarp();
-            tmem_st4(tmem + lane_off + kX + static_cast<uint32_t>(c0 + 4 * g), pk);
-            tmem_st4(tmem + lane_off + kY + static_cast<uint32_t>(c0 + 4 * g), dk);
-            *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + g) ^ (r & 7)) << 4)) =
-                make_uint4(dk[0], dk[1], dk[2], dk[3]);
+            const int off = ((ds_chunk0 + g) ^ (r & 7)) << 4;
+            *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
           }
+          tc_fence_before();
+          mbar_arrive(&bars[BWB_XYF]);
+          xy_read = true;
         };
-        if (!interior) {
+        // interior blocks: the time bias of each column pair comes from the
+        // lane's current bucket (every lane stays in it: "steady") or from one
+        // of two warp-wide buckets B_lo, B_hi (B_hi iff dt >= thr[B_hi])
+        int path = 2;  // 0 steady, 1 two buckets, 2 general
+        int32_t dt_last = 0, thr_hi = INT32_MAX;
+        float rt_lo = 0.0f, rt_hi = 0.0f;
+        if (interior) {
+          const int32_t dt_first = tt[c0] - t_own;
+          dt_last = tt[c0 + 31] - t_own;
+          if (__all_sync(full, dt_last < edge)) {
+            path = 0;
+          } else {
+            walk_to(dt_first);
+            int bl = tb;  // bucket of the block's last column
+            int32_t el = edge;
+            while (dt_last >= el) {
+              ++bl;
+              el = bl + 1 < p.Tb ? sThr[bl + 1] : INT32_MAX;
+            }
+            const int B_lo = __reduce_min_sync(full, tb), B_hi = __reduce_max_sync(full, bl);
+            if (B_hi - B_lo <= 1) {
+              path = 1;
+              rt_lo = sRt[B_lo];
+              rt_hi = sRt[B_hi];
+              thr_hi = B_hi > B_lo ? sThr[B_hi] : INT32_MAX;
+            }
+          }
+        }
+        if (path == 2) {
           general();
         } else {
           uint32_t xs[32], ys[32];
@@ -515,10 +579,12 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           tmem_ld32(tmem + lane_off + kY + static_cast<uint32_t>(c0), ys);
           tmem_ld_wait(xs);
           tmem_ld_wait(ys);
+          // S^T / dP^T are in registers: the next pair's MMAs may overwrite them
+          tc_fence_before();
+          mbar_arrive(&bars[BWB_XYF]);
+          xy_read = true;
           uint32_t px[16], py[16];
-          // interior path over column pairs: rt_pair(c) gives the pair's time
-          // bias, ds_sink(c, ds2) sees its dS; returns false (nothing written)
-          // when the block falls back to the general path
+          // rt_pair(c) gives the pair's time bias, ds_sink(c, ds2) sees its dS
           auto interior_pairs = [&](auto rt_pair, auto ds_sink) {
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
@@ -541,11 +607,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               }
             }
           };
-          bool packed = true;  // px / py hold the block's packed P^T / dS^T
-          const int32_t dt_first = tt[c0] - t_own;
-          const int32_t dt_last = tt[c0 + 31] - t_own;
-          if (__all_sync(full, dt_last < edge)) {
-            // every lane stays in its bucket: its bias is rt_cur
+          if (path == 0) {
             const uint64_t rt2 = f2_pack(rt_cur, rt_cur);
             uint64_t tg2 = f2_pack(0.0f, 0.0f);
             interior_pairs([&](int) { return rt2; },
@@ -554,56 +616,41 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             f2_unpack(tg2, a0, a1);
             tg_acc += a0 + a1;
           } else {
-            walk_to(dt_first);
-            int bl = tb;  // bucket of the block's last column
-            int32_t el = edge;
-            while (dt_last >= el) {
-              ++bl;
-              el = bl + 1 < p.Tb ? sThr[bl + 1] : INT32_MAX;
-            }
-            const int B_lo = __reduce_min_sync(full, tb), B_hi = __reduce_max_sync(full, bl);
-            if (B_hi - B_lo <= 1) {
-              // two buckets in the warp: B_hi iff dt >= thr[B_hi]
-              const float rt_lo = sRt[B_lo], rt_hi = sRt[B_hi];
-              const int32_t thr_hi = B_hi > B_lo ? sThr[B_hi] : INT32_MAX;
-              uint64_t tg2 = f2_pack(0.0f, 0.0f), hi2 = f2_pack(0.0f, 0.0f);
-              interior_pairs(
-                  [&](int c) {
-                    const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
-                    return f2_pack(t2.x - t_own >= thr_hi ? rt_hi : rt_lo,
-                                   t2.y - t_own >= thr_hi ? rt_hi : rt_lo);
-                  },
-                  [&](int c, uint64_t d) {
-                    const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
-                    float d0, d1;
-                    f2_unpack(d, d0, d1);
-                    hi2 = f2_add(hi2, f2_pack(t2.x - t_own >= thr_hi ? d0 : 0.0f,
-                                              t2.y - t_own >= thr_hi ? d1 : 0.0f));
-                    tg2 = f2_add(tg2, d);
-                  });
-              float a0, a1, h0, h1;
-              f2_unpack(tg2, a0, a1);
-              f2_unpack(hi2, h0, h1);
-              const float hsum = h0 + h1;
-              // the lane's elements below thr_hi belong to its current bucket
-              tg_acc += (a0 + a1) - hsum;
-              walk_to(dt_last);
-              tg_acc += hsum;
-            } else {
-              packed = false;
-              general();
-            }
+            uint64_t tg2 = f2_pack(0.0f, 0.0f), hi2 = f2_pack(0.0f, 0.0f);
+            interior_pairs(
+                [&](int c) {
+                  const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
+                  return f2_pack(t2.x - t_own >= thr_hi ? rt_hi : rt_lo,
+                                 t2.y - t_own >= thr_hi ? rt_hi : rt_lo);
+                },
+                [&](int c, uint64_t d) {
+                  const int2 t2 = *reinterpret_cast<const int2*>(tt + c0 + c);
+                  float d0, d1;
+                  f2_unpack(d, d0, d1);
+                  hi2 = f2_add(hi2, f2_pack(t2.x - t_own >= thr_hi ? d0 : 0.0f,
+                                            t2.y - t_own >= thr_hi ? d1 : 0.0f));
+                  tg2 = f2_add(tg2, d);
+                });
+            float a0, a1, h0, h1;
+            f2_unpack(tg2, a0, a1);
+            f2_unpack(hi2, h0, h1);
+            const float hsum = h0 + h1;
+            // the lane's elements below thr_hi belong to its current bucket
+            tg_acc += (a0 + a1) - hsum;
+            walk_to(dt_last);
+            tg_acc += hsum;
           }
-          if (packed) {
-            // dS^T rows to shared memory for the dQ MMA; the packed operands
-            // over the first 16 of the 32 columns this warp read
+          // P^T and dS^T rows to shared memory for the dQ / dV / dK MMAs
+          wait_s3();
+          if (ok) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              *reinterpret_cast<uint4*>(ds_row + (((ds_chunk0 + k) ^ (r & 7)) << 4)) =
+            for (int k = 0; k < 4; ++k) {
+              const int off = ((ds_chunk0 + k) ^ (r & 7)) << 4;
+              *reinterpret_cast<uint4*>(pt_row + off) =
+                  make_uint4(px[4 * k], px[4 * k + 1], px[4 * k + 2], px[4 * k + 3]);
+              *reinterpret_cast<uint4*>(ds_row + off) =
                   make_uint4(py[4 * k], py[4 * k + 1], py[4 * k + 2], py[4 * k + 3]);
-            __syncwarp();
-            tmem_st16(tmem + lane_off + kX + static_cast<uint32_t>(c0), px);
-            tmem_st16(tmem + lane_off + kY + static_cast<uint32_t>(c0), py);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -623,16 +670,17 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           diagB[k] = 0.0f;
           diagA[k + 1] = 0.0f;
         }
-        tmem_st_wait();
       }
+      if (!xy_read) mbar_arrive(&bars[BWB_XYF]);  // error path: keep the count
       tc_fence_before();
       mbar_arrive(&bars[BWB_P]);
+      if (it + 1 < n_st) stage_store(it + 1);
       // the previous tile pair's dQ_part, while this pair's MMAs run
       if (ok && it > 0) drain_dq(it - 1);
     }
     warp_bucket_add(sTg, tg_acc != 0.0f, tb, tg_acc);
     if (ok && n_st > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_DQ], static_cast<uint32_t>(n_st - 1) & 1u, ctl));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_S3], static_cast<uint32_t>(n_st - 1) & 1u, ctl));
       tc_fence_after();
       if (ok) drain_dq(n_st - 1);
     }
