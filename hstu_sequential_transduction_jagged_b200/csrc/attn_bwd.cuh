@@ -55,6 +55,7 @@ struct AttnBwdParams {
   int32_t hist_len;            // position-gradient entries kept in shared memory
   uint64_t timeout_ns;
   int32_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0), clamped to int32
+  int4 oct[32];                   // per octave k of dt+1: {t1, t2, t3, bucket(2^k - 1)}
 };
 
 struct BwSmem {
@@ -72,7 +73,8 @@ struct BwSmem {
   static constexpr uint32_t kThr = kBand + 2 * 256 * 8;     // Tb int32 thresholds
   static constexpr uint32_t kRt = kThr + MAX_TIME_BUCKETS * 4;  // Tb floats (rab_time row)
   static constexpr uint32_t kTg = kRt + MAX_TIME_BUCKETS * 4;   // Tb floats (time gradient)
-  static constexpr uint32_t kBars = kTg + MAX_TIME_BUCKETS * 4; // 16 barriers
+  static constexpr uint32_t kOct = kTg + MAX_TIME_BUCKETS * 4;  // 32 int4 octave entries
+  static constexpr uint32_t kBars = kOct + 32 * 16;             // 16 barriers
   static constexpr uint32_t kMisc = kBars + 16 * 8;
   // per element warp two 64-float diagonal buffers (odd lanes, even lanes)
   static constexpr uint32_t kDiag = kMisc + 64;
@@ -194,6 +196,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   int32_t* sThr = reinterpret_cast<int32_t*>(smem + BwSmem::kThr);
   float* sRt = reinterpret_cast<float*>(smem + BwSmem::kRt);
   float* sTg = reinterpret_cast<float*>(smem + BwSmem::kTg);
+  int4* sOct = reinterpret_cast<int4*>(smem + BwSmem::kOct);
   float* sPg = reinterpret_cast<float*>(smem + BwSmem::kPg);
   float* sDiag = reinterpret_cast<float*>(smem + BwSmem::kDiag);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BwSmem::kBars);
@@ -227,6 +230,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     sRt[k] = p.rab_time[static_cast<int64_t>(h) * p.Tb + k];
     sTg[k] = 0.0f;
   }
+  if (tid < 32) sOct[tid] = p.oct[tid];
   for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
   for (int k = tid; k < BW_ELEM_WARPS * 128; k += BW_THREADS) sDiag[k] = 0.0f;
   tc_fence_before();
@@ -408,16 +412,11 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (mv) advance(dt);
       }
     };
-    // the same for one lane on its own (the general path, where lanes sit in
-    // many different buckets): the running sum goes to global memory with a
-    // reduction that does not return
+    // the general path, where lanes sit in many different buckets, takes each
+    // element's bucket straight from the octave table; a lane's running sum
+    // goes to global memory (a reduction that does not return) when its
+    // bucket changes
     float* drt = p.drab_time + static_cast<int64_t>(h) * p.Tb;
-    auto walk_lane = [&](int32_t dt) {
-      if (dt >= edge) {
-        if (tg_acc != 0.0f) atomicAdd(&drt[tb], tg_acc);
-        advance(dt);
-      }
-    };
     // position-table gradient: this warp's 32 x 32 block adds dS to its 63
     // diagonals k = cc - lane + 31 (D = i - j = dg0 + k - 31).  Odd lanes add
     // into diagB[k], even lanes into diagA[k + 1], so that the two diagonals of
@@ -481,7 +480,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // the user's end) and no pair in the clamped position bucket
         const bool interior = it > 0 && sbase + c0 + 32 <= n &&
                               sbase + c0 + 31 - (o0 + q4 * 32) < p.P - 1;
-        // General path: per element visibility, walk and clamp.  A rolled loop
+        // General path: per element visibility, bucket and clamp.  A rolled loop
         // over four 8-column groups (the rare blocks keep their code small)
         // that reads S^T / dP^T from tensor memory and writes each group's
         // packed P^T / dS^T to shared memory.
@@ -509,7 +508,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int cc = 8 * g + c + e;
                 float pp = 0.0f, ds = 0.0f, dsp = 0.0f;
                 if (cc >= c_lo && cc <= c_hi) {
-                  walk_lane(tt[c0 + cc] - t_own);
+                  const int b = time_bucket_octave(tt[c0 + cc] - t_own, sOct);
+                  if (b != tb) {
+                    if (tg_acc != 0.0f) atomicAdd(&drt[tb], tg_acc);
+                    tg_acc = 0.0f;
+                    tb = b;
+                    rt_cur = sRt[b];
+                  }
                   const int dpos = (sbase + c0 + cc) - orow;  // D = i - j
                   float b0, b1;
                   f2_unpack(bp[cc], b0, b1);
@@ -539,13 +544,14 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
           }
+          edge = tb + 1 < p.Tb ? sThr[tb + 1] : INT32_MAX;
           tc_fence_before();
           mbar_arrive(&bars[BWB_XYF]);
           xy_read = true;
         };
         // interior blocks: the time bias of each column pair comes from the
-        // lane's current bucket (every lane stays in it: "steady") or from one
-        // of two warp-wide buckets B_lo, B_hi (B_hi iff dt >= thr[B_hi])
+        // lane's current bucket (every lane stays in it: "steady") or from the
+        // lane's current bucket and the next one (hi iff dt >= thr_hi)
         int path = 2;  // 0 steady, 1 two buckets, 2 general
         int32_t dt_last = 0, thr_hi = INT32_MAX;
         float rt_lo = 0.0f, rt_hi = 0.0f;
@@ -556,18 +562,13 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             path = 0;
           } else {
             walk_to(dt_first);
-            int bl = tb;  // bucket of the block's last column
-            int32_t el = edge;
-            while (dt_last >= el) {
-              ++bl;
-              el = bl + 1 < p.Tb ? sThr[bl + 1] : INT32_MAX;
-            }
-            const int B_lo = __reduce_min_sync(full, tb), B_hi = __reduce_max_sync(full, bl);
-            if (B_hi - B_lo <= 1) {
+            // every lane spans at most two buckets (its current one and the
+            // next): per element, bucket tb + 1 iff dt >= edge
+            if (__all_sync(full, tb + 2 >= p.Tb || dt_last < sThr[tb + 2])) {
               path = 1;
-              rt_lo = sRt[B_lo];
-              rt_hi = sRt[B_hi];
-              thr_hi = B_hi > B_lo ? sThr[B_hi] : INT32_MAX;
+              rt_lo = rt_cur;
+              rt_hi = tb + 1 < p.Tb ? sRt[tb + 1] : rt_cur;
+              thr_hi = edge;
             }
           }
         }

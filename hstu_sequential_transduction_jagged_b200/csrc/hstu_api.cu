@@ -641,6 +641,7 @@ hstu_status_t launch_attn_bwd(const hstu_layer_cfg_t* c, const hstu_jagged_t* ja
   const int64_t* thr = thresholds_for(Tb);
   for (int b = 0; b < Tb; ++b)
     p.thr[b] = thr[b] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(thr[b]) : INT32_MAX;
+  if (!compute_octaves(Tb, thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
   const size_t smem = BwSmem::bytes(p.hist_len);
   if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
   // dQ is accumulated into (one vector atomic per element per key tile)
