@@ -52,7 +52,6 @@ struct AttnBwdParams {
   float* drab_time;            // [H, Tb]
   int32_t B, H, P, Tb, max_len;
   int32_t phi2;
-  int32_t hist_len;            // position-gradient entries kept in shared memory
   uint64_t timeout_ns;
   int32_t thr[MAX_TIME_BUCKETS];  // time-bucket thresholds (thr[0] = 0), clamped to int32
   int4 oct[32];                   // per octave k of dt+1: {t1, t2, t3, bucket(2^k - 1)}
@@ -78,10 +77,10 @@ struct BwSmem {
   static constexpr uint32_t kMisc = kBars + 16 * 8;
   // per element warp two 64-float diagonal buffers (odd lanes, even lanes)
   static constexpr uint32_t kDiag = kMisc + 64;
-  static constexpr uint32_t kPg = kDiag + BW_ELEM_WARPS * 128 * 4;  // hist_len floats (position gradient)
-  static constexpr uint32_t bytes(int hist_len) {
-    return kPg + static_cast<uint32_t>(hist_len) * 4u + 1024u;
-  }
+  // dQ_part of one tile pair in fp32 for the TMA reduce-add: two 32-column
+  // boxes of 128 rows (128B-swizzled rows of 128 bytes), 16 KB each
+  static constexpr uint32_t kDqs = (kDiag + BW_ELEM_WARPS * 128 * 4 + 1023u) & ~1023u;
+  static constexpr uint32_t kBytes = kDqs + 2 * BW_TILE_BYTES + 1024u;
 };
 
 enum : int {
@@ -168,7 +167,7 @@ template <int PHI, bool F16>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const __grid_constant__ AttnBwdParams p) {
+                     const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ AttnBwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -197,7 +196,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   float* sRt = reinterpret_cast<float*>(smem + BwSmem::kRt);
   float* sTg = reinterpret_cast<float*>(smem + BwSmem::kTg);
   int4* sOct = reinterpret_cast<int4*>(smem + BwSmem::kOct);
-  float* sPg = reinterpret_cast<float*>(smem + BwSmem::kPg);
+  uint8_t* sDqs = smem + BwSmem::kDqs;
   float* sDiag = reinterpret_cast<float*>(smem + BwSmem::kDiag);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BwSmem::kBars);
   uint32_t* sTmemBase = reinterpret_cast<uint32_t*>(smem + BwSmem::kMisc);
@@ -231,7 +230,6 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     sTg[k] = 0.0f;
   }
   if (tid < 32) sOct[tid] = p.oct[tid];
-  for (int k = tid; k < p.hist_len; k += BW_THREADS) sPg[k] = 0.0f;
   for (int k = tid; k < BW_ELEM_WARPS * 128; k += BW_THREADS) sDiag[k] = 0.0f;
   tc_fence_before();
   __syncthreads();
@@ -370,19 +368,37 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t* ds_row = sDs + (cg >> 1) * BW_TILE_BYTES + r * 128;
     uint8_t* pt_row = ds_row + (BwSmem::kPt - BwSmem::kDs);  // the same slice of P^T
     const int ds_chunk0 = (cg & 1) * 4;
-    // the previous tile pair's dQ_part (rows = its queries) into global dQ
-    auto drain_dq = [&](int j) {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_off + kDq + 64u * static_cast<uint32_t>(j & 1) +
-                    static_cast<uint32_t>(cg * 16), v);
-      tmem_ld_wait(v);
-      const int qrow = (ot + j) * BW_COLS + r;
-      if (qrow < n) {
-        float4* d4 = reinterpret_cast<float4*>(p.dq + (start + qrow) * p.ld_g + h * ATT_HD + cg * 16);
+    // Tile pair j's dQ_part (rows = its queries) into global dQ.  Each lane
+    // quarter (32 query rows; the four warps of 16 columns that share it)
+    // stages its rows in the two swizzled fp32 boxes, then one thread of the
+    // quarter adds them to dQ with two TMA reduce-adds.  The quarter's barrier
+    // is taken on every call, `live` or not, so that no warp waits on one that
+    // gave up; the staging rows are rewritten only after the issuing thread has
+    // seen its previous reduce read them (bulk_wait_read0 before the CTA
+    // barrier at the top of each iteration, or before the last call).
+    const bool dq_issuer = cg == 0 && lane == 0;
+    uint8_t* dq_stage = sDqs + (cg >> 1) * BW_TILE_BYTES + q4 * 4096 + lane * 128;
+    auto drain_dq = [&](int j, bool live) {
+      if (live) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_off + kDq + 64u * static_cast<uint32_t>(j & 1) +
+                      static_cast<uint32_t>(cg * 16), v);
+        tmem_ld_wait(v);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          atomicAdd(d4 + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(dq_stage + ((((cg & 1) * 4 + k) ^ (lane & 7)) << 4)) =
+              make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        fence_proxy_async_smem();
+      }
+      named_barrier_sync(2 + q4, 4 * 32);
+      const int qrow0 = (ot + j) * BW_COLS + q4 * 32;
+      if (live && dq_issuer && qrow0 < n) {
+        // rows past the user's end hold exact zeros (no visible key)
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+          tma_reduce_add_2d(&tm_dq, sDqs + b * BW_TILE_BYTES + q4 * 4096, h * ATT_HD + 32 * b,
+                            static_cast<int32_t>(start + qrow0));
+        bulk_commit();
       }
     };
     // Time-bucket walk over this thread's visible pairs in the order visited:
@@ -417,6 +433,7 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // goes to global memory (a reduction that does not return) when its
     // bucket changes
     float* drt = p.drab_time + static_cast<int64_t>(h) * p.Tb;
+    float* drp = p.drab_pos + static_cast<int64_t>(h) * p.P;
     // position-table gradient: this warp's 32 x 32 block adds dS to its 63
     // diagonals k = cc - lane + 31 (D = i - j = dg0 + k - 31).  Odd lanes add
     // into diagB[k], even lanes into diagA[k + 1], so that the two diagonals of
@@ -429,8 +446,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     float* dlp = ((lane & 1) ? diagB : diagA + 1) + 31 - lane;  // dlp[cc]: this lane's entry
     // Staging of tile pair j's 128 query times and 255-entry position-bias
     // band (entry e: rab_pos[min(D, P - 1)] for D = i - j = (j's first query -
-    // o0) + e - 127, 0 for D < 0, paired with entry e + 1): the global loads of
-    // the next pair are issued before this pair's work and stored after it.
+    // o0) + e - 127, 0 for D < 0, paired with entry e + 1), written for the
+    // next pair once this pair's element work is done.
     int64_t pf_t = 0;
     float pf_b0 = 0.0f, pf_b1 = 0.0f;
     auto stage_load = [&](int j) {
@@ -460,8 +477,8 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int sbase = (ot + it) * BW_COLS;  // first query of the tile
       const int32_t* tt = sTimes + (it & 1) * 128;
       const uint64_t* bandp = reinterpret_cast<const uint64_t*>(sBand) + (it & 1) * 256;
+      if (dq_issuer) bulk_wait_read0();
       named_barrier_sync(1, BW_ELEM_WARPS * 32);
-      if (it + 1 < n_st) stage_load(it + 1);
       if (ok) ok = mbar_wait(&bars[BWB_S], static_cast<uint32_t>(it) & 1u, ctl);
       ok = __all_sync(full, ok);
       bool xy_read = false;  // this thread arrived on BWB_XYF for the pair
@@ -655,19 +672,16 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
         }
         fence_proxy_async_smem();
-        // this block's diagonals into the CTA histogram (0 <= D < P - 1 there:
-        // clamped pairs went to pg_clamp; entries past the shared histogram go
-        // to global memory), and the buffers cleared
+        // this block's diagonals into drab_pos (0 <= D < P - 1 there: clamped
+        // pairs went to pg_clamp; consecutive lanes add to consecutive entries,
+        // with reductions that do not return), and the buffers cleared
         __syncwarp();
         const int dg0 = (sbase + c0) - (o0 + q4 * 32);
 #pragma unroll
         for (int k = lane; k < 63; k += 32) {
           const float v = diagB[k] + diagA[k + 1];
           const int dd = dg0 + k - 31;
-          if (v != 0.0f && dd >= 0 && dd < p.P - 1) {
-            if (dd < p.hist_len) atomicAdd(&sPg[dd], v);
-            else atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + dd], v);
-          }
+          if (v != 0.0f && dd >= 0 && dd < p.P - 1) atomicAdd(&drp[dd], v);
           diagB[k] = 0.0f;
           diagA[k + 1] = 0.0f;
         }
@@ -675,16 +689,22 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!xy_read) mbar_arrive(&bars[BWB_XYF]);  // error path: keep the count
       tc_fence_before();
       mbar_arrive(&bars[BWB_P]);
-      if (it + 1 < n_st) stage_store(it + 1);
+      if (it + 1 < n_st) {
+        stage_load(it + 1);
+        stage_store(it + 1);
+      }
       // the previous tile pair's dQ_part, while this pair's MMAs run
-      if (ok && it > 0) drain_dq(it - 1);
+      if (it > 0) drain_dq(it - 1, ok);
     }
     warp_bucket_add(sTg, tg_acc != 0.0f, tb, tg_acc);
-    if (ok && n_st > 0) {
+    if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[BWB_S3], static_cast<uint32_t>(n_st - 1) & 1u, ctl));
       tc_fence_after();
-      if (ok) drain_dq(n_st - 1);
     }
+    if (dq_issuer) bulk_wait_read0();
+    named_barrier_sync(2 + q4, 4 * 32);
+    drain_dq(n_st - 1, ok);
+    if (dq_issuer) bulk_wait_all();
     // ---------------- epilogue: the accumulators (rows of the own tile); the
     // four column groups take 16 of the 64 accumulator columns each
     if (ok) ok = mbar_wait(&bars[BWB_DONE], 0, ctl);
@@ -709,14 +729,9 @@ hstu_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (pg_clamp != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + p.P - 1], pg_clamp);
   }
 
-  // ---------------- table gradients and teardown
+  // ---------------- time-table gradient and teardown
   tc_fence_before();
   __syncthreads();
-  const int lim = min(p.hist_len, p.P - 1);
-  for (int k = tid; k < lim; k += BW_THREADS) {
-    const float g = sPg[k];
-    if (g != 0.0f) atomicAdd(&p.drab_pos[static_cast<int64_t>(h) * p.P + k], g);
-  }
   for (int k = tid; k < p.Tb; k += BW_THREADS) {
     const float g = sTg[k];
     if (g != 0.0f) atomicAdd(&p.drab_time[static_cast<int64_t>(h) * p.Tb + k], g);

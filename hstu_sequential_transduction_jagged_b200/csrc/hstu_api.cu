@@ -197,7 +197,7 @@ AttnKernelFn attn_kernel_ptr(bool cand, int phi, bool pairs, bool f16, bool fuse
 }
 
 using AttnBwdFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                          const CUtensorMap, const AttnBwdParams);
+                          const CUtensorMap, const CUtensorMap, const AttnBwdParams);
 
 template <bool F16>
 AttnBwdFn attn_bwd_kernel_for(int phi) {
@@ -633,23 +633,21 @@ hstu_status_t launch_attn_bwd(const hstu_layer_cfg_t* c, const hstu_jagged_t* ja
   p.Tb = Tb;
   p.max_len = jag->max_len;
   p.phi2 = c->phi2;
-  // position-gradient entries kept in shared memory (the rest go to global
-  // memory with one atomic per touched entry)
-  const int hist_cap = static_cast<int>((227u * 1024u - BwSmem::bytes(0)) / 4u);
-  p.hist_len = std::min(std::min(P, jag->max_len), hist_cap);
   p.timeout_ns = kDefaultTimeoutNs;
   const int64_t* thr = thresholds_for(Tb);
   for (int b = 0; b < Tb; ++b)
     p.thr[b] = thr[b] < static_cast<int64_t>(INT32_MAX) ? static_cast<int32_t>(thr[b]) : INT32_MAX;
   if (!compute_octaves(Tb, thr, p.oct)) return HSTU_ERR_UNSUPPORTED;
-  const size_t smem = BwSmem::bytes(p.hist_len);
-  if (smem > 227u * 1024u) return HSTU_ERR_UNSUPPORTED;
-  // dQ is accumulated into (one vector atomic per element per key tile)
+  const size_t smem = BwSmem::kBytes;
+  static_assert(BwSmem::kBytes <= 227u * 1024u, "backward shared memory");
+  // dQ is accumulated into (a TMA reduce-add per tile pair)
+  CUtensorMap mdq;
+  if ((s = make_out_map(&mdq, dq, true, T, hv, ld_g)) != HSTU_OK) return s;
   HSTU_CHECK_CUDA(cudaMemset2DAsync(dq, sizeof(float) * ld_g, 0, sizeof(float) * hv, T, st));
   dim3 grid(H, jag->batch, (jag->max_len + BW_ROWS - 1) / BW_ROWS);
   {
     ProfScope prof(K_ATTN_BWD, st);
-    attn_bwd_kernel_ptr(c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, p);
+    attn_bwd_kernel_ptr(c->phi2, f16)<<<grid, BW_THREADS, smem, st>>>(mq, mk, mv, mo, mdq, p);
     HSTU_CHECK_CUDA(cudaGetLastError());
   }
   return HSTU_OK;
