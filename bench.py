@@ -668,7 +668,8 @@ def measure_train(ctx, steps, warmup, sample_clocks=False, batch=None):
         roof = {"kernel": "hstu_attn_bwd_kernel (dK, dV and dQ, one launch per layer)",
                 "bound": "tensor",
                 "achieved": ach, "peak": ctx.peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / ctx.peaks["bf16_tflops"], "traffic": None,
+                "frac": ach / ctx.peaks["bf16_tflops"],
+                "traffic": traffic_from_profiles("attention_bwd"),
                 "peak_source": f"{ctx.peak_src} bf16 dense, burst ({PEAK_RULE})",
                 "algorithmic_flop_per_launch": bwd_flop,
                 "flop_rule": "5 x 2 x 64 flop per visible (i, j, head): S, dP, dV, dQ, dK",
