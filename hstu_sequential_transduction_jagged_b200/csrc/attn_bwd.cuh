@@ -7,24 +7,30 @@
 // One tcgen05 kernel over fp16 (or bf16) Q, K, V, dO with fp32 accumulation
 // in tensor memory and fp32 outputs.  A CTA owns one (head, user, 128-key
 // tile) and walks the query tiles at and after its keys.  For each tile pair:
-//   S^T = K Q^T and dP^T = V dO^T go to tensor memory; the element warps turn
-//   them into P^T and dS^T (16-bit, over the columns they read) and also write
-//   dS^T to shared memory; then
-//   dQ_part = dS K (A = dS^T read transposed from shared memory) goes to one of
-//   two tensor-memory buffers, and dV += P^T dO, dK += dS^T Q accumulate.
-// While the tensor core runs the next tile pair's MMAs the element warps add
-// the previous dQ_part into dQ in global memory (fp32 vector atomics: the
-// caller's dQ is zeroed first, and the order of the additions is not fixed).
-// dK and dV rows belong to one CTA and are stored once at the end.  The table
-// gradients collect in shared memory (position: a per-warp diagonal buffer
-// flushed per tile pair; time: a running sum per row, flushed when the bucket
-// changes) and go to global memory with one atomic per touched entry at the end.
+//   S^T = K Q^T and dP^T = V dO^T go to tensor memory; the element warps read
+//   them into registers (after which the next pair's S^T / dP^T may be issued,
+//   so they run during this pair's element work), form P^T and dS^T and write
+//   both, 16-bit, to shared memory; then
+//   dQ_part = dS K (A = dS^T read transposed) goes to one of two tensor-memory
+//   buffers, and dV += P^T dO, dK += dS^T Q accumulate in tensor memory.
+// While the tensor core runs the next pair the element warps stage the
+// previous dQ_part in shared memory and add it to dQ with TMA reduce-adds (the
+// caller's dQ is zeroed first; the order of the additions is not fixed).  dK
+// and dV rows belong to one CTA and are stored once at the end.
+// Table gradients: the position-table gradient goes through per-warp buffers
+// of the 63 diagonals of each 32 x 32 block and then straight to drab_pos
+// (coalesced reductions); the time-table gradient is a running sum per lane,
+// flushed when its bucket changes (per warp aggregated into shared memory, or
+// to global memory in the general path), and the shared sums go to drab_time
+// at the end.
 // Warp roles (576 threads): warps 0-15 element work (thread = one key row:
 // lane quarter warp & 3; 32 of the query tile's 128 rows: column group
-// warp >> 2), warp 16 TMA producer, warp 17 MMA issue (one elected lane).  Per
-// element the time bucket comes from an exact incremental walk over the
-// thread's increasing time differences, and the position bias from the tile
-// pair's 255-entry band staged in shared memory.  Every wait is bounded.
+// warp >> 2), warp 16 TMA producer, warp 17 MMA issue (one elected lane).
+// The time bias of a block comes from the lane's current bucket ("steady"),
+// its current bucket or the next one (a compare per element), or, in the
+// general path, the octave table per element; the position bias from the tile
+// pair's 255-entry band staged in shared memory.  Timestamps are
+// non-decreasing within a user.  Every wait is bounded.
 #pragma once
 
 #include "attn.cuh"

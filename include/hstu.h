@@ -204,11 +204,14 @@ typedef struct {
  *               HSTU_FP32 return HSTU_ERR_UNSUPPORTED
  *   jag         causal only (segments must be NULL)
  *   q, k, v, d_o device [T, H*64] in the operand type, 16-byte aligned
- *   dq, dk, dv  device [T, H*64] fp32, written
+ *   dq, dk, dv  device [T, H*64] fp32, written (dq is zeroed, then accumulated
+ *               one key tile at a time with TMA reduce-adds: its summation
+ *               order, and so its last bits, vary from run to run)
  *   drab_pos    device [H, P] fp32, drab_time device [H, Tb] fp32: overwritten
- *               (zeroed, then accumulated with atomics: the summation order,
- *               and so the last bits, vary from run to run)
- * Runs two tcgen05 kernels (dK/dV with the table gradients, then dQ). */
+ *               (zeroed, then accumulated with atomics; the same holds)
+ * Timestamps must be non-decreasing within each user.  Runs one tcgen05 kernel
+ * (one CTA per head, user and 128-key tile).  HSTU_ERR_UNSUPPORTED when the
+ * time-bucket table does not fit the octave lookup (as for the forward). */
 hstu_status_t hstu_attn_bwd(const hstu_layer_cfg_t* cfg, const hstu_jagged_t* jag,
                             const void* q, const void* k, const void* v, const void* d_o,
                             const float* rab_pos, const float* rab_time, float* dq, float* dk,
@@ -287,7 +290,7 @@ size_t hstu_layer_bwd_workspace_bytes(const hstu_layer_cfg_t* cfg, int64_t total
  * passes.  Then:
  *   dG = dY W2, dW2 = dY^T G, db2 = sum dY                  (GEMMs: cuBLAS, TF32)
  *   dU, dAV, dgamma, dbeta through G = LayerNorm(AV) (.) U  (one warp per row)
- *   dQ, dK, dV, drab_pos, drab_time                         (hstu_attn_bwd's kernels)
+ *   dQ, dK, dV, drab_pos, drab_time                         (hstu_attn_bwd's kernel)
  *   dZ = [dU | dV | dQ | dK] (.) phi1', db1 = sum dZ,
  *   dW1 = dZ^T X, dX = dY + dZ W1                           (GEMMs: cuBLAS, TF32)
  *   cfg       dtype HSTU_BF16; phi1 ReLU (ReLU'(0) = 0) or identity; phi2
