@@ -36,8 +36,8 @@ def _check(got, want, what):
     assert rel <= REL and ma <= ABS, f"{what}: rel_l2={rel:.3e} max_abs/scale={ma:.3e}"
 
 
-def _run(H, lengths, phi2, dtype, P=512, Tb=128, heads=2, seed=81):
-    ac = make_attn_case(lengths, heads, P, Tb, seed=seed, dtype=dtype)
+def _run(H, lengths, phi2, dtype, P=512, Tb=128, heads=2, seed=81, gap_kind="exp"):
+    ac = make_attn_case(lengths, heads, P, Tb, seed=seed, dtype=dtype, gap_kind=gap_kind)
     rng = np.random.default_rng(seed + 1)
     T = int(ac.offsets[-1])
     do = to_dtype(rng.standard_normal((T, heads * 64), dtype=np.float32) * 0.5, dtype)
@@ -93,6 +93,16 @@ def test_attention_backward_clamped_tables(H):
 def test_attention_backward_long_user(H):
     """A 2000-row user with 8 heads (16 key tiles, the longest-first order)."""
     _run(H, [2000, 77], "silu", "fp16", P=4096, heads=8, seed=85)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_attention_backward_lognormal_timeline(H, dtype):
+    """The long-sequence workload's timeline (log-normal gaps, mu 7, sigma 2):
+    dense bucket changes near the diagonal, slow ones far from it, so the
+    steady, two-bucket and general element paths all occur (a host simulation
+    of the kernel's path choice over these two users: 12% steady, 53%
+    two-bucket, 35% general 32 x 32 blocks)."""
+    _run(H, [1500, 900], "silu", dtype, P=4096, heads=4, seed=87, gap_kind="lognormal")
 
 
 def test_attention_backward_rejects_softmax_and_masks(H):
