@@ -467,14 +467,14 @@ def measure_forward(ctx, name, steps, warmup, with_e2e, sample_clocks=True, batc
         if roof is not None:
             roof["algorithmic_flop_attention"] = counts["attn_flop_per_layer"]
             roof["algorithmic_flop_f2"] = counts["f2_flop_per_layer"]
-            if name == "long-bf16":
+            if name == "long-bf16-fused" and batch is None:
                 roof["traffic"] = traffic_from_profiles("attention_f2_fused")
     else:
         attn_name = "attention" if bf16 else "fp32_attention"
         roof = _roofline(ctx, kernels, attn_name, counts["attn_flop_per_layer"],
                          "hstu_attn_kernel (causal)" if bf16 else "hstu_f32_attn_kernel (causal)",
                          "tensor" if bf16 else "alu")
-        if roof is not None and name == "long-bf16":
+        if roof is not None and name == "long-bf16" and batch is None:
             roof["traffic"] = traffic_from_profiles("attention")
     kern = _kernel_table(kernels)
     for kname, key in (("f1_gemm", "f1_flop_per_layer"), ("f2_gemm", "f2_flop_per_layer")):
@@ -669,7 +669,7 @@ def measure_train(ctx, steps, warmup, sample_clocks=False, batch=None):
                 "bound": "tensor",
                 "achieved": ach, "peak": ctx.peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": ach / ctx.peaks["bf16_tflops"],
-                "traffic": traffic_from_profiles("attention_bwd"),
+                "traffic": traffic_from_profiles("attention_bwd") if batch is None else None,
                 "peak_source": f"{ctx.peak_src} bf16 dense, burst ({PEAK_RULE})",
                 "algorithmic_flop_per_launch": bwd_flop,
                 "flop_rule": "5 x 2 x 64 flop per visible (i, j, head): S, dP, dV, dQ, dK",
