@@ -257,7 +257,9 @@ def attn_fwd_f32(cfg: LayerConfig, jag: Jagged, q, k, v, rab_pos, rab_time, av_o
 
 def attn_bwd(cfg: LayerConfig, jag: Jagged, q, k, v, d_o, rab_pos, rab_time, stream=None):
     """Backward of the causal attention: returns dq, dk, dv ([T, H*64] fp32) and
-    drab_pos [H, P], drab_time [H, Tb] (fp32) for dO = d_o."""
+    drab_pos [H, P], drab_time [H, Tb] (fp32) for dO = d_o.  dq and the table
+    gradients are sums of reductions in no fixed order: their last bits vary
+    from run to run."""
     dev = rab_pos.device
     T, hv = jag.total_tokens, cfg.num_heads * cfg.dv
     dq, dk, dv = (torch.empty((max(T, 1), hv), dtype=torch.float32, device=dev) for _ in range(3))
